@@ -1,0 +1,163 @@
+"""Pins for the oracle's FP8 E4M3 codec and per-group quantizer (CPU only).
+
+The codec is pinned to the format definition (fixed points from the specification, a brute
+force nearest-value search, ties-to-even at every midpoint); the quantizer to the IEEE fp32
+rounding of its scale (numpy float32 arithmetic) and to the half-spacing error bound.
+"""
+import math
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _all_finite_codes():
+    return np.array([c for c in range(256) if (c & 0x7F) != 0x7F], dtype=np.uint8)
+
+
+def test_spec_points():
+    for line in open(os.path.join(GOLDEN, "e4m3_spec_points.txt")):
+        line = line.split("#")[0].strip()
+        if not line:
+            continue
+        code, val = line.split()
+        got = float(oracle.e4m3_decode(np.uint8(int(code, 16))))
+        if val == "nan":
+            assert math.isnan(got)
+        else:
+            assert got == float(val), (code, got, val)
+            if val.startswith("-"):
+                assert math.copysign(1.0, got) < 0
+
+
+def test_decode_table_structure():
+    codes = _all_finite_codes()
+    assert len(codes) == 254
+    vals = oracle.e4m3_decode(codes)
+    pos = oracle.e4m3_decode(np.arange(0, 0x7F, dtype=np.uint8))
+    # strictly increasing in the code for the positive half, sign bit mirrors
+    assert np.all(np.diff(pos) > 0)
+    neg = oracle.e4m3_decode(np.arange(0x80, 0xFF, dtype=np.uint8))
+    assert np.array_equal(neg, -pos)
+    assert vals.max() == 448.0 and vals.min() == -448.0
+    # 3 mantissa bits: every positive normal value times 8 / 2^floor(log2 v) is an integer in [8, 16)
+    for v in pos[8:]:
+        e = math.floor(math.log2(v))
+        m = v / 2.0 ** e * 8
+        assert m == int(m) and 8 <= m < 16
+
+
+def _brute_encode(x: float, table_codes, table_vals) -> int:
+    """Nearest finite E4M3 value by exhaustive search; a tie goes to the even code; values beyond
+    the largest finite magnitude saturate."""
+    if x > 448.0:
+        x = 448.0
+    if x < -448.0:
+        x = -448.0
+    d = np.abs(table_vals - x)
+    best = d.min()
+    cands = [int(c) for c, dd in zip(table_codes, d) if dd == best]
+    if len(cands) > 1:
+        cands = [c for c in cands if c % 2 == 0] or cands
+        # +0 / -0 tie: follow the sign of x
+        if set(cands) == {0x00, 0x80}:
+            return 0x80 if math.copysign(1.0, x) < 0 else 0x00
+    if len(cands) == 2 and set(cands) == {0x00, 0x80}:
+        return 0x80 if math.copysign(1.0, x) < 0 else 0x00
+    return cands[0]
+
+
+def test_encode_matches_exhaustive_search():
+    codes = _all_finite_codes()
+    vals = oracle.e4m3_decode(codes)
+    rng = np.random.default_rng(123)
+    xs = np.concatenate([
+        rng.standard_normal(3000).astype(np.float32) * np.float32(50),
+        rng.standard_normal(2000).astype(np.float32) * np.float32(0.01),
+        rng.uniform(-500, 500, 1000).astype(np.float32),
+    ])
+    enc = oracle.e4m3_encode(xs)
+    for x, c in zip(xs, enc):
+        assert int(c) == _brute_encode(float(x), codes, vals), (x, c)
+
+
+def test_round_trip_and_midpoints_ties_to_even():
+    codes = np.arange(0, 0x7F, dtype=np.uint8)
+    vals = oracle.e4m3_decode(codes)
+    assert np.array_equal(oracle.e4m3_encode(vals.astype(np.float32)), codes)
+    mids = ((vals[:-1] + vals[1:]) / 2).astype(np.float32)
+    assert np.array_equal(mids.astype(np.float64), (vals[:-1] + vals[1:]) / 2)  # exact in fp32
+    enc = oracle.e4m3_encode(mids).astype(int)
+    lo, hi = codes[:-1].astype(int), codes[1:].astype(int)
+    expect = np.where(lo % 2 == 0, lo, hi)
+    assert np.array_equal(enc, expect)
+    # negative side mirrors
+    assert np.array_equal(oracle.e4m3_encode(-mids).astype(int), expect | 0x80)
+    # saturation just above the largest finite value, and far above
+    for x in (448.0 * (1 + 2 ** -10), 464.0, 479.0, 480.0, 1e6):
+        assert int(oracle.e4m3_encode(np.float32(x))) == 0x7E
+        assert int(oracle.e4m3_encode(np.float32(-x))) == 0xFE
+
+
+def test_quantize_scale_rule_and_error_bound():
+    rng = np.random.default_rng(7)
+    x = rng.standard_normal((64, 128)).astype(np.float32)
+    x[3] = 0.0
+    x[5, :] = np.float32(1e-30)
+    codes, scales = oracle.quantize_rows(x, 128)
+    amax = np.abs(x).max(axis=1)
+    with np.errstate(divide="ignore"):
+        exp_scale = np.where(amax == 0, np.float32(1), amax / np.float32(448))
+    assert np.array_equal(scales[:, 0], exp_scale.astype(np.float32))
+    assert np.all(codes[3] == 0) and scales[3, 0] == 1.0
+    # the amax element maps to the largest code magnitude
+    for r in range(64):
+        if amax[r] > 0:
+            j = int(np.abs(x[r]).argmax())
+            assert (int(codes[r, j]) & 0x7F) == 0x7E
+    # dequantization error <= half the E4M3 spacing at the scaled value, times the scale
+    deq = oracle.dequantize_rows(codes, scales, 128)
+    with np.errstate(divide="ignore"):
+        inv = np.where(amax == 0, 0, (np.float32(448) / amax).astype(np.float32))
+    y = np.abs(x.astype(np.float64) * inv[:, None].astype(np.float64))
+    spacing = np.where(y < 2.0 ** -6, 2.0 ** -9, 2.0 ** (np.floor(np.log2(np.maximum(y, 1e-300))) - 3))
+    bound = 0.5 * spacing * scales[:, :1].astype(np.float64) * (1 + 1e-6) + 1e-45
+    assert np.all(np.abs(deq - x) <= bound + np.abs(x) * 1e-6)
+
+
+def test_group_32_variant_shares_scales_per_group():
+    rng = np.random.default_rng(8)
+    x = rng.standard_normal((4, 128)).astype(np.float32)
+    x[:, 32:64] *= 100
+    codes, scales = oracle.quantize_rows(x, 32)
+    assert scales.shape == (4, 4)
+    for g in range(4):
+        sub_c, sub_s = oracle.quantize_rows(np.ascontiguousarray(x[:, 32 * g:32 * (g + 1)]), 32)
+        assert np.array_equal(sub_c, codes[:, 32 * g:32 * (g + 1)])
+        assert np.array_equal(sub_s[:, 0], scales[:, g])
+
+
+def test_pages_quantization_table_and_storage_claim():
+    rows = {}
+    claim = None
+    for line in open(os.path.join(GOLDEN, "tiered_quantization.txt")):
+        line = line.split("#")[0].strip()
+        if not line:
+            continue
+        parts = line.split()
+        if parts[0] == "index_storage_ratio_claim":
+            claim = float(parts[1])
+        else:
+            rows[parts[0]] = (parts[1], int(parts[2]))
+    assert rows["index_qk"] == ("fp8", 32) and rows["kv_cache"] == ("fp8", 128)
+    # FP8 key of 128 dims: one byte per element plus the fp32 scales, against two bytes per
+    # element in bf16.  Per-key scale (this build's index cache) and group-32 scales both land
+    # near the pages' "about half".
+    D = 128
+    for group in (D, rows["index_qk"][1]):
+        ratio = (D + 4 * (D // group)) / (2 * D)
+        assert abs(ratio - claim) < 0.07, ratio
