@@ -1,0 +1,214 @@
+/*
+ * hsa.h -- C ABI of the sparse index attention library (libhsa.so) for NVIDIA B200 (sm_100a).
+ *
+ * The path, as the source pages state the problem ("Day 0 Inference Adaptation and
+ * Optimization for Hybrid Attention Models", section "Sparse Attention Pipeline Optimization";
+ * "Inference Adaptation and Performance Optimization for a Domestically Developed LLM's New
+ * Architecture", section 3):
+ *   1. a lightweight indexer scores every causal history position of every query row,
+ *        I[t,s] = sum_j w[t,j] * ReLU( q_I[t,j,:] . k_I[s,:] ),   0 <= s <= p_t;
+ *   2. a per-row Top-K keeps the K best positions (ties toward the lower position; rows with
+ *      p_t + 1 <= K keep all of them);
+ *   3. sparse MLA attention reads only the selected rows of the paged latent KV cache
+ *      (latent c_kv || rope part per position, shared by every head) and attends over them.
+ * FP8 storage of index keys and latent KV ("Hierarchical Quantization" on the first page;
+ * the table of section 4 on the fifth) is written by hsa_quantize_index / hsa_quantize_kv.
+ *
+ * Conventions shared by every call
+ *  - Memory: every tensor is caller-owned device memory, row-major and contiguous unless a
+ *    stride is given.  The library never allocates device memory.  Calls that need scratch take
+ *    a workspace pointer and size; hsa_*_workspace_size() reports the bytes needed.
+ *  - Streams: every call is asynchronous on the cudaStream_t passed in as `stream` (NULL = the
+ *    legacy default stream).  Host-side argument checks happen before anything is enqueued.
+ *  - Errors: every call returns an hsa_status_t.  HSA_ERR_INVALID_ARG: null pointer, size out of
+ *    range, misaligned pointer; HSA_ERR_UNSUPPORTED: a dtype / shape combination no kernel
+ *    implements; HSA_ERR_WORKSPACE: workspace too small; HSA_ERR_CUDA: a launch failed
+ *    (hsa_last_error_message() names it).  Nothing is enqueued when a call returns an error.
+ *  - Device-side checks: every kernel validates the page ids it reads from the block table, the
+ *    positions it reads (q_pos < seq_len, selected index in [0, q_pos]) and the row grouping it
+ *    relies on.  A failed check never faults: the access is skipped or redirected to page 0 and
+ *    a bit is OR-ed into *seq->status (if non-null), so results are then undefined but the
+ *    context stays usable.  Bits: HSA_DEV_BAD_PAGE, HSA_DEV_BAD_POS, HSA_DEV_BAD_GROUP.
+ *  - Threading: no mutable global state beyond a per-thread error message; calls on different
+ *    streams may be issued from different host threads.
+ */
+#ifndef HSA_H_
+#define HSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define HSA_API __attribute__((visibility("default")))
+#else
+#define HSA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum hsa_status {
+    HSA_OK = 0,
+    HSA_ERR_INVALID_ARG = 1,
+    HSA_ERR_UNSUPPORTED = 2,
+    HSA_ERR_CUDA = 3,
+    HSA_ERR_WORKSPACE = 4
+} hsa_status_t;
+
+typedef enum hsa_dtype {
+    HSA_F32 = 0,   /* IEEE binary32 */
+    HSA_BF16 = 1,  /* bfloat16 */
+    HSA_E4M3 = 2   /* OCP FP8 E4M3 code, one byte; paired with fp32 scales */
+} hsa_dtype_t;
+
+/* device status bits (OR-ed into *hsa_paged_seq_t.status) */
+#define HSA_DEV_BAD_PAGE 1u   /* block_table entry outside [0, num_pages) */
+#define HSA_DEV_BAD_POS 2u    /* q_pos >= seq_len, or a selected index outside [0, q_pos] */
+#define HSA_DEV_BAD_GROUP 4u  /* rows of one q_run disagree on their sequence */
+
+/* Paged sequences and query rows.
+ * Position s of sequence b lives in physical slot
+ *     block_table[b * bt_stride + s / page_size] * page_size + s % page_size
+ * of every paged cache ("reads from the paged K cache", first page, "Sparse Attention Pipeline
+ * Optimization"; gather through the page table, third page, 3.1).  Query row t belongs to
+ * sequence q_seq[t] at absolute position q_pos[t] and sees positions 0..q_pos[t] (the causal
+ * mask is generated from q_pos inside the kernels, with per-row offsets instead of a
+ * per-sequence host loop, third page 3.1).  Top-K outputs are positions in this logical
+ * numbering, the representation shared with the cache layer (third page, section 4). */
+typedef struct hsa_paged_seq {
+    int32_t B;                   /* number of sequences, >= 1 */
+    const int32_t* seq_lens;     /* device [B]: context length of each sequence */
+    const int32_t* block_table;  /* device [B, bt_stride]: physical page of each logical page */
+    int64_t bt_stride;           /* elements between consecutive sequences' rows */
+    int32_t page_size;           /* slots per page, >= 1 */
+    int32_t num_pages;           /* physical pages in every paged cache */
+    int32_t max_seq_len;         /* host-side upper bound of seq_lens[] (sizes launch grids) */
+    int32_t T_q;                 /* number of query rows, >= 0 */
+    const int32_t* q_seq;        /* device [T_q]: sequence of each query row */
+    const int32_t* q_pos;        /* device [T_q]: absolute position of each query row */
+    int32_t q_run;               /* rows come in runs of q_run consecutive rows of one sequence
+                                    (the last run may be shorter); 1 = no promise */
+    uint32_t* status;            /* device, nullable: device-side check bits are OR-ed here */
+} hsa_paged_seq_t;
+
+/* ---- 1. index score ---------------------------------------------------------------------
+ * scores[t, s] = sum_{j<H_I} w[t,j] * max(0, sum_{d<D_I} q_I[t,j,d] * k(slot(t,s), d))
+ * for 0 <= s <= q_pos[t]; entries s > q_pos[t] are not written.
+ *   q_I      device [T_q, H_I, D_I], q_dtype F32 or BF16
+ *   w        device fp32 [T_q, H_I] (head weights)
+ *   k_cache  device [num_pages * page_size, D_I] of k_dtype F32, BF16 or E4M3
+ *   k_scale  device fp32 [num_pages * page_size] when k_dtype == E4M3 (key = code * scale),
+ *            else NULL
+ *   scores   device fp32 [T_q, ld_scores], ld_scores >= max_seq_len
+ * Pages: first page "Sparse Attention Pipeline Optimization" (correlation scoring with
+ * head-weight weighted summation over the paged K cache); fifth page 3.1 (LI); BF16 and
+ * quantized index paths, second page 3.1.  The tensor-core kernel serves q BF16, k BF16/E4M3,
+ * H_I = 64, D_I = 128, page_size a multiple of 8; other shapes use a CUDA-core kernel. */
+HSA_API hsa_status_t hsa_index_score(const hsa_paged_seq_t* seq, const void* q_I, hsa_dtype_t q_dtype,
+                             const float* w, int32_t H_I, int32_t D_I, const void* k_cache,
+                             hsa_dtype_t k_dtype, const float* k_scale, float* scores,
+                             int64_t ld_scores, void* stream);
+
+/* ---- 2. Top-K -----------------------------------------------------------------------------
+ * For row t with n = q_pos[t] + 1 candidate positions:
+ *   n <= K : idx[t] = 0, 1, ..., n-1, then -1 up to K;
+ *   n >  K : the K positions first in the order (score descending, position ascending),
+ *            written in ascending position order.  +0.0 and -0.0 are equal; NaN is outside the
+ *            contract.
+ *   scores  device fp32 [T_q, ld_scores] (entries past q_pos[t] are ignored)
+ *   idx     device int32 [T_q, K], 1 <= K <= 65536
+ * Pages: first page "Sparse Attention Pipeline Optimization" (Top-K of the weighted scores);
+ * third page 3.1 (selection).  Needs no workspace. */
+HSA_API hsa_status_t hsa_topk(const hsa_paged_seq_t* seq, const float* scores, int64_t ld_scores,
+                      int32_t K, int32_t* idx, void* stream);
+
+/* ---- 3. sparse MLA attention -----------------------------------------------------------
+ * For row t, head h, over S_t = { idx[t,k] != -1 }:
+ *   z_n = softmax_scale * sum_{d<D_qk} q[t,h,d] * key(n, d)
+ *   out[t,h,:] = sum_n e^{z_n - m} * key(n, 0:D_v) / sum_n e^{z_n - m},  m = max_n z_n
+ *   lse[t,h]   = m + log sum_n e^{z_n - m}        (empty S_t: out = 0, lse = -inf)
+ * where key(n, :) is cache row slot(t, n): the latent part (D_v values, also the value) followed
+ * by the rope part (D_qk - D_v values).
+ *   q        device [T_q, H, D_qk], q_dtype F32 or BF16
+ *   kv       kv_dtype F32 / BF16: device [slots, D_qk] packed latent || rope; kv_rope = NULL
+ *            kv_dtype E4M3: device uint8 [slots, D_v] latent codes, kv_scale fp32 [slots]
+ *            (one per token), kv_rope BF16 [slots, D_qk - D_v]
+ *   idx      device int32 [T_q, K]: positions in [0, q_pos[t]] or -1
+ *   out      device [T_q, H, D_v] of out_dtype (F32 or BF16)
+ *   lse      device fp32 [T_q, H] or NULL
+ *   ws       workspace of at least hsa_sparse_mla_workspace_size() bytes, 256-byte aligned
+ * Pages: first page "Sparse Attention Pipeline Optimization" (indexed reads, block-wise fused
+ * attention); third page 3.2 (partition by query, aggregate over the selected positions,
+ * stage them in shared memory); fifth page 3 (SFA).  The tensor-core kernel serves q BF16,
+ * kv BF16 or E4M3, H = 128, D_qk = 576, D_v = 512; other shapes use a CUDA-core kernel. */
+HSA_API size_t hsa_sparse_mla_workspace_size(const hsa_paged_seq_t* seq, int32_t H, int32_t D_qk,
+                                     int32_t D_v, int32_t K);
+HSA_API hsa_status_t hsa_sparse_mla_attn(const hsa_paged_seq_t* seq, const void* q, hsa_dtype_t q_dtype,
+                                 int32_t H, int32_t D_qk, int32_t D_v, const void* kv,
+                                 hsa_dtype_t kv_dtype, const float* kv_scale, const void* kv_rope,
+                                 const int32_t* idx, int32_t K, float softmax_scale, void* out,
+                                 hsa_dtype_t out_dtype, float* lse, void* ws, size_t ws_bytes,
+                                 void* stream);
+
+/* ---- 4. fused decode step -----------------------------------------------------------------
+ * hsa_index_score -> hsa_topk -> hsa_sparse_mla_attn on the same rows, results bitwise equal
+ * to the three calls in sequence.  scores ([T_q, ld_scores] fp32) and idx ([T_q, K] int32) are
+ * caller buffers that hold the intermediate results afterwards.  With stream_aux != NULL the
+ * rows are split in two halves; the second half runs on stream_aux, overlapping the first
+ * half's attention (event-ordered; stream_main waits for stream_aux before returning work to
+ * the caller).  Pages: first page "Sparse Attention Pipeline Optimization" (fuse where
+ * possible, parallelize where possible: indexer then sparse attention kernel; multi-stream
+ * orchestration); fifth page 3.3 (operators on independent streams with event
+ * synchronization). */
+typedef struct hsa_index_args {
+    const void* q_I; hsa_dtype_t q_dtype; const float* w; int32_t H_I; int32_t D_I;
+    const void* k_cache; hsa_dtype_t k_dtype; const float* k_scale;
+} hsa_index_args_t;
+
+typedef struct hsa_attn_args {
+    const void* q; hsa_dtype_t q_dtype; int32_t H; int32_t D_qk; int32_t D_v;
+    const void* kv; hsa_dtype_t kv_dtype; const float* kv_scale; const void* kv_rope;
+    float softmax_scale; void* out; hsa_dtype_t out_dtype; float* lse;
+} hsa_attn_args_t;
+
+HSA_API size_t hsa_fused_decode_workspace_size(const hsa_paged_seq_t* seq, const hsa_attn_args_t* attn,
+                                       int32_t K);
+HSA_API hsa_status_t hsa_fused_decode(const hsa_paged_seq_t* seq, const hsa_index_args_t* index,
+                              const hsa_attn_args_t* attn, int32_t K, float* scores,
+                              int64_t ld_scores, int32_t* idx, void* ws, size_t ws_bytes,
+                              void* stream_main, void* stream_aux);
+
+/* ---- 5. FP8 quantizers (cache write) --------------------------------------------------------
+ * Per row r and group g of `group` consecutive elements:
+ *   amax = max |x|; scale = amax / 448 (fp32, round to nearest); inv = 448 / amax (fp32);
+ *   code = E4M3(round-to-nearest-even, saturating, of x * inv);   amax == 0: scale 1, codes 0.
+ * Row r is written to physical slot slot_mapping[r] (slot_mapping NULL: slot r).
+ * hsa_quantize_index: src [n_rows, D] F32/BF16 -> codes uint8 [slots, D], scales fp32
+ *   [slots, D / group].  group = D gives one scale per key (the layout hsa_index_score reads);
+ *   group = 32 is the pages' group size (MXFP8-style granularity with fp32 scales).
+ * hsa_quantize_kv: src [n_rows, D_v + D_rope] F32/BF16 (latent || rope) -> latent codes uint8
+ *   [slots, D_v], scales fp32 [slots, D_v / group], rope copied to rope_cache BF16
+ *   [slots, D_rope].  group = D_v gives one scale per token (the layout hsa_sparse_mla_attn
+ *   reads); group = 128 is the pages' tile size.
+ * Pages: first page "Hierarchical Quantization"; second page 4.1 and 4.2; fifth page 4 (table:
+ * index Q/K group 32, KV cache tile 128, dynamic scales). */
+HSA_API hsa_status_t hsa_quantize_index(const void* src, hsa_dtype_t src_dtype, int64_t n_rows,
+                                int32_t D, int32_t group, const int64_t* slot_mapping,
+                                int64_t num_slots, uint8_t* codes, float* scales, void* stream);
+HSA_API hsa_status_t hsa_quantize_kv(const void* src, hsa_dtype_t src_dtype, int64_t n_rows, int32_t D_v,
+                             int32_t D_rope, int32_t group, const int64_t* slot_mapping,
+                             int64_t num_slots, uint8_t* codes, float* scales, void* rope_cache,
+                             void* stream);
+
+/* ---- diagnostics -------------------------------------------------------------------------- */
+HSA_API const char* hsa_status_string(hsa_status_t s);
+/* Text of the last error raised by a call on this host thread ("" if none). */
+HSA_API const char* hsa_last_error_message(void);
+/* Library version, major * 10000 + minor * 100 + patch. */
+HSA_API int32_t hsa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* HSA_H_ */

@@ -1,1 +1,287 @@
-"""Sparse index attention on B200: indexer score -> Top-K -> sparse MLA over a paged latent cache."""
+"""Sparse index attention on B200: indexer score -> Top-K -> sparse MLA over a paged latent cache.
+
+Thin Python binding of ``libhsa.so`` (C ABI in ``include/hsa.h``).  Every function here only
+marshals torch tensors into pointers and sizes and calls the C entry point of the same name; all
+computation happens in the library's CUDA kernels.  Output tensors that the caller does not pass
+are allocated with torch on the input's device (PyTorch provides device memory and streams).
+
+The library is loaded on first use; if ``libhsa.so`` has not been built the call raises
+``RuntimeError`` -- there is no fallback path.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libhsa.so")
+
+HSA_OK, HSA_ERR_INVALID_ARG, HSA_ERR_UNSUPPORTED, HSA_ERR_CUDA, HSA_ERR_WORKSPACE = 0, 1, 2, 3, 4
+HSA_F32, HSA_BF16, HSA_E4M3 = 0, 1, 2
+HSA_DEV_BAD_PAGE, HSA_DEV_BAD_POS, HSA_DEV_BAD_GROUP = 1, 2, 4
+
+_P = ctypes.c_void_p
+_i32, _i64, _sz, _f32 = ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t, ctypes.c_float
+
+
+class hsa_paged_seq_t(ctypes.Structure):
+    _fields_ = [("B", _i32), ("seq_lens", _P), ("block_table", _P), ("bt_stride", _i64),
+                ("page_size", _i32), ("num_pages", _i32), ("max_seq_len", _i32), ("T_q", _i32),
+                ("q_seq", _P), ("q_pos", _P), ("q_run", _i32), ("status", _P)]
+
+
+class hsa_index_args_t(ctypes.Structure):
+    _fields_ = [("q_I", _P), ("q_dtype", ctypes.c_int), ("w", _P), ("H_I", _i32), ("D_I", _i32),
+                ("k_cache", _P), ("k_dtype", ctypes.c_int), ("k_scale", _P)]
+
+
+class hsa_attn_args_t(ctypes.Structure):
+    _fields_ = [("q", _P), ("q_dtype", ctypes.c_int), ("H", _i32), ("D_qk", _i32), ("D_v", _i32),
+                ("kv", _P), ("kv_dtype", ctypes.c_int), ("kv_scale", _P), ("kv_rope", _P),
+                ("softmax_scale", _f32), ("out", _P), ("out_dtype", ctypes.c_int), ("lse", _P)]
+
+
+SYMBOLS = {
+    "hsa_index_score": (ctypes.c_int, [_P, _P, ctypes.c_int, _P, _i32, _i32, _P, ctypes.c_int, _P,
+                                       _P, _i64, _P]),
+    "hsa_topk": (ctypes.c_int, [_P, _P, _i64, _i32, _P, _P]),
+    "hsa_sparse_mla_workspace_size": (_sz, [_P, _i32, _i32, _i32, _i32]),
+    "hsa_sparse_mla_attn": (ctypes.c_int, [_P, _P, ctypes.c_int, _i32, _i32, _i32, _P, ctypes.c_int,
+                                           _P, _P, _P, _i32, _f32, _P, ctypes.c_int, _P, _P, _sz,
+                                           _P]),
+    "hsa_fused_decode_workspace_size": (_sz, [_P, _P, _i32]),
+    "hsa_fused_decode": (ctypes.c_int, [_P, _P, _P, _i32, _P, _i64, _P, _P, _sz, _P, _P]),
+    "hsa_quantize_index": (ctypes.c_int, [_P, ctypes.c_int, _i64, _i32, _i32, _P, _i64, _P, _P, _P]),
+    "hsa_quantize_kv": (ctypes.c_int, [_P, ctypes.c_int, _i64, _i32, _i32, _i32, _P, _i64, _P, _P,
+                                       _P, _P]),
+    "hsa_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "hsa_last_error_message": (ctypes.c_char_p, []),
+    "hsa_version": (_i32, []),
+}
+
+_lock = threading.Lock()
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libhsa.so (raises RuntimeError if it was not built)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                raise RuntimeError(
+                    f"{LIB_PATH} is missing: build it with `python -m sparse_index_attention_b200.build`"
+                    " (the CUDA library is required; there is no fallback)")
+            L = ctypes.CDLL(LIB_PATH)
+            for name, (res, args) in SYMBOLS.items():
+                f = getattr(L, name)
+                f.restype = res
+                f.argtypes = args
+            _lib = L
+    return _lib
+
+
+class HsaError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        L = lib()
+        msg = L.hsa_last_error_message().decode()
+        super().__init__(f"{where}: {L.hsa_status_string(status).decode()}: {msg}")
+        self.status = status
+
+
+def _check(rc: int, where: str):
+    if rc != HSA_OK:
+        raise HsaError(rc, where)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    if t is None:
+        return None
+    if not t.is_contiguous():
+        raise ValueError("tensor must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _dtype(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return HSA_F32
+    if t.dtype == torch.bfloat16:
+        return HSA_BF16
+    if t.dtype in (torch.uint8, getattr(torch, "float8_e4m3fn", torch.uint8)):
+        return HSA_E4M3
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _stream(s) -> ctypes.c_void_p:
+    if s is None:
+        s = torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+class PagedSeq:
+    """Paged sequences + query rows (hsa_paged_seq_t).  Keeps its tensors alive."""
+
+    def __init__(self, seq_lens, block_table, page_size: int, num_pages: int, q_seq, q_pos,
+                 max_seq_len: Optional[int] = None, q_run: int = 1, status=None):
+        self.seq_lens = seq_lens.to(torch.int32).contiguous()
+        self.block_table = block_table.to(torch.int32).contiguous()
+        self.q_seq = q_seq.to(torch.int32).contiguous()
+        self.q_pos = q_pos.to(torch.int32).contiguous()
+        self.status = status
+        self.page_size, self.num_pages, self.q_run = int(page_size), int(num_pages), int(q_run)
+        self.max_seq_len = int(max_seq_len if max_seq_len is not None else self.seq_lens.max().item())
+        self.T_q = int(self.q_seq.shape[0])
+        self.B = int(self.seq_lens.shape[0])
+        self.c = hsa_paged_seq_t(self.B, _ptr(self.seq_lens), _ptr(self.block_table),
+                                 int(self.block_table.shape[1]), self.page_size, self.num_pages,
+                                 self.max_seq_len, self.T_q, _ptr(self.q_seq), _ptr(self.q_pos),
+                                 self.q_run, _ptr(status))
+
+    def rows(self, r0: int, r1: int, q_run: Optional[int] = None) -> "PagedSeq":
+        """Descriptor of query rows [r0, r1) (same sequences and caches)."""
+        return PagedSeq(self.seq_lens, self.block_table, self.page_size, self.num_pages,
+                        self.q_seq[r0:r1], self.q_pos[r0:r1], self.max_seq_len,
+                        q_run if q_run is not None else self.q_run, self.status)
+
+    @property
+    def ref(self):
+        return ctypes.byref(self.c)
+
+
+# ------------------------------------------------------------------------------ entry points
+def hsa_index_score(seq: PagedSeq, q_I, w, k_cache, k_scale=None, scores=None, ld: Optional[int] = None,
+                    stream=None):
+    T_q, H_I, D_I = q_I.shape
+    if scores is None:
+        ld = ld or seq.max_seq_len
+        scores = torch.empty((T_q, ld), dtype=torch.float32, device=q_I.device)
+    ld = scores.shape[1]
+    _check(lib().hsa_index_score(seq.ref, _ptr(q_I), _dtype(q_I), _ptr(w), H_I, D_I, _ptr(k_cache),
+                                 _dtype(k_cache), _ptr(k_scale), _ptr(scores), ld, _stream(stream)),
+           "hsa_index_score")
+    return scores
+
+
+def hsa_topk(seq: PagedSeq, scores, K: int, idx=None, stream=None):
+    if idx is None:
+        idx = torch.empty((seq.T_q, K), dtype=torch.int32, device=scores.device)
+    _check(lib().hsa_topk(seq.ref, _ptr(scores), scores.shape[1], K, _ptr(idx), _stream(stream)),
+           "hsa_topk")
+    return idx
+
+
+def hsa_sparse_mla_workspace_size(seq: PagedSeq, H: int, D_qk: int, D_v: int, K: int) -> int:
+    return int(lib().hsa_sparse_mla_workspace_size(seq.ref, H, D_qk, D_v, K))
+
+
+def _workspace(nbytes: int, device, ws):
+    if ws is not None:
+        return ws
+    return torch.empty(max(nbytes, 1), dtype=torch.uint8, device=device)
+
+
+def hsa_sparse_mla_attn(seq: PagedSeq, q, kv, idx, D_v: int, softmax_scale: float, kv_scale=None,
+                        kv_rope=None, out=None, out_dtype=None, lse=True, ws=None, stream=None):
+    """Returns (out [T_q, H, D_v], lse [T_q, H] or None).  kv is the packed [slots, D_qk] cache
+    (fp32/bf16) or the uint8 latent codes [slots, D_v] with kv_scale and kv_rope."""
+    T_q, H, D_qk = q.shape
+    K = idx.shape[1]
+    if out is None:
+        out = torch.empty((T_q, H, D_v), dtype=out_dtype or q.dtype, device=q.device)
+    if lse is True:
+        lse = torch.empty((T_q, H), dtype=torch.float32, device=q.device)
+    elif lse is False:
+        lse = None
+    need = hsa_sparse_mla_workspace_size(seq, H, D_qk, D_v, K)
+    ws = _workspace(need, q.device, ws)
+    _check(lib().hsa_sparse_mla_attn(seq.ref, _ptr(q), _dtype(q), H, D_qk, D_v, _ptr(kv), _dtype(kv),
+                                     _ptr(kv_scale), _ptr(kv_rope), _ptr(idx), K,
+                                     float(softmax_scale), _ptr(out), _dtype(out), _ptr(lse),
+                                     _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
+           "hsa_sparse_mla_attn")
+    return out, lse
+
+
+def _attn_struct(q, kv, D_v, softmax_scale, kv_scale, kv_rope, out, lse):
+    T_q, H, D_qk = q.shape
+    return hsa_attn_args_t(_ptr(q), _dtype(q), H, D_qk, D_v, _ptr(kv), _dtype(kv), _ptr(kv_scale),
+                           _ptr(kv_rope), float(softmax_scale), _ptr(out), _dtype(out), _ptr(lse))
+
+
+def hsa_fused_decode_workspace_size(seq: PagedSeq, q, kv, D_v: int, K: int) -> int:
+    T_q, H, D_qk = q.shape
+    at = hsa_attn_args_t(None, _dtype(q), H, D_qk, D_v, None, _dtype(kv), None, None, 1.0, None,
+                         _dtype(q), None)
+    return int(lib().hsa_fused_decode_workspace_size(seq.ref, ctypes.byref(at), K))
+
+
+def hsa_fused_decode(seq: PagedSeq, q_I, w, k_cache, k_scale, q, kv, kv_scale, kv_rope, K: int,
+                     D_v: int, softmax_scale: float, scores=None, idx=None, out=None, lse=True,
+                     ws=None, stream=None, aux_stream=None):
+    """index score -> Top-K -> sparse MLA in one call.  Returns (out, lse, idx, scores)."""
+    T_q, H_I, D_I = q_I.shape
+    _, H, D_qk = q.shape
+    dev = q.device
+    if scores is None:
+        scores = torch.empty((T_q, seq.max_seq_len), dtype=torch.float32, device=dev)
+    if idx is None:
+        idx = torch.empty((T_q, K), dtype=torch.int32, device=dev)
+    if out is None:
+        out = torch.empty((T_q, H, D_v), dtype=q.dtype, device=dev)
+    if lse is True:
+        lse = torch.empty((T_q, H), dtype=torch.float32, device=dev)
+    elif lse is False:
+        lse = None
+    ws = _workspace(hsa_fused_decode_workspace_size(seq, q, kv, D_v, K), dev, ws)
+    ia = hsa_index_args_t(_ptr(q_I), _dtype(q_I), _ptr(w), H_I, D_I, _ptr(k_cache), _dtype(k_cache),
+                          _ptr(k_scale))
+    at = _attn_struct(q, kv, D_v, softmax_scale, kv_scale, kv_rope, out, lse)
+    _check(lib().hsa_fused_decode(seq.ref, ctypes.byref(ia), ctypes.byref(at), K, _ptr(scores),
+                                  scores.shape[1], _ptr(idx), _ptr(ws), ws.numel(), _stream(stream),
+                                  None if aux_stream is None else ctypes.c_void_p(aux_stream.cuda_stream)),
+           "hsa_fused_decode")
+    return out, lse, idx, scores
+
+
+def hsa_quantize_index(src, group: int, slot_mapping=None, num_slots: Optional[int] = None,
+                       codes=None, scales=None, stream=None):
+    """Rows [n, D] -> (codes uint8 [slots, D], scales fp32 [slots, D/group])."""
+    n, D = src.shape
+    num_slots = num_slots if num_slots is not None else n
+    if codes is None:
+        codes = torch.zeros((num_slots, D), dtype=torch.uint8, device=src.device)
+    if scales is None:
+        scales = torch.zeros((num_slots, D // group), dtype=torch.float32, device=src.device)
+    _check(lib().hsa_quantize_index(_ptr(src), _dtype(src), n, D, group, _ptr(slot_mapping),
+                                    num_slots, _ptr(codes), _ptr(scales), _stream(stream)),
+           "hsa_quantize_index")
+    return codes, scales
+
+
+def hsa_quantize_kv(src, D_v: int, group: int, slot_mapping=None, num_slots: Optional[int] = None,
+                    codes=None, scales=None, rope_cache=None, stream=None):
+    """Rows [n, D_v + D_rope] (latent || rope) -> (codes [slots, D_v], scales [slots, D_v/group],
+    rope bf16 [slots, D_rope])."""
+    n, D = src.shape
+    D_rope = D - D_v
+    num_slots = num_slots if num_slots is not None else n
+    dev = src.device
+    if codes is None:
+        codes = torch.zeros((num_slots, D_v), dtype=torch.uint8, device=dev)
+    if scales is None:
+        scales = torch.zeros((num_slots, D_v // group), dtype=torch.float32, device=dev)
+    if rope_cache is None:
+        rope_cache = torch.zeros((num_slots, max(D_rope, 0)), dtype=torch.bfloat16, device=dev)
+    _check(lib().hsa_quantize_kv(_ptr(src), _dtype(src), n, D_v, D_rope, group, _ptr(slot_mapping),
+                                 num_slots, _ptr(codes), _ptr(scales), _ptr(rope_cache),
+                                 _stream(stream)),
+           "hsa_quantize_kv")
+    return codes, scales, rope_cache
+
+
+def hsa_version() -> int:
+    return int(lib().hsa_version())

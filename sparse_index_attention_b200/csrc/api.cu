@@ -1,0 +1,415 @@
+// api.cu -- the C ABI of libhsa (declared in include/hsa.h): argument validation, kernel
+// dispatch and the two-stream fused decode step.  Every entry point validates its arguments on
+// the host before enqueuing anything and reports failures as hsa_status_t.
+#include <stdarg.h>
+#include <stdio.h>
+
+#include <string>
+
+#include "kernels.h"
+
+namespace {
+
+thread_local std::string g_last_error;
+
+hsa_status_t fail(hsa_status_t s, const char* fmt, ...) __attribute__((format(printf, 2, 3)));
+hsa_status_t fail(hsa_status_t s, const char* fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof(buf), fmt, ap);
+    va_end(ap);
+    g_last_error = buf;
+    return s;
+}
+
+hsa_status_t cuda_status(cudaError_t e, const char* what) {
+    if (e == cudaSuccess) return HSA_OK;
+    return fail(HSA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+#define HSA_REQUIRE(cond, code, ...)                                  \
+    do {                                                              \
+        if (!(cond)) return fail((code), __VA_ARGS__);                \
+    } while (0)
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+size_t dtype_size(hsa_dtype_t d) { return d == HSA_F32 ? 4 : (d == HSA_BF16 ? 2 : 1); }
+
+hsa_status_t check_seq(const hsa_paged_seq_t* s) {
+    HSA_REQUIRE(s != nullptr, HSA_ERR_INVALID_ARG, "seq is NULL");
+    HSA_REQUIRE(s->B >= 1, HSA_ERR_INVALID_ARG, "B = %d must be >= 1", s->B);
+    HSA_REQUIRE(s->seq_lens && s->block_table, HSA_ERR_INVALID_ARG, "seq_lens / block_table NULL");
+    HSA_REQUIRE(s->page_size >= 1 && s->num_pages >= 1, HSA_ERR_INVALID_ARG,
+                "page_size = %d, num_pages = %d must be >= 1", s->page_size, s->num_pages);
+    HSA_REQUIRE(s->max_seq_len >= 1, HSA_ERR_INVALID_ARG, "max_seq_len = %d must be >= 1",
+                s->max_seq_len);
+    HSA_REQUIRE(s->bt_stride >= hsa::ceil_div(s->max_seq_len, s->page_size), HSA_ERR_INVALID_ARG,
+                "bt_stride = %lld cannot hold ceil(max_seq_len / page_size) pages",
+                (long long)s->bt_stride);
+    HSA_REQUIRE(s->T_q >= 0, HSA_ERR_INVALID_ARG, "T_q = %d < 0", s->T_q);
+    HSA_REQUIRE(s->T_q == 0 || (s->q_seq && s->q_pos), HSA_ERR_INVALID_ARG, "q_seq / q_pos NULL");
+    HSA_REQUIRE(s->q_run >= 1, HSA_ERR_INVALID_ARG, "q_run = %d must be >= 1", s->q_run);
+    return HSA_OK;
+}
+
+hsa::SeqView view(const hsa_paged_seq_t* s) { return hsa::make_view(*s); }
+
+// Row window [t0, t0 + n) of a descriptor (used by the fused call's two halves).
+hsa_paged_seq_t sub_rows(const hsa_paged_seq_t& s, int32_t t0, int32_t n) {
+    hsa_paged_seq_t r = s;
+    r.T_q = n;
+    r.q_seq = s.q_seq + t0;
+    r.q_pos = s.q_pos + t0;
+    return r;
+}
+
+hsa_status_t check_index(const hsa_paged_seq_t* seq, const void* q_I, hsa_dtype_t q_dtype,
+                         const float* w, int32_t H_I, int32_t D_I, const void* k_cache,
+                         hsa_dtype_t k_dtype, const float* k_scale, const float* scores,
+                         int64_t ld) {
+    hsa_status_t st = check_seq(seq);
+    if (st != HSA_OK) return st;
+    HSA_REQUIRE(H_I >= 1 && H_I <= 256 && D_I >= 1 && D_I <= 1024, HSA_ERR_INVALID_ARG,
+                "H_I = %d, D_I = %d out of range", H_I, D_I);
+    HSA_REQUIRE((size_t)H_I * D_I * 4 <= 160 * 1024, HSA_ERR_UNSUPPORTED,
+                "H_I * D_I = %d too large", H_I * D_I);
+    HSA_REQUIRE(q_dtype == HSA_F32 || q_dtype == HSA_BF16, HSA_ERR_UNSUPPORTED,
+                "q_I dtype must be F32 or BF16");
+    HSA_REQUIRE(k_dtype == HSA_F32 || k_dtype == HSA_BF16 || k_dtype == HSA_E4M3,
+                HSA_ERR_UNSUPPORTED, "k dtype must be F32, BF16 or E4M3");
+    HSA_REQUIRE(ld >= seq->max_seq_len, HSA_ERR_INVALID_ARG, "ld_scores = %lld < max_seq_len",
+                (long long)ld);
+    if (seq->T_q > 0) {
+        HSA_REQUIRE(q_I && w && k_cache && scores, HSA_ERR_INVALID_ARG, "NULL tensor pointer");
+        HSA_REQUIRE(k_dtype != HSA_E4M3 || k_scale, HSA_ERR_INVALID_ARG,
+                    "E4M3 keys need k_scale");
+        HSA_REQUIRE(aligned(q_I, dtype_size(q_dtype)) && aligned(w, 4) && aligned(scores, 4) &&
+                        aligned(k_cache, dtype_size(k_dtype)),
+                    HSA_ERR_INVALID_ARG, "misaligned tensor pointer");
+    }
+    return HSA_OK;
+}
+
+hsa_status_t check_attn(const hsa_paged_seq_t* seq, const void* q, hsa_dtype_t q_dtype, int32_t H,
+                        int32_t D_qk, int32_t D_v, const void* kv, hsa_dtype_t kv_dtype,
+                        const float* kv_scale, const void* kv_rope, const int32_t* idx, int32_t K,
+                        const void* out, hsa_dtype_t out_dtype) {
+    hsa_status_t st = check_seq(seq);
+    if (st != HSA_OK) return st;
+    HSA_REQUIRE(H >= 1 && H <= 1024, HSA_ERR_INVALID_ARG, "H = %d out of range", H);
+    HSA_REQUIRE(D_v >= 1 && D_v <= D_qk && D_qk <= 2048, HSA_ERR_INVALID_ARG,
+                "D_qk = %d, D_v = %d out of range", D_qk, D_v);
+    HSA_REQUIRE(K >= 1 && K <= 65536, HSA_ERR_INVALID_ARG, "K = %d out of range", K);
+    HSA_REQUIRE(q_dtype == HSA_F32 || q_dtype == HSA_BF16, HSA_ERR_UNSUPPORTED,
+                "q dtype must be F32 or BF16");
+    HSA_REQUIRE(out_dtype == HSA_F32 || out_dtype == HSA_BF16, HSA_ERR_UNSUPPORTED,
+                "out dtype must be F32 or BF16");
+    HSA_REQUIRE(kv_dtype == HSA_F32 || kv_dtype == HSA_BF16 || kv_dtype == HSA_E4M3,
+                HSA_ERR_UNSUPPORTED, "kv dtype must be F32, BF16 or E4M3");
+    if (seq->T_q > 0) {
+        HSA_REQUIRE(q && kv && idx && out, HSA_ERR_INVALID_ARG, "NULL tensor pointer");
+        if (kv_dtype == HSA_E4M3) {
+            HSA_REQUIRE(kv_scale && (kv_rope || D_qk == D_v), HSA_ERR_INVALID_ARG,
+                        "E4M3 latent cache needs kv_scale and kv_rope");
+        } else {
+            HSA_REQUIRE(kv_rope == nullptr, HSA_ERR_INVALID_ARG,
+                        "kv_rope must be NULL for a packed F32/BF16 cache");
+        }
+        HSA_REQUIRE(aligned(q, dtype_size(q_dtype)) && aligned(out, dtype_size(out_dtype)) &&
+                        aligned(idx, 4) && aligned(kv, dtype_size(kv_dtype)),
+                    HSA_ERR_INVALID_ARG, "misaligned tensor pointer");
+    }
+    return HSA_OK;
+}
+
+hsa::IndexScoreArgs index_args(const hsa_paged_seq_t* seq, const void* q_I, hsa_dtype_t q_dtype,
+                               const float* w, int32_t H_I, int32_t D_I, const void* k_cache,
+                               hsa_dtype_t k_dtype, const float* k_scale, float* scores,
+                               int64_t ld) {
+    hsa::IndexScoreArgs a;
+    a.seq = view(seq);
+    a.max_seq_len = seq->max_seq_len;
+    a.q_run = seq->q_run;
+    a.q_I = q_I;
+    a.q_dtype = q_dtype;
+    a.w = w;
+    a.H_I = H_I;
+    a.D_I = D_I;
+    a.k_cache = k_cache;
+    a.k_dtype = k_dtype;
+    a.k_scale = k_scale;
+    a.scores = scores;
+    a.ld = ld;
+    return a;
+}
+
+hsa_status_t run_index(const hsa::IndexScoreArgs& a, cudaStream_t st) {
+    if (a.seq.T_q == 0) return HSA_OK;
+    if (hsa::index_score_tc_supported(a))
+        return cuda_status(hsa::launch_index_score_tc(a, st), "index_score (tensor core)");
+    return cuda_status(hsa::launch_index_score_simt(a, st), "index_score");
+}
+
+hsa::SparseMlaArgs attn_args(const hsa_paged_seq_t* seq, const hsa_attn_args_t& at,
+                             const int32_t* idx, int32_t K, void* ws, size_t ws_bytes) {
+    hsa::SparseMlaArgs a;
+    a.seq = view(seq);
+    a.max_seq_len = seq->max_seq_len;
+    a.q = at.q;
+    a.q_dtype = at.q_dtype;
+    a.H = at.H;
+    a.D_qk = at.D_qk;
+    a.D_v = at.D_v;
+    a.kv = at.kv;
+    a.kv_dtype = at.kv_dtype;
+    a.kv_scale = at.kv_scale;
+    a.kv_rope = at.kv_rope;
+    a.idx = idx;
+    a.K = K;
+    a.softmax_scale = at.softmax_scale;
+    a.out = at.out;
+    a.out_dtype = at.out_dtype;
+    a.lse = at.lse;
+    a.ws = ws;
+    a.ws_bytes = ws_bytes;
+    return a;
+}
+
+size_t attn_ws_bytes(const hsa::SparseMlaArgs& a) {
+    return hsa::sparse_mla_tc_supported(a) ? hsa::sparse_mla_tc_workspace(a.seq.T_q, a.K) : 0;
+}
+
+hsa_status_t run_attn(const hsa::SparseMlaArgs& a, cudaStream_t st) {
+    if (a.seq.T_q == 0) return HSA_OK;
+    if (hsa::sparse_mla_tc_supported(a)) {
+        const size_t need = hsa::sparse_mla_tc_workspace(a.seq.T_q, a.K);
+        HSA_REQUIRE(a.ws_bytes >= need && (need == 0 || (a.ws && aligned(a.ws, 256))),
+                    HSA_ERR_WORKSPACE, "workspace of %zu bytes needed (256-byte aligned), got %zu",
+                    need, a.ws_bytes);
+        return cuda_status(hsa::launch_sparse_mla_tc(a, st), "sparse_mla_attn (tensor core)");
+    }
+    return cuda_status(hsa::launch_sparse_mla_simt(a, st), "sparse_mla_attn");
+}
+
+hsa_attn_args_t make_attn(const void* q, hsa_dtype_t q_dtype, int32_t H, int32_t D_qk, int32_t D_v,
+                          const void* kv, hsa_dtype_t kv_dtype, const float* kv_scale,
+                          const void* kv_rope, float softmax_scale, void* out,
+                          hsa_dtype_t out_dtype, float* lse) {
+    hsa_attn_args_t a;
+    a.q = q;
+    a.q_dtype = q_dtype;
+    a.H = H;
+    a.D_qk = D_qk;
+    a.D_v = D_v;
+    a.kv = kv;
+    a.kv_dtype = kv_dtype;
+    a.kv_scale = kv_scale;
+    a.kv_rope = kv_rope;
+    a.softmax_scale = softmax_scale;
+    a.out = out;
+    a.out_dtype = out_dtype;
+    a.lse = lse;
+    return a;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* hsa_status_string(hsa_status_t s) {
+    switch (s) {
+        case HSA_OK: return "HSA_OK";
+        case HSA_ERR_INVALID_ARG: return "HSA_ERR_INVALID_ARG";
+        case HSA_ERR_UNSUPPORTED: return "HSA_ERR_UNSUPPORTED";
+        case HSA_ERR_CUDA: return "HSA_ERR_CUDA";
+        case HSA_ERR_WORKSPACE: return "HSA_ERR_WORKSPACE";
+    }
+    return "HSA_ERR_UNKNOWN";
+}
+
+const char* hsa_last_error_message(void) { return g_last_error.c_str(); }
+
+int32_t hsa_version(void) { return 100; }
+
+hsa_status_t hsa_index_score(const hsa_paged_seq_t* seq, const void* q_I, hsa_dtype_t q_dtype,
+                             const float* w, int32_t H_I, int32_t D_I, const void* k_cache,
+                             hsa_dtype_t k_dtype, const float* k_scale, float* scores,
+                             int64_t ld_scores, void* stream) {
+    g_last_error.clear();
+    hsa_status_t st = check_index(seq, q_I, q_dtype, w, H_I, D_I, k_cache, k_dtype, k_scale,
+                                  scores, ld_scores);
+    if (st != HSA_OK) return st;
+    return run_index(index_args(seq, q_I, q_dtype, w, H_I, D_I, k_cache, k_dtype, k_scale, scores,
+                                ld_scores),
+                     (cudaStream_t)stream);
+}
+
+hsa_status_t hsa_topk(const hsa_paged_seq_t* seq, const float* scores, int64_t ld_scores,
+                      int32_t K, int32_t* idx, void* stream) {
+    g_last_error.clear();
+    hsa_status_t st = check_seq(seq);
+    if (st != HSA_OK) return st;
+    HSA_REQUIRE(K >= 1 && K <= 65536, HSA_ERR_INVALID_ARG, "K = %d out of range", K);
+    HSA_REQUIRE(ld_scores >= seq->max_seq_len, HSA_ERR_INVALID_ARG, "ld_scores < max_seq_len");
+    if (seq->T_q == 0) return HSA_OK;
+    HSA_REQUIRE(scores && idx && aligned(scores, 4) && aligned(idx, 4), HSA_ERR_INVALID_ARG,
+                "NULL or misaligned scores / idx");
+    return cuda_status(hsa::launch_topk(view(seq), seq->max_seq_len, scores, ld_scores, K, idx,
+                                        (cudaStream_t)stream),
+                       "topk");
+}
+
+size_t hsa_sparse_mla_workspace_size(const hsa_paged_seq_t* seq, int32_t H, int32_t D_qk,
+                                     int32_t D_v, int32_t K) {
+    if (seq == nullptr || seq->T_q <= 0) return 0;
+    // the tensor-core kernel's need only depends on the shape, not on the pointers
+    hsa_attn_args_t at = make_attn(nullptr, HSA_BF16, H, D_qk, D_v, nullptr, HSA_BF16, nullptr,
+                                   nullptr, 1.f, nullptr, HSA_BF16, nullptr);
+    return attn_ws_bytes(attn_args(seq, at, nullptr, K, nullptr, 0));
+}
+
+hsa_status_t hsa_sparse_mla_attn(const hsa_paged_seq_t* seq, const void* q, hsa_dtype_t q_dtype,
+                                 int32_t H, int32_t D_qk, int32_t D_v, const void* kv,
+                                 hsa_dtype_t kv_dtype, const float* kv_scale, const void* kv_rope,
+                                 const int32_t* idx, int32_t K, float softmax_scale, void* out,
+                                 hsa_dtype_t out_dtype, float* lse, void* ws, size_t ws_bytes,
+                                 void* stream) {
+    g_last_error.clear();
+    hsa_status_t st = check_attn(seq, q, q_dtype, H, D_qk, D_v, kv, kv_dtype, kv_scale, kv_rope,
+                                 idx, K, out, out_dtype);
+    if (st != HSA_OK) return st;
+    hsa_attn_args_t at = make_attn(q, q_dtype, H, D_qk, D_v, kv, kv_dtype, kv_scale, kv_rope,
+                                   softmax_scale, out, out_dtype, lse);
+    return run_attn(attn_args(seq, at, idx, K, ws, ws_bytes), (cudaStream_t)stream);
+}
+
+size_t hsa_fused_decode_workspace_size(const hsa_paged_seq_t* seq, const hsa_attn_args_t* attn,
+                                       int32_t K) {
+    if (seq == nullptr || attn == nullptr || seq->T_q <= 0) return 0;
+    // each half of a two-stream call needs its own region; the sum of the halves' needs is
+    // reported (the workspace need grows with the row count), rounded to 256 bytes each
+    const int32_t t1 = seq->T_q / 2;
+    hsa_paged_seq_t a = sub_rows(*seq, 0, t1), b = sub_rows(*seq, t1, seq->T_q - t1);
+    size_t na = t1 > 0 ? attn_ws_bytes(attn_args(&a, *attn, nullptr, K, nullptr, 0)) : 0;
+    size_t nb = attn_ws_bytes(attn_args(&b, *attn, nullptr, K, nullptr, 0));
+    size_t nall = attn_ws_bytes(attn_args(seq, *attn, nullptr, K, nullptr, 0));
+    na = (na + 255) / 256 * 256;
+    nb = (nb + 255) / 256 * 256;
+    return na + nb > nall ? na + nb : nall;
+}
+
+hsa_status_t hsa_fused_decode(const hsa_paged_seq_t* seq, const hsa_index_args_t* ix,
+                              const hsa_attn_args_t* at, int32_t K, float* scores,
+                              int64_t ld_scores, int32_t* idx, void* ws, size_t ws_bytes,
+                              void* stream_main, void* stream_aux) {
+    g_last_error.clear();
+    HSA_REQUIRE(ix && at, HSA_ERR_INVALID_ARG, "index / attn args NULL");
+    hsa_status_t st = check_index(seq, ix->q_I, ix->q_dtype, ix->w, ix->H_I, ix->D_I, ix->k_cache,
+                                  ix->k_dtype, ix->k_scale, scores, ld_scores);
+    if (st != HSA_OK) return st;
+    st = check_attn(seq, at->q, at->q_dtype, at->H, at->D_qk, at->D_v, at->kv, at->kv_dtype,
+                    at->kv_scale, at->kv_rope, idx, K, at->out, at->out_dtype);
+    if (st != HSA_OK) return st;
+    HSA_REQUIRE(K >= 1 && K <= 65536, HSA_ERR_INVALID_ARG, "K = %d out of range", K);
+    if (seq->T_q == 0) return HSA_OK;
+    HSA_REQUIRE(idx && aligned(idx, 4), HSA_ERR_INVALID_ARG, "idx NULL or misaligned");
+    const size_t need = hsa_fused_decode_workspace_size(seq, at, K);
+    HSA_REQUIRE(ws_bytes >= need && (need == 0 || (ws && aligned(ws, 256))), HSA_ERR_WORKSPACE,
+                "workspace of %zu bytes needed (256-byte aligned), got %zu", need, ws_bytes);
+
+    cudaStream_t s0 = (cudaStream_t)stream_main, s1 = (cudaStream_t)stream_aux;
+    // split point: half the rows, on a run boundary so no run is cut
+    int32_t t1 = seq->T_q / 2;
+    t1 -= t1 % seq->q_run;
+    const bool two = s1 != nullptr && t1 > 0 && t1 < seq->T_q;
+
+    auto one_part = [&](int32_t r0, int32_t n, void* pws, size_t pws_bytes, cudaStream_t s,
+                        cudaEvent_t after_topk) -> hsa_status_t {
+        hsa_paged_seq_t part = sub_rows(*seq, r0, n);
+        const size_t qI = (size_t)r0 * ix->H_I * ix->D_I * dtype_size(ix->q_dtype);
+        hsa::IndexScoreArgs ia = index_args(
+            &part, static_cast<const char*>(ix->q_I) + qI, ix->q_dtype, ix->w + (size_t)r0 * ix->H_I,
+            ix->H_I, ix->D_I, ix->k_cache, ix->k_dtype, ix->k_scale, scores + (size_t)r0 * ld_scores,
+            ld_scores);
+        hsa_status_t r = run_index(ia, s);
+        if (r != HSA_OK) return r;
+        r = cuda_status(hsa::launch_topk(view(&part), part.max_seq_len,
+                                         scores + (size_t)r0 * ld_scores, ld_scores, K,
+                                         idx + (size_t)r0 * K, s),
+                        "topk");
+        if (r != HSA_OK) return r;
+        if (after_topk) {
+            r = cuda_status(cudaEventRecord(after_topk, s), "cudaEventRecord");
+            if (r != HSA_OK) return r;
+        }
+        hsa_attn_args_t pa = *at;
+        pa.q = static_cast<const char*>(at->q) + (size_t)r0 * at->H * at->D_qk * dtype_size(at->q_dtype);
+        pa.out = static_cast<char*>(at->out) + (size_t)r0 * at->H * at->D_v * dtype_size(at->out_dtype);
+        pa.lse = at->lse ? at->lse + (size_t)r0 * at->H : nullptr;
+        return run_attn(attn_args(&part, pa, idx + (size_t)r0 * K, K, pws, pws_bytes), s);
+    };
+
+    if (!two) return one_part(0, seq->T_q, ws, ws_bytes, s0, nullptr);
+
+    // stream_main: rows [0, t1) index -> topk -> (event) -> attention
+    // stream_aux : waits for that event, then rows [t1, T_q) index -> topk -> attention, so the
+    //              second half's index stream overlaps the first half's attention
+    cudaEvent_t ev_topk = nullptr, ev_done = nullptr;
+    hsa_status_t r = cuda_status(cudaEventCreateWithFlags(&ev_topk, cudaEventDisableTiming), "event");
+    if (r == HSA_OK) r = cuda_status(cudaEventCreateWithFlags(&ev_done, cudaEventDisableTiming), "event");
+    hsa_paged_seq_t first = sub_rows(*seq, 0, t1);
+    size_t ws0 = attn_ws_bytes(attn_args(&first, *at, nullptr, K, nullptr, 0));
+    ws0 = (ws0 + 255) / 256 * 256;
+    if (r == HSA_OK) r = one_part(0, t1, ws, ws0, s0, ev_topk);
+    if (r == HSA_OK) r = cuda_status(cudaStreamWaitEvent(s1, ev_topk, 0), "cudaStreamWaitEvent");
+    if (r == HSA_OK)
+        r = one_part(t1, seq->T_q - t1, static_cast<char*>(ws) + ws0, ws_bytes - ws0, s1, nullptr);
+    if (r == HSA_OK) r = cuda_status(cudaEventRecord(ev_done, s1), "cudaEventRecord");
+    if (r == HSA_OK) r = cuda_status(cudaStreamWaitEvent(s0, ev_done, 0), "cudaStreamWaitEvent");
+    if (ev_topk) cudaEventDestroy(ev_topk);
+    if (ev_done) cudaEventDestroy(ev_done);
+    return r;
+}
+
+hsa_status_t hsa_quantize_index(const void* src, hsa_dtype_t src_dtype, int64_t n_rows,
+                                int32_t D, int32_t group, const int64_t* slot_mapping,
+                                int64_t num_slots, uint8_t* codes, float* scales, void* stream) {
+    g_last_error.clear();
+    HSA_REQUIRE(src_dtype == HSA_F32 || src_dtype == HSA_BF16, HSA_ERR_UNSUPPORTED,
+                "source dtype must be F32 or BF16");
+    HSA_REQUIRE(n_rows >= 0 && D >= 1 && group >= 1 && D % group == 0, HSA_ERR_INVALID_ARG,
+                "need n_rows >= 0, D >= 1, group | D (n_rows=%lld D=%d group=%d)",
+                (long long)n_rows, D, group);
+    HSA_REQUIRE(num_slots >= 0 && (slot_mapping || n_rows <= num_slots), HSA_ERR_INVALID_ARG,
+                "identity slot mapping needs n_rows <= num_slots");
+    if (n_rows == 0) return HSA_OK;
+    HSA_REQUIRE(src && codes && scales, HSA_ERR_INVALID_ARG, "NULL tensor pointer");
+    return cuda_status(hsa::launch_quantize_rows(src, src_dtype, n_rows, D, D, group, slot_mapping,
+                                                 num_slots, codes, scales, 0, nullptr,
+                                                 (cudaStream_t)stream),
+                       "quantize_index");
+}
+
+hsa_status_t hsa_quantize_kv(const void* src, hsa_dtype_t src_dtype, int64_t n_rows, int32_t D_v,
+                             int32_t D_rope, int32_t group, const int64_t* slot_mapping,
+                             int64_t num_slots, uint8_t* codes, float* scales, void* rope_cache,
+                             void* stream) {
+    g_last_error.clear();
+    HSA_REQUIRE(src_dtype == HSA_F32 || src_dtype == HSA_BF16, HSA_ERR_UNSUPPORTED,
+                "source dtype must be F32 or BF16");
+    HSA_REQUIRE(n_rows >= 0 && D_v >= 1 && D_rope >= 0 && group >= 1 && D_v % group == 0,
+                HSA_ERR_INVALID_ARG, "need n_rows >= 0, D_v >= 1, D_rope >= 0, group | D_v");
+    HSA_REQUIRE(num_slots >= 0 && (slot_mapping || n_rows <= num_slots), HSA_ERR_INVALID_ARG,
+                "identity slot mapping needs n_rows <= num_slots");
+    if (n_rows == 0) return HSA_OK;
+    HSA_REQUIRE(src && codes && scales && (D_rope == 0 || rope_cache), HSA_ERR_INVALID_ARG,
+                "NULL tensor pointer");
+    return cuda_status(hsa::launch_quantize_rows(src, src_dtype, n_rows, D_v + D_rope, D_v, group,
+                                                 slot_mapping, num_slots, codes, scales, D_rope,
+                                                 rope_cache, (cudaStream_t)stream),
+                       "quantize_kv");
+}
+
+}  // extern "C"

@@ -1,0 +1,90 @@
+"""Shared test plumbing: turn a seeded workload into library descriptors / oracle inputs, and the
+tolerance checks the parity tests use.  No method arithmetic lives here: scores, selections and
+attention come from the library (GPU side) or from ``oracle`` (reference side)."""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import oracle
+import sparse_index_attention_b200 as hsa
+from sparse_index_attention_b200 import workloads
+
+
+def paged_seq(wl: workloads.Workload, status=None) -> hsa.PagedSeq:
+    return hsa.PagedSeq(wl.seq_lens, wl.block_table, wl.page_size, wl.num_pages, wl.q_seq, wl.q_pos,
+                        max_seq_len=int(wl.seq_lens.max().item()), q_run=wl.q_run, status=status)
+
+
+def oracle_paging(wl: workloads.Workload, rows=None) -> oracle.Paging:
+    pg = oracle.Paging(wl.seq_lens, wl.block_table, wl.page_size, wl.num_pages, wl.q_seq, wl.q_pos)
+    return pg if rows is None else pg.subset(rows)
+
+
+class GpuCaches:
+    """The caches the GPU path reads, written by the library's own quantizers when FP8."""
+
+    def __init__(self, wl: workloads.Workload):
+        self.k_scale = None
+        self.kv_scale = None
+        self.kv_rope = None
+        if wl.index_fp8:
+            self.k, sc = hsa.hsa_quantize_index(wl.k_I, wl.D_I)
+            self.k_scale = sc.view(-1)
+        else:
+            self.k = wl.k_I
+        if wl.kv_fp8:
+            self.kv, sc, self.kv_rope = hsa.hsa_quantize_kv(wl.kv, wl.D_v, wl.D_v)
+            self.kv_scale = sc.view(-1)
+        else:
+            self.kv = wl.kv
+
+
+class OracleCaches:
+    """Exact values of the caches as the oracle reads them (its own quantizer for FP8)."""
+
+    def __init__(self, wl: workloads.Workload, need_kv: bool = True):
+        if wl.index_fp8:
+            codes, sc = oracle.quantize_rows(wl.k_I.float().cpu(), wl.D_I)
+            self.k = oracle.dequantize_rows(codes, sc, wl.D_I)
+        else:
+            self.k = wl.k_I.cpu()
+        if need_kv:
+            kv = wl.kv.float().cpu().numpy().astype(np.float64)
+            if wl.kv_fp8:
+                codes, sc = oracle.quantize_rows(wl.kv[:, :wl.D_v].float().cpu(), wl.D_v)
+                kv[:, :wl.D_v] = oracle.dequantize_rows(codes, sc, wl.D_v)
+            self.kv = kv
+
+
+def index_tolerance_ok(gpu, ref, mag, rel=1e-3):
+    """|I_gpu - I_ref| <= rel * (|I_ref| + M) elementwise, M = sum_j |w_j| ReLU(q_j . k_s)."""
+    gpu = np.asarray(gpu, dtype=np.float64)
+    err = np.abs(gpu - ref)
+    bound = rel * (np.abs(ref) + mag)
+    return bool(np.all(err <= bound)), float(np.max(err / np.maximum(bound, 1e-300)))
+
+
+def attn_close(gpu, ref, tol):
+    gpu = np.asarray(gpu, dtype=np.float64)
+    err = np.abs(gpu - ref)
+    ok = err <= tol + tol * np.abs(ref)
+    return bool(np.all(ok)), float(err.max())
+
+
+def stable_topk_reference(scores: torch.Tensor, q_pos: torch.Tensor, K: int) -> torch.Tensor:
+    """Selection from the same fp32 scores with torch's stable sort (descending score, ties by
+    position), re-sorted ascending: the reference for the bit-exact Top-K check."""
+    T, ld = scores.shape
+    out = torch.full((T, K), -1, dtype=torch.int32, device=scores.device)
+    pos = q_pos.tolist()
+    for t in range(T):
+        n = pos[t] + 1
+        if n <= K:
+            out[t, :n] = torch.arange(n, dtype=torch.int32, device=scores.device)
+            continue
+        row = scores[t, :n].clone()
+        row[row == 0] = 0.0                          # -0.0 == +0.0
+        order = torch.sort(row, descending=True, stable=True).indices[:K]
+        out[t] = order.sort().values.to(torch.int32)
+    return out

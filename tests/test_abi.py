@@ -1,0 +1,64 @@
+"""The C-ABI library loads and exports every entry point that include/hsa.h declares; argument
+validation rejects bad calls before anything reaches a GPU (CPU only: no compute is launched)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import sparse_index_attention_b200 as hsa
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    text = open(os.path.join(ROOT, "include", "hsa.h")).read()
+    return sorted(set(re.findall(r"HSA_API\s+[\w\s\*]+?\b(hsa_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_path():
+    names = _declared()
+    for n in ("hsa_index_score", "hsa_topk", "hsa_sparse_mla_attn", "hsa_fused_decode",
+              "hsa_quantize_index", "hsa_quantize_kv"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol():
+    L = hsa.lib()
+    for name in _declared():
+        assert hasattr(L, name), name
+        assert name in hsa.SYMBOLS, f"binding lacks {name}"
+    assert hsa.hsa_version() >= 100
+
+
+def test_validation_without_gpu():
+    L = hsa.lib()
+    # NULL descriptor
+    rc = L.hsa_topk(None, None, 0, 8, None, None)
+    assert rc == hsa.HSA_ERR_INVALID_ARG
+    assert b"seq" in L.hsa_last_error_message()
+    # a descriptor with fake (never dereferenced) device pointers and bad sizes
+    fake = ctypes.c_void_p(0x1000)
+    seq = hsa.hsa_paged_seq_t(1, fake, fake, 4, 16, 4, 64, 2, fake, fake, 1, None)
+    assert L.hsa_topk(ctypes.byref(seq), fake, 64, 0, fake, None) == hsa.HSA_ERR_INVALID_ARG
+    assert L.hsa_topk(ctypes.byref(seq), fake, 32, 8, fake, None) == hsa.HSA_ERR_INVALID_ARG  # ld < max_seq_len
+    bad = hsa.hsa_paged_seq_t(1, fake, fake, 2, 16, 4, 64, 2, fake, fake, 1, None)  # bt_stride too small
+    assert L.hsa_topk(ctypes.byref(bad), fake, 64, 8, fake, None) == hsa.HSA_ERR_INVALID_ARG
+    rc = L.hsa_index_score(ctypes.byref(seq), fake, hsa.HSA_E4M3, fake, 4, 32, fake, hsa.HSA_BF16,
+                           None, fake, 64, None)
+    assert rc == hsa.HSA_ERR_UNSUPPORTED                       # e4m3 queries are not a supported type
+    rc = L.hsa_index_score(ctypes.byref(seq), fake, hsa.HSA_BF16, fake, 4, 32, fake, hsa.HSA_E4M3,
+                           None, fake, 64, None)
+    assert rc == hsa.HSA_ERR_INVALID_ARG                       # E4M3 keys without scales
+    rc = L.hsa_quantize_index(fake, hsa.HSA_BF16, 10, 128, 48, None, 10, fake, fake, None)
+    assert rc == hsa.HSA_ERR_INVALID_ARG                       # group does not divide D
+    # zero rows is a no-op, not an error
+    empty = hsa.hsa_paged_seq_t(1, fake, fake, 4, 16, 4, 64, 0, None, None, 1, None)
+    assert L.hsa_topk(ctypes.byref(empty), None, 64, 8, None, None) == hsa.HSA_OK
+
+
+def test_missing_library_fails_loudly(monkeypatch):
+    monkeypatch.setattr(hsa, "_lib", None)
+    monkeypatch.setattr(hsa, "LIB_PATH", "/nonexistent/libhsa.so")
+    with pytest.raises(RuntimeError, match="no fallback"):
+        hsa.lib()

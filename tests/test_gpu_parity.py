@@ -1,0 +1,207 @@
+"""GPU parity: every C-ABI entry point against the float64 oracle on seeded inputs that span
+several tiles and a ragged tail.  Tolerances (written here, per element):
+  index score    |I_gpu - I_ref| <= 1e-3 (|I_ref| + M),  M = sum_j |w_j| ReLU(q_j . k_s)
+  Top-K          bit-exact (same fp32 scores on both sides)
+  attention      |o_gpu - o_ref| <= 2e-2 + 2e-2 |o_ref| (bf16), 6e-2 for FP8 caches, 1e-4 fp32
+  quantizers     bit-exact codes and scales
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import sparse_index_attention_b200 as hsa
+from sparse_index_attention_b200 import workloads
+
+from helpers import (GpuCaches, OracleCaches, attn_close, index_tolerance_ok, oracle_paging,
+                     paged_seq, stable_topk_reference)
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def _index_vs_oracle(wl, rows=None):
+    gc = GpuCaches(wl)
+    seq = paged_seq(wl)
+    sc = hsa.hsa_index_score(seq, wl.q_I, wl.w, gc.k, gc.k_scale)
+    torch.cuda.synchronize()
+    rows = list(range(wl.T_q)) if rows is None else rows
+    oc = OracleCaches(wl, need_kv=False)
+    pg = oracle_paging(wl, rows)
+    qI, w = wl.q_I[rows].cpu(), wl.w[rows].cpu()
+    ref = oracle.index_score(pg, qI, w, oc.k, ld=sc.shape[1])
+    mag = oracle.index_score(pg, qI, w.abs(), oc.k, ld=sc.shape[1])
+    got = sc[rows].cpu().numpy()
+    for i, t in enumerate(rows):
+        n = int(wl.q_pos[t]) + 1
+        ok, worst = index_tolerance_ok(got[i, :n], ref[i, :n], mag[i, :n])
+        assert ok, (wl.name, t, worst)
+    return sc
+
+
+@pytest.mark.parametrize("name,kw", [
+    ("tiny_decode_fp32", {}),
+    ("decode_bf16", dict(B=6, L_min=100, L_max=1500)),
+    ("decode_fp8", dict(B=3, L=700)),
+    ("prefill_bf16", dict(T=700)),
+    ("prefill_long_zigzag", dict(T=1024, n_chunks=4)),
+])
+def test_index_score_vs_oracle(name, kw):
+    _index_vs_oracle(workloads.make(name, DEV, **kw))
+
+
+def test_index_score_integer_inputs_bit_exact():
+    wl = workloads.make("decode_bf16", DEV, B=3, L_min=200, L_max=900)
+    g = torch.Generator(device=DEV).manual_seed(77)
+    wl.q_I = torch.randint(-2, 3, wl.q_I.shape, generator=g, device=DEV).to(torch.bfloat16)
+    wl.k_I = torch.randint(-2, 3, wl.k_I.shape, generator=g, device=DEV).to(torch.bfloat16)
+    e = torch.randint(-3, 4, wl.w.shape, generator=g, device=DEV).float()
+    wl.w = torch.exp2(e) * torch.where(torch.rand(wl.w.shape, generator=g, device=DEV) < 0.5, -1.0, 1.0)
+    sc = hsa.hsa_index_score(paged_seq(wl), wl.q_I, wl.w, wl.k_I)
+    ref = oracle.index_score(oracle_paging(wl), wl.q_I.cpu(), wl.w.cpu(), wl.k_I.cpu(), ld=sc.shape[1])
+    got = sc.cpu().numpy()
+    for t in range(wl.T_q):
+        n = int(wl.q_pos[t]) + 1
+        assert np.array_equal(got[t, :n].astype(np.float64), ref[t, :n]), t
+
+
+def test_index_score_paging_invariance_bitwise():
+    wl = workloads.make("decode_bf16", DEV, B=4, L_min=300, L_max=1000)
+    base = hsa.hsa_index_score(paged_seq(wl), wl.q_I, wl.w, wl.k_I)
+    perm = torch.randperm(wl.num_pages, generator=torch.Generator().manual_seed(3)).to(DEV)
+    moved = torch.empty_like(wl.k_I).view(wl.num_pages, wl.page_size, -1)
+    moved[perm] = wl.k_I.view(wl.num_pages, wl.page_size, -1)
+    wl2 = workloads.make("decode_bf16", DEV, B=4, L_min=300, L_max=1000)
+    wl2.block_table = perm.to(torch.int32)[wl.block_table.long()]
+    got = hsa.hsa_index_score(paged_seq(wl2), wl.q_I, wl.w, moved.view(-1, wl.D_I))
+    for t in range(wl.T_q):
+        n = int(wl.q_pos[t]) + 1
+        assert torch.equal(got[t, :n], base[t, :n])
+
+
+@pytest.mark.parametrize("ties", [False, True])
+def test_topk_vs_oracle_bit_exact(ties):
+    K = 64
+    lens = [1, 63, 64, 65, 66, 200, 1000, 4097, 33, 64 * 1024 + 17, 70000, 2]
+    T = len(lens)
+    ld = max(lens)
+    sc = workloads.random_scores(T, ld, seed=21, device=DEV, ties=ties)
+    seq = hsa.PagedSeq(torch.tensor([ld], device=DEV), torch.zeros((1, ld), dtype=torch.int32, device=DEV),
+                       1, ld, torch.zeros(T, dtype=torch.int32, device=DEV),
+                       torch.tensor([n - 1 for n in lens], dtype=torch.int32, device=DEV), max_seq_len=ld)
+    idx = hsa.hsa_topk(seq, sc, K)
+    ref = oracle.topk(sc.cpu(), np.array(lens, dtype=np.int32), K)
+    assert np.array_equal(idx.cpu().numpy(), ref)
+    # short rows: staged in shared memory
+    seq2 = hsa.PagedSeq(torch.tensor([3000], device=DEV), torch.zeros((1, 3000), dtype=torch.int32, device=DEV),
+                        1, 3000, torch.zeros(5, dtype=torch.int32, device=DEV),
+                        torch.tensor([2999, 100, 64, 63, 1500], dtype=torch.int32, device=DEV), max_seq_len=3000)
+    sc2 = sc[:5, :3000].contiguous()
+    idx2 = hsa.hsa_topk(seq2, sc2, K)
+    ref2 = oracle.topk(sc2.cpu(), np.array([3000, 101, 65, 64, 1501], dtype=np.int32), K)
+    assert np.array_equal(idx2.cpu().numpy(), ref2)
+
+
+def _attn_vs_oracle(wl, tol, idx=None):
+    gc = GpuCaches(wl)
+    seq = paged_seq(wl)
+    if idx is None:
+        idx = workloads.random_selection(wl.q_pos, wl.K, seed=wl.seed + 50)
+    idx_d = idx.to(DEV)
+    out, lse = hsa.hsa_sparse_mla_attn(seq, wl.q, gc.kv, idx_d, wl.D_v, wl.softmax_scale,
+                                       kv_scale=gc.kv_scale, kv_rope=gc.kv_rope)
+    torch.cuda.synchronize()
+    oc = OracleCaches(wl)
+    ref, rlse = oracle.sparse_mla(oracle_paging(wl), wl.q.cpu(), oc.kv, idx, wl.D_v, wl.softmax_scale)
+    ok, worst = attn_close(out.float().cpu().numpy(), ref, tol)
+    assert ok, (wl.name, worst)
+    l = lse.cpu().numpy()
+    fin = np.isfinite(rlse)
+    assert np.array_equal(np.isfinite(l), fin)
+    np.testing.assert_allclose(l[fin], rlse[fin], rtol=1e-4, atol=1e-4)
+    return out, lse
+
+
+@pytest.mark.parametrize("name,kw,tol", [
+    ("tiny_decode_fp32", {}, 1e-4),
+    ("decode_bf16", dict(B=5, L_min=100, L_max=4000), 2e-2),
+    ("decode_fp8", dict(B=3, L=3000), 6e-2),
+    ("prefill_bf16", dict(T=2100), 2e-2),
+])
+def test_sparse_mla_vs_oracle(name, kw, tol):
+    _attn_vs_oracle(workloads.make(name, DEV, **kw), tol)
+
+
+def test_sparse_mla_empty_rows_and_constant_values():
+    wl = workloads.make("decode_bf16", DEV, B=4, L_min=100, L_max=3000)
+    idx = workloads.random_selection(wl.q_pos, wl.K, seed=5)
+    idx[1] = -1                       # a row that selects nothing
+    idx[2, 1::2] = -1                 # holes inside a row
+    out, lse = _attn_vs_oracle(wl, 2e-2, idx)
+    assert torch.all(out[1] == 0) and torch.all(torch.isneginf(lse[1]))
+    wl.kv[:, :wl.D_v] = 1.0           # every value row is all ones -> output is ones
+    out2, _ = hsa.hsa_sparse_mla_attn(paged_seq(wl), wl.q, wl.kv, idx.to(DEV), wl.D_v, wl.softmax_scale)
+    for t in (0, 2, 3):
+        assert torch.allclose(out2[t].float(), torch.ones_like(out2[t].float()), atol=1e-2)
+
+
+@pytest.mark.parametrize("group", [None, 32])
+def test_quantize_index_bit_exact(group):
+    wl = workloads.make("decode_fp8", DEV, B=2, L=2000)
+    grp = wl.D_I if group is None else group
+    n = wl.k_I.shape[0]
+    perm = torch.randperm(n, generator=torch.Generator().manual_seed(1))
+    slots = perm.to(DEV).to(torch.int64)
+    codes, scales = hsa.hsa_quantize_index(wl.k_I, grp, slot_mapping=slots, num_slots=n)
+    rc, rs = oracle.quantize_rows(wl.k_I.float().cpu(), grp)
+    assert np.array_equal(codes.cpu()[perm].numpy(), rc)
+    assert np.array_equal(scales.cpu()[perm].numpy(), rs)
+
+
+def test_quantize_kv_bit_exact_and_rounding_ties():
+    wl = workloads.make("decode_fp8", DEV, B=2, L=1024)
+    codes, scales, rope = hsa.hsa_quantize_kv(wl.kv, wl.D_v, wl.D_v)
+    rc, rs = oracle.quantize_rows(wl.kv[:, :wl.D_v].float().cpu(), wl.D_v)
+    assert np.array_equal(codes.cpu().numpy(), rc) and np.array_equal(scales.cpu().numpy(), rs)
+    assert torch.equal(rope, wl.kv[:, wl.D_v:])
+    # rows whose max is 448 have scale 1 and are rounded as they are: every midpoint between
+    # adjacent E4M3 values, and 4e6 random fp32 values, against the library's conversion
+    vals = oracle.e4m3_decode(np.arange(0, 0x7F, dtype=np.uint8))
+    mids = ((vals[:-1] + vals[1:]) / 2).astype(np.float32)
+    g = torch.Generator().manual_seed(9)
+    rnd = (torch.randn(4_000_000, generator=g) * 60).clamp(-447, 447)
+    x = torch.cat([torch.from_numpy(mids), -torch.from_numpy(mids), rnd])
+    D = 126
+    pad = (-x.numel()) % (D - 1)
+    x = torch.cat([x, torch.zeros(pad)]).view(-1, D - 1)
+    x = torch.cat([torch.full((x.shape[0], 1), 448.0), x], dim=1).contiguous()
+    gcodes, gscales = hsa.hsa_quantize_index(x.to(DEV), D)
+    assert torch.all(gscales == 1.0)
+    ref = oracle.e4m3_encode(x.numpy().ravel()).reshape(x.shape)
+    assert np.array_equal(gcodes.cpu().numpy(), ref)
+
+
+def test_device_checks_flag_instead_of_faulting():
+    wl = workloads.make("decode_bf16", DEV, B=3, L_min=200, L_max=600)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    bad = wl.block_table.clone()
+    bad[1, 0] = wl.num_pages + 5      # page id out of range
+    seq = hsa.PagedSeq(wl.seq_lens, bad, wl.page_size, wl.num_pages, wl.q_seq, wl.q_pos, q_run=1,
+                       status=status)
+    hsa.hsa_index_score(seq, wl.q_I, wl.w, wl.k_I)
+    torch.cuda.synchronize()
+    assert int(status.item()) & hsa.HSA_DEV_BAD_PAGE
+    status.zero_()
+    qpos = wl.q_pos.clone()
+    qpos[0] = int(wl.seq_lens[0]) + 3  # position past the sequence end
+    seq2 = hsa.PagedSeq(wl.seq_lens, wl.block_table, wl.page_size, wl.num_pages, wl.q_seq, qpos,
+                        max_seq_len=int(wl.seq_lens.max()) + 8, status=status)
+    hsa.hsa_topk(seq2, torch.zeros((3, int(wl.seq_lens.max()) + 8), device=DEV), 16)
+    torch.cuda.synchronize()
+    assert int(status.item()) & hsa.HSA_DEV_BAD_POS
+    status.zero_()
+    idx = workloads.random_selection(wl.q_pos, 64, seed=1).to(DEV)
+    idx[0, 0] = int(wl.q_pos[0]) + 1   # selected position beyond the causal window
+    hsa.hsa_sparse_mla_attn(paged_seq(wl, status), wl.q, wl.kv, idx, wl.D_v, wl.softmax_scale)
+    torch.cuda.synchronize()
+    assert int(status.item()) & hsa.HSA_DEV_BAD_POS

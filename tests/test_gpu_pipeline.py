@@ -1,0 +1,123 @@
+"""GPU parity of the whole path (index score -> Top-K -> sparse MLA) against the oracle, run end
+to end on both sides from the same seeded inputs, plus the fused/two-stream invariants.
+
+Checks per the path's contract:
+  (i)   Top-K bit-exact against a reference selection (torch stable sort) on the GPU's own scores;
+  (ii)  the oracle's own float64 selection agrees on >= 99.9% of positions, and every position in
+        the symmetric difference is a near tie of the oracle's K-th score within the index-score
+        tolerance;
+  (iii) index scores within 1e-3 (|I_ref| + M); attention outputs within 2e-2 abs/rel (bf16),
+        6e-2 (FP8 caches), 1e-4 (fp32) of the oracle's end-to-end output;
+  (iv)  fused == unfused and two-stream == one-stream, bitwise.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import sparse_index_attention_b200 as hsa
+from sparse_index_attention_b200 import workloads
+
+from helpers import (GpuCaches, OracleCaches, attn_close, index_tolerance_ok, oracle_paging,
+                     paged_seq, stable_topk_reference)
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+TOL = {"f32": 1e-4, "bf16": 2e-2}
+
+
+def run_fused(wl, gc, aux=False):
+    seq = paged_seq(wl)
+    aux_stream = torch.cuda.Stream() if aux else None
+    out, lse, idx, sc = hsa.hsa_fused_decode(seq, wl.q_I, wl.w, gc.k, gc.k_scale, wl.q, gc.kv,
+                                             gc.kv_scale, gc.kv_rope, wl.K, wl.D_v,
+                                             wl.softmax_scale, aux_stream=aux_stream)
+    torch.cuda.synchronize()
+    return out, lse, idx, sc
+
+
+def check_against_oracle(wl, rows, sc, idx, out):
+    """(i)-(iii) on the sampled rows."""
+    K = wl.K
+    ref_sel = stable_topk_reference(sc[rows], wl.q_pos[rows], K)
+    assert torch.equal(idx[rows], ref_sel), "Top-K differs from the stable-sort selection"
+    oc = OracleCaches(wl)
+    pg = oracle_paging(wl, rows)
+    qI, w = wl.q_I[rows].cpu(), wl.w[rows].cpu()
+    ld = sc.shape[1]
+    ref_sc = oracle.index_score(pg, qI, w, oc.k, ld=ld)
+    mag = oracle.index_score(pg, qI, w.abs(), oc.k, ld=ld)
+    got_sc = sc[rows].cpu().numpy()
+    n_valid = (wl.q_pos[rows] + 1).cpu().numpy().astype(np.int32)
+    for i in range(len(rows)):
+        n = n_valid[i]
+        ok, worst = index_tolerance_ok(got_sc[i, :n], ref_sc[i, :n], mag[i, :n])
+        assert ok, ("index score", rows[i], worst)
+    ref_idx = oracle.topk(ref_sc, n_valid, K)
+    gidx = idx[rows].cpu().numpy()
+    agree = total = 0
+    for i in range(len(rows)):
+        a = set(gidx[i][gidx[i] >= 0].tolist())
+        b = set(ref_idx[i][ref_idx[i] >= 0].tolist())
+        total += len(b)
+        agree += len(a & b)
+        n = n_valid[i]
+        if n > K:
+            kth = np.sort(ref_sc[i, :n])[::-1][K - 1]
+            for s in a ^ b:
+                m = max(mag[i, s], mag[i, :n][ref_sc[i, :n] == kth].max())
+                assert abs(ref_sc[i, s] - kth) <= 1e-3 * (abs(kth) + m), ("not a near tie", rows[i], s)
+    assert agree >= 0.999 * total, (agree, total)
+    ref_out, _ = oracle.sparse_mla(pg, wl.q[rows].cpu(), oc.kv, ref_idx, wl.D_v, wl.softmax_scale)
+    tol = 6e-2 if (wl.kv_fp8 or wl.index_fp8) else TOL[wl.dtype]
+    ok, worst = attn_close(out[rows].float().cpu().numpy(), ref_out, tol)
+    assert ok, ("attention", worst)
+
+
+@pytest.mark.parametrize("name,kw", [
+    ("tiny_decode_fp32", {}),
+    ("decode_bf16", dict(B=8, L_min=1500, L_max=5000)),
+    ("decode_fp8", dict(B=4, L=4500)),
+])
+def test_pipeline_vs_oracle_small(name, kw):
+    wl = workloads.make(name, DEV, **kw)
+    gc = GpuCaches(wl)
+    out, lse, idx, sc = run_fused(wl, gc)
+    check_against_oracle(wl, list(range(wl.T_q)), sc, idx, out)
+
+
+@pytest.mark.parametrize("name,kw", [
+    ("tiny_decode_fp32", {}),
+    ("decode_bf16", dict(B=8, L_min=1500, L_max=5000)),
+    ("decode_fp8", dict(B=6, L=3000)),
+])
+def test_fused_equals_unfused_and_two_streams(name, kw):
+    wl = workloads.make(name, DEV, **kw)
+    gc = GpuCaches(wl)
+    out1, lse1, idx1, sc1 = run_fused(wl, gc, aux=False)
+    out2, lse2, idx2, sc2 = run_fused(wl, gc, aux=True)
+    seq = paged_seq(wl)
+    sc3 = hsa.hsa_index_score(seq, wl.q_I, wl.w, gc.k, gc.k_scale)
+    idx3 = hsa.hsa_topk(seq, sc3, wl.K)
+    out3, lse3 = hsa.hsa_sparse_mla_attn(seq, wl.q, gc.kv, idx3, wl.D_v, wl.softmax_scale,
+                                         kv_scale=gc.kv_scale, kv_rope=gc.kv_rope)
+    torch.cuda.synchronize()
+    for t in range(wl.T_q):
+        n = int(wl.q_pos[t]) + 1
+        assert torch.equal(sc1[t, :n], sc2[t, :n]) and torch.equal(sc1[t, :n], sc3[t, :n])
+    assert torch.equal(idx1, idx2) and torch.equal(idx1, idx3)
+    assert torch.equal(out1, out2) and torch.equal(out1, out3)
+    assert torch.equal(lse1, lse2) and torch.equal(lse1, lse3)
+
+
+def test_decode_bf16_full_size_sampled():
+    """The benchmark's workload and launch configuration (64 sequences, contexts 8192..32768,
+    Top-2048, 128 heads, latent 512 + rope 64, two streams): Top-K bit-exact on every row,
+    oracle checks on sampled rows."""
+    wl = workloads.make("decode_bf16", DEV)
+    gc = GpuCaches(wl)
+    out, lse, idx, sc = run_fused(wl, gc, aux=True)
+    ref_sel = stable_topk_reference(sc, wl.q_pos, wl.K)
+    assert torch.equal(idx, ref_sel)
+    rows = [0, 17, 40, 63]
+    check_against_oracle(wl, rows, sc, idx, out)
