@@ -1,0 +1,372 @@
+"""Benchmark of the sparse index attention decode step on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Workload: the bf16 decode batch -- 64 sequences with contexts uniform in [8192, 32768], one query
+token each, a 64-head x 128-dim indexer, Top-2048, sparse MLA with 128 heads over a paged
+latent cache of 512 + 64 dims (page 64), softmax scale 1/sqrt(576).  Synthetic seeded inputs,
+resident in HBM before the timed region.
+
+One step = one pass of the whole path over the batch: hsa_fused_decode on two streams (index
+score -> Top-K -> sparse MLA, the second half of the batch on the auxiliary stream).  L2 is
+flushed (256 MiB memset) before every timed step; each step is timed with CUDA events on the
+launching stream, the time reported is the sum over the K steps (max over ranks when N > 1).
+Multi-GPU runs are independent replicas (the decode batch shards by sequence; no collective is
+on the data path): every rank runs the full batch on its own GPU.
+
+The JSON line also carries: the roofline of the dominant kernel (per-kernel CUDA-event times
+from a second timed loop that issues the three C-ABI calls separately on one stream), the
+end-to-end throughput through the C ABI with host buffers (H2D of the step's query inputs and
+D2H of its output inside the timed region), the oracle timed on a bounded sample on the host
+cores, and the SM clocks sampled during the timed region.
+
+--impl reference runs the float64 CPU oracle (the only reference implementation of this path)
+on the same workload, one query row per step, and prints the same JSON line with
+"impl": "reference".
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from sparse_index_attention_b200 import workloads  # noqa: E402
+
+METRIC = "decode & prefill tokens/s on 1 B200; % of HBM / tensor-core roofline"
+UNIT = "tokens/s"
+WORKLOAD = "decode_bf16"
+FLUSH_BYTES = 256 << 20
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        d = json.load(open(p))
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                "source": "fallback"}
+
+
+def workload_config(wl):
+    lens = wl.seq_lens.tolist()
+    return {"workload": WORKLOAD, "B": wl.B, "context_min": min(lens), "context_max": max(lens),
+            "context_mean": round(sum(lens) / len(lens), 1), "query_rows": wl.T_q,
+            "index_heads": wl.H_I, "index_dim": wl.D_I, "top_k": wl.K, "heads": wl.H,
+            "latent_dim": wl.D_v, "rope_dim": wl.D_rope, "page_size": wl.page_size,
+            "softmax_scale": wl.softmax_scale, "seed": wl.seed,
+            "l2": "flushed (256 MiB memset) before every timed step"}
+
+
+def algorithmic_work(wl):
+    """Bytes (and flops) each kernel must move, from the workload's shape (per launch over the
+    whole batch).  Index score: 256 B per key read + 4 B score written per key, plus q_I and w;
+    Top-K: 4 B per score read + 4 B per index written; attention: 1152 B per selected latent
+    row + q and output."""
+    n = (wl.q_pos.long() + 1).cpu()
+    sel = torch.clamp(n, max=wl.K)
+    esz = 2
+    idx_bytes = int(n.sum()) * (wl.D_I * esz + 4) + wl.T_q * wl.H_I * (wl.D_I * esz + 4)
+    topk_bytes = int(n.sum()) * 4 + wl.T_q * wl.K * 4
+    attn_bytes = int(sel.sum()) * wl.D_qk * esz + wl.T_q * wl.H * (wl.D_qk + wl.D_v) * esz + \
+        wl.T_q * wl.K * 4 + wl.T_q * wl.H * 4
+    idx_flops = int(n.sum()) * wl.H_I * wl.D_I * 2
+    attn_flops = int(sel.sum()) * wl.H * (wl.D_qk + wl.D_v) * 2
+    return {"index_score": {"bytes": idx_bytes, "flops": idx_flops},
+            "topk": {"bytes": topk_bytes, "flops": 0},
+            "sparse_mla": {"bytes": attn_bytes, "flops": attn_flops}}
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while the timed region runs."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x100: "display_clock_setting"}
+
+    def __init__(self, index: int, period_s: float = 0.02):
+        self.samples, self.reasons = [], set()
+        self.period = period_s
+        self.ok = False
+        self.max_mhz = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.nv = None
+        self._stop = threading.Event()
+        self._t = None
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                mask = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for bit, name in self.REASONS.items():
+                    if mask & bit and name != "gpu_idle":
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self._t:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                    "samples": 0}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+def cpu_baseline(wl, rows, timer_label="oracle"):
+    """The float64 oracle (as it is) on a sample of query rows: index score -> Top-K -> sparse
+    MLA for those rows over their full contexts.  Returns (tokens/s, seconds, threads)."""
+    import oracle
+    pg = oracle.Paging(wl.seq_lens, wl.block_table, wl.page_size, wl.num_pages, wl.q_seq, wl.q_pos)
+    k = wl.k_I.float().cpu().numpy().astype(np.float64)
+    kv = wl.kv.float().cpu().numpy().astype(np.float64)
+    qI, w, q = wl.q_I[rows].cpu(), wl.w[rows].cpu(), wl.q[rows].cpu()
+    t0 = time.perf_counter()
+    oracle.sparse_index_attention(pg.subset(rows), qI, w, k, q, kv, wl.K, wl.D_v, wl.softmax_scale)
+    dt = time.perf_counter() - t0
+    return len(rows) / dt, dt, oracle.num_threads()
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    import oracle
+    wl = workloads.make(WORKLOAD, "cpu")
+    pg = oracle.Paging(wl.seq_lens, wl.block_table, wl.page_size, wl.num_pages, wl.q_seq, wl.q_pos)
+    k = wl.k_I.float().numpy().astype(np.float64)
+    kv = wl.kv.float().numpy().astype(np.float64)
+
+    def step(i):
+        r = i % wl.T_q
+        oracle.sparse_index_attention(pg.subset([r]), wl.q_I[r:r + 1], wl.w[r:r + 1], k,
+                                      wl.q[r:r + 1], kv, wl.K, wl.D_v, wl.softmax_scale)
+
+    for i in range(args.warmup):
+        step(i)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        step(args.warmup + i)
+    dt = time.perf_counter() - t0
+    value = args.steps / dt
+    threads = oracle.num_threads()
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": workload_config(wl),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                             "sample": "one query row per step (index score over its whole "
+                                       "context, Top-2048, 128-head sparse MLA), rows in turn"},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args, rank, world, local_rank):
+    import sparse_index_attention_b200 as hsa
+    dist = None
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", device_id=dev, timeout=datetime.timedelta(seconds=120))
+
+    wl = workloads.make(WORKLOAD, dev)
+    seq = hsa.PagedSeq(wl.seq_lens, wl.block_table, wl.page_size, wl.num_pages, wl.q_seq, wl.q_pos,
+                       q_run=wl.q_run)
+    ld = seq.max_seq_len
+    scores = torch.empty((wl.T_q, ld), dtype=torch.float32, device=dev)
+    idx = torch.empty((wl.T_q, wl.K), dtype=torch.int32, device=dev)
+    out = torch.empty((wl.T_q, wl.H, wl.D_v), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((wl.T_q, wl.H), dtype=torch.float32, device=dev)
+    ws = torch.empty(max(1, hsa.hsa_fused_decode_workspace_size(seq, wl.q, wl.kv, wl.D_v, wl.K)),
+                     dtype=torch.uint8, device=dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    main = torch.cuda.current_stream()
+    aux = torch.cuda.Stream()
+
+    def step(q_I=wl.q_I, w=wl.w, q=wl.q):
+        hsa.hsa_fused_decode(seq, q_I, w, wl.k_I, None, q, wl.kv, None, None, wl.K, wl.D_v,
+                             wl.softmax_scale, scores=scores, idx=idx, out=out, lse=lse, ws=ws,
+                             stream=main, aux_stream=aux)
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    def max_over_ranks(x: float) -> float:
+        if dist is None:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+
+    # ---- timed region: K fused steps, L2 flushed before each ----
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    barrier()
+    torch.cuda.synchronize()
+    launches0 = hsa.hsa_launch_count()
+    wall0 = time.perf_counter()
+    with ClockSampler(local_rank) as clocks:
+        for i in range(args.steps):
+            flush.zero_()
+            starts[i].record(main)
+            step()
+            ends[i].record(main)
+        torch.cuda.synchronize()
+    wall = time.perf_counter() - wall0
+    barrier()
+    launches = hsa.hsa_launch_count() - launches0
+    t_ms = sum(s.elapsed_time(e) for s, e in zip(starts, ends))
+    t_ms = max_over_ranks(t_ms)
+    value = world * wl.T_q * args.steps / (t_ms * 1e-3)
+
+    # ---- per-kernel times: the three C-ABI calls on one stream, events between them ----
+    reps = max(3, min(args.steps, 50))
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(reps)]
+    for i in range(reps):
+        flush.zero_()
+        ev[i][0].record(main)
+        hsa.hsa_index_score(seq, wl.q_I, wl.w, wl.k_I, None, scores=scores, stream=main)
+        ev[i][1].record(main)
+        hsa.hsa_topk(seq, scores, wl.K, idx=idx, stream=main)
+        ev[i][2].record(main)
+        hsa.hsa_sparse_mla_attn(seq, wl.q, wl.kv, idx, wl.D_v, wl.softmax_scale, out=out, lse=lse,
+                                ws=ws, stream=main)
+        ev[i][3].record(main)
+    torch.cuda.synchronize()
+    names = ["index_score", "topk", "sparse_mla"]
+    stage_ms = {n: statistics.mean(e[j].elapsed_time(e[j + 1]) for e in ev) for j, n in enumerate(names)}
+    work = algorithmic_work(wl)
+    peaks = load_peaks()
+    stages = {}
+    for n in names:
+        ms = stage_ms[n]
+        stages[n] = {"ms": round(ms, 4), "GB/s": round(work[n]["bytes"] / (ms * 1e-3) / 1e9, 1),
+                     "TFLOP/s": round(work[n]["flops"] / (ms * 1e-3) / 1e12, 2),
+                     "bytes": work[n]["bytes"], "flops": work[n]["flops"]}
+    dom = max(names, key=lambda n: stage_ms[n])
+    achieved = work[dom]["bytes"] / (stage_ms[dom] * 1e-3) / 1e9
+    traffic = None
+    tpath = os.path.join(ROOT, "profiles", "traffic.json")
+    if os.path.exists(tpath):
+        try:
+            traffic = json.load(open(tpath)).get(dom)
+        except Exception:
+            traffic = None
+    roofline = {"kernel": dom, "bound": "hbm", "achieved": round(achieved, 1),
+                "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
+                "traffic": traffic, "peak_source": f"{peaks['source']} (MEASURED_PEAKS.json hbm_gbs)"
+                if peaks["source"] == "measured" else "fallback 6.65 TB/s"}
+
+    # ---- end to end through the C ABI with host buffers ----
+    h_qI = torch.empty_like(wl.q_I, device="cpu").pin_memory()
+    h_w = torch.empty_like(wl.w, device="cpu").pin_memory()
+    h_q = torch.empty_like(wl.q, device="cpu").pin_memory()
+    h_out = torch.empty_like(out, device="cpu").pin_memory()
+    h_qI.copy_(wl.q_I)
+    h_w.copy_(wl.w)
+    h_q.copy_(wl.q)
+    d_qI, d_w, d_q = torch.empty_like(wl.q_I), torch.empty_like(wl.w), torch.empty_like(wl.q)
+    e_steps = max(3, min(args.steps, 50))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    barrier()
+    e0.record(main)
+    for i in range(e_steps):
+        d_qI.copy_(h_qI, non_blocking=True)
+        d_w.copy_(h_w, non_blocking=True)
+        d_q.copy_(h_q, non_blocking=True)
+        step(d_qI, d_w, d_q)
+        h_out.copy_(out, non_blocking=True)
+    e1.record(main)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1))
+    h2d = h_qI.numel() * h_qI.element_size() + h_w.numel() * 4 + h_q.numel() * h_q.element_size()
+    d2h = h_out.numel() * h_out.element_size()
+    e2e = {"value": world * wl.T_q * e_steps / (e2e_ms * 1e-3), "unit": UNIT,
+           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e_steps,
+           "note": "L2 not flushed between end-to-end steps"}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rows = list(range(args.cpu_rows))
+        v, secs, threads = cpu_baseline(wl, rows)
+        cpu = {"value": v, "unit": UNIT, "cores": threads, "kind": "oracle",
+               "sample": f"{len(rows)} query rows of the batch (index score over each full context, "
+                         f"Top-2048, 128-head sparse MLA), {secs:.1f} s"}
+
+    if dist is not None:
+        dist.barrier()
+    if rank == 0:
+        line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": t_ms / args.steps,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+                "data": "synthetic", "config": workload_config(wl),
+                "parallelism": f"replicas x{world} (independent decode batches, no collective on the data path)",
+                "roofline": roofline, "stages": stages, "cpu_baseline": cpu, "e2e": e2e,
+                "gpu_launches": launches, "clocks": clocks.summary(),
+                "wall_s_timed_region": round(wall, 3)}
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.destroy_process_group()
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--cpu-rows", type=int, default=16, help="query rows for the oracle baseline")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+    else:
+        run_ours(args, rank, world, local_rank)
+
+
+if __name__ == "__main__":
+    main()

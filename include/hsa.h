@@ -205,6 +205,9 @@ HSA_API hsa_status_t hsa_quantize_kv(const void* src, hsa_dtype_t src_dtype, int
 HSA_API const char* hsa_status_string(hsa_status_t s);
 /* Text of the last error raised by a call on this host thread ("" if none). */
 HSA_API const char* hsa_last_error_message(void);
+/* Number of kernels this library has launched from the calling host thread since it was loaded
+ * (a diagnostic for benchmarks: every kernel of the path is counted once per launch). */
+HSA_API uint64_t hsa_launch_count(void);
 /* Library version, major * 10000 + minor * 100 + patch. */
 HSA_API int32_t hsa_version(void);
 

@@ -61,6 +61,7 @@ SYMBOLS = {
     "hsa_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "hsa_last_error_message": (ctypes.c_char_p, []),
     "hsa_version": (_i32, []),
+    "hsa_launch_count": (ctypes.c_uint64, []),
 }
 
 _lock = threading.Lock()
@@ -285,3 +286,8 @@ def hsa_quantize_kv(src, D_v: int, group: int, slot_mapping=None, num_slots: Opt
 
 def hsa_version() -> int:
     return int(lib().hsa_version())
+
+
+def hsa_launch_count() -> int:
+    """Kernels launched by the library from this host thread so far."""
+    return int(lib().hsa_launch_count())

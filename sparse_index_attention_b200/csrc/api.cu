@@ -216,7 +216,14 @@ hsa_attn_args_t make_attn(const void* q, hsa_dtype_t q_dtype, int32_t H, int32_t
 
 }  // namespace
 
+uint64_t& hsa::launch_counter() {
+    thread_local uint64_t n = 0;
+    return n;
+}
+
 extern "C" {
+
+uint64_t hsa_launch_count(void) { return hsa::launch_counter(); }
 
 const char* hsa_status_string(hsa_status_t s) {
     switch (s) {

@@ -104,4 +104,8 @@ __device__ __forceinline__ float load_any(const void* p, hsa_dtype_t dt, int64_t
 
 __host__ __device__ constexpr int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
+// Kernel launches issued by the calling host thread (reported by hsa_launch_count()).
+uint64_t& launch_counter();
+inline void count_launch(int n = 1) { launch_counter() += (uint64_t)n; }
+
 }  // namespace hsa

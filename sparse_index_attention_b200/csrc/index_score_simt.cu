@@ -63,6 +63,7 @@ cudaError_t launch_t(const IndexScoreArgs& a, cudaStream_t st) {
     }
     k<<<grid, kThreads, smem, st>>>(a.seq, reinterpret_cast<const QT*>(a.q_I), a.w, a.H_I, a.D_I,
                                     a.k_cache, a.k_scale, a.scores, a.ld);
+    count_launch();
     return cudaGetLastError();
 }
 

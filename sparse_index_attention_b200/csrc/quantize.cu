@@ -69,12 +69,14 @@ cudaError_t launch_t(const void* src, int64_t n_rows, int32_t src_stride, int32_
     quantize_groups_kernel<T><<<(unsigned)blocks, kThreads, 0, st>>>(
         reinterpret_cast<const T*>(src), n_rows, src_stride, D, group, slot_mapping, num_slots,
         codes, scales);
+    count_launch();
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess || copy_cols == 0) return e;
     const int64_t n = n_rows * copy_cols;
     copy_cols_kernel<T><<<(unsigned)ceil_div(n, kThreads), kThreads, 0, st>>>(
         reinterpret_cast<const T*>(src), n_rows, src_stride, D, copy_cols, slot_mapping, num_slots,
         reinterpret_cast<__nv_bfloat16*>(copy_dst));
+    count_launch();
     return cudaGetLastError();
 }
 

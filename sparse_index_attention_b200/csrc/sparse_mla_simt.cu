@@ -155,6 +155,7 @@ cudaError_t launch_t(const SparseMlaArgs& a, cudaStream_t st) {
                                     a.kv, a.kv_scale,
                                     reinterpret_cast<const __nv_bfloat16*>(a.kv_rope), a.idx, a.K,
                                     a.softmax_scale, reinterpret_cast<OT*>(a.out), a.lse);
+    count_launch();
     return cudaGetLastError();
 }
 

@@ -162,8 +162,10 @@ cudaError_t launch_topk(const SeqView& seq, int32_t max_seq_len, const float* sc
         cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
         k<<<seq.T_q, kThreads, smem, st>>>(seq, scores, ld, K, idx);
+    count_launch();
     } else {
         topk_kernel<false><<<seq.T_q, kThreads, base, st>>>(seq, scores, ld, K, idx);
+    count_launch();
     }
     return cudaGetLastError();
 }
