@@ -28,7 +28,9 @@
  *    positions it reads (q_pos < seq_len, selected index in [0, q_pos]) and the row grouping it
  *    relies on.  A failed check never faults: the access is skipped or redirected to page 0 and
  *    a bit is OR-ed into *seq->status (if non-null), so results are then undefined but the
- *    context stays usable.  Bits: HSA_DEV_BAD_PAGE, HSA_DEV_BAD_POS, HSA_DEV_BAD_GROUP.
+ *    context stays usable.  Bits: HSA_DEV_BAD_PAGE, HSA_DEV_BAD_POS, HSA_DEV_BAD_GROUP,
+ *    HSA_DEV_TIMEOUT (every wait inside a kernel is bounded; one that gives up makes the kernel
+ *    leave early and sets this bit instead of hanging the GPU).
  *  - Threading: no mutable global state beyond a per-thread error message; calls on different
  *    streams may be issued from different host threads.
  */
@@ -66,6 +68,7 @@ typedef enum hsa_dtype {
 #define HSA_DEV_BAD_PAGE 1u   /* block_table entry outside [0, num_pages) */
 #define HSA_DEV_BAD_POS 2u    /* q_pos >= seq_len, or a selected index outside [0, q_pos] */
 #define HSA_DEV_BAD_GROUP 4u  /* rows of one q_run disagree on their sequence */
+#define HSA_DEV_TIMEOUT 8u    /* a pipeline wait inside a kernel gave up (the kernel returned early) */
 
 /* Paged sequences and query rows.
  * Position s of sequence b lives in physical slot

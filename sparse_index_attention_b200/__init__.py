@@ -22,7 +22,7 @@ LIB_PATH = os.path.join(_HERE, "libhsa.so")
 
 HSA_OK, HSA_ERR_INVALID_ARG, HSA_ERR_UNSUPPORTED, HSA_ERR_CUDA, HSA_ERR_WORKSPACE = 0, 1, 2, 3, 4
 HSA_F32, HSA_BF16, HSA_E4M3 = 0, 1, 2
-HSA_DEV_BAD_PAGE, HSA_DEV_BAD_POS, HSA_DEV_BAD_GROUP = 1, 2, 4
+HSA_DEV_BAD_PAGE, HSA_DEV_BAD_POS, HSA_DEV_BAD_GROUP, HSA_DEV_TIMEOUT = 1, 2, 4, 8
 
 _P = ctypes.c_void_p
 _i32, _i64, _sz, _f32 = ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t, ctypes.c_float

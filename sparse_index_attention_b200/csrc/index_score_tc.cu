@@ -1,7 +1,454 @@
-// index_score_tc.cu -- tensor-core (tcgen05) index score; filled in below.
+// index_score_tc.cu -- tensor-core index score for the 64-head x 128-dim indexer (sm_100a).
+//
+// I[t,s] = sum_j w[t,j] ReLU(q_I[t,j,:] . k[s,:])  ("Day 0 Inference Adaptation and Optimization
+// for Hybrid Attention Models", "Sparse Attention Pipeline Optimization": scoring over the paged
+// K cache and head-weight weighted summation; fifth page, 3.1).
+//
+// Mapping.  One tcgen05 MMA tile is D[128 keys x G*64] = K_tile[128 x 128] . Q_group^T, with the
+// keys on M (TMEM lanes) and G query rows x 64 index heads on N (TMEM columns).  The epilogue
+// thread that owns TMEM lane r owns key s = tile*128 + r and reduces its 64 head columns per
+// query row in registers: no cross-thread reduction.  Accumulators are double-buffered in TMEM
+// so the epilogue of tile i overlaps the MMA of tile i+1.
+//
+// Schedule.  Work is the flat list of (query group, key tile) pairs, where a group is G
+// consecutive rows of one sequence and its key range is [0, max position of the group].  Each
+// persistent CTA takes one contiguous slice of that list (load balance without atomics), so
+// it walks the keys of one group in order and reloads the group's queries only when the group
+// changes.  Every CTA derives the list itself from q_pos (prefix sum in shared memory).
+//
+// Data movement.  Keys come through the block table page by page with 2D TMA loads (128-byte
+// swizzle, two 64-column halves per page); FP8 keys are loaded raw and widened to bf16 in
+// shared memory by four converter warps (e4m3 -> bf16 is exact), and the per-key fp32 scale
+// multiplies the finished score (the scale is positive, so it commutes with the ReLU sum).
+//
+// Warp roles: 0 TMA producer, 1 MMA issuer (one elected thread each), 2-5 epilogue
+// (TMEM lane quarters 2,3,0,1), 6-9 FP8 converters (FP8 variant only).
+#include <algorithm>
+
 #include "kernels.h"
+#include "tc_common.cuh"
 
 namespace hsa {
-bool index_score_tc_supported(const IndexScoreArgs&) { return false; }
-cudaError_t launch_index_score_tc(const IndexScoreArgs&, cudaStream_t) { return cudaErrorNotSupported; }
+
+namespace {
+
+constexpr int kBM = 128;                 // keys per tile = MMA M
+constexpr int kDI = 128;                 // index dim
+constexpr int kHI = 64;                  // index heads
+constexpr int kHalfBytes = kBM * 128;    // one 64-column swizzled half of a key tile: 16 KB
+constexpr int kTileBytes = 2 * kHalfBytes;
+
+template <int G, bool kFp8>
+struct Cfg {
+    static constexpr int N = G * kHI;
+    static constexpr int kQBytes = N * kDI * 2;
+    static constexpr int kStages = kFp8 ? (G == 1 ? 4 : (G == 2 ? 3 : 2)) : (G == 1 ? 6 : (G == 2 ? 5 : 4));
+    static constexpr int kRawStages = kFp8 ? 4 : 0;          // FP8 staging tiles (16 KB each)
+    static constexpr int kMaxGroups = G == 1 ? 2048 : 4096;
+    static constexpr int kTmemCols = 2 * N;                   // 128, 256 or 512
+    static constexpr int kThreads = kFp8 ? 320 : 192;
+    static constexpr size_t kSmem = 1024 + (size_t)kStages * kTileBytes + (size_t)kRawStages * (kBM * kDI) +
+                                    kQBytes + 4 * (kMaxGroups + 1) + 4 * N + 256;
+    static_assert(kSmem <= 232448, "shared memory budget");
+};
+
+struct GroupInfo {
+    int32_t b;        // sequence (of the group's first valid row)
+    int32_t pos_max;  // largest valid position in the group, -1 if none
+};
+
+__device__ __forceinline__ GroupInfo group_info(const SeqView& v, int g, int G, bool flag) {
+    GroupInfo gi{-1, -1};
+    for (int j = 0; j < G; ++j) {
+        const int t = g * G + j;
+        if (t >= v.T_q) break;
+        RowInfo r = load_row(v, t);
+        if (r.pos < 0) continue;
+        if (gi.b < 0) gi.b = r.b;
+        if (r.b != gi.b) {
+            if (flag) flag_status(v, HSA_DEV_BAD_GROUP);
+            continue;
+        }
+        gi.pos_max = max(gi.pos_max, r.pos);
+    }
+    return gi;
+}
+
+// (group, key tile) of flat tile index f, advancing a monotone cursor.
+__device__ __forceinline__ void locate(const int32_t* prefix, int n_groups, int64_t f, int& g, int& kt) {
+    while (g + 1 < n_groups && prefix[g + 1] <= f) ++g;
+    kt = (int)(f - prefix[g]);
+}
+
+__device__ __forceinline__ int first_group(const int32_t* prefix, int n_groups, int64_t f) {
+    int lo = 0, hi = n_groups - 1;  // last g with prefix[g] <= f
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (prefix[mid] <= f) lo = mid; else hi = mid - 1;
+    }
+    return lo;
+}
+
+template <int G, bool kFp8>
+__global__ void __launch_bounds__(Cfg<G, kFp8>::kThreads, 1)
+index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_q,
+                      SeqView v, int32_t q_row0, const float* __restrict__ w,
+                      const float* __restrict__ k_scale, float* __restrict__ scores, int64_t ld,
+                      int32_t box_rows) {
+    using C = Cfg<G, kFp8>;
+    constexpr int N = C::N;
+    constexpr int S = C::kStages;
+    constexpr uint32_t kIdesc = tc::idesc_bf16_f32(kBM, N, 0, 0);
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* tiles = base;                                          // S x 32 KB (bf16, swizzled)
+    uint8_t* raw = tiles + (size_t)S * kTileBytes;                  // FP8 staging
+    uint8_t* qbuf = raw + (size_t)C::kRawStages * (kBM * kDI);      // N x 128 bf16, swizzled
+    // barriers first (8-byte alignment), then the variable-size arrays
+    uint64_t* bars = reinterpret_cast<uint64_t*>(qbuf + C::kQBytes);
+    uint64_t* full = bars;                 // [S]  keys landed (bf16 tile ready)
+    uint64_t* empty = full + S;            // [S]  MMA done with the tile
+    uint64_t* acc_full = empty + S;        // [2]
+    uint64_t* acc_empty = acc_full + 2;    // [2]
+    uint64_t* q_full = acc_empty + 2;
+    uint64_t* q_empty = q_full + 1;
+    uint64_t* raw_full = q_empty + 1;      // [4] FP8 bytes landed
+    uint64_t* raw_empty = raw_full + 4;    // [4] converters done with the staging tile
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(raw_empty + 4);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+    static_assert((2 * S + 2 + 2 + 2 + 8) * 8 + 8 <= 256, "barrier block");
+    int32_t* prefix = reinterpret_cast<int32_t*>(reinterpret_cast<uint8_t*>(bars) + 256);
+    float* w_s = reinterpret_cast<float*>(prefix + C::kMaxGroups + 1);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int n_groups = (int)ceil_div(v.T_q, G);
+
+    if (tid == 0) {
+        for (int i = 0; i < S; ++i) {
+            tc::mbar_init(&full[i], kFp8 ? 128 : 1);
+            tc::mbar_init(&empty[i], 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            tc::mbar_init(&acc_full[i], 1);
+            tc::mbar_init(&acc_empty[i], 4);
+        }
+        tc::mbar_init(q_full, 1);
+        tc::mbar_init(q_empty, 1);
+        for (int i = 0; i < 4; ++i) {
+            tc::mbar_init(&raw_full[i], 1);
+            tc::mbar_init(&raw_empty[i], 128);
+        }
+        *abort_flag = 0;
+        tc::fence_barrier_init();
+    }
+    if (warp == 1) {
+        tc::tmem_alloc(tmem_holder, C::kTmemCols);
+        tc::tmem_relinquish();
+    }
+    // tiles per group, then an exclusive prefix sum (warp 0)
+    for (int g = tid; g < n_groups; g += blockDim.x) {
+        const GroupInfo gi = group_info(v, g, G, blockIdx.x == 0);
+        prefix[g] = gi.pos_max >= 0 ? (int32_t)ceil_div(gi.pos_max + 1, kBM) : 0;
+    }
+    __syncthreads();
+    if (warp == 0) {
+        int32_t carry = 0;
+        for (int g0 = 0; g0 < n_groups; g0 += 32) {
+            const int g = g0 + lane;
+            int32_t x = g < n_groups ? prefix[g] : 0;
+            int32_t incl = x;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += y;
+            }
+            if (g < n_groups) prefix[g] = carry + incl - x;
+            carry += __shfl_sync(0xffffffffu, incl, 31);
+        }
+        if (lane == 0) prefix[n_groups] = carry;
+    }
+    tc::tc_fence_before();
+    __syncthreads();
+    tc::tc_fence_after();
+    const uint32_t tmem_base = *tmem_holder;
+    const int64_t total = n_groups > 0 ? prefix[n_groups] : 0;
+    const int64_t f_begin = total * blockIdx.x / gridDim.x;
+    const int64_t f_end = total * (blockIdx.x + 1) / gridDim.x;
+
+    if (f_begin < f_end) {
+        if (warp == 0) {
+            // ------------------------------------------------------------ TMA producer
+            if (tc::elect_one()) {
+                tc::tma_prefetch_desc(&tmap_k);
+                tc::tma_prefetch_desc(&tmap_q);
+                int g = first_group(prefix, n_groups, f_begin), kt, cur = -1;
+                uint32_t stage = 0, phase = 0, qe_phase = 0;
+                GroupInfo gi{0, -1};
+                for (int64_t f = f_begin; f < f_end; ++f) {
+                    locate(prefix, n_groups, f, g, kt);
+                    if (g != cur) {
+                        if (cur >= 0) {
+                            if (!tc::mbar_wait(q_empty, qe_phase, abort_flag)) break;
+                            qe_phase ^= 1;
+                        }
+                        tc::mbar_arrive_expect_tx(q_full, C::kQBytes);
+                        const int32_t qrow = q_row0 + g * G * kHI;
+                        tc::tma_load_2d(qbuf, &tmap_q, q_full, 0, qrow);
+                        tc::tma_load_2d(qbuf + N * 128, &tmap_q, q_full, 64, qrow);
+                        gi = group_info(v, g, G, false);
+                        cur = g;
+                    }
+                    const int s0 = kt * kBM;
+                    const int n_keys = min(kBM, gi.pos_max + 1 - s0);
+                    const int n_boxes = (int)ceil_div(n_keys, box_rows);
+                    uint64_t* bar = kFp8 ? &raw_full[stage & 3] : &full[stage];
+                    if (kFp8) {
+                        if (!tc::mbar_wait(&raw_empty[stage & 3], ((stage >> 2) & 1) ^ 1, abort_flag)) break;
+                    } else {
+                        if (!tc::mbar_wait(&empty[stage], phase ^ 1, abort_flag)) break;
+                    }
+                    tc::mbar_arrive_expect_tx(bar, (uint32_t)(n_boxes * box_rows * (kFp8 ? 128 : 256)));
+                    for (int j = 0; j < n_boxes; ++j) {
+                        const int s = s0 + j * box_rows;
+                        const int32_t row = (int32_t)paged_slot(v, gi.b, s);
+                        if (kFp8) {
+                            uint8_t* dst = raw + (size_t)(stage & 3) * (kBM * kDI) + (size_t)j * box_rows * 128;
+                            tc::tma_load_2d(dst, &tmap_k, bar, 0, row);
+                        } else {
+                            uint8_t* dst = tiles + (size_t)stage * kTileBytes + (size_t)j * box_rows * 128;
+                            tc::tma_load_2d(dst, &tmap_k, bar, 0, row);
+                            tc::tma_load_2d(dst + kHalfBytes, &tmap_k, bar, 64, row);
+                        }
+                    }
+                    if (kFp8) {
+                        ++stage;   // staging ring of 4; the bf16 ring is advanced by the converters
+                    } else if (++stage == (uint32_t)S) {
+                        stage = 0;
+                        phase ^= 1;
+                    }
+                }
+            }
+            __syncwarp();
+        } else if (warp == 1) {
+            // ------------------------------------------------------------ MMA issuer
+            if (tc::elect_one()) {
+                int g = first_group(prefix, n_groups, f_begin), kt, cur = -1;
+                uint32_t stage = 0, phase = 0, acc = 0, acc_phase = 0, q_phase = 0;
+                const uint32_t q_addr = tc::smem_u32(qbuf);
+                for (int64_t f = f_begin; f < f_end; ++f) {
+                    locate(prefix, n_groups, f, g, kt);
+                    if (g != cur) {
+                        if (!tc::mbar_wait(q_full, q_phase, abort_flag)) break;
+                        q_phase ^= 1;
+                        cur = g;
+                    }
+                    if (!tc::mbar_wait(&full[stage], phase, abort_flag)) break;
+                    if (!tc::mbar_wait(&acc_empty[acc], acc_phase ^ 1, abort_flag)) break;
+                    tc::tc_fence_after();
+                    const uint32_t a_addr = tc::smem_u32(tiles + (size_t)stage * kTileBytes);
+                    const uint32_t d = tmem_base + acc * N;
+#pragma unroll
+                    for (int k = 0; k < kDI / 16; ++k) {
+                        const uint32_t koff = (uint32_t)((k >> 2) * kHalfBytes + (k & 3) * 32);
+                        const uint32_t qoff = (uint32_t)((k >> 2) * (N * 128) + (k & 3) * 32);
+                        tc::mma_bf16(d, tc::sw128_desc(a_addr + koff, 16, 1024),
+                                     tc::sw128_desc(q_addr + qoff, 16, 1024), kIdesc, k > 0 ? 1u : 0u);
+                    }
+                    tc::mma_commit(&empty[stage]);
+                    tc::mma_commit(&acc_full[acc]);
+                    int g2 = g, kt2;
+                    if (f + 1 < f_end) locate(prefix, n_groups, f + 1, g2, kt2);
+                    if (f + 1 == f_end || g2 != g) tc::mma_commit(q_empty);
+                    if (++stage == (uint32_t)S) {
+                        stage = 0;
+                        phase ^= 1;
+                    }
+                    acc ^= 1;
+                    if (acc == 0) acc_phase ^= 1;
+                }
+            }
+            __syncwarp();
+        } else if (warp < 6) {
+            // ------------------------------------------------------------ epilogue
+            const int quarter = warp & 3;
+            const int r_in_tile = quarter * 32 + lane;
+            const int et = tid - 64;  // 0..127
+            int g = first_group(prefix, n_groups, f_begin), kt, cur = -1;
+            uint32_t acc = 0, acc_phase = 0;
+            int32_t row_pos[G];
+            int32_t seq_b = 0;
+            for (int64_t f = f_begin; f < f_end; ++f) {
+                locate(prefix, n_groups, f, g, kt);
+                if (g != cur) {
+                    tc::named_barrier(1, 128);
+                    for (int i = et; i < N; i += 128) {
+                        const int t = g * G + i / kHI;
+                        w_s[i] = t < v.T_q ? w[(int64_t)t * kHI + (i % kHI)] : 0.f;
+                    }
+                    const GroupInfo gi = group_info(v, g, G, false);
+                    seq_b = gi.b < 0 ? 0 : gi.b;
+#pragma unroll
+                    for (int j = 0; j < G; ++j) {
+                        const int t = g * G + j;
+                        row_pos[j] = -1;
+                        if (t < v.T_q) {
+                            RowInfo r = load_row(v, t);
+                            if (r.pos >= 0 && r.b == gi.b) row_pos[j] = r.pos;
+                        }
+                    }
+                    tc::named_barrier(1, 128);
+                    cur = g;
+                }
+                if (!tc::mbar_wait(&acc_full[acc], acc_phase, abort_flag)) break;
+                tc::tc_fence_after();
+                const int s = kt * kBM + r_in_tile;
+                const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + acc * N;
+                float kscale = 1.f;
+                if (kFp8) {
+                    int pmax = -1;
+#pragma unroll
+                    for (int j = 0; j < G; ++j) pmax = max(pmax, row_pos[j]);
+                    if (s <= pmax) kscale = __ldg(k_scale + paged_slot(v, seq_b, s));
+                }
+#pragma unroll
+                for (int j = 0; j < G; ++j) {
+                    float a[64];
+                    tc::tmem_ld32(taddr + j * kHI, a);
+                    tc::tmem_ld32(taddr + j * kHI + 32, a + 32);
+                    tc::tmem_ld_wait();
+                    float sc = 0.f;
+                    const float* wj = w_s + j * kHI;
+#pragma unroll
+                    for (int h = 0; h < kHI; ++h) sc = fmaf(wj[h], fmaxf(a[h], 0.f), sc);
+                    if (kFp8) sc *= kscale;   // positive per-key scale factors out of the ReLU sum
+                    if (s <= row_pos[j]) scores[(int64_t)(g * G + j) * ld + s] = sc;
+                }
+                tc::tc_fence_before();
+                __syncwarp();
+                if (lane == 0) tc::mbar_arrive(&acc_empty[acc]);
+                acc ^= 1;
+                if (acc == 0) acc_phase ^= 1;
+            }
+        } else if (kFp8) {
+            // ------------------------------------------------------------ FP8 -> bf16 converters
+            // thread r widens key row r of the staging tile (128 codes) into the two 64-column
+            // swizzled halves of the bf16 tile the MMA reads (e4m3 -> f16 -> bf16 is exact)
+            const int r = tid - 192;  // 0..127
+            uint32_t stage = 0, phase = 0;
+            uint32_t n = 0;
+            for (int64_t f = f_begin; f < f_end; ++f, ++n) {
+                if (!tc::mbar_wait(&raw_full[n & 3], (n >> 2) & 1, abort_flag)) break;
+                if (!tc::mbar_wait(&empty[stage], phase ^ 1, abort_flag)) break;
+                const uint8_t* src = raw + (size_t)(n & 3) * (kBM * kDI) + (size_t)r * 128;
+                uint8_t* dst = tiles + (size_t)stage * kTileBytes + (size_t)r * 128;
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {               // 16 codes -> 32 bytes of bf16
+                    const uint4 in = *reinterpret_cast<const uint4*>(src + c * 16);
+                    const uint32_t words[4] = {in.x, in.y, in.z, in.w};
+                    uint32_t outw[8];
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+#pragma unroll
+                        for (int hlf = 0; hlf < 2; ++hlf) {
+                            const __nv_fp8x2_storage_t pair = (__nv_fp8x2_storage_t)(words[q] >> (16 * hlf));
+                            const __half2_raw h2 = __nv_cvt_fp8x2_to_halfraw2(pair, __NV_E4M3);
+                            const float2 f2 = __half22float2(__half2(h2));
+                            const __nv_bfloat162 b2 = __floats2bfloat162_rn(f2.x, f2.y);
+                            outw[q * 2 + hlf] = *reinterpret_cast<const uint32_t*>(&b2);
+                        }
+                    }
+                    const int half = c >> 2;                 // which 64-column half
+                    const int chunk = (c & 3) * 2;           // 16-byte chunk within the 128-byte row
+                    uint8_t* hbase = dst + half * kHalfBytes;
+                    *reinterpret_cast<uint4*>(hbase + (((chunk) ^ (r & 7)) * 16)) =
+                        make_uint4(outw[0], outw[1], outw[2], outw[3]);
+                    *reinterpret_cast<uint4*>(hbase + (((chunk + 1) ^ (r & 7)) * 16)) =
+                        make_uint4(outw[4], outw[5], outw[6], outw[7]);
+                }
+                tc::fence_async_smem();
+                tc::mbar_arrive(&raw_empty[n & 3]);
+                tc::mbar_arrive(&full[stage]);
+                if (++stage == (uint32_t)S) {
+                    stage = 0;
+                    phase ^= 1;
+                }
+            }
+        }
+    }
+    __syncthreads();
+    if (warp == 1) {
+        tc::tc_fence_after();
+        tc::tmem_dealloc(tmem_base, C::kTmemCols);
+    }
+    if (tid == 0 && *abort_flag) flag_status(v, HSA_DEV_TIMEOUT);
+}
+
+int num_sms() {
+    static int n = 0;
+    if (n == 0) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        if (n <= 0) n = 148;
+    }
+    return n;
+}
+
+template <int G, bool kFp8>
+cudaError_t launch_g(const IndexScoreArgs& a, cudaStream_t st) {
+    using C = Cfg<G, kFp8>;
+    const int box_rows = a.seq.page_size <= kBM ? a.seq.page_size : kBM;
+    const uint64_t slots = (uint64_t)a.seq.num_pages * a.seq.page_size;
+    CUtensorMap tk, tq;
+    bool ok = kFp8 ? make_tensor_map_2d(&tk, a.k_cache, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, slots, kDI,
+                                        kDI, kDI, box_rows, CU_TENSOR_MAP_SWIZZLE_NONE)
+                   : make_tensor_map_2d(&tk, a.k_cache, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, slots,
+                                        kDI, kDI * 2, 64, box_rows, CU_TENSOR_MAP_SWIZZLE_128B);
+    ok = ok && make_tensor_map_2d(&tq, a.q_I, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                                  (uint64_t)a.seq.T_q * kHI, kDI, kDI * 2, 64, C::N,
+                                  CU_TENSOR_MAP_SWIZZLE_128B);
+    if (!ok) return cudaErrorInvalidValue;
+    auto kern = index_score_tc_kernel<G, kFp8>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::kSmem);
+    if (e != cudaSuccess) return e;
+    const int rows_per_launch = C::kMaxGroups * G;
+    for (int t0 = 0; t0 < a.seq.T_q; t0 += rows_per_launch) {
+        SeqView v = a.seq;
+        v.T_q = min(rows_per_launch, a.seq.T_q - t0);
+        v.q_seq += t0;
+        v.q_pos += t0;
+        const int64_t groups = ceil_div(v.T_q, G);
+        const int grid = (int)std::min<int64_t>(num_sms(), std::max<int64_t>(1, groups * 64));
+        kern<<<grid, C::kThreads, C::kSmem, st>>>(tk, tq, v, t0 * kHI, a.w + (int64_t)t0 * kHI,
+                                                   a.k_scale, a.scores + (int64_t)t0 * a.ld, a.ld,
+                                                   box_rows);
+        count_launch();
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+}
+
+}  // namespace
+
+bool index_score_tc_supported(const IndexScoreArgs& a) {
+    if (a.q_dtype != HSA_BF16 || (a.k_dtype != HSA_BF16 && a.k_dtype != HSA_E4M3)) return false;
+    if (a.k_dtype == HSA_E4M3 && a.k_scale == nullptr) return false;
+    if (a.H_I != kHI || a.D_I != kDI) return false;
+    const int p = a.seq.page_size;
+    if (p % 8 != 0) return false;
+    if (p <= kBM ? (kBM % p != 0) : (p % kBM != 0)) return false;
+    if ((reinterpret_cast<uintptr_t>(a.q_I) & 15) || (reinterpret_cast<uintptr_t>(a.k_cache) & 15)) return false;
+    if ((uint64_t)a.seq.num_pages * p >= (1ull << 31) || (uint64_t)a.seq.T_q * kHI >= (1ull << 31)) return false;
+    return true;
+}
+
+cudaError_t launch_index_score_tc(const IndexScoreArgs& a, cudaStream_t st) {
+    const bool fp8 = a.k_dtype == HSA_E4M3;
+    if (a.q_run % 4 == 0) return fp8 ? launch_g<4, true>(a, st) : launch_g<4, false>(a, st);
+    if (a.q_run % 2 == 0) return fp8 ? launch_g<2, true>(a, st) : launch_g<2, false>(a, st);
+    return fp8 ? launch_g<1, true>(a, st) : launch_g<1, false>(a, st);
+}
+
 }  // namespace hsa

@@ -50,6 +50,21 @@ def test_index_score_vs_oracle(name, kw):
     _index_vs_oracle(workloads.make(name, DEV, **kw))
 
 
+@pytest.mark.parametrize("q_run,T", [(1, 2500), (2, 600), (4, 300)])
+def test_index_score_row_groupings(q_run, T):
+    """The tensor-core kernel groups q_run-aligned rows (1, 2 or 4 per MMA tile) and splits
+    launches past its group limit; every grouping must give the same per-row contract."""
+    wl = workloads.make("prefill_bf16", DEV, T=T)
+    wl.q_run = q_run
+    _index_vs_oracle(wl, rows=sorted(set(range(0, T, 7)) | {T - 1}))
+
+
+@pytest.mark.parametrize("page_size", [16, 128, 256])
+def test_index_score_page_sizes(page_size):
+    _index_vs_oracle(workloads.make("decode_bf16", DEV, B=4, L_min=200, L_max=1300, page_size=page_size))
+    _index_vs_oracle(workloads.make("decode_fp8", DEV, B=2, L=900, page_size=page_size))
+
+
 def test_index_score_integer_inputs_bit_exact():
     wl = workloads.make("decode_bf16", DEV, B=3, L_min=200, L_max=900)
     g = torch.Generator(device=DEV).manual_seed(77)
