@@ -115,9 +115,10 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
     uint64_t* q_empty = q_full + 1;
     uint64_t* raw_full = q_empty + 1;      // [4] FP8 bytes landed
     uint64_t* raw_empty = raw_full + 4;    // [4] converters done with the staging tile
-    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(raw_empty + 4);
+    uint64_t* epi_bar = raw_empty + 4;     // the four epilogue warps
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(epi_bar + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
-    static_assert((2 * S + 2 + 2 + 2 + 8) * 8 + 8 <= 256, "barrier block");
+    static_assert((2 * S + 2 + 2 + 2 + 8 + 1) * 8 + 8 <= 256, "barrier block");
     int32_t* prefix = reinterpret_cast<int32_t*>(reinterpret_cast<uint8_t*>(bars) + 256);
     float* w_s = reinterpret_cast<float*>(prefix + C::kMaxGroups + 1);
 
@@ -139,6 +140,7 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
             tc::mbar_init(&raw_full[i], 1);
             tc::mbar_init(&raw_empty[i], 128);
         }
+        tc::mbar_init(epi_bar, 4);
         *abort_flag = 0;
         tc::fence_barrier_init();
     }
@@ -278,10 +280,11 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
             uint32_t acc = 0, acc_phase = 0;
             int32_t row_pos[G];
             int32_t seq_b = 0;
+            tc::WarpSetSync epi_sync{epi_bar, 0};
             for (int64_t f = f_begin; f < f_end; ++f) {
                 locate(prefix, n_groups, f, g, kt);
                 if (g != cur) {
-                    tc::named_barrier(1, 128);
+                    if (!epi_sync.sync(abort_flag)) break;   // everyone is done with the old weights
                     for (int i = et; i < N; i += 128) {
                         const int t = g * G + i / kHI;
                         w_s[i] = t < v.T_q ? w[(int64_t)t * kHI + (i % kHI)] : 0.f;
@@ -297,7 +300,7 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
                             if (r.pos >= 0 && r.b == gi.b) row_pos[j] = r.pos;
                         }
                     }
-                    tc::named_barrier(1, 128);
+                    if (!epi_sync.sync(abort_flag)) break;   // the new weights are in place
                     cur = g;
                 }
                 if (!tc::mbar_wait(&acc_full[acc], acc_phase, abort_flag)) break;

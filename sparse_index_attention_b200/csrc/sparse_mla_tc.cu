@@ -5,8 +5,10 @@
 // Inference Adaptation for Very Large Hybrid-Attention Models", 3.2: partition by query,
 // aggregate over the selected positions, stage them in shared memory.
 //
-// Per query row t the selected latent rows are gathered in tiles of 64 (TMA tile::gather4
-// through the block table) and every tile is shared by all 128 heads:
+// Per query row t the selected latent rows are gathered in tiles of 64 through the block table
+// (cp.async by four producer warps: one warp instruction moves one row's 512-byte half, so every
+// request is a full, coalesced line; the 128-byte / 64-byte swizzles the MMA expects are applied
+// to the destination addresses) and every tile is shared by all 128 heads:
 //     S = Q_t . KV^T            (M = 128 heads, N = 64 rows, K = 576)
 //     P = online softmax(S)     (fp32, base-2 exponent, lazy rescale)
 //     O += P . V                (M = 128 heads, N = 512 latent dims, K = 64 rows)
@@ -19,16 +21,28 @@
 // decisions).  Each CTA then accumulates its half of O.  No gathered byte and no MMA is
 // duplicated between the two CTAs.
 //
-// Shared memory per CTA: Q (72 KB: four 64-dim 128-byte-swizzled blocks + one 32-dim
-// 64-byte-swizzled rope block), three KV stages of 64 rows (36 KB each, same block structure;
-// the stage is the K-major B operand of Q.KV^T and, read MN-major, the B operand of P.V), and a
-// 32 KB exchange buffer that receives the peer's partial S; after it is read, P (bf16, 16 KB)
-// is written over it.  Ordering needs no extra barrier: the peer only sends tile n after this
-// CTA's P.V of tile n-1 completed (its MMA commit is multicast to the peer), so receiving tile n
-// also proves that the previous P is no longer in use.
+// Shared memory per CTA: the rope part of Q (8 KB, 64-byte swizzle), four KV stages of 64
+// gathered rows (36 KB each: four 64-dim 128-byte-swizzled blocks + one 32-dim 64-byte-swizzled
+// rope block; the stage is the K-major B operand of Q.KV^T and, read MN-major, the B operand of
+// P.V), two 32 KB exchange buffers that receive the peer's partial S (P, bf16, is written over
+// the buffer once it has been read), and the physical slots of the next 2048 selected entries.
+// The latent part of Q lives in TMEM (A operand of Q.KV^T), next to O (256 columns) and the two
+// partial-S buffers (2 x 64 columns).
 //
-// Warp roles: 0 TMA producer (gather), 1 MMA issuer, 2-5 softmax / exchange / epilogue (thread h
-// owns head h = TMEM lane h).  Persistent: each cluster loops over query rows.
+// Pipeline per tile n: the softmax warps send their partial S(n+1) to the peer before they
+// compute softmax(n), so the distributed-shared-memory hop overlaps the exponentials, and the
+// tensor core runs Q.KV^T(n+1) and P.V(n-1) while softmax(n) runs.  The peer may overwrite an
+// exchange buffer only after this CTA's P.V of the tile that used it (MMA commit multicast to the
+// peer), which is also what makes receiving tile n prove that P.V(n-2) has finished.
+//
+// (A TMA tile::gather4 version of the gather -- four 128-byte rows per instruction, 80 per tile
+// and CTA -- delivered only about 0.75 TB/s here: the MMA warp waited on the gathered tiles for
+// three quarters of the kernel.  Plain 16-byte asynchronous copies from 128 threads keep far more
+// bytes in flight.)
+//
+// Warp roles: 0-3 producers (slot window + gather; warp w owns rows 16w..16w+15 of every tile,
+// warp 0 also loads the rope part of Q by TMA), 4 MMA issuer, 5-8 softmax / exchange / epilogue
+// (thread h owns head h = TMEM lane h).  Persistent: each cluster loops over query rows.
 #include <algorithm>
 
 #include "kernels.h"
@@ -42,24 +56,29 @@ constexpr int kH = 128;          // heads = MMA M = TMEM lanes
 constexpr int kDqk = 576;
 constexpr int kDv = 512;
 constexpr int kBN = 64;          // gathered rows per tile
-constexpr int kStages = 3;
-constexpr int kThreads = 192;
+constexpr int kStages = 4;
+constexpr int kThreads = 288;
+constexpr int kCopyDepth = 2;    // cp.async groups in flight per producer thread beyond the newest
+constexpr int kSlotWin = 2048;   // selected entries whose slots are resolved at once
 
-constexpr int kQBlk = kH * 128;                    // 128 heads x 64 dims bf16, SW128
-constexpr int kQRope = kH * 64;                    // 128 heads x 32 dims bf16, SW64
-constexpr int kQBytes = 4 * kQBlk + kQRope;        // 72 KB
+constexpr int kQRopeBytes = kH * 64;               // 128 heads x 32 dims bf16, SW64
 constexpr int kKvBlk = kBN * 128;                  // 64 rows x 64 dims
 constexpr int kKvRope = kBN * 64;                  // 64 rows x 32 dims
 constexpr int kStageBytes = 4 * kKvBlk + kKvRope;  // 36 KB
-constexpr int kOffStages = kQBytes;
-constexpr int kOffRecv = kOffStages + kStages * kStageBytes;
 constexpr int kRecvBytes = kH * kBN * 4;           // 32 KB of fp32 partial S
-constexpr int kOffBars = kOffRecv + kRecvBytes;
+constexpr int kOffStages = kQRopeBytes;
+constexpr int kOffRecv = kOffStages + kStages * kStageBytes;
+constexpr int kOffSlots = kOffRecv + 2 * kRecvBytes;
+constexpr int kOffMasks = kOffSlots + 4 * kSlotWin;
+constexpr int kOffBars = kOffMasks + 8 * kStages;
+constexpr int kKvRowBytes = kDqk * 2;   // 1152
 constexpr size_t kSmem = 1024 + kOffBars + 256;
 static_assert(kSmem <= 232448, "shared memory budget");
+static_assert(kOffStages % 1024 == 0 && kStageBytes % 1024 == 0 && kOffRecv % 1024 == 0, "swizzle alignment");
 
 constexpr uint32_t kTmemO = 0;       // 256 columns: this CTA's half of O
 constexpr uint32_t kTmemS = 256;     // 2 x 64 columns: partial S, double-buffered
+constexpr uint32_t kTmemQ = 384;     // 128 columns: this CTA's 256 latent dims of Q (bf16 pairs)
 constexpr uint32_t kTmemCols = 512;
 
 constexpr uint32_t kIdescQK = tc::idesc_bf16_f32(kH, kBN, 0, 0);
@@ -67,20 +86,22 @@ constexpr uint32_t kIdescPV = tc::idesc_bf16_f32(kH, 256, 0, 1);
 constexpr float kRescaleLog2 = 8.f;  // rescale O only when the running max grows by > 2^8
 
 struct Bars {
-    uint64_t q_full, q_empty;
+    uint64_t q_full;      // Q of the row in place: latent part in TMEM, rope part in smem (4 warps)
+    uint64_t q_empty;     // last Q.KV^T of the row done
     uint64_t kv_full[kStages], kv_empty[kStages];
     uint64_t s_full[2], s_empty[2];
     uint64_t p_full;
-    uint64_t peer_free;   // the peer's P.V of the previous tile is done (its buffer is free)
-    uint64_t recv_full;   // the peer's partial S of this tile has landed here
+    uint64_t pv_done;     // this CTA's P.V of a tile completed
+    uint64_t peer_free[2];  // the peer's P.V of a tile of parity b completed (its buffer b is free)
+    uint64_t recv_full[2];
     uint64_t o_ready, o_free;
+    uint64_t buf_read;    // the four softmax warps finished reading an exchange buffer
     uint32_t tmem;
     int abort;
 };
 static_assert(sizeof(Bars) <= 256, "barrier block");
 
-// Number of leading entries of idx row t that can hold a selection (1 + last index != -1),
-// computed by a whole warp scanning from the end.
+// 1 + the last index of idx row that is not -1 (0 if none), by a whole warp scanning from the end.
 __device__ __forceinline__ int row_extent(const int32_t* __restrict__ idx_row, int K, int lane) {
     for (int k0 = ((K - 1) / 32) * 32; k0 >= 0; k0 -= 32) {
         const int k = k0 + lane;
@@ -91,38 +112,25 @@ __device__ __forceinline__ int row_extent(const int32_t* __restrict__ idx_row, i
     return 0;
 }
 
-// Physical slot of selected entry k of a row (0 for padding or an invalid entry, which the
-// softmax masks out).
-__device__ __forceinline__ int32_t entry_slot(const SeqView& v, const int32_t* __restrict__ idx_row,
-                                              int K, int k, int b, int pos) {
-    if (k >= K) return 0;
-    const int n = __ldg(idx_row + k);
-    if (n < 0 || n > pos) return 0;
-    return (int32_t)paged_slot(v, b, n);
-}
-
-__device__ __forceinline__ bool entry_valid(const int32_t* __restrict__ idx_row, int K, int k, int pos,
-                                            const SeqView& v, bool flag) {
-    if (k >= K) return false;
-    const int n = __ldg(idx_row + k);
-    if (n == -1) return false;
-    if (n < 0 || n > pos) {
-        if (flag) flag_status(v, HSA_DEV_BAD_POS);
-        return false;
-    }
-    return true;
+__device__ __forceinline__ int row_tiles(const SeqView& v, const int32_t* __restrict__ idx, int K, int t,
+                                         int lane, RowInfo& r) {
+    r = load_row(v, t);
+    if (r.pos < 0) return 0;
+    return (int)ceil_div(row_extent(idx + (int64_t)t * K, K, lane), kBN);
 }
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
-sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q_lat, const __grid_constant__ CUtensorMap tm_q_rope,
-                     const __grid_constant__ CUtensorMap tm_kv_lat, const __grid_constant__ CUtensorMap tm_kv_rope,
-                     SeqView v, const int32_t* __restrict__ idx, int K, float scale_log2,
-                     __nv_bfloat16* __restrict__ out, float* __restrict__ lse) {
+sparse_mla_tc_kernel(SeqView v,
+                     const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ kv,
+                     const int32_t* __restrict__ idx, int K,
+                     float scale_log2, __nv_bfloat16* __restrict__ out, float* __restrict__ lse) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t* qs = base;
+    uint8_t* q_rope = base;
     uint8_t* stages = base + kOffStages;
     uint8_t* recv = base + kOffRecv;
+    int32_t* slots = reinterpret_cast<int32_t*>(base + kOffSlots);
+    volatile uint64_t* masks = reinterpret_cast<volatile uint64_t*>(base + kOffMasks);
     Bars* bars = reinterpret_cast<Bars*>(base + kOffBars);
     volatile int* abort_flag = &bars->abort;
 
@@ -133,25 +141,28 @@ sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q_lat, const __grid_
     const int n_clusters = gridDim.x >> 1;
 
     if (tid == 0) {
-        tc::mbar_init(&bars->q_full, 1);
+        tc::mbar_init(&bars->q_full, 4);
         tc::mbar_init(&bars->q_empty, 1);
         for (int i = 0; i < kStages; ++i) {
-            tc::mbar_init(&bars->kv_full[i], 1);
+            tc::mbar_init(&bars->kv_full[i], 128);   // every producer thread, after its copies landed
             tc::mbar_init(&bars->kv_empty[i], 1);
         }
         for (int i = 0; i < 2; ++i) {
             tc::mbar_init(&bars->s_full[i], 1);
             tc::mbar_init(&bars->s_empty[i], 4);
+            tc::mbar_init(&bars->recv_full[i], 1);
         }
         tc::mbar_init(&bars->p_full, 4);
-        tc::mbar_init(&bars->peer_free, 1);
-        tc::mbar_init(&bars->recv_full, 1);
+        tc::mbar_init(&bars->pv_done, 1);
+        tc::mbar_init(&bars->peer_free[0], 1);
+        tc::mbar_init(&bars->peer_free[1], 1);
         tc::mbar_init(&bars->o_ready, 1);
         tc::mbar_init(&bars->o_free, 4);
+        tc::mbar_init(&bars->buf_read, 4);
         bars->abort = 0;
         tc::fence_barrier_init();
     }
-    if (warp == 1) {
+    if (warp == 4) {
         tc::tmem_alloc(&bars->tmem, kTmemCols);
         tc::tmem_relinquish();
     }
@@ -161,62 +172,88 @@ sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q_lat, const __grid_
     tc::tc_fence_after();
     const uint32_t tmem_base = bars->tmem;
 
-    if (warp == 0) {
-        // ---------------------------------------------------------------- producer (TMA)
-        if (lane == 0) {
-            tc::tma_prefetch_desc(&tm_q_lat);
-            tc::tma_prefetch_desc(&tm_q_rope);
-            tc::tma_prefetch_desc(&tm_kv_lat);
-            tc::tma_prefetch_desc(&tm_kv_rope);
-        }
-        uint32_t n = 0, qr = 0;
+    if (warp < 4) {
+        // ---------------------------------------------------------------- producers (gather)
+        const uint8_t* kv_bytes = reinterpret_cast<const uint8_t*>(kv);
+        int32_t* my_slots = slots + warp * (kSlotWin / 4);   // this warp's 16 rows of 32 tiles
+        uint16_t* masks16 = reinterpret_cast<uint16_t*>(const_cast<uint64_t*>(masks));
+        uint32_t n = 0, landed = 0;
         bool stop = false;
+        // the copies of tile `landed` are complete for this thread: publish them
+        auto publish = [&]() {
+            tc::fence_async_smem();   // generic-proxy writes -> visible to the tensor core
+            tc::mbar_arrive(&bars->kv_full[landed % kStages]);
+            ++landed;
+        };
         for (int t = cluster; t < v.T_q && !stop; t += n_clusters) {
-            const RowInfo r = load_row(v, t);
-            const int32_t* idx_row = idx + (int64_t)t * K;
-            const int ntiles = r.pos < 0 ? 0 : (int)ceil_div(row_extent(idx_row, K, lane), kBN);
+            RowInfo r;
+            const int ntiles = row_tiles(v, idx, K, t, lane, r);
             if (ntiles == 0) continue;
-            if (qr > 0 && !tc::mbar_wait(&bars->q_empty, (qr - 1) & 1, abort_flag)) break;
-            if (lane == 0) {
-                tc::mbar_arrive_expect_tx(&bars->q_full, kQBytes);
-                for (int kb = 0; kb < 4; ++kb)
-                    tc::tma_load_2d(qs + kb * kQBlk, &tm_q_lat, &bars->q_full, 256 * rank + 64 * kb, t * kH);
-                tc::tma_load_2d(qs + 4 * kQBlk, &tm_q_rope, &bars->q_full, 512 + 32 * rank, t * kH);
-            }
-            ++qr;
+            const int32_t* idx_row = idx + (int64_t)t * K;
             for (int j = 0; j < ntiles; ++j, ++n) {
+                if (j % (kSlotWin / kBN) == 0) {
+                    // physical slots of this warp's rows for the next 32 tiles (-1: none), eight
+                    // independent lookups per lane in flight at a time
+#pragma unroll 1
+                    for (int e0 = 0; e0 < kSlotWin / 4; e0 += 32 * 8) {
+                        int32_t nn[8];
+#pragma unroll
+                        for (int u = 0; u < 8; ++u) {
+                            const int e = e0 + lane + 32 * u;
+                            const int k = (j + e / 16) * kBN + warp * 16 + (e % 16);
+                            nn[u] = k < K ? __ldg(idx_row + k) : -1;
+                        }
+#pragma unroll
+                        for (int u = 0; u < 8; ++u) {
+                            int32_t sl = -1;
+                            if (nn[u] >= 0 && nn[u] <= r.pos) sl = (int32_t)paged_slot(v, r.b, nn[u]);
+                            else if (nn[u] != -1 && rank == 0) flag_status(v, HSA_DEV_BAD_POS);
+                            my_slots[e0 + lane + 32 * u] = sl;
+                        }
+                    }
+                    __syncwarp();
+                }
                 const uint32_t st = n % kStages;
                 if (!tc::mbar_wait(&bars->kv_empty[st], ((n / kStages) & 1) ^ 1, abort_flag)) {
                     stop = true;
                     break;
                 }
-                const int k0 = j * kBN;
-                const int32_t slot_a = entry_slot(v, idx_row, K, k0 + lane, r.b, r.pos);
-                const int32_t slot_b = entry_slot(v, idx_row, K, k0 + 32 + lane, r.b, r.pos);
+                const int32_t* ts = my_slots + (j % (kSlotWin / kBN)) * 16;
                 uint8_t* sbase = stages + st * kStageBytes;
-                if (lane == 0) tc::mbar_arrive_expect_tx(&bars->kv_full[st], kStageBytes);
-#pragma unroll 1
-                for (int g = 0; g < kBN / 4; ++g) {
-                    const int32_t src = g < 8 ? slot_a : slot_b;
-                    const int l0 = (4 * g) & 31;
-                    const int32_t y0 = __shfl_sync(0xffffffffu, src, l0);
-                    const int32_t y1 = __shfl_sync(0xffffffffu, src, l0 + 1);
-                    const int32_t y2 = __shfl_sync(0xffffffffu, src, l0 + 2);
-                    const int32_t y3 = __shfl_sync(0xffffffffu, src, l0 + 3);
-                    if (lane == 0) {
-                        for (int kb = 0; kb < 4; ++kb)
-                            tc::tma_gather4(sbase + kb * kKvBlk + g * 512, &tm_kv_lat, &bars->kv_full[st],
-                                            256 * rank + 64 * kb, y0, y1, y2, y3);
-                        tc::tma_gather4(sbase + 4 * kKvBlk + g * 256, &tm_kv_rope, &bars->kv_full[st],
-                                        512 + 32 * rank, y0, y1, y2, y3);
-                    }
+                // latent half: one row per warp instruction, lane = 16-byte chunk
+#pragma unroll 4
+                for (int k = 0; k < 16; ++k) {
+                    const int row = warp * 16 + k;
+                    const int32_t sl = ts[k];
+                    const uint8_t* src = kv_bytes + (int64_t)(sl < 0 ? 0 : sl) * kKvRowBytes + 512 * rank + lane * 16;
+                    uint8_t* dst = sbase + (lane >> 3) * kKvBlk + row * 128 + (((lane & 7) ^ (row & 7)) * 16);
+                    tc::cp_async16(dst, src, sl < 0 ? 0u : 16u);
+                }
+                // rope half: 4 chunks per row, 8 rows per instruction
+#pragma unroll
+                for (int h2 = 0; h2 < 2; ++h2) {
+                    const int row = warp * 16 + 8 * h2 + (lane >> 2);
+                    const int cc = lane & 3;
+                    const int32_t sl = ts[8 * h2 + (lane >> 2)];
+                    const uint8_t* src = kv_bytes + (int64_t)(sl < 0 ? 0 : sl) * kKvRowBytes + 1024 + 64 * rank + cc * 16;
+                    uint8_t* dst = sbase + 4 * kKvBlk + row * 64 + ((cc ^ ((row >> 1) & 3)) * 16);
+                    tc::cp_async16(dst, src, sl < 0 ? 0u : 16u);
+                }
+                const uint32_t vm = __ballot_sync(0xffffffffu, lane < 16 && ts[lane & 15] >= 0) & 0xFFFFu;
+                if (lane == 0) masks16[st * 4 + warp] = (uint16_t)vm;
+                tc::cp_async_commit();
+                if (n >= (uint32_t)kCopyDepth) {
+                    tc::cp_async_wait<kCopyDepth>();
+                    publish();
                 }
             }
         }
-    } else if (warp == 1) {
+        // drain: the last tiles' copies
+        tc::cp_async_wait<0>();
+        while (!stop && landed < n) publish();
+    } else if (warp == 4) {
         // ---------------------------------------------------------------- MMA issuer
-        const uint32_t q_addr = tc::smem_u32(qs);
-        const uint32_t p_addr = tc::smem_u32(recv);
+        const uint32_t qr_addr = tc::smem_u32(q_rope);
         uint32_t n = 0, qr = 0, rows_done = 0;
         bool stop = false;
         auto pv = [&](uint32_t m, bool first) -> bool {
@@ -224,6 +261,7 @@ sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q_lat, const __grid_
             if (first && !tc::mbar_wait(&bars->o_free, (rows_done & 1) ^ 1, abort_flag)) return false;
             tc::tc_fence_after();
             if (lane == 0) {
+                const uint32_t p_addr = tc::smem_u32(recv + (m & 1) * kRecvBytes);
                 const uint32_t v_addr = tc::smem_u32(stages + (m % kStages) * kStageBytes);
 #pragma unroll
                 for (int kk = 0; kk < kBN / 16; ++kk)
@@ -231,15 +269,15 @@ sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q_lat, const __grid_
                                  tc::sw128_desc(v_addr + kk * 2048, kKvBlk, 1024), kIdescPV,
                                  (first && kk == 0) ? 0u : 1u);
                 tc::mma_commit(&bars->kv_empty[m % kStages]);
-                tc::mma_commit_multicast(&bars->peer_free, (uint16_t)(1u << peer));
+                tc::mma_commit(&bars->pv_done);
+                tc::mma_commit_multicast(&bars->peer_free[m & 1], (uint16_t)(1u << peer));
             }
             __syncwarp();
             return true;
         };
         for (int t = cluster; t < v.T_q && !stop; t += n_clusters) {
-            const RowInfo r = load_row(v, t);
-            const int32_t* idx_row = idx + (int64_t)t * K;
-            const int ntiles = r.pos < 0 ? 0 : (int)ceil_div(row_extent(idx_row, K, lane), kBN);
+            RowInfo r;
+            const int ntiles = row_tiles(v, idx, K, t, lane, r);
             if (ntiles == 0) continue;
             if (!tc::mbar_wait(&bars->q_full, qr & 1, abort_flag)) break;
             ++qr;
@@ -255,15 +293,13 @@ sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q_lat, const __grid_
                     const uint32_t kv_addr = tc::smem_u32(stages + st * kStageBytes);
                     const uint32_t d = tmem_base + kTmemS + sb * kBN;
 #pragma unroll
-                    for (int kb = 0; kb < 4; ++kb)
-#pragma unroll
-                        for (int kk = 0; kk < 4; ++kk)
-                            tc::mma_bf16(d, tc::sw128_desc(q_addr + kb * kQBlk + kk * 32, 16, 1024),
-                                         tc::sw128_desc(kv_addr + kb * kKvBlk + kk * 32, 16, 1024),
-                                         kIdescQK, (kb | kk) ? 1u : 0u);
+                    for (int k = 0; k < 16; ++k)
+                        tc::mma_bf16_tmem_a(d, tmem_base + kTmemQ + 8 * k,
+                                            tc::sw128_desc(kv_addr + (k >> 2) * kKvBlk + (k & 3) * 32, 16, 1024),
+                                            kIdescQK, k ? 1u : 0u);
 #pragma unroll
                     for (int kk = 0; kk < 2; ++kk)
-                        tc::mma_bf16(d, tc::sw64_desc(q_addr + 4 * kQBlk + kk * 32, 512),
+                        tc::mma_bf16(d, tc::sw64_desc(qr_addr + kk * 32, 512),
                                      tc::sw64_desc(kv_addr + 4 * kKvBlk + kk * 32, 512), kIdescQK, 1u);
                     tc::mma_commit(&bars->s_full[sb]);
                     if (j == ntiles - 1) tc::mma_commit(&bars->q_empty);
@@ -283,107 +319,166 @@ sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q_lat, const __grid_
         // ---------------------------------------------------------------- softmax / exchange
         const int h = (warp & 3) * 32 + lane;          // head = TMEM lane
         const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
-        const uint32_t my_recv = tc::smem_u32(recv) + h * (kBN * 4);
-        const uint32_t peer_recv = tc::mapa_shared(my_recv, peer);
-        const uint32_t peer_bar = tc::mapa_shared(tc::smem_u32(&bars->recv_full), peer);
+        uint32_t peer_recv[2], peer_bar[2];
+        for (int b = 0; b < 2; ++b) {
+            peer_recv[b] = tc::mapa_shared(tc::smem_u32(recv + b * kRecvBytes), peer);
+            peer_bar[b] = tc::mapa_shared(tc::smem_u32(&bars->recv_full[b]), peer);
+        }
         uint32_t n = 0, rows_done = 0;
         bool stop = false;
-        for (int t = cluster; t < v.T_q && !stop; t += n_clusters) {
-            const RowInfo r = load_row(v, t);
-            const int32_t* idx_row = idx + (int64_t)t * K;
-            const int ntiles = r.pos < 0 ? 0 : (int)ceil_div(row_extent(idx_row, K, lane), kBN);
-            __nv_bfloat16* orow = out + ((int64_t)t * kH + h) * kDv + 256 * rank;
-            if (ntiles == 0) {
-                for (int c = 0; c < 256; c += 8)
-                    *reinterpret_cast<uint4*>(orow + c) = make_uint4(0, 0, 0, 0);
+        tc::WarpSetSync buf_sync{&bars->buf_read, 0};
+
+        // next row (t0, t0 + n_clusters, ...) with work; rows without any selection are written
+        // here directly (output 0, lse -inf)
+        auto next_row = [&](int t0, int& ntiles, RowInfo& r) -> int {
+            for (int t = t0; t < v.T_q; t += n_clusters) {
+                ntiles = row_tiles(v, idx, K, t, lane, r);
+                if (ntiles > 0) return t;
+                __nv_bfloat16* orow = out + ((int64_t)t * kH + h) * kDv + 256 * rank;
+                for (int c = 0; c < 256; c += 8) *reinterpret_cast<uint4*>(orow + c) = make_uint4(0, 0, 0, 0);
                 if (lse != nullptr && rank == 0) lse[(int64_t)t * kH + h] = -INFINITY;
-                continue;
             }
+            return -1;
+        };
+        // Q row t: this CTA's 256 latent dims into TMEM (thread h writes lane h) and its 32 rope
+        // dims into shared memory (64-byte swizzle: 16-byte chunk c of row h at c ^ ((h >> 1) & 3))
+        auto load_q = [&](int t) {
+            const uint4* srcr = reinterpret_cast<const uint4*>(q + ((int64_t)t * kH + h) * kDqk + 512 + 32 * rank);
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+                *reinterpret_cast<uint4*>(q_rope + h * 64 + ((c ^ ((h >> 1) & 3)) * 16)) = __ldg(srcr + c);
+            tc::fence_async_smem();
+            const uint4* src = reinterpret_cast<const uint4*>(q + ((int64_t)t * kH + h) * kDqk + 256 * rank);
+#pragma unroll 1
+            for (int c = 0; c < 4; ++c) {
+                uint32_t w[32];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const uint4 x = __ldg(src + 8 * c + i);
+                    w[4 * i] = x.x;
+                    w[4 * i + 1] = x.y;
+                    w[4 * i + 2] = x.z;
+                    w[4 * i + 3] = x.w;
+                }
+                tc::tmem_st32_u(tmem_base + lane_off + kTmemQ + 32 * c, w);
+            }
+            tc::tmem_st_wait();
+            tc::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(&bars->q_full);
+        };
+        // partial S(m) -> the peer's exchange buffer (m & 1)
+        auto send_tile = [&](uint32_t m) -> bool {
+            const uint32_t b = m & 1;
+            if (!tc::mbar_wait(&bars->s_full[b], (m >> 1) & 1, abort_flag)) return false;
+            tc::tc_fence_after();
+            float s[kBN];
+            tc::tmem_ld32(tmem_base + lane_off + kTmemS + b * kBN, s);
+            tc::tmem_ld32(tmem_base + lane_off + kTmemS + b * kBN + 32, s + 32);
+            tc::tmem_ld_wait();
+            // the peer's P.V(m-2) has released its buffer b.  One barrier per buffer: the peer
+            // cannot complete P.V(m) before it receives this send, so the barrier is never two
+            // phases ahead of this wait (a single barrier for both buffers could be, since the
+            // peer may finish P.V(m-1) first, and a parity wait would then alias).
+            if (m >= 2 && !tc::mbar_wait(&bars->peer_free[b], ((m - 2) >> 1) & 1, abort_flag)) return false;
+            if (tid == 160) tc::mbar_arrive_expect_tx(&bars->recv_full[b], kRecvBytes);
+            const uint32_t dst = peer_recv[b] + h * (kBN * 4);
+#pragma unroll
+            for (int i = 0; i < kBN / 4; ++i)
+                tc::st_async_v4(dst + ((i ^ (h & 7)) * 16), peer_bar[b], __float_as_uint(s[4 * i]),
+                                __float_as_uint(s[4 * i + 1]), __float_as_uint(s[4 * i + 2]),
+                                __float_as_uint(s[4 * i + 3]));
+            return true;
+        };
+
+        int ntiles = 0;
+        RowInfo r;
+        int t = next_row(cluster, ntiles, r);
+        if (t >= 0) {
+            load_q(t);
+            stop = !send_tile(0);
+        }
+        while (t >= 0 && !stop) {
             float m_used = -INFINITY, l = 0.f;
+            int t_next = -1, ntiles_next = 0;
+            RowInfo r_next;
             for (int j = 0; j < ntiles; ++j, ++n) {
-                const uint32_t sb = n & 1;
-                const int k0 = j * kBN;
-                const uint32_t va = __ballot_sync(0xffffffffu, entry_valid(idx_row, K, k0 + lane, r.pos, v, warp == 2 && rank == 0));
-                const uint32_t vb = __ballot_sync(0xffffffffu, entry_valid(idx_row, K, k0 + 32 + lane, r.pos, v, warp == 2 && rank == 0));
-                if (!tc::mbar_wait(&bars->s_full[sb], (n >> 1) & 1, abort_flag)) {
+                const uint32_t b = n & 1, st = n % kStages;
+                // ---- softmax(n)
+                if (!tc::mbar_wait(&bars->kv_full[st], (n / kStages) & 1, abort_flag) ||
+                    !tc::mbar_wait_cluster(&bars->recv_full[b], (n >> 1) & 1, abort_flag)) {
                     stop = true;
                     break;
                 }
+                const uint64_t valid = masks[st];
                 tc::tc_fence_after();
                 float s[kBN];
-                tc::tmem_ld32(tmem_base + lane_off + kTmemS + sb * kBN, s);
-                tc::tmem_ld32(tmem_base + lane_off + kTmemS + sb * kBN + 32, s + 32);
+                tc::tmem_ld32(tmem_base + lane_off + kTmemS + b * kBN, s);
+                tc::tmem_ld32(tmem_base + lane_off + kTmemS + b * kBN + 32, s + 32);
                 tc::tmem_ld_wait();
                 tc::tc_fence_before();
                 __syncwarp();
-                if (lane == 0) tc::mbar_arrive(&bars->s_empty[sb]);
-                // swap partial S with the peer
-                if (n > 0 && !tc::mbar_wait(&bars->peer_free, (n - 1) & 1, abort_flag)) {
-                    stop = true;
-                    break;
-                }
-                if (tid == 64) tc::mbar_arrive_expect_tx(&bars->recv_full, kRecvBytes);
-#pragma unroll
-                for (int i = 0; i < kBN / 4; ++i)
-                    tc::st_async_v4(peer_recv + 16 * i, peer_bar, __float_as_uint(s[4 * i]),
-                                    __float_as_uint(s[4 * i + 1]), __float_as_uint(s[4 * i + 2]),
-                                    __float_as_uint(s[4 * i + 3]));
-                if (!tc::mbar_wait_cluster(&bars->recv_full, n & 1, abort_flag)) {
-                    stop = true;
-                    break;
-                }
-                const float4* other = reinterpret_cast<const float4*>(recv + h * (kBN * 4));
+                if (lane == 0) tc::mbar_arrive(&bars->s_empty[b]);
+                uint8_t* buf = recv + b * kRecvBytes;
+                const float4* other = reinterpret_cast<const float4*>(buf + h * (kBN * 4));
 #pragma unroll
                 for (int i = 0; i < kBN / 4; ++i) {
-                    const float4 o = other[i];
+                    const float4 o = other[i ^ (h & 7)];
                     s[4 * i] += o.x;
                     s[4 * i + 1] += o.y;
                     s[4 * i + 2] += o.z;
                     s[4 * i + 3] += o.w;
                 }
-                tc::named_barrier(1, 128);  // every row of the buffer is read before P overwrites it
-                // online softmax over the tile (base 2)
+                if (!buf_sync.sync(abort_flag)) {  // the buffer is fully read before P overwrites it
+                    stop = true;
+                    break;
+                }
                 float mt = -INFINITY;
 #pragma unroll
                 for (int i = 0; i < kBN; ++i) {
-                    const bool ok = ((i < 32 ? va >> i : vb >> (i - 32)) & 1u) != 0;
-                    s[i] = ok ? s[i] * scale_log2 : -INFINITY;
+                    s[i] = ((valid >> i) & 1ull) ? s[i] * scale_log2 : -INFINITY;
                     mt = fmaxf(mt, s[i]);
                 }
+                // lazy rescale: a head whose running max grew by more than 2^8 rescales O and l
+                // to the new max (the decision is per head; the TMEM accesses are warp-wide)
+                float m_new = m_used;
                 if (mt != -INFINITY) {
-                    if (m_used == -INFINITY) {
-                        m_used = mt;
-                    } else if (mt > m_used + kRescaleLog2) {
-                        // O of this head is final up to P.V(n-1) (receiving tile n implies it)
-                        const float alpha = exp2f(m_used - mt);
-                        m_used = mt;
-                        l *= alpha;
-#pragma unroll 1
-                        for (int c = 0; c < 256; c += 32) {
-                            float o[32];
-                            tc::tmem_ld32(tmem_base + lane_off + kTmemO + c, o);
-                            tc::tmem_ld_wait();
-#pragma unroll
-                            for (int i = 0; i < 32; ++i) o[i] *= alpha;
-                            tc::tmem_st32(tmem_base + lane_off + kTmemO + c, o);
-                        }
-                        tc::tmem_st_wait();
-                    }
+                    if (m_used == -INFINITY) m_used = m_new = mt;
+                    else if (mt > m_used + kRescaleLog2) m_new = mt;
                 }
-                float psum = 0.f;
+                if (__any_sync(0xffffffffu, m_new != m_used)) {
+                    // O holds P.V up to tile n-1 once that P.V completed
+                    if (!tc::mbar_wait(&bars->pv_done, (n - 1) & 1, abort_flag)) {
+                        stop = true;
+                        break;
+                    }
+                    tc::tc_fence_after();
+                    const float alpha = m_new != m_used ? tc::fast_exp2(m_used - m_new) : 1.f;
+                    m_used = m_new;
+                    l *= alpha;
+#pragma unroll 1
+                    for (int c = 0; c < 256; c += 32) {
+                        float o[32];
+                        tc::tmem_ld32(tmem_base + lane_off + kTmemO + c, o);
+                        tc::tmem_ld_wait();
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) o[i] *= alpha;
+                        tc::tmem_st32(tmem_base + lane_off + kTmemO + c, o);
+                    }
+                    tc::tmem_st_wait();
+                }
+                float ps[4] = {0.f, 0.f, 0.f, 0.f};
                 uint32_t pk[kBN / 2];
 #pragma unroll
                 for (int i = 0; i < kBN; i += 2) {
-                    const float p0 = s[i] == -INFINITY ? 0.f : exp2f(s[i] - m_used);
-                    const float p1 = s[i + 1] == -INFINITY ? 0.f : exp2f(s[i + 1] - m_used);
-                    psum += p0;
-                    psum += p1;
+                    const float p0 = s[i] == -INFINITY ? 0.f : tc::fast_exp2(s[i] - m_used);
+                    const float p1 = s[i + 1] == -INFINITY ? 0.f : tc::fast_exp2(s[i + 1] - m_used);
+                    ps[(i >> 1) & 3] += p0 + p1;
                     const __nv_bfloat162 b2 = __floats2bfloat162_rn(p0, p1);
                     pk[i / 2] = *reinterpret_cast<const uint32_t*>(&b2);
                 }
-                l += psum;
-                // P row h, K-major 128-byte swizzle: 16-byte chunk c at (c ^ (h & 7))
-                uint8_t* prow = recv + h * 128;
+                l += (ps[0] + ps[1]) + (ps[2] + ps[3]);
+                uint8_t* prow = buf + h * 128;   // P: K-major, 128-byte swizzle
 #pragma unroll
                 for (int c = 0; c < 8; ++c)
                     *reinterpret_cast<uint4*>(prow + ((c ^ (h & 7)) * 16)) =
@@ -392,11 +487,33 @@ sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q_lat, const __grid_
                 tc::tc_fence_before();
                 __syncwarp();
                 if (lane == 0) tc::mbar_arrive(&bars->p_full);
+                // ---- send S(n+1): next tile of this row, or the first tile of the next row
+                if (j + 1 < ntiles) {
+                    if (!send_tile(n + 1)) {
+                        stop = true;
+                        break;
+                    }
+                } else {
+                    t_next = next_row(t + n_clusters, ntiles_next, r_next);
+                    if (t_next >= 0) {
+                        if (!tc::mbar_wait(&bars->q_empty, rows_done & 1, abort_flag)) {
+                            stop = true;
+                            break;
+                        }
+                        tc::tc_fence_after();
+                        load_q(t_next);
+                        if (!send_tile(n + 1)) {
+                            stop = true;
+                            break;
+                        }
+                    }
+                }
             }
             if (stop) break;
-            // row epilogue: O / l -> bf16 -> global
+            // ---- row epilogue: O / l -> bf16 -> global
             if (!tc::mbar_wait(&bars->o_ready, rows_done & 1, abort_flag)) break;
             tc::tc_fence_after();
+            __nv_bfloat16* orow = out + ((int64_t)t * kH + h) * kDv + 256 * rank;
             const float inv_l = l > 0.f ? 1.f / l : 0.f;
 #pragma unroll 1
             for (int c = 0; c < 256; c += 32) {
@@ -407,9 +524,9 @@ sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q_lat, const __grid_
                 for (int i = 0; i < 32; i += 8) {
                     uint32_t w4[4];
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        const __nv_bfloat162 b2 = __floats2bfloat162_rn(o[i + 2 * q] * inv_l, o[i + 2 * q + 1] * inv_l);
-                        w4[q] = *reinterpret_cast<const uint32_t*>(&b2);
+                    for (int qq = 0; qq < 4; ++qq) {
+                        const __nv_bfloat162 b2 = __floats2bfloat162_rn(o[i + 2 * qq] * inv_l, o[i + 2 * qq + 1] * inv_l);
+                        w4[qq] = *reinterpret_cast<const uint32_t*>(&b2);
                     }
                     *reinterpret_cast<uint4*>(orow + c + i) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
                 }
@@ -420,15 +537,21 @@ sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q_lat, const __grid_
             if (lse != nullptr && rank == 0)
                 lse[(int64_t)t * kH + h] = l > 0.f ? (m_used + log2f(l)) * 0.69314718055994531f : -INFINITY;
             ++rows_done;
+            t = t_next;
+            ntiles = ntiles_next;
+            r = r_next;
         }
-        // the peer's last P.V commit arrives here; take it before leaving
-        if (!stop && n > 0) tc::mbar_wait(&bars->peer_free, (n - 1) & 1, abort_flag);
+        // the peer's last two P.V commits arrive here; take them before leaving
+        if (!stop) {
+            if (n >= 2) tc::mbar_wait(&bars->peer_free[(n - 2) & 1], ((n - 2) >> 1) & 1, abort_flag);
+            if (n >= 1) tc::mbar_wait(&bars->peer_free[(n - 1) & 1], ((n - 1) >> 1) & 1, abort_flag);
+        }
     }
     __syncwarp();
     tc::tc_fence_before();
     __syncthreads();
     tc::cluster_sync_all();
-    if (warp == 1) {
+    if (warp == 4) {
         tc::tc_fence_after();
         tc::tmem_dealloc(tmem_base, kTmemCols);
     }
@@ -462,25 +585,14 @@ size_t sparse_mla_tc_workspace(int32_t, int32_t) { return 0; }
 
 cudaError_t launch_sparse_mla_tc(const SparseMlaArgs& a, cudaStream_t st) {
     if (a.seq.T_q == 0) return cudaSuccess;
-    const uint64_t slots = (uint64_t)a.seq.num_pages * a.seq.page_size;
-    const uint64_t qrows = (uint64_t)a.seq.T_q * kH;
-    CUtensorMap tql, tqr, tkl, tkr;
-    bool ok = make_tensor_map_2d(&tql, a.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, qrows, kDqk, kDqk * 2,
-                                 64, kH, CU_TENSOR_MAP_SWIZZLE_128B) &&
-              make_tensor_map_2d(&tqr, a.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, qrows, kDqk, kDqk * 2,
-                                 32, kH, CU_TENSOR_MAP_SWIZZLE_64B) &&
-              make_tensor_map_2d(&tkl, a.kv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, slots, kDqk, kDqk * 2,
-                                 64, 1, CU_TENSOR_MAP_SWIZZLE_128B) &&
-              make_tensor_map_2d(&tkr, a.kv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, slots, kDqk, kDqk * 2,
-                                 32, 1, CU_TENSOR_MAP_SWIZZLE_64B);
-    if (!ok) return cudaErrorInvalidValue;
     cudaError_t e = cudaFuncSetAttribute(sparse_mla_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)kSmem);
     if (e != cudaSuccess) return e;
     const int clusters = std::max(1, std::min(a.seq.T_q, num_sms() / 2));
     const float scale_log2 = a.softmax_scale * 1.4426950408889634f;
     sparse_mla_tc_kernel<<<2 * clusters, kThreads, kSmem, st>>>(
-        tql, tqr, tkl, tkr, a.seq, a.idx, a.K, scale_log2, reinterpret_cast<__nv_bfloat16*>(a.out), a.lse);
+        a.seq, reinterpret_cast<const __nv_bfloat16*>(a.q), reinterpret_cast<const __nv_bfloat16*>(a.kv),
+        a.idx, a.K, scale_log2, reinterpret_cast<__nv_bfloat16*>(a.out), a.lse);
     count_launch();
     return cudaGetLastError();
 }

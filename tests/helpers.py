@@ -12,8 +12,21 @@ from sparse_index_attention_b200 import workloads
 
 
 def paged_seq(wl: workloads.Workload, status=None) -> hsa.PagedSeq:
+    """Descriptor of the workload's rows.  Unless a status tensor is given, a fresh one is
+    attached so that check_status() can assert that no device-side check fired."""
+    if status is None and wl.seq_lens.is_cuda:
+        status = torch.zeros(1, dtype=torch.int32, device=wl.seq_lens.device)
     return hsa.PagedSeq(wl.seq_lens, wl.block_table, wl.page_size, wl.num_pages, wl.q_seq, wl.q_pos,
                         max_seq_len=int(wl.seq_lens.max().item()), q_run=wl.q_run, status=status)
+
+
+def check_status(seq: hsa.PagedSeq):
+    """No device-side check (bad page / position / grouping, or a pipeline wait that gave up)
+    fired during the calls made with this descriptor."""
+    if seq.status is not None:
+        torch.cuda.synchronize()
+        v = int(seq.status.item())
+        assert v == 0, f"device status bits {v:#x}"
 
 
 def oracle_paging(wl: workloads.Workload, rows=None) -> oracle.Paging:

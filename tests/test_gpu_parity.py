@@ -13,8 +13,8 @@ import oracle
 import sparse_index_attention_b200 as hsa
 from sparse_index_attention_b200 import workloads
 
-from helpers import (GpuCaches, OracleCaches, attn_close, index_tolerance_ok, oracle_paging,
-                     paged_seq, stable_topk_reference)
+from helpers import (GpuCaches, OracleCaches, attn_close, check_status, index_tolerance_ok,
+                     oracle_paging, paged_seq, stable_topk_reference)
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -24,7 +24,7 @@ def _index_vs_oracle(wl, rows=None):
     gc = GpuCaches(wl)
     seq = paged_seq(wl)
     sc = hsa.hsa_index_score(seq, wl.q_I, wl.w, gc.k, gc.k_scale)
-    torch.cuda.synchronize()
+    check_status(seq)
     rows = list(range(wl.T_q)) if rows is None else rows
     oc = OracleCaches(wl, need_kv=False)
     pg = oracle_paging(wl, rows)
@@ -125,7 +125,7 @@ def _attn_vs_oracle(wl, tol, idx=None):
     idx_d = idx.to(DEV)
     out, lse = hsa.hsa_sparse_mla_attn(seq, wl.q, gc.kv, idx_d, wl.D_v, wl.softmax_scale,
                                        kv_scale=gc.kv_scale, kv_rope=gc.kv_rope)
-    torch.cuda.synchronize()
+    check_status(seq)
     oc = OracleCaches(wl)
     ref, rlse = oracle.sparse_mla(oracle_paging(wl), wl.q.cpu(), oc.kv, idx, wl.D_v, wl.softmax_scale)
     ok, worst = attn_close(out.float().cpu().numpy(), ref, tol)
@@ -220,3 +220,16 @@ def test_device_checks_flag_instead_of_faulting():
     hsa.hsa_sparse_mla_attn(paged_seq(wl, status), wl.q, wl.kv, idx, wl.D_v, wl.softmax_scale)
     torch.cuda.synchronize()
     assert int(status.item()) & hsa.HSA_DEV_BAD_POS
+
+
+def test_sparse_mla_repeatable_and_clean():
+    """Many launches of the same call give bitwise-identical results and never trip a device-side
+    check: pipeline races between the two CTAs of a cluster would show up here first."""
+    wl = workloads.make("decode_bf16", DEV, B=24, L_min=2100, L_max=6000)
+    idx = workloads.random_selection(wl.q_pos, wl.K, seed=77).to(DEV)
+    seq = paged_seq(wl)
+    ref, ref_lse = hsa.hsa_sparse_mla_attn(seq, wl.q, wl.kv, idx, wl.D_v, wl.softmax_scale)
+    for _ in range(30):
+        out, lse = hsa.hsa_sparse_mla_attn(seq, wl.q, wl.kv, idx, wl.D_v, wl.softmax_scale)
+        assert torch.equal(out, ref) and torch.equal(lse, ref_lse)
+    check_status(seq)

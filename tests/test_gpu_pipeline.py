@@ -18,8 +18,8 @@ import oracle
 import sparse_index_attention_b200 as hsa
 from sparse_index_attention_b200 import workloads
 
-from helpers import (GpuCaches, OracleCaches, attn_close, index_tolerance_ok, oracle_paging,
-                     paged_seq, stable_topk_reference)
+from helpers import (GpuCaches, OracleCaches, attn_close, check_status, index_tolerance_ok,
+                     oracle_paging, paged_seq, stable_topk_reference)
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -32,7 +32,7 @@ def run_fused(wl, gc, aux=False):
     out, lse, idx, sc = hsa.hsa_fused_decode(seq, wl.q_I, wl.w, gc.k, gc.k_scale, wl.q, gc.kv,
                                              gc.kv_scale, gc.kv_rope, wl.K, wl.D_v,
                                              wl.softmax_scale, aux_stream=aux_stream)
-    torch.cuda.synchronize()
+    check_status(seq)
     return out, lse, idx, sc
 
 
