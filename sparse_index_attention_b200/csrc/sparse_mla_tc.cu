@@ -58,7 +58,6 @@ constexpr int kDv = 512;
 constexpr int kBN = 64;          // gathered rows per tile
 constexpr int kStages = 4;
 constexpr int kThreads = 288;
-constexpr int kCopyDepth = 2;    // cp.async groups in flight per producer thread beyond the newest
 constexpr int kSlotWin = 2048;   // selected entries whose slots are resolved at once
 
 constexpr int kQRopeBytes = kH * 64;               // 128 heads x 32 dims bf16, SW64
@@ -144,7 +143,8 @@ sparse_mla_tc_kernel(SeqView v,
         tc::mbar_init(&bars->q_full, 4);
         tc::mbar_init(&bars->q_empty, 1);
         for (int i = 0; i < kStages; ++i) {
-            tc::mbar_init(&bars->kv_full[i], 128);   // every producer thread, after its copies landed
+            // 128 producer threads when their copies land + 4 warps publishing their mask bits
+            tc::mbar_init(&bars->kv_full[i], 128 + 4);
             tc::mbar_init(&bars->kv_empty[i], 1);
         }
         for (int i = 0; i < 2; ++i) {
@@ -177,14 +177,8 @@ sparse_mla_tc_kernel(SeqView v,
         const uint8_t* kv_bytes = reinterpret_cast<const uint8_t*>(kv);
         int32_t* my_slots = slots + warp * (kSlotWin / 4);   // this warp's 16 rows of 32 tiles
         uint16_t* masks16 = reinterpret_cast<uint16_t*>(const_cast<uint64_t*>(masks));
-        uint32_t n = 0, landed = 0;
+        uint32_t n = 0;
         bool stop = false;
-        // the copies of tile `landed` are complete for this thread: publish them
-        auto publish = [&]() {
-            tc::fence_async_smem();   // generic-proxy writes -> visible to the tensor core
-            tc::mbar_arrive(&bars->kv_full[landed % kStages]);
-            ++landed;
-        };
         for (int t = cluster; t < v.T_q && !stop; t += n_clusters) {
             RowInfo r;
             const int ntiles = row_tiles(v, idx, K, t, lane, r);
@@ -239,18 +233,17 @@ sparse_mla_tc_kernel(SeqView v,
                     uint8_t* dst = sbase + 4 * kKvBlk + row * 64 + ((cc ^ ((row >> 1) & 3)) * 16);
                     tc::cp_async16(dst, src, sl < 0 ? 0u : 16u);
                 }
+                // the stage is complete when every thread's copies have landed (hardware arrive)
+                // and every warp has published its rows' validity bits
+                tc::cp_async_arrive_noinc(&bars->kv_full[st]);
                 const uint32_t vm = __ballot_sync(0xffffffffu, lane < 16 && ts[lane & 15] >= 0) & 0xFFFFu;
-                if (lane == 0) masks16[st * 4 + warp] = (uint16_t)vm;
-                tc::cp_async_commit();
-                if (n >= (uint32_t)kCopyDepth) {
-                    tc::cp_async_wait<kCopyDepth>();
-                    publish();
+                if (lane == 0) {
+                    masks16[st * 4 + warp] = (uint16_t)vm;
+                    tc::mbar_arrive(&bars->kv_full[st]);
                 }
             }
         }
-        // drain: the last tiles' copies
-        tc::cp_async_wait<0>();
-        while (!stop && landed < n) publish();
+        tc::cp_async_wait<0>();   // nothing of this thread still in flight when the CTA leaves
     } else if (warp == 4) {
         // ---------------------------------------------------------------- MMA issuer
         const uint32_t qr_addr = tc::smem_u32(q_rope);
@@ -288,6 +281,7 @@ sparse_mla_tc_kernel(SeqView v,
                     stop = true;
                     break;
                 }
+                tc::fence_async_smem();   // the gathered tile (generic-proxy copies) -> tensor core
                 tc::tc_fence_after();
                 if (lane == 0) {
                     const uint32_t kv_addr = tc::smem_u32(stages + st * kStageBytes);
