@@ -291,3 +291,53 @@ def hsa_version() -> int:
 def hsa_launch_count() -> int:
     """Kernels launched by the library from this host thread so far."""
     return int(lib().hsa_launch_count())
+
+
+def hsa_prefill_chunked(seq: PagedSeq, q_I, w, k_cache, k_scale, q, kv, kv_scale, kv_rope, K: int,
+                        D_v: int, softmax_scale: float, chunks, out=None, lse=True, idx=None,
+                        streams=None):
+    """Causal prefill over query-row windows issued in the order of `chunks` [(r0, r1), ...].
+
+    Consecutive chunks form pairs that run concurrently, one on each of two streams; with the
+    zigzag order (chunk i paired with chunk 2N-1-i, "Efficient Inference Deployment and
+    Optimization for Hybrid Attention LLMs", 5.2) every pair carries the same causal index work.
+    Each chunk is hsa_index_score -> hsa_topk -> hsa_sparse_mla_attn on its rows, so its outputs
+    land at the rows' own offsets and no restore step exists; the issue order cannot change any
+    result.  This function only slices tensors and issues C-ABI calls.  Returns (out, lse, idx).
+    """
+    T_q = q.shape[0]
+    dev = q.device
+    if out is None:
+        out = torch.empty((T_q, q.shape[1], D_v), dtype=q.dtype, device=dev)
+    if lse is True:
+        lse = torch.empty((T_q, q.shape[1]), dtype=torch.float32, device=dev)
+    elif lse is False:
+        lse = None
+    if idx is None:
+        idx = torch.empty((T_q, K), dtype=torch.int32, device=dev)
+    main = torch.cuda.current_stream()
+    if streams is None:
+        streams = (torch.cuda.Stream(), torch.cuda.Stream())
+    start = torch.cuda.Event()
+    start.record(main)
+    rows_max = max(r1 - r0 for r0, r1 in chunks)
+    bufs = []
+    for s in streams:
+        s.wait_event(start)
+        bufs.append(torch.empty((rows_max, seq.max_seq_len), dtype=torch.float32, device=dev))
+    for i, (r0, r1) in enumerate(chunks):
+        s = streams[i % 2]
+        part = seq.rows(r0, r1, q_run=min(seq.q_run, r1 - r0))
+        sc = bufs[i % 2][:r1 - r0]
+        hsa_index_score(part, q_I[r0:r1], w[r0:r1], k_cache, k_scale, scores=sc, stream=s)
+        hsa_topk(part, sc, K, idx=idx[r0:r1], stream=s)
+        hsa_sparse_mla_attn(part, q[r0:r1], kv, idx[r0:r1], D_v, softmax_scale, kv_scale=kv_scale,
+                            kv_rope=kv_rope, out=out[r0:r1], lse=None if lse is None else lse[r0:r1],
+                            stream=s)
+    for s in streams:
+        done = torch.cuda.Event()
+        done.record(s)
+        main.wait_event(done)
+    for b, s in zip(bufs, streams):
+        b.record_stream(s)
+    return out, lse, idx

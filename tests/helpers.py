@@ -101,3 +101,34 @@ def stable_topk_reference(scores: torch.Tensor, q_pos: torch.Tensor, K: int) -> 
         order = torch.sort(row, descending=True, stable=True).indices[:K]
         out[t] = order.sort().values.to(torch.int32)
     return out
+
+
+def compact_workload(wl: workloads.Workload, rows) -> workloads.Workload:
+    """A copy of the workload reduced to the given query rows and the pages of their sequences
+    (pages renumbered consecutively, contents copied).  Rows' results are unchanged: every cache
+    row is read through the block table and FP8 quantization is per row."""
+    import dataclasses
+    import math
+    rows = list(rows)
+    q_seq = wl.q_seq[rows].tolist()
+    seqs = sorted(set(q_seq))
+    pages_of = []
+    for b in seqs:
+        n = math.ceil(int(wl.seq_lens[b]) / wl.page_size)
+        pages_of.append(wl.block_table[b, :n].long())
+    old = torch.cat(pages_of)
+    P = old.numel()
+    maxp = max(p.numel() for p in pages_of)
+    bt = torch.zeros((len(seqs), maxp), dtype=torch.int32)
+    off = 0
+    for i, p in enumerate(pages_of):
+        bt[i, :p.numel()] = torch.arange(off, off + p.numel(), dtype=torch.int32)
+        off += p.numel()
+    def pages(x):
+        return x.view(wl.num_pages, wl.page_size, -1)[old.to(x.device)].reshape(P * wl.page_size, -1).cpu()
+    remap = {b: i for i, b in enumerate(seqs)}
+    return dataclasses.replace(
+        wl, B=len(seqs), seq_lens=wl.seq_lens[seqs].cpu(), block_table=bt, num_pages=P,
+        T_q=len(rows), q_seq=torch.tensor([remap[b] for b in q_seq], dtype=torch.int32),
+        q_pos=wl.q_pos[rows].cpu(), q_I=wl.q_I[rows].cpu(), w=wl.w[rows].cpu(), k_I=pages(wl.k_I),
+        q=wl.q[rows].cpu(), kv=pages(wl.kv), q_run=1)
