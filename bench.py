@@ -298,12 +298,15 @@ def run_ours(args, rank, world, local_rank):
     dom = max(names, key=lambda n: stage_ms[n])
     achieved = work[dom]["bytes"] / (stage_ms[dom] * 1e-3) / 1e9
     traffic = None
-    tpath = os.path.join(ROOT, "profiles", "traffic.json")
-    if os.path.exists(tpath):
-        try:
-            traffic = json.load(open(tpath)).get(dom)
-        except Exception:
-            traffic = None
+    tpath = os.path.join(ROOT, "profiles", "dram_traffic_decode_bf16.json")
+    try:
+        import hashlib
+        rec = json.load(open(tpath))["kernels"][dom]
+        cur = hashlib.sha256(open(os.path.join(ROOT, rec["source"]), "rb").read()).hexdigest()[:16]
+        if cur == rec["source_sha256_16"]:       # counters taken on this very kernel source
+            traffic = rec["traffic_bytes"]
+    except Exception:
+        traffic = None
     roofline = {"kernel": dom, "bound": "hbm", "achieved": round(achieved, 1),
                 "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
                 "traffic": traffic, "peak_source": f"{peaks['source']} (MEASURED_PEAKS.json hbm_gbs)"
