@@ -29,9 +29,9 @@
 // The latent part of Q lives in TMEM (A operand of Q.KV^T), next to O (256 columns) and the two
 // partial-S buffers (2 x 64 columns).
 //
-// Pipeline per tile n: the softmax warps send their partial S(n+1) to the peer before they
-// compute softmax(n), so the distributed-shared-memory hop overlaps the exponentials, and the
-// tensor core runs Q.KV^T(n+1) and P.V(n-1) while softmax(n) runs.  The peer may overwrite an
+// Pipeline per tile n: sender warps push partial S(n) to the peer as soon as Q.KV^T(n) is done,
+// independent of the softmax, so the distributed-shared-memory hop overlaps the softmax of the
+// previous tile, and the tensor core runs Q.KV^T(n+1) and P.V(n-1) while softmax(n) runs.  The peer may overwrite an
 // exchange buffer only after this CTA's P.V of the tile that used it (MMA commit multicast to the
 // peer), which is also what makes receiving tile n prove that P.V(n-2) has finished.
 //
@@ -40,9 +40,9 @@
 // three quarters of the kernel.  Plain 16-byte asynchronous copies from 128 threads keep far more
 // bytes in flight.)
 //
-// Warp roles: 0-3 producers (slot window + gather; warp w owns rows 16w..16w+15 of every tile,
-// warp 0 also loads the rope part of Q by TMA), 4 MMA issuer, 5-8 softmax / exchange / epilogue
-// (thread h owns head h = TMEM lane h).  Persistent: each cluster loops over query rows.
+// Warp roles: 0-3 producers (slot window + gather; warp w owns rows 16w..16w+15 of every tile),
+// 4 MMA issuer, 5-12 softmax / epilogue (two threads per head h = TMEM lane h, 32 columns each),
+// 13-16 senders (partial S to the peer).  Persistent: each cluster loops over query rows.
 #include <algorithm>
 
 #include "kernels.h"
@@ -57,8 +57,8 @@ constexpr int kDqk = 576;
 constexpr int kDv = 512;
 constexpr int kBN = 64;          // gathered rows per tile
 constexpr int kStages = 4;
-constexpr int kThreads = 288;
-constexpr int kSlotWin = 2048;   // selected entries whose slots are resolved at once
+constexpr int kThreads = 544;   // 4 producer, 1 MMA, 8 softmax, 4 sender warps
+constexpr int kSlotWin = 1024;   // selected entries whose slots are resolved at once (16 tiles)
 
 constexpr int kQRopeBytes = kH * 64;               // 128 heads x 32 dims bf16, SW64
 constexpr int kKvBlk = kBN * 128;                  // 64 rows x 64 dims
@@ -69,7 +69,9 @@ constexpr int kOffStages = kQRopeBytes;
 constexpr int kOffRecv = kOffStages + kStages * kStageBytes;
 constexpr int kOffSlots = kOffRecv + 2 * kRecvBytes;
 constexpr int kOffMasks = kOffSlots + 4 * kSlotWin;
-constexpr int kOffBars = kOffMasks + 8 * kStages;
+constexpr int kOffXmax = kOffMasks + 8 * kStages;              // [2 tiles][2 halves][128] fp32
+constexpr int kOffXsum = kOffXmax + 4 * 512;                   // [2 halves][128] fp32
+constexpr int kOffBars = kOffXsum + 4 * 256;
 constexpr int kKvRowBytes = kDqk * 2;   // 1152
 constexpr size_t kSmem = 1024 + kOffBars + 256;
 static_assert(kSmem <= 232448, "shared memory budget");
@@ -89,12 +91,13 @@ struct Bars {
     uint64_t q_empty;     // last Q.KV^T of the row done
     uint64_t kv_full[kStages], kv_empty[kStages];
     uint64_t s_full[2], s_empty[2];
+    uint64_t s_sent[2];     // the senders have read partial S of the buffer (P may overwrite it)
     uint64_t p_full;
     uint64_t pv_done;     // this CTA's P.V of a tile completed
     uint64_t peer_free[2];  // the peer's P.V of a tile of parity b completed (its buffer b is free)
     uint64_t recv_full[2];
     uint64_t o_ready, o_free;
-    uint64_t buf_read;    // the four softmax warps finished reading an exchange buffer
+    uint64_t buf_read;    // the eight softmax warps finished reading an exchange buffer
     uint32_t tmem;
     int abort;
 };
@@ -130,6 +133,8 @@ sparse_mla_tc_kernel(SeqView v,
     uint8_t* recv = base + kOffRecv;
     int32_t* slots = reinterpret_cast<int32_t*>(base + kOffSlots);
     volatile uint64_t* masks = reinterpret_cast<volatile uint64_t*>(base + kOffMasks);
+    float* xmax = reinterpret_cast<float*>(base + kOffXmax);
+    float* xsum = reinterpret_cast<float*>(base + kOffXsum);
     Bars* bars = reinterpret_cast<Bars*>(base + kOffBars);
     volatile int* abort_flag = &bars->abort;
 
@@ -140,7 +145,7 @@ sparse_mla_tc_kernel(SeqView v,
     const int n_clusters = gridDim.x >> 1;
 
     if (tid == 0) {
-        tc::mbar_init(&bars->q_full, 4);
+        tc::mbar_init(&bars->q_full, 8);
         tc::mbar_init(&bars->q_empty, 1);
         for (int i = 0; i < kStages; ++i) {
             // 128 producer threads when their copies land + 4 warps publishing their mask bits
@@ -149,16 +154,17 @@ sparse_mla_tc_kernel(SeqView v,
         }
         for (int i = 0; i < 2; ++i) {
             tc::mbar_init(&bars->s_full[i], 1);
-            tc::mbar_init(&bars->s_empty[i], 4);
+            tc::mbar_init(&bars->s_empty[i], 1);    // P.V of the tile whose P sits in the buffer
+            tc::mbar_init(&bars->s_sent[i], 4);     // 4 sender warps
             tc::mbar_init(&bars->recv_full[i], 1);
         }
-        tc::mbar_init(&bars->p_full, 4);
+        tc::mbar_init(&bars->p_full, 8);
         tc::mbar_init(&bars->pv_done, 1);
         tc::mbar_init(&bars->peer_free[0], 1);
         tc::mbar_init(&bars->peer_free[1], 1);
         tc::mbar_init(&bars->o_ready, 1);
-        tc::mbar_init(&bars->o_free, 4);
-        tc::mbar_init(&bars->buf_read, 4);
+        tc::mbar_init(&bars->o_free, 8);
+        tc::mbar_init(&bars->buf_read, 8);
         bars->abort = 0;
         tc::fence_barrier_init();
     }
@@ -175,7 +181,7 @@ sparse_mla_tc_kernel(SeqView v,
     if (warp < 4) {
         // ---------------------------------------------------------------- producers (gather)
         const uint8_t* kv_bytes = reinterpret_cast<const uint8_t*>(kv);
-        int32_t* my_slots = slots + warp * (kSlotWin / 4);   // this warp's 16 rows of 32 tiles
+        int32_t* my_slots = slots + warp * (kSlotWin / 4);   // this warp's 16 rows of 16 tiles
         uint16_t* masks16 = reinterpret_cast<uint16_t*>(const_cast<uint64_t*>(masks));
         uint32_t n = 0;
         bool stop = false;
@@ -254,14 +260,15 @@ sparse_mla_tc_kernel(SeqView v,
             if (first && !tc::mbar_wait(&bars->o_free, (rows_done & 1) ^ 1, abort_flag)) return false;
             tc::tc_fence_after();
             if (lane == 0) {
-                const uint32_t p_addr = tc::smem_u32(recv + (m & 1) * kRecvBytes);
+                const uint32_t p_tmem = tmem_base + kTmemS + (m & 1) * kBN;   // P (bf16 pairs) over S
                 const uint32_t v_addr = tc::smem_u32(stages + (m % kStages) * kStageBytes);
 #pragma unroll
                 for (int kk = 0; kk < kBN / 16; ++kk)
-                    tc::mma_bf16(tmem_base + kTmemO, tc::sw128_desc(p_addr + kk * 32, 16, 1024),
-                                 tc::sw128_desc(v_addr + kk * 2048, kKvBlk, 1024), kIdescPV,
-                                 (first && kk == 0) ? 0u : 1u);
+                    tc::mma_bf16_tmem_a(tmem_base + kTmemO, p_tmem + 8 * kk,
+                                        tc::sw128_desc(v_addr + kk * 2048, kKvBlk, 1024), kIdescPV,
+                                        (first && kk == 0) ? 0u : 1u);
                 tc::mma_commit(&bars->kv_empty[m % kStages]);
+                tc::mma_commit(&bars->s_empty[m & 1]);
                 tc::mma_commit(&bars->pv_done);
                 tc::mma_commit_multicast(&bars->peer_free[m & 1], (uint16_t)(1u << peer));
             }
@@ -309,15 +316,16 @@ sparse_mla_tc_kernel(SeqView v,
             __syncwarp();
             ++rows_done;
         }
-    } else {
-        // ---------------------------------------------------------------- softmax / exchange
+    } else if (warp < 13) {
+        // ---------------------------------------------------------------- softmax
+        // Two threads per head: warps 5-8 take columns 0..31 of every tile and output dims
+        // 0..127 of this CTA's half, warps 9-12 columns 32..63 and dims 128..255.  They combine
+        // their tile maxima through xmax (double-buffered by tile parity) and their row sums
+        // through xsum at the end of a row.
         const int h = (warp & 3) * 32 + lane;          // head = TMEM lane
+        const int half = (warp - 5) >> 2;              // which 32 columns / 128 output dims
         const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
-        uint32_t peer_recv[2], peer_bar[2];
-        for (int b = 0; b < 2; ++b) {
-            peer_recv[b] = tc::mapa_shared(tc::smem_u32(recv + b * kRecvBytes), peer);
-            peer_bar[b] = tc::mapa_shared(tc::smem_u32(&bars->recv_full[b]), peer);
-        }
+        const uint32_t col = (uint32_t)(32 * half);
         uint32_t n = 0, rows_done = 0;
         bool stop = false;
         tc::WarpSetSync buf_sync{&bars->buf_read, 0};
@@ -328,23 +336,24 @@ sparse_mla_tc_kernel(SeqView v,
             for (int t = t0; t < v.T_q; t += n_clusters) {
                 ntiles = row_tiles(v, idx, K, t, lane, r);
                 if (ntiles > 0) return t;
-                __nv_bfloat16* orow = out + ((int64_t)t * kH + h) * kDv + 256 * rank;
-                for (int c = 0; c < 256; c += 8) *reinterpret_cast<uint4*>(orow + c) = make_uint4(0, 0, 0, 0);
-                if (lse != nullptr && rank == 0) lse[(int64_t)t * kH + h] = -INFINITY;
+                __nv_bfloat16* orow = out + ((int64_t)t * kH + h) * kDv + 256 * rank + 128 * half;
+                for (int c = 0; c < 128; c += 8) *reinterpret_cast<uint4*>(orow + c) = make_uint4(0, 0, 0, 0);
+                if (lse != nullptr && rank == 0 && half == 0) lse[(int64_t)t * kH + h] = -INFINITY;
             }
             return -1;
         };
-        // Q row t: this CTA's 256 latent dims into TMEM (thread h writes lane h) and its 32 rope
-        // dims into shared memory (64-byte swizzle: 16-byte chunk c of row h at c ^ ((h >> 1) & 3))
+        // Q row t: this CTA's 256 latent dims into TMEM (lane h, columns 384.. as bf16 pairs) and
+        // its 32 rope dims into shared memory (64-byte swizzle: chunk c of row h at c ^ ((h>>1)&3));
+        // each of the two threads of a head moves half of it
         auto load_q = [&](int t) {
             const uint4* srcr = reinterpret_cast<const uint4*>(q + ((int64_t)t * kH + h) * kDqk + 512 + 32 * rank);
 #pragma unroll
-            for (int c = 0; c < 4; ++c)
+            for (int c = 2 * half; c < 2 * half + 2; ++c)
                 *reinterpret_cast<uint4*>(q_rope + h * 64 + ((c ^ ((h >> 1) & 3)) * 16)) = __ldg(srcr + c);
             tc::fence_async_smem();
             const uint4* src = reinterpret_cast<const uint4*>(q + ((int64_t)t * kH + h) * kDqk + 256 * rank);
 #pragma unroll 1
-            for (int c = 0; c < 4; ++c) {
+            for (int c = 2 * half; c < 2 * half + 2; ++c) {
                 uint32_t w[32];
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
@@ -361,80 +370,54 @@ sparse_mla_tc_kernel(SeqView v,
             __syncwarp();
             if (lane == 0) tc::mbar_arrive(&bars->q_full);
         };
-        // partial S(m) -> the peer's exchange buffer (m & 1)
-        auto send_tile = [&](uint32_t m) -> bool {
-            const uint32_t b = m & 1;
-            if (!tc::mbar_wait(&bars->s_full[b], (m >> 1) & 1, abort_flag)) return false;
-            tc::tc_fence_after();
-            float s[kBN];
-            tc::tmem_ld32(tmem_base + lane_off + kTmemS + b * kBN, s);
-            tc::tmem_ld32(tmem_base + lane_off + kTmemS + b * kBN + 32, s + 32);
-            tc::tmem_ld_wait();
-            // the peer's P.V(m-2) has released its buffer b.  One barrier per buffer: the peer
-            // cannot complete P.V(m) before it receives this send, so the barrier is never two
-            // phases ahead of this wait (a single barrier for both buffers could be, since the
-            // peer may finish P.V(m-1) first, and a parity wait would then alias).
-            if (m >= 2 && !tc::mbar_wait(&bars->peer_free[b], ((m - 2) >> 1) & 1, abort_flag)) return false;
-            if (tid == 160) tc::mbar_arrive_expect_tx(&bars->recv_full[b], kRecvBytes);
-            const uint32_t dst = peer_recv[b] + h * (kBN * 4);
-#pragma unroll
-            for (int i = 0; i < kBN / 4; ++i)
-                tc::st_async_v4(dst + ((i ^ (h & 7)) * 16), peer_bar[b], __float_as_uint(s[4 * i]),
-                                __float_as_uint(s[4 * i + 1]), __float_as_uint(s[4 * i + 2]),
-                                __float_as_uint(s[4 * i + 3]));
-            return true;
-        };
-
         int ntiles = 0;
         RowInfo r;
         int t = next_row(cluster, ntiles, r);
-        if (t >= 0) {
-            load_q(t);
-            stop = !send_tile(0);
-        }
+        if (t >= 0) load_q(t);
         while (t >= 0 && !stop) {
             float m_used = -INFINITY, l = 0.f;
             int t_next = -1, ntiles_next = 0;
             RowInfo r_next;
             for (int j = 0; j < ntiles; ++j, ++n) {
                 const uint32_t b = n & 1, st = n % kStages;
-                // ---- softmax(n)
+                // ---- softmax(n), columns [col, col + 32)
                 if (!tc::mbar_wait(&bars->kv_full[st], (n / kStages) & 1, abort_flag) ||
                     !tc::mbar_wait_cluster(&bars->recv_full[b], (n >> 1) & 1, abort_flag)) {
                     stop = true;
                     break;
                 }
-                const uint64_t valid = masks[st];
+                const uint32_t valid = (uint32_t)(masks[st] >> col);
                 tc::tc_fence_after();
-                float s[kBN];
-                tc::tmem_ld32(tmem_base + lane_off + kTmemS + b * kBN, s);
-                tc::tmem_ld32(tmem_base + lane_off + kTmemS + b * kBN + 32, s + 32);
+                float s[32];
+                tc::tmem_ld32(tmem_base + lane_off + kTmemS + b * kBN + col, s);
                 tc::tmem_ld_wait();
-                tc::tc_fence_before();
-                __syncwarp();
-                if (lane == 0) tc::mbar_arrive(&bars->s_empty[b]);
-                uint8_t* buf = recv + b * kRecvBytes;
-                const float4* other = reinterpret_cast<const float4*>(buf + h * (kBN * 4));
+                const float4* other = reinterpret_cast<const float4*>(recv + b * kRecvBytes + h * (kBN * 4));
 #pragma unroll
-                for (int i = 0; i < kBN / 4; ++i) {
-                    const float4 o = other[i ^ (h & 7)];
+                for (int i = 0; i < 8; ++i) {
+                    const float4 o = other[(8 * half + i) ^ (h & 7)];
                     s[4 * i] += o.x;
                     s[4 * i + 1] += o.y;
                     s[4 * i + 2] += o.z;
                     s[4 * i + 3] += o.w;
                 }
-                if (!buf_sync.sync(abort_flag)) {  // the buffer is fully read before P overwrites it
+                if (__any_sync(0xffffffffu, valid != 0xffffffffu)) {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        if (!((valid >> i) & 1u)) s[i] = -INFINITY;
+                }
+                float mt = s[0];
+#pragma unroll
+                for (int i = 1; i < 32; ++i) mt = fmaxf(mt, s[i]);
+                mt = mt == -INFINITY ? -INFINITY : mt * scale_log2;   // tile max in base-2 units
+                xmax[(n & 1) * 256 + half * 128 + h] = mt;
+                if (!buf_sync.sync(abort_flag)) {  // both halves' maxima posted
                     stop = true;
                     break;
                 }
-                float mt = -INFINITY;
-#pragma unroll
-                for (int i = 0; i < kBN; ++i) {
-                    s[i] = ((valid >> i) & 1ull) ? s[i] * scale_log2 : -INFINITY;
-                    mt = fmaxf(mt, s[i]);
-                }
+                mt = fmaxf(mt, xmax[(n & 1) * 256 + (half ^ 1) * 128 + h]);
                 // lazy rescale: a head whose running max grew by more than 2^8 rescales O and l
-                // to the new max (the decision is per head; the TMEM accesses are warp-wide)
+                // to the new max (both threads of the head take the same decision; the TMEM
+                // accesses are warp-wide)
                 float m_new = m_used;
                 if (mt != -INFINITY) {
                     if (m_used == -INFINITY) m_used = m_new = mt;
@@ -451,7 +434,7 @@ sparse_mla_tc_kernel(SeqView v,
                     m_used = m_new;
                     l *= alpha;
 #pragma unroll 1
-                    for (int c = 0; c < 256; c += 32) {
+                    for (int c = 128 * half; c < 128 * half + 128; c += 32) {
                         float o[32];
                         tc::tmem_ld32(tmem_base + lane_off + kTmemO + c, o);
                         tc::tmem_ld_wait();
@@ -461,33 +444,34 @@ sparse_mla_tc_kernel(SeqView v,
                     }
                     tc::tmem_st_wait();
                 }
+                // p = 2^(s * scale_log2 - m): one FFMA per element (masked entries are -inf -> 0);
+                // a head with nothing valid so far (m = -inf) contributes zeros
+                const float mneg = m_used == -INFINITY ? 0.f : -m_used;
+                const bool none = m_used == -INFINITY;
                 float ps[4] = {0.f, 0.f, 0.f, 0.f};
-                uint32_t pk[kBN / 2];
+                uint32_t pk[16];
 #pragma unroll
-                for (int i = 0; i < kBN; i += 2) {
-                    const float p0 = s[i] == -INFINITY ? 0.f : tc::fast_exp2(s[i] - m_used);
-                    const float p1 = s[i + 1] == -INFINITY ? 0.f : tc::fast_exp2(s[i + 1] - m_used);
+                for (int i = 0; i < 32; i += 2) {
+                    const float p0 = none ? 0.f : tc::fast_exp2(fmaf(s[i], scale_log2, mneg));
+                    const float p1 = none ? 0.f : tc::fast_exp2(fmaf(s[i + 1], scale_log2, mneg));
                     ps[(i >> 1) & 3] += p0 + p1;
                     const __nv_bfloat162 b2 = __floats2bfloat162_rn(p0, p1);
                     pk[i / 2] = *reinterpret_cast<const uint32_t*>(&b2);
                 }
                 l += (ps[0] + ps[1]) + (ps[2] + ps[3]);
-                uint8_t* prow = buf + h * 128;   // P: K-major, 128-byte swizzle
-#pragma unroll
-                for (int c = 0; c < 8; ++c)
-                    *reinterpret_cast<uint4*>(prow + ((c ^ (h & 7)) * 16)) =
-                        make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-                tc::fence_async_smem();
+                // P over this thread's 32 columns of the S buffer: rows 32*half.. -> 16 columns of
+                // bf16 pairs; the senders must have read partial S first
+                if (!tc::mbar_wait(&bars->s_sent[b], (n >> 1) & 1, abort_flag)) {
+                    stop = true;
+                    break;
+                }
+                tc::tmem_st16_u(tmem_base + lane_off + kTmemS + b * kBN + 16 * half, pk);
+                tc::tmem_st_wait();
                 tc::tc_fence_before();
                 __syncwarp();
                 if (lane == 0) tc::mbar_arrive(&bars->p_full);
-                // ---- send S(n+1): next tile of this row, or the first tile of the next row
-                if (j + 1 < ntiles) {
-                    if (!send_tile(n + 1)) {
-                        stop = true;
-                        break;
-                    }
-                } else {
+                // ---- last tile of the row: put the next row's Q in place
+                if (j + 1 == ntiles) {
                     t_next = next_row(t + n_clusters, ntiles_next, r_next);
                     if (t_next >= 0) {
                         if (!tc::mbar_wait(&bars->q_empty, rows_done & 1, abort_flag)) {
@@ -496,23 +480,21 @@ sparse_mla_tc_kernel(SeqView v,
                         }
                         tc::tc_fence_after();
                         load_q(t_next);
-                        if (!send_tile(n + 1)) {
-                            stop = true;
-                            break;
-                        }
                     }
                 }
             }
             if (stop) break;
-            // ---- row epilogue: O / l -> bf16 -> global
-            if (!tc::mbar_wait(&bars->o_ready, rows_done & 1, abort_flag)) break;
+            // ---- row epilogue: O / l -> bf16 -> global (this thread: 128 of the 256 dims)
+            xsum[half * 128 + h] = l;
+            if (!tc::mbar_wait(&bars->o_ready, rows_done & 1, abort_flag) || !buf_sync.sync(abort_flag)) break;
             tc::tc_fence_after();
-            __nv_bfloat16* orow = out + ((int64_t)t * kH + h) * kDv + 256 * rank;
-            const float inv_l = l > 0.f ? 1.f / l : 0.f;
+            const float l_all = l + xsum[(half ^ 1) * 128 + h];
+            __nv_bfloat16* orow = out + ((int64_t)t * kH + h) * kDv + 256 * rank + 128 * half;
+            const float inv_l = l_all > 0.f ? 1.f / l_all : 0.f;
 #pragma unroll 1
-            for (int c = 0; c < 256; c += 32) {
+            for (int c = 0; c < 128; c += 32) {
                 float o[32];
-                tc::tmem_ld32(tmem_base + lane_off + kTmemO + c, o);
+                tc::tmem_ld32(tmem_base + lane_off + kTmemO + 128 * half + c, o);
                 tc::tmem_ld_wait();
 #pragma unroll
                 for (int i = 0; i < 32; i += 8) {
@@ -528,17 +510,66 @@ sparse_mla_tc_kernel(SeqView v,
             tc::tc_fence_before();
             __syncwarp();
             if (lane == 0) tc::mbar_arrive(&bars->o_free);
-            if (lse != nullptr && rank == 0)
-                lse[(int64_t)t * kH + h] = l > 0.f ? (m_used + log2f(l)) * 0.69314718055994531f : -INFINITY;
+            if (lse != nullptr && rank == 0 && half == 0)
+                lse[(int64_t)t * kH + h] = l_all > 0.f ? (m_used + log2f(l_all)) * 0.69314718055994531f : -INFINITY;
             ++rows_done;
             t = t_next;
             ntiles = ntiles_next;
             r = r_next;
         }
+    } else {
+        // ---------------------------------------------------------------- senders
+        // Warps 13-16 (one per TMEM lane quarter, thread = head) push every partial S tile to
+        // the peer's exchange buffer as soon as its Q.KV^T completes, so the distributed-memory
+        // hop never waits behind a softmax.
+        const int h = (warp & 3) * 32 + lane;
+        const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+        uint32_t peer_recv[2], peer_bar[2];
+        for (int b = 0; b < 2; ++b) {
+            peer_recv[b] = tc::mapa_shared(tc::smem_u32(recv + b * kRecvBytes), peer);
+            peer_bar[b] = tc::mapa_shared(tc::smem_u32(&bars->recv_full[b]), peer);
+        }
+        uint32_t m = 0;
+        bool stop = false;
+        for (int t = cluster; t < v.T_q && !stop; t += n_clusters) {
+            RowInfo r;
+            const int ntiles = row_tiles(v, idx, K, t, lane, r);
+            for (int j = 0; j < ntiles; ++j, ++m) {
+                const uint32_t b = m & 1;
+                if (!tc::mbar_wait(&bars->s_full[b], (m >> 1) & 1, abort_flag)) {
+                    stop = true;
+                    break;
+                }
+                tc::tc_fence_after();
+                float sv[kBN];
+                tc::tmem_ld32(tmem_base + lane_off + kTmemS + b * kBN, sv);
+                tc::tmem_ld32(tmem_base + lane_off + kTmemS + b * kBN + 32, sv + 32);
+                tc::tmem_ld_wait();
+                tc::tc_fence_before();
+                __syncwarp();
+                if (lane == 0) tc::mbar_arrive(&bars->s_sent[b]);
+                // the peer's P.V(m-2) has released its buffer b.  One barrier per buffer: the
+                // peer cannot complete P.V(m) before it receives this tile, so the barrier is
+                // never two phases ahead of this wait (with a single barrier for both buffers it
+                // could be, since the peer may finish P.V(m-1) first, and a parity wait would
+                // then alias).
+                if (m >= 2 && !tc::mbar_wait(&bars->peer_free[b], ((m - 2) >> 1) & 1, abort_flag)) {
+                    stop = true;
+                    break;
+                }
+                if (warp == 13 && lane == 0) tc::mbar_arrive_expect_tx(&bars->recv_full[b], kRecvBytes);
+                const uint32_t dst = peer_recv[b] + h * (kBN * 4);
+#pragma unroll
+                for (int i = 0; i < kBN / 4; ++i)
+                    tc::st_async_v4(dst + ((i ^ (h & 7)) * 16), peer_bar[b], __float_as_uint(sv[4 * i]),
+                                    __float_as_uint(sv[4 * i + 1]), __float_as_uint(sv[4 * i + 2]),
+                                    __float_as_uint(sv[4 * i + 3]));
+            }
+        }
         // the peer's last two P.V commits arrive here; take them before leaving
         if (!stop) {
-            if (n >= 2) tc::mbar_wait(&bars->peer_free[(n - 2) & 1], ((n - 2) >> 1) & 1, abort_flag);
-            if (n >= 1) tc::mbar_wait(&bars->peer_free[(n - 1) & 1], ((n - 1) >> 1) & 1, abort_flag);
+            if (m >= 2) tc::mbar_wait(&bars->peer_free[(m - 2) & 1], ((m - 2) >> 1) & 1, abort_flag);
+            if (m >= 1) tc::mbar_wait(&bars->peer_free[(m - 1) & 1], ((m - 1) >> 1) & 1, abort_flag);
         }
     }
     __syncwarp();
@@ -568,6 +599,7 @@ int num_sms() {
 bool sparse_mla_tc_supported(const SparseMlaArgs& a) {
     if (a.q_dtype != HSA_BF16 || a.kv_dtype != HSA_BF16 || a.out_dtype != HSA_BF16) return false;
     if (a.H != kH || a.D_qk != kDqk || a.D_v != kDv) return false;
+    if (!(a.softmax_scale > 0.f)) return false;   // the kernel takes tile maxima on unscaled S
     auto al = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; };
     if (!al(a.q) || !al(a.kv) || !al(a.out)) return false;
     if ((uint64_t)a.seq.T_q * kH >= (1ull << 31)) return false;
