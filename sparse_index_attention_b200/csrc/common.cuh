@@ -7,6 +7,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "../../include/hsa.h"
 
 namespace hsa {
@@ -107,5 +109,33 @@ __host__ __device__ constexpr int64_t ceil_div(int64_t a, int64_t b) { return (a
 // Kernel launches issued by the calling host thread (reported by hsa_launch_count()).
 uint64_t& launch_counter();
 inline void count_launch(int n = 1) { launch_counter() += (uint64_t)n; }
+
+// Programmatic dependent launch.  The tensor-core path's kernels (index score, Top-K, sparse MLA)
+// are launched so that a kernel may start while the previous kernel on the stream is still
+// running.  Such a kernel reads only the row descriptors (which no kernel of this library
+// writes) before pdl_wait(), which returns once every earlier kernel on the stream has finished
+// and its writes are visible; it touches nothing else until then.  Right after its own
+// pdl_wait() it calls pdl_trigger(), which lets the next kernel launch: so when a kernel starts,
+// everything before its predecessor has finished.  Without the launch attribute both are no-ops.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+template <typename... Params, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(Params...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t st, Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+    count_launch();
+    return e;
+}
 
 }  // namespace hsa

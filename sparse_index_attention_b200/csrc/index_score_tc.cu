@@ -173,6 +173,8 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
     tc::tc_fence_before();
     __syncthreads();
     tc::tc_fence_after();
+    pdl_wait();              // queries, weights and keys may be the previous kernel's output
+    pdl_trigger();
     const uint32_t tmem_base = *tmem_holder;
     const int64_t total = n_groups > 0 ? prefix[n_groups] : 0;
     const int64_t f_begin = total * blockIdx.x / gridDim.x;
@@ -423,11 +425,9 @@ cudaError_t launch_g(const IndexScoreArgs& a, cudaStream_t st) {
         v.q_pos += t0;
         const int64_t groups = ceil_div(v.T_q, G);
         const int grid = (int)std::min<int64_t>(num_sms(), std::max<int64_t>(1, groups * 64));
-        kern<<<grid, C::kThreads, C::kSmem, st>>>(tk, tq, v, t0 * kHI, a.w + (int64_t)t0 * kHI,
-                                                   a.k_scale, a.scores + (int64_t)t0 * a.ld, a.ld,
-                                                   box_rows);
-        count_launch();
-        e = cudaGetLastError();
+        e = launch_pdl(kern, dim3(grid), dim3(C::kThreads), C::kSmem, st, tk, tq, v, t0 * kHI,
+                       a.w + (int64_t)t0 * kHI, a.k_scale, a.scores + (int64_t)t0 * a.ld, a.ld, box_rows);
+        if (e == cudaSuccess) e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
     return cudaSuccess;

@@ -177,6 +177,8 @@ sparse_mla_tc_kernel(SeqView v,
     tc::cluster_sync_all();  // the peer's barriers exist before anything remote touches them
     tc::tc_fence_after();
     const uint32_t tmem_base = bars->tmem;
+    pdl_wait();              // the selection is the previous kernel's output
+    pdl_trigger();
 
     if (warp < 4) {
         // ---------------------------------------------------------------- producers (gather)
@@ -616,11 +618,10 @@ cudaError_t launch_sparse_mla_tc(const SparseMlaArgs& a, cudaStream_t st) {
     if (e != cudaSuccess) return e;
     const int clusters = std::max(1, std::min(a.seq.T_q, num_sms() / 2));
     const float scale_log2 = a.softmax_scale * 1.4426950408889634f;
-    sparse_mla_tc_kernel<<<2 * clusters, kThreads, kSmem, st>>>(
-        a.seq, reinterpret_cast<const __nv_bfloat16*>(a.q), reinterpret_cast<const __nv_bfloat16*>(a.kv),
-        a.idx, a.K, scale_log2, reinterpret_cast<__nv_bfloat16*>(a.out), a.lse);
-    count_launch();
-    return cudaGetLastError();
+    e = launch_pdl(sparse_mla_tc_kernel, dim3(2 * clusters), dim3(kThreads), kSmem, st, a.seq,
+                   reinterpret_cast<const __nv_bfloat16*>(a.q), reinterpret_cast<const __nv_bfloat16*>(a.kv),
+                   a.idx, a.K, scale_log2, reinterpret_cast<__nv_bfloat16*>(a.out), a.lse);
+    return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 }  // namespace hsa

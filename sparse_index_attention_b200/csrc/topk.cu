@@ -3,12 +3,28 @@
 // index scores; "Day-One Inference Adaptation for Very Large Hybrid-Attention Models", 3.1).
 //
 // One 1024-thread CTA per query row.  Scores map to order-preserving 32-bit keys (-0.0 folded
-// onto +0.0).  Three histogram passes over digits of 11, 11 and 10 bits find the exact key T
-// of the K-th best element and how many elements equal to T belong to the selection.  A final
-// pass compacts the selection in ascending position order with a block-wide scan: every key
-// above T, and the lowest-position elements equal to T (ties go to the lower index).  Rows of
-// at most kSmemKeys positions are staged once in shared memory; longer rows are re-read from
-// global memory (L2) on every pass.
+// onto +0.0).  The selection is every key above T, the key of the K-th best element, and the
+// lowest-position elements equal to T (ties go to the lower index), written in ascending
+// position order.
+//
+// A histogram over the whole row is expensive here: the scores concentrate in a few exponent
+// bins, and the shared-memory atomics on those bins serialize.  So a long row is first cut down
+// to candidates:
+//   stage     the row's keys go to shared memory (float4 loads), when they fit;
+//   sample    4096 evenly spaced keys; a two-pass radix select on them gives a threshold L a few
+//             standard deviations below the sample's estimate of T, so that the row holds K or
+//             more keys >= L with overwhelming probability;
+//   collect   warps sweep contiguous segments of the row: a ballot count, a scan over the warps,
+//             and a second sweep that writes every key >= L with its position, in position order;
+//   select    a three-pass radix select (digits of 11, 11 and 10 bits) over the candidates finds
+//             T exactly and how many elements equal to T are selected;
+//   write     a ballot sweep over the candidates places each selected position.
+// Whenever the candidates cannot be used -- short rows, too few keys >= L, more than fit in
+// shared memory (heavy ties) -- the select and write steps run over the whole row instead, which
+// gives the same result.  Either way the output is exact: the threshold only decides how much
+// work the exact steps see.
+#include <algorithm>
+
 #include "kernels.h"
 
 namespace hsa {
@@ -16,9 +32,14 @@ namespace hsa {
 namespace {
 
 constexpr int kThreads = 1024;
+constexpr int kWarps = kThreads / 32;
 constexpr int kBins = 2048;
-constexpr int kItems = 16;                     // consecutive positions per thread in compaction
-constexpr int kSmemKeys = 50 * 1024;           // 200 KB of staged keys
+constexpr int kSample = 4096;
+constexpr int kSampleMinRow = 2 * kSample;     // shorter rows go straight to the exact steps
+constexpr int kSmemKeys = 40 * 1024;           // staged keys (160 KB)
+constexpr int kMaxSmem = 227 * 1024;
+// shared memory ahead of the candidates: histogram, warp sums, scalars
+constexpr int kFixedWords = kBins + 2 * kWarps + 16;
 
 __device__ __forceinline__ uint32_t score_key(float f) {
     uint32_t u = __float_as_uint(f);
@@ -26,128 +47,264 @@ __device__ __forceinline__ uint32_t score_key(float f) {
     return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-// Inclusive scan of one value per thread over the whole block; `total` gets the block sum.
-__device__ __forceinline__ uint32_t block_incl_scan(uint32_t x, uint32_t* wsum, uint32_t& total) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    constexpr int kWarps = kThreads / 32;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
-        if (lane >= o) x += y;
-    }
-    if (lane == 31) wsum[warp] = x;
-    __syncthreads();
-    if (warp == 0) {
-        uint32_t s = lane < kWarps ? wsum[lane] : 0u;
+__device__ __forceinline__ uint32_t lanemask_lt() {
+    uint32_t m;
+    asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
+    return m;
+}
+
+struct Kth {
+    uint32_t key;    // the k-th largest key (with two passes: its top 22 bits, low 10 bits zero)
+    uint32_t krem;   // how many elements equal to `key` are among the k largest (three passes)
+};
+
+// Radix select over the n keys get(0..n-1) (1 <= k <= n): digits of 11, 11 and 10 bits, most
+// significant first; each pass histograms the keys that share the digits found so far.  `hist`
+// is all zero on entry and is left all zero: the thread that reads a bin's count clears it.
+template <int kPasses, class Get>
+__device__ Kth radix_select(const Get& get, int n, uint32_t k, uint32_t* hist, uint64_t* wsum,
+                            uint32_t* misc) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    uint32_t prefix = 0u, pmask = 0u, krem = k;
+#pragma unroll 1
+    for (int pass = 0; pass < kPasses; ++pass) {
+        const int sh = pass == 0 ? 21 : (pass == 1 ? 10 : 0);
+        const uint32_t dmask = pass == 2 ? 0x3FFu : 0x7FFu;
+#pragma unroll 1
+        for (int i0 = 0; i0 < n; i0 += kThreads) {
+            const int i = i0 + tid;
+            const bool ok = i < n;
+            const uint32_t u = ok ? get(i) : 0u;
+            const bool take = ok && (u & pmask) == prefix;
+            const uint32_t bin = (u >> sh) & dmask;
+            // a warp whose lanes all take one bin (ties, constant rows) adds once
+            const uint32_t b0 = __shfl_sync(0xffffffffu, bin, 0);
+            if (__all_sync(0xffffffffu, take && bin == b0)) {
+                if (lane == 0) atomicAdd(hist + b0, 32u);
+            } else if (take) {
+                atomicAdd(hist + bin, 1u);
+            }
+        }
+        __syncthreads();
+        // thread i owns digits d0 = 2047 - 2i (higher) and d1 = 2046 - 2i: a prefix sum in this
+        // order counts the keys whose digit is >= d1
+        const int d0 = kBins - 1 - 2 * tid, d1 = d0 - 1;
+        const uint32_t h0 = hist[d0], c = h0 + hist[d1];
+        hist[d0] = 0u;
+        hist[d1] = 0u;
+        uint32_t incl = c;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
-            uint32_t y = __shfl_up_sync(0xffffffffu, s, o);
-            if (lane >= o) s += y;
+            const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
         }
-        wsum[lane] = s;
+        if (lane == 31) wsum[warp] = incl;
+        __syncthreads();
+        // every warp scans the 32 warp totals itself
+        const uint32_t wt = (uint32_t)wsum[lane];
+        uint32_t wincl = wt;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t y = __shfl_up_sync(0xffffffffu, wincl, o);
+            if (lane >= o) wincl += y;
+        }
+        const uint32_t wbefore = __shfl_sync(0xffffffffu, wincl - wt, warp);
+        const uint32_t excl = wbefore + incl - c;
+        if (excl < krem && krem <= excl + c) {
+            misc[0] = excl + h0 >= krem ? (uint32_t)d0 : (uint32_t)d1;
+            misc[1] = excl + h0 >= krem ? excl : excl + h0;
+        }
+        __syncthreads();
+        krem -= misc[1];
+        prefix |= misc[0] << sh;
+        pmask |= dmask << sh;
     }
+    return Kth{prefix, krem};
+}
+
+// Writes the selection -- keys above T, and the first krem keys equal to T -- from the n keys
+// get(0..n-1), which are in ascending position order, to out[] in that order.  Warps own
+// contiguous segments; a count sweep and a scan over the warps give each its first slot.
+template <class Get, class Pos>
+__device__ void write_selection(const Get& get, const Pos& pos, int n, uint32_t T, uint32_t krem,
+                                int K, int32_t* __restrict__ out, uint64_t* wsum) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int seg = ((n + kThreads - 1) / kThreads) * 32;
+    const int s0 = min(n, warp * seg), s1 = min(n, s0 + seg);
+    uint32_t gt = 0u, eq = 0u;
+    for (int j = s0; j < s1; j += 32) {
+        const int i = j + lane;
+        const bool ok = i < s1;
+        const uint32_t u = ok ? get(i) : 0u;
+        gt += (uint32_t)__popc(__ballot_sync(0xffffffffu, ok && u > T));
+        eq += (uint32_t)__popc(__ballot_sync(0xffffffffu, ok && u == T));
+    }
+    if (lane == 0) wsum[warp] = ((uint64_t)gt << 32) | eq;
     __syncthreads();
-    const uint32_t pre = warp > 0 ? wsum[warp - 1] : 0u;
-    total = wsum[kWarps - 1];
-    __syncthreads();
-    return x + pre;
+    uint64_t before = lane < warp ? wsum[lane] : 0ull;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) before += __shfl_xor_sync(0xffffffffu, before, o);
+    uint32_t gb = (uint32_t)(before >> 32), eb = (uint32_t)before;
+    for (int j = s0; j < s1; j += 32) {
+        const int i = j + lane;
+        const bool ok = i < s1;
+        const uint32_t u = ok ? get(i) : 0u;
+        const uint32_t bg = __ballot_sync(0xffffffffu, ok && u > T);
+        const uint32_t be = __ballot_sync(0xffffffffu, ok && u == T);
+        const uint32_t g = gb + (uint32_t)__popc(bg & lanemask_lt());
+        const uint32_t e = eb + (uint32_t)__popc(be & lanemask_lt());
+        // the output slot of a selected element is the number of selected elements at lower
+        // positions (< K by construction; the bound keeps a wrong count harmless)
+        if (ok && u > T) {
+            const uint32_t o = g + min(e, krem);
+            if (o < (uint32_t)K) out[o] = pos(i);
+        } else if (ok && u == T && e < krem && g + e < (uint32_t)K) {
+            out[g + e] = pos(i);
+        }
+        gb += (uint32_t)__popc(bg);
+        eb += (uint32_t)__popc(be);
+    }
 }
 
 template <bool kStaged>
 __global__ void __launch_bounds__(kThreads, 1)
-topk_kernel(SeqView v, const float* __restrict__ scores, int64_t ld, int K, int32_t* __restrict__ idx) {
-    extern __shared__ uint32_t sm[];
-    uint32_t* hist = sm;                 // [kBins]
-    uint32_t* wsum = sm + kBins;         // [32]
-    uint32_t* misc = wsum + 32;          // [8]
-    uint32_t* keys = misc + 8;           // [n] when staged
+topk_kernel(SeqView v, const float* __restrict__ scores, int64_t ld, int K, int cand_cap,
+            int32_t* __restrict__ idx) {
+    extern __shared__ __align__(16) uint32_t sm[];
+    uint32_t* hist = sm;                                          // [kBins]
+    uint64_t* wsum = reinterpret_cast<uint64_t*>(sm + kBins);     // [kWarps]
+    uint32_t* misc = sm + kBins + 2 * kWarps;                     // [16]
+    uint32_t* cand_key = misc + 16;                               // [cand_cap]; first the sample
+    uint32_t* cand_pos = cand_key + cand_cap;                     // [cand_cap]
+    uint32_t* keys = cand_pos + cand_cap;                         // [n] when staged
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int t = blockIdx.x;
     const RowInfo r = load_row(v, t);
+    pdl_wait();                          // the scores are the previous kernel's output
+    pdl_trigger();
     int32_t* out = idx + (int64_t)t * K;
     const int n = r.pos + 1;             // 0 for an invalid row: all -1
     if (n <= K) {
-        for (int i = threadIdx.x; i < K; i += kThreads) out[i] = i < n ? i : -1;
+        for (int i = tid; i < K; i += kThreads) out[i] = i < n ? i : -1;
         return;
     }
-    const float* row = scores + (int64_t)t * ld;
-    if (kStaged) {
-        for (int i = threadIdx.x; i < n; i += kThreads) keys[i] = score_key(row[i]);
-        __syncthreads();
-    }
-    auto key_at = [&](int i) -> uint32_t { return kStaged ? keys[i] : score_key(__ldg(row + i)); };
+    const float* src = scores + (int64_t)t * ld;
+    for (int b = tid; b < kBins; b += kThreads) hist[b] = 0u;
+    auto key_at = [&](int i) -> uint32_t { return kStaged ? keys[i] : score_key(__ldg(src + i)); };
 
-    uint32_t prefix = 0u, pmask = 0u, krem = (uint32_t)K;
+    if (kStaged) {
+        const bool vec = (reinterpret_cast<uintptr_t>(src) & 15u) == 0u;
+        constexpr int kU = 8;
 #pragma unroll 1
-    for (int pass = 0; pass < 3; ++pass) {
-        const int sh = pass == 0 ? 21 : (pass == 1 ? 10 : 0);
-        const uint32_t dmask = pass == 2 ? 0x3FFu : 0x7FFu;
-        for (int b = threadIdx.x; b < kBins; b += kThreads) hist[b] = 0u;
-        __syncthreads();
-        for (int i = threadIdx.x; i < n; i += kThreads) {
-            const uint32_t u = key_at(i);
-            if ((u & pmask) == prefix) atomicAdd(&hist[(u >> sh) & dmask], 1u);
-        }
-        __syncthreads();
-        // thread i owns digits d0 = 2047 - 2i (higher) and d1 = 2046 - 2i: a prefix scan in this
-        // order counts the elements whose digit is >= d1
-        const int d0 = kBins - 1 - 2 * threadIdx.x, d1 = d0 - 1;
-        const uint32_t h0 = hist[d0], c = h0 + hist[d1];
-        uint32_t total;
-        const uint32_t incl = block_incl_scan(c, wsum, total);
-        const uint32_t excl = incl - c;
-        if (excl < krem && krem <= incl) {
-            if (excl + h0 >= krem) {
-                misc[0] = (uint32_t)d0;
-                misc[1] = excl;
-            } else {
-                misc[0] = (uint32_t)d1;
-                misc[1] = excl + h0;
+        for (int base = 0; base < n; base += kThreads * 4 * kU) {
+            float4 f[kU];
+#pragma unroll
+            for (int a = 0; a < kU; ++a) {
+                const int i = base + (a * kThreads + tid) * 4;
+                if (vec && i + 3 < n) {
+                    f[a] = __ldg(reinterpret_cast<const float4*>(src + i));
+                } else {
+                    f[a].x = i + 0 < n ? __ldg(src + i + 0) : 0.f;
+                    f[a].y = i + 1 < n ? __ldg(src + i + 1) : 0.f;
+                    f[a].z = i + 2 < n ? __ldg(src + i + 2) : 0.f;
+                    f[a].w = i + 3 < n ? __ldg(src + i + 3) : 0.f;
+                }
+            }
+#pragma unroll
+            for (int a = 0; a < kU; ++a) {
+                const int i = base + (a * kThreads + tid) * 4;
+                const uint4 u = make_uint4(score_key(f[a].x), score_key(f[a].y), score_key(f[a].z),
+                                           score_key(f[a].w));
+                if (i + 3 < n) {
+                    *reinterpret_cast<uint4*>(keys + i) = u;
+                } else {
+                    if (i + 0 < n) keys[i + 0] = u.x;
+                    if (i + 1 < n) keys[i + 1] = u.y;
+                    if (i + 2 < n) keys[i + 2] = u.z;
+                }
             }
         }
-        __syncthreads();
-        const uint32_t digit = misc[0], above = misc[1];
-        krem -= above;
-        prefix |= digit << sh;
-        pmask |= dmask << sh;
-        __syncthreads();
     }
-    // prefix is the exact key T of the K-th best element; krem (>= 1) elements equal to T are
-    // selected, the ones at the lowest positions.
-    const uint32_t T = prefix;
-    uint32_t run_gt = 0u, run_eq = 0u;
-#pragma unroll 1
-    for (int base = 0; base < n; base += kThreads * kItems) {
-        const int p0 = base + threadIdx.x * kItems;
-        uint32_t u[kItems];
-        uint32_t gt = 0u, eq = 0u;
+    __syncthreads();
+
+    // candidates: the keys >= a threshold taken from a sample, in position order
+    int n_cand = -1;                     // -1: the exact steps run over the whole row
+    if (n >= kSampleMinRow) {
+        const float ps = (float)K * (float)kSample / (float)n;   // expected sample keys >= T
+        const int rank = (int)ceilf(ps + 4.f * sqrtf(ps) + 8.f);
+        if (rank < kSample / 2) {
+            uint32_t* sample = cand_key;
+            for (int s = tid; s < kSample; s += kThreads)
+                sample[s] = key_at((int)(((int64_t)s * n) / kSample));
+            __syncthreads();
+            const uint32_t L = radix_select<2>([&](int i) { return sample[i]; }, kSample,
+                                               (uint32_t)rank, hist, wsum, misc).key;
+            // warp segments of whole 128-key chunks, swept four keys per lane at a time
+            const int seg = ((n + kWarps * 128 - 1) / (kWarps * 128)) * 128;
+            const int s0 = min(n, warp * seg), s1 = min(n, s0 + seg);
+            uint32_t c = 0u;
+            for (int j = s0; j < s1; j += 128) {
 #pragma unroll
-        for (int k = 0; k < kItems; ++k) {
-            u[k] = (p0 + k < n) ? key_at(p0 + k) : 0u;
-            gt += (p0 + k < n) && u[k] > T;
-            eq += (p0 + k < n) && u[k] == T;
-        }
-        // both counts fit in 16 bits (at most kThreads * kItems = 16384 per chunk)
-        uint32_t total;
-        const uint32_t incl = block_incl_scan((gt << 16) | eq, wsum, total);
-        const uint32_t excl = incl - ((gt << 16) | eq);
-        uint32_t gb = run_gt + (excl >> 16), eb = run_eq + (excl & 0xFFFFu);
+                for (int a = 0; a < 4; ++a) {
+                    const int i = j + 32 * a + lane;
+                    c += (uint32_t)__popc(__ballot_sync(0xffffffffu, i < s1 && key_at(i) >= L));
+                }
+            }
+            if (lane == 0) wsum[warp] = c;
+            __syncthreads();
+            uint32_t before = lane < warp ? (uint32_t)wsum[lane] : 0u;
+            uint32_t total = (uint32_t)wsum[lane];
 #pragma unroll
-        for (int k = 0; k < kItems; ++k) {
-            if (p0 + k >= n) break;
-            // the output slot of a selected element is the number of selected elements at
-            // lower positions (< K by construction; the bound keeps a wrong count harmless)
-            if (u[k] > T) {
-                const uint32_t o = gb + min(eb, krem);
-                if (o < (uint32_t)K) out[o] = p0 + k;
-                ++gb;
-            } else if (u[k] == T) {
-                if (eb < krem && gb + eb < (uint32_t)K) out[gb + eb] = p0 + k;
-                ++eb;
+            for (int o = 16; o > 0; o >>= 1) {
+                before += __shfl_xor_sync(0xffffffffu, before, o);
+                total += __shfl_xor_sync(0xffffffffu, total, o);
+            }
+            __syncthreads();
+            if (total >= (uint32_t)K && total <= (uint32_t)cand_cap) {     // the same in every thread
+                const uint32_t lt = lanemask_lt();
+                for (int j = s0; j < s1; j += 128) {
+                    uint32_t u[4], bal[4];
+#pragma unroll
+                    for (int a = 0; a < 4; ++a) {
+                        const int i = j + 32 * a + lane;
+                        u[a] = i < s1 ? key_at(i) : 0u;
+                        bal[a] = __ballot_sync(0xffffffffu, i < s1 && u[a] >= L);
+                    }
+#pragma unroll
+                    for (int a = 0; a < 4; ++a) {
+                        if ((bal[a] >> lane) & 1u) {
+                            const uint32_t p = before + (uint32_t)__popc(bal[a] & lt);
+                            cand_key[p] = u[a];
+                            cand_pos[p] = (uint32_t)(j + 32 * a + lane);
+                        }
+                        before += (uint32_t)__popc(bal[a]);
+                    }
+                }
+                n_cand = (int)total;
+                __syncthreads();
             }
         }
-        run_gt += total >> 16;
-        run_eq += total & 0xFFFFu;
     }
+
+    if (n_cand >= 0) {
+        auto get = [&](int i) { return cand_key[i]; };
+        const Kth kth = radix_select<3>(get, n_cand, (uint32_t)K, hist, wsum, misc);
+        write_selection(get, [&](int i) { return (int32_t)cand_pos[i]; }, n_cand, kth.key, kth.krem,
+                        K, out, wsum);
+    } else {
+        const Kth kth = radix_select<3>(key_at, n, (uint32_t)K, hist, wsum, misc);
+        write_selection(key_at, [](int i) { return (int32_t)i; }, n, kth.key, kth.krem, K, out, wsum);
+    }
+}
+
+template <bool kStaged>
+cudaError_t launch_variant(const SeqView& seq, const float* scores, int64_t ld, int32_t K,
+                           int cand_cap, size_t smem, int32_t* idx, cudaStream_t st) {
+    auto k = topk_kernel<kStaged>;
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    e = launch_pdl(k, dim3(seq.T_q), dim3(kThreads), smem, st, seq, scores, ld, (int)K, cand_cap, idx);
+    return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 }  // namespace
@@ -155,19 +312,14 @@ topk_kernel(SeqView v, const float* __restrict__ scores, int64_t ld, int K, int3
 cudaError_t launch_topk(const SeqView& seq, int32_t max_seq_len, const float* scores, int64_t ld,
                         int32_t K, int32_t* idx, cudaStream_t st) {
     if (seq.T_q == 0) return cudaSuccess;
-    const size_t base = sizeof(uint32_t) * (kBins + 32 + 8);
-    if (max_seq_len <= kSmemKeys) {
-        const size_t smem = base + sizeof(uint32_t) * (size_t)max_seq_len;
-        auto k = topk_kernel<true>;
-        cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        k<<<seq.T_q, kThreads, smem, st>>>(seq, scores, ld, K, idx);
-    count_launch();
-    } else {
-        topk_kernel<false><<<seq.T_q, kThreads, base, st>>>(seq, scores, ld, K, idx);
-    count_launch();
-    }
-    return cudaGetLastError();
+    const bool staged = max_seq_len <= kSmemKeys;
+    const int staged_words = staged ? ((max_seq_len + 3) & ~3) : 0;
+    // candidates (key and position) fill the rest; always room for the sample
+    const int cand_cap = ((kMaxSmem / 4 - kFixedWords - staged_words) / 2) & ~3;
+    const size_t smem = sizeof(uint32_t) * ((size_t)kFixedWords + 2 * (size_t)cand_cap + staged_words);
+    static_assert((kMaxSmem / 4 - kFixedWords - kSmemKeys) / 2 >= kSample, "no room for the sample");
+    return staged ? launch_variant<true>(seq, scores, ld, K, cand_cap, smem, idx, st)
+                  : launch_variant<false>(seq, scores, ld, K, cand_cap, smem, idx, st);
 }
 
 }  // namespace hsa

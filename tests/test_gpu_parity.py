@@ -117,6 +117,39 @@ def test_topk_vs_oracle_bit_exact(ties):
     assert np.array_equal(idx2.cpu().numpy(), ref2)
 
 
+@pytest.mark.parametrize("T,ld,K", [
+    (64, 9000, 2048),     # staged in shared memory, just long enough to sample
+    (64, 20001, 2048),    # staged, odd row stride (unaligned row starts)
+    (160, 40000, 2048),   # staged, the longest staged rows
+    (12, 70001, 2048),    # read from L2, odd row stride
+    (10, 131072, 2048),   # read from L2, the longest prefill context
+    (80, 60003, 512),     # read from L2, small K
+])
+@pytest.mark.parametrize("dist", ["normal", "ties", "narrow", "constant"])
+def test_topk_launch_variants_bit_exact(T, ld, K, dist):
+    """Every path of the Top-K kernel (rows staged in shared memory or read from L2, aligned or
+    unaligned row starts, sampled candidates or the whole row) on score distributions that
+    stress each step: spread values, heavy ties with +-0.0, values that all share their top 22
+    key bits, and constant rows whose candidates overflow shared memory."""
+    g = torch.Generator().manual_seed(T * 7 + ld)
+    lens = torch.randint(1, ld + 1, (T,), generator=g)
+    lens[0], lens[1], lens[2], lens[3] = ld, K, K + 1, min(ld, 3 * K + 5)
+    sc = workloads.random_scores(T, ld, seed=ld % 97, device=DEV, ties=(dist == "ties"))
+    if dist == "narrow":
+        sc = 1.0 + sc.abs() * 1e-6
+    elif dist == "constant":
+        sc = torch.full_like(sc, 0.75)
+        sc[1::2] = -0.0
+    seq = hsa.PagedSeq(torch.tensor([ld], device=DEV), torch.zeros((1, ld), dtype=torch.int32, device=DEV),
+                       1, ld, torch.zeros(T, dtype=torch.int32, device=DEV),
+                       (lens - 1).to(torch.int32).to(DEV), max_seq_len=ld,
+                       status=torch.zeros(1, dtype=torch.int32, device=DEV))
+    idx = hsa.hsa_topk(seq, sc, K)
+    check_status(seq)
+    ref = oracle.topk(sc.cpu(), lens.numpy().astype(np.int32), K)
+    assert np.array_equal(idx.cpu().numpy(), ref)
+
+
 def _attn_vs_oracle(wl, tol, idx=None):
     gc = GpuCaches(wl)
     seq = paged_seq(wl)
