@@ -24,16 +24,20 @@
 // Shared memory per CTA: the rope part of Q (8 KB, 64-byte swizzle), four KV stages of 64
 // gathered rows (36 KB each: four 64-dim 128-byte-swizzled blocks + one 32-dim 64-byte-swizzled
 // rope block; the stage is the K-major B operand of Q.KV^T and, read MN-major, the B operand of
-// P.V), two 32 KB exchange buffers that receive the peer's partial S (P, bf16, is written over
-// the buffer once it has been read), and the physical slots of the next 2048 selected entries.
-// The latent part of Q lives in TMEM (A operand of Q.KV^T), next to O (256 columns) and the two
-// partial-S buffers (2 x 64 columns).
+// P.V), two 32 KB exchange buffers that receive the peer's partial S (fp32, laid out
+// [4-column chunk][head][4] so that every warp-wide store and load covers 512 contiguous bytes),
+// and the physical slots of the next 1024 selected entries.  Tensor memory: O (256 columns), two
+// partial-S buffers (2 x 64 columns; P, bf16 pairs, overwrites the first half of its S buffer and
+// is the TMEM A operand of P.V) and the latent part of Q (128 columns, the A operand of Q.KV^T).
 //
 // Pipeline per tile n: sender warps push partial S(n) to the peer as soon as Q.KV^T(n) is done,
 // independent of the softmax, so the distributed-shared-memory hop overlaps the softmax of the
-// previous tile, and the tensor core runs Q.KV^T(n+1) and P.V(n-1) while softmax(n) runs.  The peer may overwrite an
-// exchange buffer only after this CTA's P.V of the tile that used it (MMA commit multicast to the
-// peer), which is also what makes receiving tile n prove that P.V(n-2) has finished.
+// previous tile, and the tensor core runs Q.KV^T(n+1) and P.V(n-1) while softmax(n) runs.  The
+// peer may overwrite an exchange buffer only after this CTA's P.V of the tile that used it (MMA
+// commit multicast to the peer), which is also what makes receiving tile n prove that P.V(n-2)
+// has finished.  Measured on B200: one tcgen05.mma issues in about 60 cycles whatever its N, so
+// Q.KV^T (18 MMAs of N = 64) costs more issue time than its flops; the cluster network moves the
+// 32 KB exchange in about 1 us when warp stores are contiguous (1.8 us with one row per thread).
 //
 // (A TMA tile::gather4 version of the gather -- four 128-byte rows per instruction, 80 per tile
 // and CTA -- delivered only about 0.75 TB/s here: the MMA warp waited on the gathered tiles for
@@ -41,8 +45,9 @@
 // bytes in flight.)
 //
 // Warp roles: 0-3 producers (slot window + gather; warp w owns rows 16w..16w+15 of every tile),
-// 4 MMA issuer, 5-12 softmax / epilogue (two threads per head h = TMEM lane h, 32 columns each),
-// 13-16 senders (partial S to the peer).  Persistent: each cluster loops over query rows.
+// 4 MMA issuer, 5-12 softmax / epilogue (two threads per head h = TMEM lane h, 32 columns each;
+// warps w and w + 4 share heads and swap tile maxima through a two-warp barrier), 13-16 senders
+// (partial S to the peer).  Persistent: each cluster loops over query rows.
 #include <algorithm>
 
 #include "kernels.h"
@@ -97,7 +102,7 @@ struct Bars {
     uint64_t peer_free[2];  // the peer's P.V of a tile of parity b completed (its buffer b is free)
     uint64_t recv_full[2];
     uint64_t o_ready, o_free;
-    uint64_t buf_read;    // the eight softmax warps finished reading an exchange buffer
+    uint64_t pair_sync[4];  // the two softmax warps of a head quarter (maxima / row sums posted)
     uint32_t tmem;
     int abort;
 };
@@ -164,7 +169,7 @@ sparse_mla_tc_kernel(SeqView v,
         tc::mbar_init(&bars->peer_free[1], 1);
         tc::mbar_init(&bars->o_ready, 1);
         tc::mbar_init(&bars->o_free, 8);
-        tc::mbar_init(&bars->buf_read, 8);
+        for (int i = 0; i < 4; ++i) tc::mbar_init(&bars->pair_sync[i], 2);
         bars->abort = 0;
         tc::fence_barrier_init();
     }
@@ -330,7 +335,7 @@ sparse_mla_tc_kernel(SeqView v,
         const uint32_t col = (uint32_t)(32 * half);
         uint32_t n = 0, rows_done = 0;
         bool stop = false;
-        tc::WarpSetSync buf_sync{&bars->buf_read, 0};
+        tc::WarpSetSync pair_sync{&bars->pair_sync[(warp - 5) & 3], 0};   // warps w and w + 4
 
         // next row (t0, t0 + n_clusters, ...) with work; rows without any selection are written
         // here directly (output 0, lse -inf)
@@ -383,8 +388,10 @@ sparse_mla_tc_kernel(SeqView v,
             for (int j = 0; j < ntiles; ++j, ++n) {
                 const uint32_t b = n & 1, st = n % kStages;
                 // ---- softmax(n), columns [col, col + 32)
+                // own partial S(n) is complete once the senders have read it (s_sent), which
+                // also frees its columns for P; it is loaded while the peer's half is in flight
                 if (!tc::mbar_wait(&bars->kv_full[st], (n / kStages) & 1, abort_flag) ||
-                    !tc::mbar_wait_cluster(&bars->recv_full[b], (n >> 1) & 1, abort_flag)) {
+                    !tc::mbar_wait(&bars->s_sent[b], (n >> 1) & 1, abort_flag)) {
                     stop = true;
                     break;
                 }
@@ -393,10 +400,14 @@ sparse_mla_tc_kernel(SeqView v,
                 float s[32];
                 tc::tmem_ld32(tmem_base + lane_off + kTmemS + b * kBN + col, s);
                 tc::tmem_ld_wait();
-                const float4* other = reinterpret_cast<const float4*>(recv + b * kRecvBytes + h * (kBN * 4));
+                if (!tc::mbar_wait_cluster(&bars->recv_full[b], (n >> 1) & 1, abort_flag)) {
+                    stop = true;
+                    break;
+                }
+                const float4* other = reinterpret_cast<const float4*>(recv + b * kRecvBytes) + h;
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
-                    const float4 o = other[(8 * half + i) ^ (h & 7)];
+                    const float4 o = other[(8 * half + i) * kH];
                     s[4 * i] += o.x;
                     s[4 * i + 1] += o.y;
                     s[4 * i + 2] += o.z;
@@ -412,7 +423,7 @@ sparse_mla_tc_kernel(SeqView v,
                 for (int i = 1; i < 32; ++i) mt = fmaxf(mt, s[i]);
                 mt = mt == -INFINITY ? -INFINITY : mt * scale_log2;   // tile max in base-2 units
                 xmax[(n & 1) * 256 + half * 128 + h] = mt;
-                if (!buf_sync.sync(abort_flag)) {  // both halves' maxima posted
+                if (!pair_sync.sync(abort_flag)) {  // both halves' maxima posted
                     stop = true;
                     break;
                 }
@@ -462,11 +473,8 @@ sparse_mla_tc_kernel(SeqView v,
                 }
                 l += (ps[0] + ps[1]) + (ps[2] + ps[3]);
                 // P over this thread's 32 columns of the S buffer: rows 32*half.. -> 16 columns of
-                // bf16 pairs; the senders must have read partial S first
-                if (!tc::mbar_wait(&bars->s_sent[b], (n >> 1) & 1, abort_flag)) {
-                    stop = true;
-                    break;
-                }
+                // bf16 pairs (the senders have read partial S, and the other half of the head read
+                // its columns before the maxima were exchanged)
                 tc::tmem_st16_u(tmem_base + lane_off + kTmemS + b * kBN + 16 * half, pk);
                 tc::tmem_st_wait();
                 tc::tc_fence_before();
@@ -488,7 +496,7 @@ sparse_mla_tc_kernel(SeqView v,
             if (stop) break;
             // ---- row epilogue: O / l -> bf16 -> global (this thread: 128 of the 256 dims)
             xsum[half * 128 + h] = l;
-            if (!tc::mbar_wait(&bars->o_ready, rows_done & 1, abort_flag) || !buf_sync.sync(abort_flag)) break;
+            if (!tc::mbar_wait(&bars->o_ready, rows_done & 1, abort_flag) || !pair_sync.sync(abort_flag)) break;
             tc::tc_fence_after();
             const float l_all = l + xsum[(half ^ 1) * 128 + h];
             __nv_bfloat16* orow = out + ((int64_t)t * kH + h) * kDv + 256 * rank + 128 * half;
@@ -560,10 +568,13 @@ sparse_mla_tc_kernel(SeqView v,
                     break;
                 }
                 if (warp == 13 && lane == 0) tc::mbar_arrive_expect_tx(&bars->recv_full[b], kRecvBytes);
-                const uint32_t dst = peer_recv[b] + h * (kBN * 4);
+                // chunk i (columns 4i..4i+3) of every head lies at [i][head]: each warp instruction
+                // writes 512 contiguous bytes, which the cluster network moves about twice as fast
+                // as one row per thread
+                const uint32_t dst = peer_recv[b] + h * 16;
 #pragma unroll
                 for (int i = 0; i < kBN / 4; ++i)
-                    tc::st_async_v4(dst + ((i ^ (h & 7)) * 16), peer_bar[b], __float_as_uint(sv[4 * i]),
+                    tc::st_async_v4(dst + i * (kH * 16), peer_bar[b], __float_as_uint(sv[4 * i]),
                                     __float_as_uint(sv[4 * i + 1]), __float_as_uint(sv[4 * i + 2]),
                                     __float_as_uint(sv[4 * i + 3]));
             }
