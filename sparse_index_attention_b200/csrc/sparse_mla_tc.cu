@@ -77,7 +77,9 @@ constexpr int kOffMasks = kOffSlots + 4 * kSlotWin;
 constexpr int kOffXmax = kOffMasks + 8 * kStages;              // [2 tiles][2 halves][128] fp32
 constexpr int kOffXsum = kOffXmax + 4 * 512;                   // [2 halves][128] fp32
 constexpr int kOffBars = kOffXsum + 4 * 256;
-constexpr int kKvRowBytes = kDqk * 2;   // 1152
+constexpr int kKvRowBytes = kDqk * 2;   // 1152: bf16 latent ‖ rope
+constexpr int kKv8RowBytes = kDv;       // 512: e4m3 latent codes (FP8 cache)
+constexpr int kRopeRowBytes = 128;      // bf16 rope of the FP8 cache
 constexpr size_t kSmem = 1024 + kOffBars + 256;
 static_assert(kSmem <= 232448, "shared memory budget");
 static_assert(kOffStages % 1024 == 0 && kStageBytes % 1024 == 0 && kOffRecv % 1024 == 0, "swizzle alignment");
@@ -126,10 +128,14 @@ __device__ __forceinline__ int row_tiles(const SeqView& v, const int32_t* __rest
     return (int)ceil_div(row_extent(idx + (int64_t)t * K, K, lane), kBN);
 }
 
+// kFp8Kv: the latent part of the cache is e4m3 codes with one fp32 scale per row and the rope part
+// a separate bf16 array; the producers widen code x scale to bf16 on the way into the stage.
+template <bool kFp8Kv>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 sparse_mla_tc_kernel(SeqView v,
-                     const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ kv,
-                     const int32_t* __restrict__ idx, int K,
+                     const __nv_bfloat16* __restrict__ q, const uint8_t* __restrict__ kv_bytes,
+                     const float* __restrict__ kv_scale, const uint8_t* __restrict__ rope_bytes,
+                     int64_t rope_row_bytes, const int32_t* __restrict__ idx, int K,
                      float scale_log2, __nv_bfloat16* __restrict__ out, float* __restrict__ lse) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -187,7 +193,6 @@ sparse_mla_tc_kernel(SeqView v,
 
     if (warp < 4) {
         // ---------------------------------------------------------------- producers (gather)
-        const uint8_t* kv_bytes = reinterpret_cast<const uint8_t*>(kv);
         int32_t* my_slots = slots + warp * (kSlotWin / 4);   // this warp's 16 rows of 16 tiles
         uint16_t* masks16 = reinterpret_cast<uint16_t*>(const_cast<uint64_t*>(masks));
         uint32_t n = 0;
@@ -227,14 +232,53 @@ sparse_mla_tc_kernel(SeqView v,
                 }
                 const int32_t* ts = my_slots + (j % (kSlotWin / kBN)) * 16;
                 uint8_t* sbase = stages + st * kStageBytes;
-                // latent half: one row per warp instruction, lane = 16-byte chunk
+                if (!kFp8Kv) {
+                    // latent half: one row per warp instruction, lane = 16-byte chunk
 #pragma unroll 4
-                for (int k = 0; k < 16; ++k) {
-                    const int row = warp * 16 + k;
-                    const int32_t sl = ts[k];
-                    const uint8_t* src = kv_bytes + (int64_t)(sl < 0 ? 0 : sl) * kKvRowBytes + 512 * rank + lane * 16;
-                    uint8_t* dst = sbase + (lane >> 3) * kKvBlk + row * 128 + (((lane & 7) ^ (row & 7)) * 16);
-                    tc::cp_async16(dst, src, sl < 0 ? 0u : 16u);
+                    for (int k = 0; k < 16; ++k) {
+                        const int row = warp * 16 + k;
+                        const int32_t sl = ts[k];
+                        const uint8_t* src = kv_bytes + (int64_t)(sl < 0 ? 0 : sl) * kKvRowBytes + 512 * rank + lane * 16;
+                        uint8_t* dst = sbase + (lane >> 3) * kKvBlk + row * 128 + (((lane & 7) ^ (row & 7)) * 16);
+                        tc::cp_async16(dst, src, sl < 0 ? 0u : 16u);
+                    }
+                } else {
+                    // latent half: 256 codes per row, two rows per warp instruction (half-warp =
+                    // row, lane = 16 codes); widened to bf16 (code x row scale, rounded once) and
+                    // stored as the two 16-byte chunks the swizzled stage expects
+                    const int sub = lane >> 4, cl = lane & 15;
+                    uint4 raw[8];
+                    float scl[8];
+#pragma unroll
+                    for (int k2 = 0; k2 < 8; ++k2) {
+                        const int32_t sl = ts[2 * k2 + sub];
+                        raw[k2] = sl < 0 ? make_uint4(0u, 0u, 0u, 0u)
+                                         : __ldg(reinterpret_cast<const uint4*>(kv_bytes + (int64_t)sl * kKv8RowBytes + 256 * rank) + cl);
+                        scl[k2] = sl < 0 ? 0.f : __ldg(kv_scale + sl);
+                    }
+#pragma unroll
+                    for (int k2 = 0; k2 < 8; ++k2) {
+                        const int row = warp * 16 + 2 * k2 + sub;
+                        const uint32_t words[4] = {raw[k2].x, raw[k2].y, raw[k2].z, raw[k2].w};
+                        uint32_t outw[8];
+#pragma unroll
+                        for (int qq = 0; qq < 4; ++qq) {
+#pragma unroll
+                            for (int hlf = 0; hlf < 2; ++hlf) {
+                                const __nv_fp8x2_storage_t pair = (__nv_fp8x2_storage_t)(words[qq] >> (16 * hlf));
+                                const float2 f2 = __half22float2(__half2(__nv_cvt_fp8x2_to_halfraw2(pair, __NV_E4M3)));
+                                const __nv_bfloat162 b2 = __floats2bfloat162_rn(f2.x * scl[k2], f2.y * scl[k2]);
+                                outw[qq * 2 + hlf] = *reinterpret_cast<const uint32_t*>(&b2);
+                            }
+                        }
+                        // codes 16cl..16cl+15 are dims of 16-byte chunks 2cl and 2cl+1
+                        uint8_t* rbase = sbase + (cl >> 2) * kKvBlk + row * 128;
+                        *reinterpret_cast<uint4*>(rbase + ((((2 * cl) & 7) ^ (row & 7)) * 16)) =
+                            make_uint4(outw[0], outw[1], outw[2], outw[3]);
+                        *reinterpret_cast<uint4*>(rbase + ((((2 * cl + 1) & 7) ^ (row & 7)) * 16)) =
+                            make_uint4(outw[4], outw[5], outw[6], outw[7]);
+                    }
+                    tc::fence_async_smem();   // these generic stores -> the tensor core
                 }
                 // rope half: 4 chunks per row, 8 rows per instruction
 #pragma unroll
@@ -242,7 +286,7 @@ sparse_mla_tc_kernel(SeqView v,
                     const int row = warp * 16 + 8 * h2 + (lane >> 2);
                     const int cc = lane & 3;
                     const int32_t sl = ts[8 * h2 + (lane >> 2)];
-                    const uint8_t* src = kv_bytes + (int64_t)(sl < 0 ? 0 : sl) * kKvRowBytes + 1024 + 64 * rank + cc * 16;
+                    const uint8_t* src = rope_bytes + (int64_t)(sl < 0 ? 0 : sl) * rope_row_bytes + 64 * rank + cc * 16;
                     uint8_t* dst = sbase + 4 * kKvBlk + row * 64 + ((cc ^ ((row >> 1) & 3)) * 16);
                     tc::cp_async16(dst, src, sl < 0 ? 0u : 16u);
                 }
@@ -250,6 +294,7 @@ sparse_mla_tc_kernel(SeqView v,
                 // and every warp has published its rows' validity bits
                 tc::cp_async_arrive_noinc(&bars->kv_full[st]);
                 const uint32_t vm = __ballot_sync(0xffffffffu, lane < 16 && ts[lane & 15] >= 0) & 0xFFFFu;
+                __syncwarp();             // orders the warp's generic stores before lane 0's arrive
                 if (lane == 0) {
                     masks16[st * 4 + warp] = (uint16_t)vm;
                     tc::mbar_arrive(&bars->kv_full[st]);
@@ -610,11 +655,14 @@ int num_sms() {
 }  // namespace
 
 bool sparse_mla_tc_supported(const SparseMlaArgs& a) {
-    if (a.q_dtype != HSA_BF16 || a.kv_dtype != HSA_BF16 || a.out_dtype != HSA_BF16) return false;
+    if (a.q_dtype != HSA_BF16 || a.out_dtype != HSA_BF16) return false;
+    if (a.kv_dtype != HSA_BF16 && a.kv_dtype != HSA_E4M3) return false;
+    if (a.kv_dtype == HSA_E4M3 && (a.kv_scale == nullptr || a.kv_rope == nullptr)) return false;
     if (a.H != kH || a.D_qk != kDqk || a.D_v != kDv) return false;
     if (!(a.softmax_scale > 0.f)) return false;   // the kernel takes tile maxima on unscaled S
     auto al = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; };
     if (!al(a.q) || !al(a.kv) || !al(a.out)) return false;
+    if (a.kv_dtype == HSA_E4M3 && (!al(a.kv_rope) || (reinterpret_cast<uintptr_t>(a.kv_scale) & 3))) return false;
     if ((uint64_t)a.seq.T_q * kH >= (1ull << 31)) return false;
     if ((uint64_t)a.seq.num_pages * a.seq.page_size >= (1ull << 31)) return false;
     return true;
@@ -624,13 +672,18 @@ size_t sparse_mla_tc_workspace(int32_t, int32_t) { return 0; }
 
 cudaError_t launch_sparse_mla_tc(const SparseMlaArgs& a, cudaStream_t st) {
     if (a.seq.T_q == 0) return cudaSuccess;
-    cudaError_t e = cudaFuncSetAttribute(sparse_mla_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)kSmem);
+    const bool fp8 = a.kv_dtype == HSA_E4M3;
+    auto kern = fp8 ? sparse_mla_tc_kernel<true> : sparse_mla_tc_kernel<false>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmem);
     if (e != cudaSuccess) return e;
     const int clusters = std::max(1, std::min(a.seq.T_q, num_sms() / 2));
     const float scale_log2 = a.softmax_scale * 1.4426950408889634f;
-    e = launch_pdl(sparse_mla_tc_kernel, dim3(2 * clusters), dim3(kThreads), kSmem, st, a.seq,
-                   reinterpret_cast<const __nv_bfloat16*>(a.q), reinterpret_cast<const __nv_bfloat16*>(a.kv),
+    const uint8_t* kv = reinterpret_cast<const uint8_t*>(a.kv);
+    // the bf16 cache packs the rope dims after the latent ones in each 1152-byte row
+    const uint8_t* rope = fp8 ? reinterpret_cast<const uint8_t*>(a.kv_rope) : kv + 2 * kDv;
+    const int64_t rope_row = fp8 ? kRopeRowBytes : kKvRowBytes;
+    e = launch_pdl(kern, dim3(2 * clusters), dim3(kThreads), kSmem, st, a.seq,
+                   reinterpret_cast<const __nv_bfloat16*>(a.q), kv, fp8 ? a.kv_scale : nullptr, rope, rope_row,
                    a.idx, a.K, scale_log2, reinterpret_cast<__nv_bfloat16*>(a.out), a.lse);
     return e != cudaSuccess ? e : cudaGetLastError();
 }

@@ -180,15 +180,21 @@ def test_sparse_mla_vs_oracle(name, kw, tol):
     _attn_vs_oracle(workloads.make(name, DEV, **kw), tol)
 
 
-def test_sparse_mla_empty_rows_and_constant_values():
-    wl = workloads.make("decode_bf16", DEV, B=4, L_min=100, L_max=3000)
+@pytest.mark.parametrize("name,kw,tol", [
+    ("decode_bf16", dict(B=4, L_min=100, L_max=3000), 2e-2),
+    ("decode_fp8", dict(B=4, L=3000), 6e-2),
+])
+def test_sparse_mla_empty_rows_and_constant_values(name, kw, tol):
+    wl = workloads.make(name, DEV, **kw)
     idx = workloads.random_selection(wl.q_pos, wl.K, seed=5)
     idx[1] = -1                       # a row that selects nothing
     idx[2, 1::2] = -1                 # holes inside a row
-    out, lse = _attn_vs_oracle(wl, 2e-2, idx)
+    out, lse = _attn_vs_oracle(wl, tol, idx)
     assert torch.all(out[1] == 0) and torch.all(torch.isneginf(lse[1]))
     wl.kv[:, :wl.D_v] = 1.0           # every value row is all ones -> output is ones
-    out2, _ = hsa.hsa_sparse_mla_attn(paged_seq(wl), wl.q, wl.kv, idx.to(DEV), wl.D_v, wl.softmax_scale)
+    gc = GpuCaches(wl)
+    out2, _ = hsa.hsa_sparse_mla_attn(paged_seq(wl), wl.q, gc.kv, idx.to(DEV), wl.D_v, wl.softmax_scale,
+                                      kv_scale=gc.kv_scale, kv_rope=gc.kv_rope)
     for t in (0, 2, 3):
         assert torch.allclose(out2[t].float(), torch.ones_like(out2[t].float()), atol=1e-2)
 
