@@ -23,7 +23,8 @@ The JSON line also carries: the roofline of the dominant kernel (per-kernel CUDA
 from a second timed loop that issues the three C-ABI calls separately on one stream), the
 end-to-end throughput through the C ABI with host buffers (H2D of the step's query inputs and
 D2H of its output inside the timed region), the oracle timed on a bounded sample on the host
-cores, and the SM clocks sampled during the timed region.
+cores, the SM clocks sampled during the timed region, and (one GPU) "other_workloads": the FP8
+decode batch, the bf16 causal prefill and the KV quantizer, each with its roofline fraction.
 
 --impl reference runs the float64 CPU oracle (the only reference implementation of this path)
 on the same workload, one query row per step, and prints the same JSON line with
@@ -197,6 +198,103 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
+def _timed(fn, reps, flush_l2, main):
+    """Median of `reps` CUDA-event timings (ms) of fn() on `main`, L2 flushed before each."""
+    ts = []
+    for _ in range(reps):
+        flush_l2()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(main)
+        fn()
+        b.record(main)
+        torch.cuda.synchronize()
+        ts.append(a.elapsed_time(b))
+    return statistics.median(ts)
+
+
+def secondary(dev, flush_l2, main, peaks, reps):
+    """The path's other workloads, each measured once per bench run (rank 0, one GPU): the FP8
+    decode batch, the bf16 causal prefill and the KV-cache quantizer.  Each entry gives tokens/s
+    and the fraction of the bound that applies to it (HBM bytes, or bf16 tensor flops for
+    prefill; algorithmic counts from the shapes)."""
+    import sparse_index_attention_b200 as hsa
+    out = {}
+    hbm = peaks["hbm_gbs"] * 1e9
+
+    # FP8 decode: 128 sequences x 65536 keys, FP8 index keys and FP8 latent cache
+    wl = workloads.make("decode_fp8", dev)
+    k8, ks = hsa.hsa_quantize_index(wl.k_I, wl.D_I)
+    kv8, kvs, rope = hsa.hsa_quantize_kv(wl.kv, wl.D_v, wl.D_v)
+    ks, kvs = ks.view(-1), kvs.view(-1)
+    seq = hsa.PagedSeq(wl.seq_lens, wl.block_table, wl.page_size, wl.num_pages, wl.q_seq, wl.q_pos,
+                       q_run=wl.q_run)
+    sc = torch.empty((wl.T_q, seq.max_seq_len), dtype=torch.float32, device=dev)
+    idx = torch.empty((wl.T_q, wl.K), dtype=torch.int32, device=dev)
+    o = torch.empty((wl.T_q, wl.H, wl.D_v), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((wl.T_q, wl.H), dtype=torch.float32, device=dev)
+    ws = torch.empty(max(1, hsa.hsa_fused_decode_workspace_size(seq, wl.q, kv8, wl.D_v, wl.K)),
+                     dtype=torch.uint8, device=dev)
+
+    def fp8_step():
+        hsa.hsa_fused_decode(seq, wl.q_I, wl.w, k8, ks, wl.q, kv8, kvs, rope, wl.K, wl.D_v,
+                             wl.softmax_scale, scores=sc, idx=idx, out=o, lse=lse, ws=ws, stream=main)
+    for _ in range(3):
+        fp8_step()
+    ms = _timed(fp8_step, reps, flush_l2, main)
+    n = (wl.q_pos.long() + 1).cpu()
+    sel = int(torch.clamp(n, max=wl.K).sum())
+    byt = int(n.sum()) * (wl.D_I + 4 + 4) + sel * (wl.D_v + 4 + 2 * (wl.D_qk - wl.D_v)) + \
+        wl.T_q * wl.H * (wl.D_qk + wl.D_v) * 2 + wl.T_q * wl.H_I * (wl.D_I * 2 + 4)
+    out["decode_fp8"] = {"workload": "128 sequences x 65536 keys, FP8 index keys (fp32 scale per key), "
+                                     "FP8 latent (fp32 scale per token) + bf16 rope, Top-2048, 128 heads",
+                         "ms_per_step": round(ms, 4), "value": wl.T_q / (ms * 1e-3), "unit": UNIT,
+                         "bound": "hbm", "bytes": byt,
+                         "frac": round(byt / (ms * 1e-3) / hbm, 4)}
+    # KV-cache quantizer on the same cache (8.4 M rows): read 1152 B, write 512 + 4 + 128 B per row
+    nrow = wl.kv.shape[0]
+
+    def quant():
+        hsa.hsa_quantize_kv(wl.kv, wl.D_v, wl.D_v, codes=kv8, scales=kvs.view(-1, 1), rope_cache=rope,
+                            stream=main)
+    quant()
+    ms = _timed(quant, reps, flush_l2, main)
+    byt = nrow * (wl.D_qk * 2 + wl.D_v + 4 + 2 * (wl.D_qk - wl.D_v))
+    out["quantize_kv"] = {"workload": f"{nrow} cache rows of 512 latent + 64 rope bf16",
+                          "ms": round(ms, 4), "value": nrow / (ms * 1e-3), "unit": "rows/s",
+                          "bound": "hbm", "bytes": byt, "frac": round(byt / (ms * 1e-3) / hbm, 4)}
+    del wl, k8, ks, kv8, kvs, rope, sc, idx, o, lse, ws, seq
+    torch.cuda.empty_cache()
+
+    # bf16 causal prefill: one sequence of 16384 tokens, every token a query, 4 query chunks of
+    # 4096 issued in zigzag pairs on two streams
+    wl = workloads.make("prefill_bf16", dev)
+    seq = hsa.PagedSeq(wl.seq_lens, wl.block_table, wl.page_size, wl.num_pages, wl.q_seq, wl.q_pos,
+                       q_run=wl.q_run)
+    chunks = workloads.zigzag_chunks(wl.T_q, 4)
+    o = torch.empty((wl.T_q, wl.H, wl.D_v), dtype=torch.bfloat16, device=dev)
+    idx = torch.empty((wl.T_q, wl.K), dtype=torch.int32, device=dev)
+    streams = (torch.cuda.Stream(), torch.cuda.Stream())
+
+    def prefill():
+        hsa.hsa_prefill_chunked(seq, wl.q_I, wl.w, wl.k_I, None, wl.q, wl.kv, None, None, wl.K,
+                                wl.D_v, wl.softmax_scale, chunks, out=o, lse=False, idx=idx,
+                                streams=streams)
+    prefill()
+    ms = _timed(prefill, max(2, reps // 4), flush_l2, main)
+    n = (wl.q_pos.long() + 1).cpu()
+    flops = int(n.sum()) * wl.H_I * wl.D_I * 2 + int(torch.clamp(n, max=wl.K).sum()) * wl.H * (wl.D_qk + wl.D_v) * 2
+    peak = peaks["bf16_tflops_sustained"] * 1e12
+    out["prefill_bf16"] = {"workload": "one sequence of 16384 tokens, every token a query, Top-2048, "
+                                       "4 chunks of 4096 in zigzag pairs",
+                           "ms_per_step": round(ms, 3), "value": wl.T_q / (ms * 1e-3), "unit": UNIT,
+                           "bound": "tensor", "flops": flops,
+                           "frac": round(flops / (ms * 1e-3) / peak, 4),
+                           "peak": "bf16_tflops_sustained (MEASURED_PEAKS.json)"}
+    del wl, seq, o, idx
+    torch.cuda.empty_cache()
+    return out
+
+
 def run_ours(args, rank, world, local_rank):
     import sparse_index_attention_b200 as hsa
     dist = None
@@ -347,6 +445,10 @@ def run_ours(args, rank, world, local_rank):
            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e_steps,
            "note": "L2 not flushed between end-to-end steps"}
 
+    other = None
+    if rank == 0 and world == 1 and not args.no_secondary:
+        other = secondary(dev, flush_l2, main, load_peaks(), reps=max(3, min(args.steps, 10)))
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         rows = list(range(args.cpu_rows))
@@ -366,7 +468,7 @@ def run_ours(args, rank, world, local_rank):
                 "roofline": roofline, "stages": stages,
                 "two_stream": {"ms_per_step": round(two_ms, 4),
                                "value": world * wl.T_q / (two_ms * 1e-3), "unit": UNIT},
-                "cpu_baseline": cpu, "e2e": e2e,
+                "cpu_baseline": cpu, "e2e": e2e, "other_workloads": other,
                 "gpu_launches": launches, "clocks": clocks.summary(),
                 "wall_s_timed_region": round(wall, 3)}
         print(json.dumps(line), flush=True)
@@ -382,6 +484,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-rows", type=int, default=16, help="query rows for the oracle baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-secondary", action="store_true",
+                    help="skip the FP8 decode, prefill and quantizer measurements")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
