@@ -198,6 +198,28 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
+def rank_ops(dist, dev):
+    """(barrier, max_over_ranks) over the process group `dist` (the torch.distributed module after
+    init_process_group, or None for one process).  Every rank calls both at the same points."""
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    def max_over_ranks(x: float) -> float:
+        if dist is None:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+    return barrier, max_over_ranks
+
+
+def replica_throughput(world: int, rows_per_step: int, steps: int, t_ms_max: float) -> float:
+    """Whole-job rows/s of `world` replicas that each ran `steps` steps of `rows_per_step` query
+    rows, from the slowest rank's time (ms)."""
+    return world * rows_per_step * steps / (t_ms_max * 1e-3)
+
+
 def _timed(fn, reps, flush_l2, main):
     """Median of `reps` CUDA-event timings (ms) of fn() on `main`, L2 flushed before each."""
     ts = []
@@ -329,16 +351,7 @@ def run_ours(args, rank, world, local_rank):
                              out=out if out_t is None else out_t, lse=lse, ws=ws,
                              stream=main, aux_stream=aux_stream)
 
-    def barrier():
-        if dist is not None:
-            dist.barrier()
-
-    def max_over_ranks(x: float) -> float:
-        if dist is None:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    barrier, max_over_ranks = rank_ops(dist, dev)
 
     for _ in range(args.warmup):
         step()
@@ -363,7 +376,7 @@ def run_ours(args, rank, world, local_rank):
     launches = hsa.hsa_launch_count() - launches0
     t_ms = sum(s.elapsed_time(e) for s, e in zip(starts, ends))
     t_ms = max_over_ranks(t_ms)
-    value = world * wl.T_q * args.steps / (t_ms * 1e-3)
+    value = replica_throughput(world, wl.T_q, args.steps, t_ms)
 
     # ---- the same step on two streams (hsa_fused_decode with an auxiliary stream)
     reps2 = max(3, min(args.steps, 50))
