@@ -337,19 +337,25 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
             }
         } else if (kFp8) {
             // ------------------------------------------------------------ FP8 -> bf16 converters
-            // thread r widens key row r of the staging tile (128 codes) into the two 64-column
-            // swizzled halves of the bf16 tile the MMA reads (e4m3 -> f16 -> bf16 is exact)
-            const int r = tid - 192;  // 0..127
+            // eight lanes widen one key row of the staging tile (16 codes each), four rows per warp
+            // instruction, into the two 64-column swizzled halves of the bf16 tile the MMA reads
+            // (e4m3 -> f16 -> bf16 is exact); a row's eight lanes read 128 contiguous bytes, so
+            // the staging reads are free of bank conflicts
+            const int cw = (tid - 192) >> 5;           // converter warp 0..3: rows 32cw..32cw+31
+            const int c = lane & 7;                    // 16-code chunk of the row
+            const int half = c >> 2;                   // which 64-column half it lands in
+            const int chunk = (c & 3) * 2;             // first of its two 16-byte chunks there
             uint32_t stage = 0, phase = 0;
             uint32_t n = 0;
             for (int64_t f = f_begin; f < f_end; ++f, ++n) {
                 if (!tc::mbar_wait(&raw_full[n & 3], (n >> 2) & 1, abort_flag)) break;
                 if (!tc::mbar_wait(&empty[stage], phase ^ 1, abort_flag)) break;
-                const uint8_t* src = raw + (size_t)(n & 3) * (kBM * kDI) + (size_t)r * 128;
-                uint8_t* dst = tiles + (size_t)stage * kTileBytes + (size_t)r * 128;
-#pragma unroll
-                for (int c = 0; c < 8; ++c) {               // 16 codes -> 32 bytes of bf16
-                    const uint4 in = *reinterpret_cast<const uint4*>(src + c * 16);
+                const uint8_t* src = raw + (size_t)(n & 3) * (kBM * kDI);
+                uint8_t* dst = tiles + (size_t)stage * kTileBytes + half * kHalfBytes;
+#pragma unroll 2
+                for (int i = 0; i < 8; ++i) {
+                    const int r = 32 * cw + 4 * i + (lane >> 3);
+                    const uint4 in = *reinterpret_cast<const uint4*>(src + r * 128 + c * 16);
                     const uint32_t words[4] = {in.x, in.y, in.z, in.w};
                     uint32_t outw[8];
 #pragma unroll
@@ -363,12 +369,10 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
                             outw[q * 2 + hlf] = *reinterpret_cast<const uint32_t*>(&b2);
                         }
                     }
-                    const int half = c >> 2;                 // which 64-column half
-                    const int chunk = (c & 3) * 2;           // 16-byte chunk within the 128-byte row
-                    uint8_t* hbase = dst + half * kHalfBytes;
-                    *reinterpret_cast<uint4*>(hbase + (((chunk) ^ (r & 7)) * 16)) =
+                    uint8_t* rbase = dst + r * 128;
+                    *reinterpret_cast<uint4*>(rbase + ((chunk ^ (r & 7)) * 16)) =
                         make_uint4(outw[0], outw[1], outw[2], outw[3]);
-                    *reinterpret_cast<uint4*>(hbase + (((chunk + 1) ^ (r & 7)) * 16)) =
+                    *reinterpret_cast<uint4*>(rbase + (((chunk + 1) ^ (r & 7)) * 16)) =
                         make_uint4(outw[4], outw[5], outw[6], outw[7]);
                 }
                 tc::fence_async_smem();

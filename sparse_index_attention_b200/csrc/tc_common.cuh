@@ -100,6 +100,15 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, u
 
 // 2D gather of four rows (y0..y3) of one box width at column x; the tensor map's box is one
 // row high.  The four rows land consecutively in shared memory.
+// Untiled bulk copy global -> shared of `bytes` (both addresses 16-byte aligned, bytes a multiple
+// of 16) that completes that many bytes of the mbarrier's transaction count.
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+        ::"r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar))
+        : "memory");
+}
+
 __device__ __forceinline__ void tma_gather4(void* dst, const CUtensorMap* map, uint64_t* bar,
                                             int32_t x, int32_t y0, int32_t y1, int32_t y2,
                                             int32_t y3) {

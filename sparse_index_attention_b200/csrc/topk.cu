@@ -26,6 +26,7 @@
 #include <algorithm>
 
 #include "kernels.h"
+#include "tc_common.cuh"
 
 namespace hsa {
 
@@ -176,7 +177,8 @@ topk_kernel(SeqView v, const float* __restrict__ scores, int64_t ld, int K, int 
     uint32_t* misc = sm + kBins + 2 * kWarps;                     // [16]
     uint32_t* cand_key = misc + 16;                               // [cand_cap]; first the sample
     uint32_t* cand_pos = cand_key + cand_cap;                     // [cand_cap]
-    uint32_t* keys = cand_pos + cand_cap;                         // [n] when staged
+    uint32_t* keys_raw = cand_pos + cand_cap;                     // [n + 4] when staged
+    uint32_t* keys = keys_raw;           // staged keys: key i of the row at keys[i]
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int t = blockIdx.x;
     const RowInfo r = load_row(v, t);
@@ -193,37 +195,38 @@ topk_kernel(SeqView v, const float* __restrict__ scores, int64_t ld, int K, int 
     auto key_at = [&](int i) -> uint32_t { return kStaged ? keys[i] : score_key(__ldg(src + i)); };
 
     if (kStaged) {
-        const bool vec = (reinterpret_cast<uintptr_t>(src) & 15u) == 0u;
-        constexpr int kU = 8;
-#pragma unroll 1
-        for (int base = 0; base < n; base += kThreads * 4 * kU) {
-            float4 f[kU];
-#pragma unroll
-            for (int a = 0; a < kU; ++a) {
-                const int i = base + (a * kThreads + tid) * 4;
-                if (vec && i + 3 < n) {
-                    f[a] = __ldg(reinterpret_cast<const float4*>(src + i));
-                } else {
-                    f[a].x = i + 0 < n ? __ldg(src + i + 0) : 0.f;
-                    f[a].y = i + 1 < n ? __ldg(src + i + 1) : 0.f;
-                    f[a].z = i + 2 < n ? __ldg(src + i + 2) : 0.f;
-                    f[a].w = i + 3 < n ? __ldg(src + i + 3) : 0.f;
-                }
-            }
-#pragma unroll
-            for (int a = 0; a < kU; ++a) {
-                const int i = base + (a * kThreads + tid) * 4;
-                const uint4 u = make_uint4(score_key(f[a].x), score_key(f[a].y), score_key(f[a].z),
-                                           score_key(f[a].w));
-                if (i + 3 < n) {
-                    *reinterpret_cast<uint4*>(keys + i) = u;
-                } else {
-                    if (i + 0 < n) keys[i + 0] = u.x;
-                    if (i + 1 < n) keys[i + 1] = u.y;
-                    if (i + 2 < n) keys[i + 2] = u.z;
-                }
+        // the row's 16-byte-aligned body arrives by one bulk copy (the copy engine streams a
+        // contiguous row much faster than per-thread loads from L2), the unaligned tail by plain
+        // loads; then every thread turns its share of the scores into keys in place
+        const uintptr_t a0 = reinterpret_cast<uintptr_t>(src) & ~uintptr_t(15);
+        const uintptr_t a1 = reinterpret_cast<uintptr_t>(src + n) & ~uintptr_t(15);
+        const int head = (int)((reinterpret_cast<uintptr_t>(src) - a0) >> 2);   // 0..3 floats
+        keys = keys_raw + head;          // element i of the row lands at keys[i]
+        uint64_t* bar = reinterpret_cast<uint64_t*>(misc + 10);
+        volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 12);
+        const uint32_t bytes = (uint32_t)(a1 - a0);
+        if (tid == 0) {
+            *abort_flag = 0;
+            tc::mbar_init(bar, 1);
+            tc::fence_barrier_init();
+        }
+        __syncthreads();
+        if (tid == 0) {
+            if (bytes > 0) {
+                tc::mbar_arrive_expect_tx(bar, bytes);
+                tc::bulk_load(keys_raw, reinterpret_cast<const void*>(a0), bytes, bar);
+            } else {
+                tc::mbar_arrive(bar);
             }
         }
+        const int body = max(0, (int)(bytes >> 2) - head);   // row elements the copy covers
+        for (int i = body + tid; i < n; i += kThreads) keys[i] = __float_as_uint(__ldg(src + i));
+        const bool landed = tc::mbar_wait(bar, 0, abort_flag);
+        if (!__syncthreads_and(landed)) {   // the copy never completed: report, skip the row
+            if (tid == 0) flag_status(v, HSA_DEV_TIMEOUT);
+            return;
+        }
+        for (int i = tid; i < n; i += kThreads) keys[i] = score_key(__uint_as_float(keys[i]));
     }
     __syncthreads();
 
@@ -313,7 +316,7 @@ cudaError_t launch_topk(const SeqView& seq, int32_t max_seq_len, const float* sc
                         int32_t K, int32_t* idx, cudaStream_t st) {
     if (seq.T_q == 0) return cudaSuccess;
     const bool staged = max_seq_len <= kSmemKeys;
-    const int staged_words = staged ? ((max_seq_len + 3) & ~3) : 0;
+    const int staged_words = staged ? ((max_seq_len + 3) & ~3) + 4 : 0;   // + up to 3 floats of head
     // candidates (key and position) fill the rest; always room for the sample
     const int cand_cap = ((kMaxSmem / 4 - kFixedWords - staged_words) / 2) & ~3;
     const size_t smem = sizeof(uint32_t) * ((size_t)kFixedWords + 2 * (size_t)cand_cap + staged_words);
