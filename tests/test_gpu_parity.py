@@ -80,6 +80,36 @@ def test_index_score_integer_inputs_bit_exact():
         assert np.array_equal(got[t, :n].astype(np.float64), ref[t, :n]), t
 
 
+def test_index_score_fp8_every_code_bit_exact():
+    """Every finite E4M3 code through the FP8 key path: key s holds one code in all 128 dims, and
+    two index heads read dim 0 with q = +1 and -1 and weights +1 and -1, so the score is exactly
+    decode(code) x scale (scales are powers of two).  Pins the kernel's widening of the codes,
+    subnormals and signed zero included, bit for bit against the E4M3 definition."""
+    wl = workloads.make("decode_fp8", DEV, B=1, L=1024)
+    slots = wl.num_pages * wl.page_size
+    code_of_slot = torch.arange(slots, dtype=torch.int64) % 256
+    code_of_slot[(code_of_slot & 0x7F) == 0x7F] = 0           # NaN codes are outside the contract
+    k8 = code_of_slot.to(torch.uint8)[:, None].expand(slots, wl.D_I).contiguous().to(DEV)
+    scale = torch.exp2(-(torch.arange(slots) % 5).float()).to(DEV)
+    q = torch.zeros((1, wl.H_I, wl.D_I), dtype=torch.bfloat16)
+    q[0, 0, 0], q[0, 1, 0] = 1.0, -1.0
+    w = torch.zeros((1, wl.H_I), dtype=torch.float32)
+    w[0, 0], w[0, 1] = 1.0, -1.0
+    seq = hsa.PagedSeq(wl.seq_lens, wl.block_table, wl.page_size, wl.num_pages,
+                       wl.q_seq[:1], wl.q_pos[:1], max_seq_len=int(wl.seq_lens.max()),
+                       status=torch.zeros(1, dtype=torch.int32, device=DEV))
+    sc = hsa.hsa_index_score(seq, q.to(DEV), w.to(DEV), k8, scale)
+    check_status(seq)
+    n = int(wl.q_pos[0]) + 1
+    bt = wl.block_table[0].cpu().long()
+    pos = torch.arange(n)
+    slot = bt[pos // wl.page_size] * wl.page_size + pos % wl.page_size
+    codes = code_of_slot[slot].numpy().astype(np.uint8)
+    ref = (oracle.e4m3_decode(codes) * scale.cpu()[slot].double().numpy()).astype(np.float32)
+    assert len(set(codes.tolist())) == 254                   # every finite code is exercised
+    assert np.array_equal(sc[0, :n].cpu().numpy(), ref)
+
+
 def test_index_score_paging_invariance_bitwise():
     wl = workloads.make("decode_bf16", DEV, B=4, L_min=300, L_max=1000)
     base = hsa.hsa_index_score(paged_seq(wl), wl.q_I, wl.w, wl.k_I)
