@@ -197,7 +197,10 @@ topk_kernel(SeqView v, const float* __restrict__ scores, int64_t ld, int K, int 
     if (kStaged) {
         // the row's 16-byte-aligned body arrives by one bulk copy (the copy engine streams a
         // contiguous row much faster than per-thread loads from L2), the unaligned tail by plain
-        // loads; then every thread turns its share of the scores into keys in place
+        // loads; then every thread turns its share of the scores into keys in place.  The copy
+        // starts at the 16-byte boundary at or below the row (up to three floats of the previous
+        // row, never before the allocation, which is at least 16-byte aligned) and ends at or
+        // below the row's end.
         const uintptr_t a0 = reinterpret_cast<uintptr_t>(src) & ~uintptr_t(15);
         const uintptr_t a1 = reinterpret_cast<uintptr_t>(src + n) & ~uintptr_t(15);
         const int head = (int)((reinterpret_cast<uintptr_t>(src) - a0) >> 2);   // 0..3 floats
