@@ -135,8 +135,11 @@ HSA_API hsa_status_t hsa_topk(const hsa_paged_seq_t* seq, const float* scores, i
  * by the rope part (D_qk - D_v values).
  *   q        device [T_q, H, D_qk], q_dtype F32 or BF16
  *   kv       kv_dtype F32 / BF16: device [slots, D_qk] packed latent || rope; kv_rope = NULL
- *            kv_dtype E4M3: device uint8 [slots, D_v] latent codes, kv_scale fp32 [slots]
- *            (one per token), kv_rope BF16 [slots, D_qk - D_v]
+ *            kv_dtype E4M3: device uint8 [slots, D_v] latent codes, kv_scale fp32
+ *            [slots, D_v / kv_scale_group] (one scale per kv_scale_group consecutive latent dims
+ *            of a token: D_v = one per token, 128 = the pages' tile; a multiple of 16 that
+ *            divides D_v), kv_rope BF16 [slots, D_qk - D_v]; F32 / BF16 caches: kv_scale_group
+ *            is ignored
  *   idx      device int32 [T_q, K]: positions in [0, q_pos[t]] or -1
  *   out      device [T_q, H, D_v] of out_dtype (F32 or BF16)
  *   lse      device fp32 [T_q, H] or NULL
@@ -149,8 +152,9 @@ HSA_API size_t hsa_sparse_mla_workspace_size(const hsa_paged_seq_t* seq, int32_t
                                      int32_t D_v, int32_t K);
 HSA_API hsa_status_t hsa_sparse_mla_attn(const hsa_paged_seq_t* seq, const void* q, hsa_dtype_t q_dtype,
                                  int32_t H, int32_t D_qk, int32_t D_v, const void* kv,
-                                 hsa_dtype_t kv_dtype, const float* kv_scale, const void* kv_rope,
-                                 const int32_t* idx, int32_t K, float softmax_scale, void* out,
+                                 hsa_dtype_t kv_dtype, const float* kv_scale, int32_t kv_scale_group,
+                                 const void* kv_rope, const int32_t* idx, int32_t K,
+                                 float softmax_scale, void* out,
                                  hsa_dtype_t out_dtype, float* lse, void* ws, size_t ws_bytes,
                                  void* stream);
 
@@ -171,7 +175,8 @@ typedef struct hsa_index_args {
 
 typedef struct hsa_attn_args {
     const void* q; hsa_dtype_t q_dtype; int32_t H; int32_t D_qk; int32_t D_v;
-    const void* kv; hsa_dtype_t kv_dtype; const float* kv_scale; const void* kv_rope;
+    const void* kv; hsa_dtype_t kv_dtype; const float* kv_scale; int32_t kv_scale_group;
+    const void* kv_rope;
     float softmax_scale; void* out; hsa_dtype_t out_dtype; float* lse;
 } hsa_attn_args_t;
 

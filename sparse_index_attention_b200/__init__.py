@@ -41,7 +41,8 @@ class hsa_index_args_t(ctypes.Structure):
 
 class hsa_attn_args_t(ctypes.Structure):
     _fields_ = [("q", _P), ("q_dtype", ctypes.c_int), ("H", _i32), ("D_qk", _i32), ("D_v", _i32),
-                ("kv", _P), ("kv_dtype", ctypes.c_int), ("kv_scale", _P), ("kv_rope", _P),
+                ("kv", _P), ("kv_dtype", ctypes.c_int), ("kv_scale", _P), ("kv_scale_group", _i32),
+                ("kv_rope", _P),
                 ("softmax_scale", _f32), ("out", _P), ("out_dtype", ctypes.c_int), ("lse", _P)]
 
 
@@ -51,7 +52,7 @@ SYMBOLS = {
     "hsa_topk": (ctypes.c_int, [_P, _P, _i64, _i32, _P, _P]),
     "hsa_sparse_mla_workspace_size": (_sz, [_P, _i32, _i32, _i32, _i32]),
     "hsa_sparse_mla_attn": (ctypes.c_int, [_P, _P, ctypes.c_int, _i32, _i32, _i32, _P, ctypes.c_int,
-                                           _P, _P, _P, _i32, _f32, _P, ctypes.c_int, _P, _P, _sz,
+                                           _P, _i32, _P, _P, _i32, _f32, _P, ctypes.c_int, _P, _P, _sz,
                                            _P]),
     "hsa_fused_decode_workspace_size": (_sz, [_P, _P, _i32]),
     "hsa_fused_decode": (ctypes.c_int, [_P, _P, _P, _i32, _P, _i64, _P, _P, _sz, _P, _P]),
@@ -185,10 +186,21 @@ def _workspace(nbytes: int, device, ws):
     return torch.empty(max(nbytes, 1), dtype=torch.uint8, device=device)
 
 
+def _kv_group(kv, kv_scale, D_v: int) -> int:
+    """Latent dims per KV scale: an FP8 cache's kv_scale holds D_v / group scales per slot."""
+    if kv_scale is None or kv.dtype != torch.uint8:
+        return D_v
+    per_slot = kv_scale.numel() // kv.shape[0]
+    if per_slot < 1 or kv_scale.numel() != per_slot * kv.shape[0] or D_v % per_slot:
+        raise ValueError(f"kv_scale with {kv_scale.numel()} entries does not fit {kv.shape[0]} slots")
+    return D_v // per_slot
+
+
 def hsa_sparse_mla_attn(seq: PagedSeq, q, kv, idx, D_v: int, softmax_scale: float, kv_scale=None,
                         kv_rope=None, out=None, out_dtype=None, lse=True, ws=None, stream=None):
     """Returns (out [T_q, H, D_v], lse [T_q, H] or None).  kv is the packed [slots, D_qk] cache
-    (fp32/bf16) or the uint8 latent codes [slots, D_v] with kv_scale and kv_rope."""
+    (fp32/bf16) or the uint8 latent codes [slots, D_v] with kv_scale ([slots] or
+    [slots, D_v / group]: one scale per token or per group of latent dims) and kv_rope."""
     T_q, H, D_qk = q.shape
     K = idx.shape[1]
     if out is None:
@@ -200,7 +212,8 @@ def hsa_sparse_mla_attn(seq: PagedSeq, q, kv, idx, D_v: int, softmax_scale: floa
     need = hsa_sparse_mla_workspace_size(seq, H, D_qk, D_v, K)
     ws = _workspace(need, q.device, ws)
     _check(lib().hsa_sparse_mla_attn(seq.ref, _ptr(q), _dtype(q), H, D_qk, D_v, _ptr(kv), _dtype(kv),
-                                     _ptr(kv_scale), _ptr(kv_rope), _ptr(idx), K,
+                                     _ptr(kv_scale), _kv_group(kv, kv_scale, D_v), _ptr(kv_rope),
+                                     _ptr(idx), K,
                                      float(softmax_scale), _ptr(out), _dtype(out), _ptr(lse),
                                      _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
            "hsa_sparse_mla_attn")
@@ -210,12 +223,13 @@ def hsa_sparse_mla_attn(seq: PagedSeq, q, kv, idx, D_v: int, softmax_scale: floa
 def _attn_struct(q, kv, D_v, softmax_scale, kv_scale, kv_rope, out, lse):
     T_q, H, D_qk = q.shape
     return hsa_attn_args_t(_ptr(q), _dtype(q), H, D_qk, D_v, _ptr(kv), _dtype(kv), _ptr(kv_scale),
-                           _ptr(kv_rope), float(softmax_scale), _ptr(out), _dtype(out), _ptr(lse))
+                           _kv_group(kv, kv_scale, D_v), _ptr(kv_rope), float(softmax_scale), _ptr(out),
+                           _dtype(out), _ptr(lse))
 
 
 def hsa_fused_decode_workspace_size(seq: PagedSeq, q, kv, D_v: int, K: int) -> int:
     T_q, H, D_qk = q.shape
-    at = hsa_attn_args_t(None, _dtype(q), H, D_qk, D_v, None, _dtype(kv), None, None, 1.0, None,
+    at = hsa_attn_args_t(None, _dtype(q), H, D_qk, D_v, None, _dtype(kv), None, D_v, None, 1.0, None,
                          _dtype(q), None)
     return int(lib().hsa_fused_decode_workspace_size(seq.ref, ctypes.byref(at), K))
 

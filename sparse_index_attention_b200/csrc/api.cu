@@ -94,8 +94,8 @@ hsa_status_t check_index(const hsa_paged_seq_t* seq, const void* q_I, hsa_dtype_
 
 hsa_status_t check_attn(const hsa_paged_seq_t* seq, const void* q, hsa_dtype_t q_dtype, int32_t H,
                         int32_t D_qk, int32_t D_v, const void* kv, hsa_dtype_t kv_dtype,
-                        const float* kv_scale, const void* kv_rope, const int32_t* idx, int32_t K,
-                        const void* out, hsa_dtype_t out_dtype) {
+                        const float* kv_scale, int32_t kv_scale_group, const void* kv_rope,
+                        const int32_t* idx, int32_t K, const void* out, hsa_dtype_t out_dtype) {
     hsa_status_t st = check_seq(seq);
     if (st != HSA_OK) return st;
     HSA_REQUIRE(H >= 1 && H <= 1024, HSA_ERR_INVALID_ARG, "H = %d out of range", H);
@@ -113,6 +113,10 @@ hsa_status_t check_attn(const hsa_paged_seq_t* seq, const void* q, hsa_dtype_t q
         if (kv_dtype == HSA_E4M3) {
             HSA_REQUIRE(kv_scale && (kv_rope || D_qk == D_v), HSA_ERR_INVALID_ARG,
                         "E4M3 latent cache needs kv_scale and kv_rope");
+            HSA_REQUIRE(kv_scale_group >= 16 && kv_scale_group % 16 == 0 && D_v % kv_scale_group == 0,
+                        HSA_ERR_INVALID_ARG,
+                        "kv_scale_group = %d must be a multiple of 16 that divides D_v = %d",
+                        kv_scale_group, D_v);
         } else {
             HSA_REQUIRE(kv_rope == nullptr, HSA_ERR_INVALID_ARG,
                         "kv_rope must be NULL for a packed F32/BF16 cache");
@@ -165,6 +169,7 @@ hsa::SparseMlaArgs attn_args(const hsa_paged_seq_t* seq, const hsa_attn_args_t& 
     a.kv = at.kv;
     a.kv_dtype = at.kv_dtype;
     a.kv_scale = at.kv_scale;
+    a.kv_scale_group = at.kv_dtype == HSA_E4M3 ? at.kv_scale_group : at.D_v;
     a.kv_rope = at.kv_rope;
     a.idx = idx;
     a.K = K;
@@ -195,7 +200,7 @@ hsa_status_t run_attn(const hsa::SparseMlaArgs& a, cudaStream_t st) {
 
 hsa_attn_args_t make_attn(const void* q, hsa_dtype_t q_dtype, int32_t H, int32_t D_qk, int32_t D_v,
                           const void* kv, hsa_dtype_t kv_dtype, const float* kv_scale,
-                          const void* kv_rope, float softmax_scale, void* out,
+                          int32_t kv_scale_group, const void* kv_rope, float softmax_scale, void* out,
                           hsa_dtype_t out_dtype, float* lse) {
     hsa_attn_args_t a;
     a.q = q;
@@ -206,6 +211,7 @@ hsa_attn_args_t make_attn(const void* q, hsa_dtype_t q_dtype, int32_t H, int32_t
     a.kv = kv;
     a.kv_dtype = kv_dtype;
     a.kv_scale = kv_scale;
+    a.kv_scale_group = kv_scale_group;
     a.kv_rope = kv_rope;
     a.softmax_scale = softmax_scale;
     a.out = out;
@@ -238,7 +244,7 @@ const char* hsa_status_string(hsa_status_t s) {
 
 const char* hsa_last_error_message(void) { return g_last_error.c_str(); }
 
-int32_t hsa_version(void) { return 100; }
+int32_t hsa_version(void) { return 200; }
 
 hsa_status_t hsa_index_score(const hsa_paged_seq_t* seq, const void* q_I, hsa_dtype_t q_dtype,
                              const float* w, int32_t H_I, int32_t D_I, const void* k_cache,
@@ -273,21 +279,22 @@ size_t hsa_sparse_mla_workspace_size(const hsa_paged_seq_t* seq, int32_t H, int3
     if (seq == nullptr || seq->T_q <= 0) return 0;
     // the tensor-core kernel's need only depends on the shape, not on the pointers
     hsa_attn_args_t at = make_attn(nullptr, HSA_BF16, H, D_qk, D_v, nullptr, HSA_BF16, nullptr,
-                                   nullptr, 1.f, nullptr, HSA_BF16, nullptr);
+                                   D_v, nullptr, 1.f, nullptr, HSA_BF16, nullptr);
     return attn_ws_bytes(attn_args(seq, at, nullptr, K, nullptr, 0));
 }
 
 hsa_status_t hsa_sparse_mla_attn(const hsa_paged_seq_t* seq, const void* q, hsa_dtype_t q_dtype,
                                  int32_t H, int32_t D_qk, int32_t D_v, const void* kv,
-                                 hsa_dtype_t kv_dtype, const float* kv_scale, const void* kv_rope,
-                                 const int32_t* idx, int32_t K, float softmax_scale, void* out,
+                                 hsa_dtype_t kv_dtype, const float* kv_scale, int32_t kv_scale_group,
+                                 const void* kv_rope, const int32_t* idx, int32_t K,
+                                 float softmax_scale, void* out,
                                  hsa_dtype_t out_dtype, float* lse, void* ws, size_t ws_bytes,
                                  void* stream) {
     g_last_error.clear();
-    hsa_status_t st = check_attn(seq, q, q_dtype, H, D_qk, D_v, kv, kv_dtype, kv_scale, kv_rope,
+    hsa_status_t st = check_attn(seq, q, q_dtype, H, D_qk, D_v, kv, kv_dtype, kv_scale, kv_scale_group, kv_rope,
                                  idx, K, out, out_dtype);
     if (st != HSA_OK) return st;
-    hsa_attn_args_t at = make_attn(q, q_dtype, H, D_qk, D_v, kv, kv_dtype, kv_scale, kv_rope,
+    hsa_attn_args_t at = make_attn(q, q_dtype, H, D_qk, D_v, kv, kv_dtype, kv_scale, kv_scale_group, kv_rope,
                                    softmax_scale, out, out_dtype, lse);
     return run_attn(attn_args(seq, at, idx, K, ws, ws_bytes), (cudaStream_t)stream);
 }
@@ -317,7 +324,7 @@ hsa_status_t hsa_fused_decode(const hsa_paged_seq_t* seq, const hsa_index_args_t
                                   ix->k_dtype, ix->k_scale, scores, ld_scores);
     if (st != HSA_OK) return st;
     st = check_attn(seq, at->q, at->q_dtype, at->H, at->D_qk, at->D_v, at->kv, at->kv_dtype,
-                    at->kv_scale, at->kv_rope, idx, K, at->out, at->out_dtype);
+                    at->kv_scale, at->kv_scale_group, at->kv_rope, idx, K, at->out, at->out_dtype);
     if (st != HSA_OK) return st;
     HSA_REQUIRE(K >= 1 && K <= 65536, HSA_ERR_INVALID_ARG, "K = %d out of range", K);
     if (seq->T_q == 0) return HSA_OK;

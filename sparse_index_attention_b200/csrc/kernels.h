@@ -42,6 +42,7 @@ struct SparseMlaArgs {
     const void* kv;
     hsa_dtype_t kv_dtype;
     const float* kv_scale;
+    int32_t kv_scale_group;   // E4M3: latent dims per scale (divides D_v); else D_v
     const void* kv_rope;
     const int32_t* idx;
     int32_t K;

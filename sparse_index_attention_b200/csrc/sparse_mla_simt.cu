@@ -19,7 +19,7 @@ constexpr int kRows = 32;  // kHeads * kRows == kThreads: one logit per thread p
 template <typename QT, int KVT, typename OT>  // KVT: 0 fp32 packed, 1 bf16 packed, 2 e4m3 + bf16 rope
 __global__ void __launch_bounds__(kThreads)
 sparse_mla_simt_kernel(SeqView v, const QT* __restrict__ q, int H, int D_qk, int D_v,
-                       const void* __restrict__ kv, const float* __restrict__ kv_scale,
+                       const void* __restrict__ kv, const float* __restrict__ kv_scale, int kv_group,
                        const __nv_bfloat16* __restrict__ kv_rope, const int32_t* __restrict__ idx,
                        int K, float softmax_scale, OT* __restrict__ out, float* __restrict__ lse) {
     extern __shared__ float smem[];
@@ -77,7 +77,8 @@ sparse_mla_simt_kernel(SeqView v, const QT* __restrict__ q, int H, int D_qk, int
                 } else if (KVT == 1) {
                     x = __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(kv)[s * D_qk + d]);
                 } else {
-                    x = d < D_v ? e4m3_to_f32(reinterpret_cast<const uint8_t*>(kv)[s * D_v + d]) * kv_scale[s]
+                    x = d < D_v ? e4m3_to_f32(reinterpret_cast<const uint8_t*>(kv)[s * D_v + d]) *
+                                      kv_scale[s * (D_v / kv_group) + d / kv_group]
                                 : __bfloat162float(kv_rope[s * D_rope + (d - D_v)]);
                 }
             }
@@ -152,7 +153,7 @@ cudaError_t launch_t(const SparseMlaArgs& a, cudaStream_t st) {
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     k<<<grid, kThreads, smem, st>>>(a.seq, reinterpret_cast<const QT*>(a.q), a.H, a.D_qk, a.D_v,
-                                    a.kv, a.kv_scale,
+                                    a.kv, a.kv_scale, a.kv_scale_group,
                                     reinterpret_cast<const __nv_bfloat16*>(a.kv_rope), a.idx, a.K,
                                     a.softmax_scale, reinterpret_cast<OT*>(a.out), a.lse);
     count_launch();

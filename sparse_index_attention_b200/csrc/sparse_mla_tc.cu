@@ -134,7 +134,7 @@ template <bool kFp8Kv>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 sparse_mla_tc_kernel(SeqView v,
                      const __nv_bfloat16* __restrict__ q, const uint8_t* __restrict__ kv_bytes,
-                     const float* __restrict__ kv_scale, const uint8_t* __restrict__ rope_bytes,
+                     const float* __restrict__ kv_scale, int kv_group, const uint8_t* __restrict__ rope_bytes,
                      int64_t rope_row_bytes, const int32_t* __restrict__ idx, int K,
                      float scale_log2, __nv_bfloat16* __restrict__ out, float* __restrict__ lse) {
     extern __shared__ uint8_t smem_raw[];
@@ -247,6 +247,8 @@ sparse_mla_tc_kernel(SeqView v,
                     // row, lane = 16 codes); widened to bf16 (code x row scale, rounded once) and
                     // stored as the two 16-byte chunks the swizzled stage expects
                     const int sub = lane >> 4, cl = lane & 15;
+                    // this lane's 16 codes lie in one scale group (groups are multiples of 16)
+                    const int n_groups = kDv / kv_group, my_group = (256 * (int)rank + 16 * cl) / kv_group;
                     uint4 raw[8];
                     float scl[8];
 #pragma unroll
@@ -254,7 +256,7 @@ sparse_mla_tc_kernel(SeqView v,
                         const int32_t sl = ts[2 * k2 + sub];
                         raw[k2] = sl < 0 ? make_uint4(0u, 0u, 0u, 0u)
                                          : __ldg(reinterpret_cast<const uint4*>(kv_bytes + (int64_t)sl * kKv8RowBytes + 256 * rank) + cl);
-                        scl[k2] = sl < 0 ? 0.f : __ldg(kv_scale + sl);
+                        scl[k2] = sl < 0 ? 0.f : __ldg(kv_scale + (int64_t)sl * n_groups + my_group);
                     }
 #pragma unroll
                     for (int k2 = 0; k2 < 8; ++k2) {
@@ -658,6 +660,8 @@ bool sparse_mla_tc_supported(const SparseMlaArgs& a) {
     if (a.q_dtype != HSA_BF16 || a.out_dtype != HSA_BF16) return false;
     if (a.kv_dtype != HSA_BF16 && a.kv_dtype != HSA_E4M3) return false;
     if (a.kv_dtype == HSA_E4M3 && (a.kv_scale == nullptr || a.kv_rope == nullptr)) return false;
+    if (a.kv_dtype == HSA_E4M3 && (a.kv_scale_group < 16 || a.kv_scale_group % 16 || kDv % a.kv_scale_group))
+        return false;
     if (a.H != kH || a.D_qk != kDqk || a.D_v != kDv) return false;
     if (!(a.softmax_scale > 0.f)) return false;   // the kernel takes tile maxima on unscaled S
     auto al = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; };
@@ -683,7 +687,8 @@ cudaError_t launch_sparse_mla_tc(const SparseMlaArgs& a, cudaStream_t st) {
     const uint8_t* rope = fp8 ? reinterpret_cast<const uint8_t*>(a.kv_rope) : kv + 2 * kDv;
     const int64_t rope_row = fp8 ? kRopeRowBytes : kKvRowBytes;
     e = launch_pdl(kern, dim3(2 * clusters), dim3(kThreads), kSmem, st, a.seq,
-                   reinterpret_cast<const __nv_bfloat16*>(a.q), kv, fp8 ? a.kv_scale : nullptr, rope, rope_row,
+                   reinterpret_cast<const __nv_bfloat16*>(a.q), kv, fp8 ? a.kv_scale : nullptr,
+                   fp8 ? a.kv_scale_group : kDv, rope, rope_row,
                    a.idx, a.K, scale_log2, reinterpret_cast<__nv_bfloat16*>(a.out), a.lse);
     return e != cudaSuccess ? e : cudaGetLastError();
 }

@@ -35,9 +35,10 @@ def oracle_paging(wl: workloads.Workload, rows=None) -> oracle.Paging:
 
 
 class GpuCaches:
-    """The caches the GPU path reads, written by the library's own quantizers when FP8."""
+    """The caches the GPU path reads, written by the library's own quantizers when FP8
+    (latent scales per token, or per `kv_group` latent dims)."""
 
-    def __init__(self, wl: workloads.Workload):
+    def __init__(self, wl: workloads.Workload, kv_group=None):
         self.k_scale = None
         self.kv_scale = None
         self.kv_rope = None
@@ -47,8 +48,8 @@ class GpuCaches:
         else:
             self.k = wl.k_I
         if wl.kv_fp8:
-            self.kv, sc, self.kv_rope = hsa.hsa_quantize_kv(wl.kv, wl.D_v, wl.D_v)
-            self.kv_scale = sc.view(-1)
+            self.kv, sc, self.kv_rope = hsa.hsa_quantize_kv(wl.kv, wl.D_v, kv_group or wl.D_v)
+            self.kv_scale = sc if kv_group else sc.view(-1)
         else:
             self.kv = wl.kv
 
@@ -56,7 +57,7 @@ class GpuCaches:
 class OracleCaches:
     """Exact values of the caches as the oracle reads them (its own quantizer for FP8)."""
 
-    def __init__(self, wl: workloads.Workload, need_kv: bool = True):
+    def __init__(self, wl: workloads.Workload, need_kv: bool = True, kv_group=None):
         if wl.index_fp8:
             codes, sc = oracle.quantize_rows(wl.k_I.float().cpu(), wl.D_I)
             self.k = oracle.dequantize_rows(codes, sc, wl.D_I)
@@ -65,8 +66,9 @@ class OracleCaches:
         if need_kv:
             kv = wl.kv.float().cpu().numpy().astype(np.float64)
             if wl.kv_fp8:
-                codes, sc = oracle.quantize_rows(wl.kv[:, :wl.D_v].float().cpu(), wl.D_v)
-                kv[:, :wl.D_v] = oracle.dequantize_rows(codes, sc, wl.D_v)
+                grp = kv_group or wl.D_v
+                codes, sc = oracle.quantize_rows(wl.kv[:, :wl.D_v].float().cpu(), grp)
+                kv[:, :wl.D_v] = oracle.dequantize_rows(codes, sc, grp)
             self.kv = kv
 
 

@@ -52,6 +52,13 @@ def test_validation_without_gpu():
     assert rc == hsa.HSA_ERR_INVALID_ARG                       # E4M3 keys without scales
     rc = L.hsa_quantize_index(fake, hsa.HSA_BF16, 10, 128, 48, None, 10, fake, fake, None)
     assert rc == hsa.HSA_ERR_INVALID_ARG                       # group does not divide D
+    # E4M3 latent cache: the scale group must be a multiple of 16 that divides D_v
+    for group, want in ((24, hsa.HSA_ERR_INVALID_ARG), (48, hsa.HSA_ERR_INVALID_ARG)):
+        rc = L.hsa_sparse_mla_attn(ctypes.byref(seq), fake, hsa.HSA_BF16, 8, 80, 64, fake, hsa.HSA_E4M3,
+                                   fake, group, fake, fake, 32, 0.1, fake, hsa.HSA_BF16, None, None, 0,
+                                   None)
+        assert rc == want, group
+        assert b"kv_scale_group" in L.hsa_last_error_message()
     # zero rows is a no-op, not an error
     empty = hsa.hsa_paged_seq_t(1, fake, fake, 4, 16, 4, 64, 0, None, None, 1, None)
     assert L.hsa_topk(ctypes.byref(empty), None, 64, 8, None, None) == hsa.HSA_OK

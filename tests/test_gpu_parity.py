@@ -180,8 +180,8 @@ def test_topk_launch_variants_bit_exact(T, ld, K, dist):
     assert np.array_equal(idx.cpu().numpy(), ref)
 
 
-def _attn_vs_oracle(wl, tol, idx=None):
-    gc = GpuCaches(wl)
+def _attn_vs_oracle(wl, tol, idx=None, kv_group=None):
+    gc = GpuCaches(wl, kv_group)
     seq = paged_seq(wl)
     if idx is None:
         idx = workloads.random_selection(wl.q_pos, wl.K, seed=wl.seed + 50)
@@ -189,7 +189,7 @@ def _attn_vs_oracle(wl, tol, idx=None):
     out, lse = hsa.hsa_sparse_mla_attn(seq, wl.q, gc.kv, idx_d, wl.D_v, wl.softmax_scale,
                                        kv_scale=gc.kv_scale, kv_rope=gc.kv_rope)
     check_status(seq)
-    oc = OracleCaches(wl)
+    oc = OracleCaches(wl, kv_group=kv_group)
     ref, rlse = oracle.sparse_mla(oracle_paging(wl), wl.q.cpu(), oc.kv, idx, wl.D_v, wl.softmax_scale)
     ok, worst = attn_close(out.float().cpu().numpy(), ref, tol)
     assert ok, (wl.name, worst)
@@ -208,6 +208,15 @@ def _attn_vs_oracle(wl, tol, idx=None):
 ])
 def test_sparse_mla_vs_oracle(name, kw, tol):
     _attn_vs_oracle(workloads.make(name, DEV, **kw), tol)
+
+
+@pytest.mark.parametrize("kv_group", [512, 128, 64])
+@pytest.mark.parametrize("H", [128, 16])
+def test_sparse_mla_fp8_scale_groups(kv_group, H):
+    """FP8 latent cache with one scale per token (512), per the pages' 128-dim tile, and per 64
+    dims, on the tensor-core kernel (128 heads) and the CUDA-core kernel (16 heads)."""
+    wl = workloads.make("decode_fp8", DEV, B=3, L=2500, H=H)
+    _attn_vs_oracle(wl, 6e-2, kv_group=kv_group)
 
 
 @pytest.mark.parametrize("name,kw,tol", [

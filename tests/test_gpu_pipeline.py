@@ -86,14 +86,15 @@ def test_pipeline_vs_oracle_small(name, kw):
     check_against_oracle(wl, list(range(wl.T_q)), sc, idx, out)
 
 
-@pytest.mark.parametrize("name,kw", [
-    ("tiny_decode_fp32", {}),
-    ("decode_bf16", dict(B=8, L_min=1500, L_max=5000)),
-    ("decode_fp8", dict(B=6, L=3000)),
+@pytest.mark.parametrize("name,kw,kv_group", [
+    ("tiny_decode_fp32", {}, None),
+    ("decode_bf16", dict(B=8, L_min=1500, L_max=5000), None),
+    ("decode_fp8", dict(B=6, L=3000), None),
+    ("decode_fp8", dict(B=6, L=3000), 128),
 ])
-def test_fused_equals_unfused_and_two_streams(name, kw):
+def test_fused_equals_unfused_and_two_streams(name, kw, kv_group):
     wl = workloads.make(name, DEV, **kw)
-    gc = GpuCaches(wl)
+    gc = GpuCaches(wl, kv_group)
     out1, lse1, idx1, sc1 = run_fused(wl, gc, aux=False)
     out2, lse2, idx2, sc2 = run_fused(wl, gc, aux=True)
     seq = paged_seq(wl)
