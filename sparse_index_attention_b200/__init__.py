@@ -262,6 +262,43 @@ def hsa_fused_decode(seq: PagedSeq, q_I, w, k_cache, k_scale, q, kv, kv_scale, k
     return out, lse, idx, scores
 
 
+class DecodeGraph:
+    """One hsa_fused_decode step captured as a CUDA graph (the decode step in "graph mode"):
+    replay() reruns the same kernels on the same buffers with a single graph launch and no
+    per-step host work in the library.  The graph reads the tensors given here: write the next
+    step's query rows into q_I, w and q (and the caches) before replay(); results land in
+    .out, .lse, .idx and .scores.  With aux=True the step uses the two-stream form."""
+
+    def __init__(self, seq: PagedSeq, q_I, w, k_cache, k_scale, q, kv, kv_scale, kv_rope, K: int,
+                 D_v: int, softmax_scale: float, aux: bool = False):
+        dev = q.device
+        T_q, H, _ = q.shape
+        self.scores = torch.empty((T_q, seq.max_seq_len), dtype=torch.float32, device=dev)
+        self.idx = torch.empty((T_q, K), dtype=torch.int32, device=dev)
+        self.out = torch.empty((T_q, H, D_v), dtype=q.dtype, device=dev)
+        self.lse = torch.empty((T_q, H), dtype=torch.float32, device=dev)
+        self.ws = _workspace(hsa_fused_decode_workspace_size(seq, q, kv, D_v, K), dev, None)
+        self._aux = torch.cuda.Stream(device=dev) if aux else None
+        args = (seq, q_I, w, k_cache, k_scale, q, kv, kv_scale, kv_rope, K, D_v, softmax_scale)
+        cap = torch.cuda.Stream(device=dev)
+
+        def step(stream):
+            hsa_fused_decode(*args, scores=self.scores, idx=self.idx, out=self.out, lse=self.lse,
+                             ws=self.ws, stream=stream, aux_stream=self._aux)
+        cap.wait_stream(torch.cuda.current_stream(dev))
+        with torch.cuda.stream(cap):
+            step(cap)                       # first call outside the capture (kernel attributes)
+        cap.synchronize()
+        self.graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.graph, stream=cap, capture_error_mode="relaxed"):
+            step(cap)
+        self._args = args                   # keep every captured tensor alive
+
+    def replay(self):
+        self.graph.replay()
+        return self.out, self.lse, self.idx, self.scores
+
+
 def hsa_quantize_index(src, group: int, slot_mapping=None, num_slots: Optional[int] = None,
                        codes=None, scales=None, stream=None):
     """Rows [n, D] -> (codes uint8 [slots, D], scales fp32 [slots, D/group])."""

@@ -122,3 +122,26 @@ def test_decode_bf16_full_size_sampled():
     assert torch.equal(idx, ref_sel)
     rows = [0, 17, 40, 63]
     check_against_oracle(wl, rows, sc, idx, out)
+
+
+@pytest.mark.parametrize("aux", [False, True])
+def test_decode_graph_replays_bitwise(aux):
+    """The fused decode step captured as a CUDA graph equals the direct call bitwise, and a
+    replay after new query rows are written into the captured inputs follows them."""
+    wl = workloads.make("decode_bf16", DEV, B=8, L_min=1500, L_max=5000)
+    gc = GpuCaches(wl)
+    seq = paged_seq(wl)
+    g = hsa.DecodeGraph(seq, wl.q_I, wl.w, gc.k, gc.k_scale, wl.q, gc.kv, gc.kv_scale, gc.kv_rope,
+                        wl.K, wl.D_v, wl.softmax_scale, aux=aux)
+    for it in range(2):
+        if it == 1:                                  # next step's queries, same buffers
+            wl.q.mul_(-1.0)
+            wl.q_I.copy_(torch.roll(wl.q_I, 1, dims=0))
+        out_g, lse_g, idx_g, _ = (t.clone() for t in g.replay())
+        torch.cuda.synchronize()
+        out_d, lse_d, idx_d, _ = hsa.hsa_fused_decode(seq, wl.q_I, wl.w, gc.k, gc.k_scale, wl.q, gc.kv,
+                                                      gc.kv_scale, gc.kv_rope, wl.K, wl.D_v,
+                                                      wl.softmax_scale)
+        torch.cuda.synchronize()
+        assert torch.equal(idx_g, idx_d) and torch.equal(out_g, out_d) and torch.equal(lse_g, lse_d)
+    check_status(seq)
