@@ -73,8 +73,8 @@ typedef enum hsa_dtype {
 /* Paged sequences and query rows.
  * Position s of sequence b lives in physical slot
  *     block_table[b * bt_stride + s / page_size] * page_size + s % page_size
- * of every paged cache ("reads from the paged K cache", first page, "Sparse Attention Pipeline
- * Optimization"; gather through the page table, third page, 3.1).  Query row t belongs to
+ * of every paged cache (the indexer reads keys straight out of the paged cache: first page,
+ * "Sparse Attention Pipeline Optimization"; gather through the page table, third page, 3.1).  Query row t belongs to
  * sequence q_seq[t] at absolute position q_pos[t] and sees positions 0..q_pos[t] (the causal
  * mask is generated from q_pos inside the kernels, with per-row offsets instead of a
  * per-sequence host loop, third page 3.1).  Top-K outputs are positions in this logical
@@ -104,8 +104,8 @@ typedef struct hsa_paged_seq {
  *   k_scale  device fp32 [num_pages * page_size] when k_dtype == E4M3 (key = code * scale),
  *            else NULL
  *   scores   device fp32 [T_q, ld_scores], ld_scores >= max_seq_len
- * Pages: first page "Sparse Attention Pipeline Optimization" (correlation scoring with
- * head-weight weighted summation over the paged K cache); fifth page 3.1 (LI); BF16 and
+ * Pages: first page "Sparse Attention Pipeline Optimization" (per-head scores over the paged K
+ * cache, summed with per-head weights); fifth page 3.1 (LI); BF16 and
  * quantized index paths, second page 3.1.  The tensor-core kernel serves q BF16, k BF16/E4M3,
  * H_I = 64, D_I = 128, page_size a multiple of 8; other shapes use a CUDA-core kernel. */
 HSA_API hsa_status_t hsa_index_score(const hsa_paged_seq_t* seq, const void* q_I, hsa_dtype_t q_dtype,
@@ -164,9 +164,9 @@ HSA_API hsa_status_t hsa_sparse_mla_attn(const hsa_paged_seq_t* seq, const void*
  * caller buffers that hold the intermediate results afterwards.  With stream_aux != NULL the
  * rows are split in two halves; the second half runs on stream_aux, overlapping the first
  * half's attention (event-ordered; stream_main waits for stream_aux before returning work to
- * the caller).  Pages: first page "Sparse Attention Pipeline Optimization" (fuse where
- * possible, parallelize where possible: indexer then sparse attention kernel; multi-stream
- * orchestration); fifth page 3.3 (operators on independent streams with event
+ * the caller).  Pages: first page "Sparse Attention Pipeline Optimization" (fusing the decode
+ * operators and running independent ones concurrently: indexer, then the sparse attention
+ * kernel; several streams); fifth page 3.3 (operators on independent streams with event
  * synchronization). */
 typedef struct hsa_index_args {
     const void* q_I; hsa_dtype_t q_dtype; const float* w; int32_t H_I; int32_t D_I;

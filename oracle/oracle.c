@@ -13,7 +13,8 @@
  * Sources (page title, section):
  *  [P1]  "Day 0 Inference Adaptation and Optimization for Hybrid Attention Models",
  *        "Sparse Attention Pipeline Optimization" (indexer scores every history position,
- *        head-weight weighted sum, Top-K, sparse attention reading only selected KV) and
+ *        per-head scores combined with per-head weights, Top-K, sparse attention reading only
+ *        the selected KV rows) and
  *        "Hierarchical Quantization" (index path 8-bit, KV cache FP8 block quantization).
  *  [P2]  "Efficient Inference Deployment and Optimization for Hybrid Attention LLMs",
  *        sections 3.1 (indexer then sparse attention), 4.1/4.2 (quantization granularity),
@@ -27,8 +28,8 @@
  *
  * The pages never write the indexer as a formula.  The oracle uses
  *     I[t,s] = sum_j w[t,j] * ReLU( sum_d q_I[t,j,d] * k_I[s,d] ),   s <= p_t,
- * which is the plainest reading of "relevance scoring" + "head-weight weighted summation"
- * ([P1], [P5] s3) with one key per position shared by all index heads.
+ * which is the plainest reading of the pages' per-head scoring followed by a weighted sum over
+ * heads ([P1], [P5] s3), with one key per position shared by all index heads.
  *
  * Parity pins: see tests/test_oracle_*.py (closed forms, invariants, brute force, library
  * routines).  No function here is "parity unpinned".
@@ -152,7 +153,7 @@ int oracle_dequantize_rows(const uint8_t* codes, const float* scales, int64_t n_
 /* ------------------------------------------------------------------------------------------
  * Paged cache addressing.  A sequence b stores position s in physical slot
  *     block_table[b][s / page_size] * page_size + s % page_size
- * ([P1] "reads from the paged K cache"; [P3] 3.1 gather).  Returns -1 for an address outside
+ * ([P1]: the indexer reads keys straight out of the paged cache; [P3] 3.1 gather).  Returns -1 for an address outside
  * the cache, which the callers report as a bad argument.
  * ------------------------------------------------------------------------------------------ */
 static int64_t paged_slot(const int32_t* block_table, int64_t bt_stride, int32_t page_size,

@@ -1,8 +1,8 @@
 // index_score_tc.cu -- tensor-core index score for the 64-head x 128-dim indexer (sm_100a).
 //
 // I[t,s] = sum_j w[t,j] ReLU(q_I[t,j,:] . k[s,:])  ("Day 0 Inference Adaptation and Optimization
-// for Hybrid Attention Models", "Sparse Attention Pipeline Optimization": scoring over the paged
-// K cache and head-weight weighted summation; fifth page, 3.1).
+// for Hybrid Attention Models", "Sparse Attention Pipeline Optimization": per-head scores over
+// the paged K cache, combined with the per-head weights; fifth page, 3.1).
 //
 // Mapping.  One tcgen05 MMA tile is D[128 keys x G*64] = K_tile[128 x 128] . Q_group^T, with the
 // keys on M (TMEM lanes) and G query rows x 64 index heads on N (TMEM columns).  The epilogue

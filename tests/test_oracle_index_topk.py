@@ -2,7 +2,7 @@
 
 Index score I[t,s] = sum_j w[t,j] * ReLU(q_I[t,j] . k_I[s]) over causal positions s <= p_t
 ("Day 0 Inference Adaptation and Optimization for Hybrid Attention Models", "Sparse Attention
-Pipeline Optimization": relevance scoring over the paged K cache, head-weight weighted sum).
+Pipeline Optimization": per-head scores over the paged K cache, summed with per-head weights).
 Pinned by: a one-head special case against numpy's matmul, linearity in w with one-hot weights
 (head indexing), exact integer arithmetic, sign/causal special cases, paging invariance and
 positive homogeneity (the FP8 scale factoring).
