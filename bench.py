@@ -236,9 +236,9 @@ def _timed(fn, reps, flush_l2, main):
 
 def secondary(dev, flush_l2, main, peaks, reps):
     """The path's other workloads, each measured once per bench run (rank 0, one GPU): the FP8
-    decode batch, the bf16 causal prefill and the KV-cache quantizer.  Each entry gives tokens/s
-    and the fraction of the bound that applies to it (HBM bytes, or bf16 tensor flops for
-    prefill; algorithmic counts from the shapes)."""
+    decode batch, the draft-verify decode batch, the bf16 causal prefill and the KV-cache
+    quantizer.  Each entry gives tokens/s and the fraction of the bound that applies to it (HBM
+    bytes, or bf16 tensor flops for prefill; algorithmic counts from the shapes)."""
     import sparse_index_attention_b200 as hsa
     out = {}
     hbm = peaks["hbm_gbs"] * 1e9
@@ -285,6 +285,43 @@ def secondary(dev, flush_l2, main, peaks, reps):
                           "ms": round(ms, 4), "value": nrow / (ms * 1e-3), "unit": "rows/s",
                           "bound": "hbm", "bytes": byt, "frac": round(byt / (ms * 1e-3) / hbm, 4)}
     del wl, k8, ks, kv8, kvs, rope, sc, idx, o, lse, ws, seq
+    torch.cuda.empty_cache()
+
+    # draft-verify decode: the bf16 decode batch with 4 query rows per sequence (the last 4
+    # positions).  The four rows of a sequence share one pass over its index keys; the bytes
+    # counted are the keys once per sequence plus the distinct cache rows the four selections
+    # name (measured from the step's own idx), q, q_I, w and the outputs.
+    wl = workloads.make("decode_draft_bf16", dev)
+    seq = hsa.PagedSeq(wl.seq_lens, wl.block_table, wl.page_size, wl.num_pages, wl.q_seq, wl.q_pos,
+                       q_run=wl.q_run)
+    sc = torch.empty((wl.T_q, seq.max_seq_len), dtype=torch.float32, device=dev)
+    idx = torch.empty((wl.T_q, wl.K), dtype=torch.int32, device=dev)
+    o = torch.empty((wl.T_q, wl.H, wl.D_v), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((wl.T_q, wl.H), dtype=torch.float32, device=dev)
+    ws = torch.empty(max(1, hsa.hsa_fused_decode_workspace_size(seq, wl.q, wl.kv, wl.D_v, wl.K)),
+                     dtype=torch.uint8, device=dev)
+
+    def draft_step():
+        hsa.hsa_fused_decode(seq, wl.q_I, wl.w, wl.k_I, None, wl.q, wl.kv, None, None, wl.K,
+                             wl.D_v, wl.softmax_scale, scores=sc, idx=idx, out=o, lse=lse, ws=ws,
+                             stream=main)
+    for _ in range(3):
+        draft_step()
+    ms = _timed(draft_step, reps, flush_l2, main)
+    main.synchronize()
+    rows_read = 0
+    for b in range(wl.B):
+        sel = idx[b * wl.q_run:(b + 1) * wl.q_run]
+        rows_read += int(torch.unique(sel[sel >= 0]).numel())
+    byt = int(wl.seq_lens.long().sum()) * wl.D_I * 2 + rows_read * wl.D_qk * 2 + \
+        wl.T_q * wl.H * (wl.D_qk + wl.D_v) * 2 + wl.T_q * wl.H_I * (wl.D_I * 2 + 4)
+    out["decode_draft_bf16"] = {
+        "workload": f"{wl.B} sequences x 8192..32768 keys, {wl.q_run} draft rows per sequence "
+                    "(draft-verify), bf16 caches, Top-2048, 128 heads",
+        "ms_per_step": round(ms, 4), "value": wl.T_q / (ms * 1e-3), "unit": UNIT,
+        "bound": "hbm", "bytes": byt, "distinct_rows_gathered": rows_read,
+        "frac": round(byt / (ms * 1e-3) / hbm, 4)}
+    del wl, sc, idx, o, lse, ws, seq
     torch.cuda.empty_cache()
 
     # bf16 causal prefill: one sequence of 16384 tokens, every token a query, 4 query chunks of

@@ -180,6 +180,23 @@ def decode_fp8(device="cpu", seed=3, B=128, L=65536, page_size=64, H_I=64, D_I=1
                   1.0 / math.sqrt(D_qk), True, True)
 
 
+def decode_draft_bf16(device="cpu", seed=5, B=64, n_draft=4, L_min=8192, L_max=32768,
+                      page_size=64, H_I=64, D_I=128, H=128, D_v=512, D_rope=64, K=2048):
+    """Draft-verify decode: each sequence checks n_draft drafted tokens in one step, so it has
+    n_draft query rows at its last n_draft positions, each causal over its own prefix
+    ("Day 0 Inference Adaptation and Optimization for Hybrid Attention Models", decoding
+    acceleration reuse: the draft-verify paradigm; "Inference Adaptation and Performance
+    Optimization for a Domestically Developed LLM's New Architecture", 6: speculative
+    inference).  Same shapes and value recipe as decode_bf16 otherwise."""
+    lens = _lengths(B, max(L_min, n_draft), max(L_max, n_draft), seed)
+    D_qk = D_v + D_rope
+    q_seq = [b for b in range(B) for _ in range(n_draft)]
+    q_pos = [L - n_draft + i for L in lens for i in range(n_draft)]
+    return _build("decode_draft_bf16", seed, device, "bf16", lens, page_size, q_seq, q_pos,
+                  n_draft, H_I, D_I, 1.0 / 8, H, D_qk, D_v, 0.5, K, 1.0 / math.sqrt(D_qk),
+                  False, False)
+
+
 def zigzag_chunks(T: int, n_chunks: int) -> List[Tuple[int, int]]:
     """Query-row ranges issued as pairs (i, n_chunks-1-i) ("Efficient Inference Deployment and
     Optimization for Hybrid Attention LLMs", 5.2: segment i goes with segment 2N-1-i)."""
@@ -206,6 +223,7 @@ RECIPES = {
     "decode_bf16": decode_bf16,
     "prefill_bf16": prefill_bf16,
     "decode_fp8": decode_fp8,
+    "decode_draft_bf16": decode_draft_bf16,
     "prefill_long_zigzag": prefill_long_zigzag,
 }
 

@@ -78,6 +78,8 @@ def check_against_oracle(wl, rows, sc, idx, out):
     ("tiny_decode_fp32", {}),
     ("decode_bf16", dict(B=8, L_min=1500, L_max=5000)),
     ("decode_fp8", dict(B=4, L=4500)),
+    ("decode_draft_bf16", dict(B=5, L_min=1500, L_max=5000)),
+    ("decode_draft_bf16", dict(B=3, n_draft=2, L_min=2040, L_max=2052)),
 ])
 def test_pipeline_vs_oracle_small(name, kw):
     wl = workloads.make(name, DEV, **kw)
@@ -91,6 +93,7 @@ def test_pipeline_vs_oracle_small(name, kw):
     ("decode_bf16", dict(B=8, L_min=1500, L_max=5000), None),
     ("decode_fp8", dict(B=6, L=3000), None),
     ("decode_fp8", dict(B=6, L=3000), 128),
+    ("decode_draft_bf16", dict(B=6, L_min=1500, L_max=5000), None),
 ])
 def test_fused_equals_unfused_and_two_streams(name, kw, kv_group):
     wl = workloads.make(name, DEV, **kw)
@@ -121,6 +124,20 @@ def test_decode_bf16_full_size_sampled():
     ref_sel = stable_topk_reference(sc, wl.q_pos, wl.K)
     assert torch.equal(idx, ref_sel)
     rows = [0, 17, 40, 63]
+    check_against_oracle(wl, rows, sc, idx, out)
+
+
+def test_decode_draft_full_size_sampled():
+    """Draft-verify decode at full size (64 sequences, contexts 8192..32768, four query rows per
+    sequence at its last four positions, Top-2048, 128 heads): the four rows of a sequence share
+    one pass over its index keys.  Top-K bit-exact on every row; oracle checks on all four rows
+    of three sequences."""
+    wl = workloads.make("decode_draft_bf16", DEV)
+    gc = GpuCaches(wl)
+    out, lse, idx, sc = run_fused(wl, gc)
+    ref_sel = stable_topk_reference(sc, wl.q_pos, wl.K)
+    assert torch.equal(idx, ref_sel)
+    rows = [r for b in (0, 29, 63) for r in range(4 * b, 4 * b + 4)]
     check_against_oracle(wl, rows, sc, idx, out)
 
 

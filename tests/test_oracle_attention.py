@@ -153,3 +153,35 @@ def test_zigzag_rule_and_balanced_load():
         # causal pairs of a query chunk [a0, a1): sum_{t} (t + 1), counted by brute force sum
         loads.append(sum(range(a0 + 1, a1 + 1)) + sum(range(b0 + 1, b1 + 1)))
     assert set(loads) == {int(spec["pairs_per_pair"][0])}
+
+
+def test_draft_rows_see_only_their_own_prefix():
+    """Draft-verify decode (several query rows per sequence at its last positions): each row's
+    result equals a one-row decode of the same sequence cut after that row's position, so no
+    row reads a key past its own position, and the rows of a sequence differ."""
+    kw = dict(B=3, n_draft=3, L_min=40, L_max=90, page_size=16, H_I=4, D_I=32, H=8, D_v=64,
+              D_rope=16, K=16)
+    wl = workloads.make("decode_draft_bf16", **kw)
+    assert wl.T_q == 9 and wl.q_run == 3
+    for b in range(wl.B):
+        L = int(wl.seq_lens[b])
+        assert wl.q_seq[3 * b:3 * b + 3].tolist() == [b] * 3
+        assert wl.q_pos[3 * b:3 * b + 3].tolist() == [L - 3, L - 2, L - 1]
+    pg = oracle.Paging(wl.seq_lens, wl.block_table, wl.page_size, wl.num_pages, wl.q_seq, wl.q_pos)
+    sc, idx, out, lse = oracle.sparse_index_attention(pg, wl.q_I, wl.w, wl.k_I, wl.q, wl.kv,
+                                                      wl.K, wl.D_v, wl.softmax_scale)
+    for t in range(wl.T_q):
+        b, p = int(wl.q_seq[t]), int(wl.q_pos[t])
+        assert idx[t].max() <= p
+        lens = wl.seq_lens.clone()
+        lens[b] = p + 1
+        one = oracle.Paging(lens, wl.block_table, wl.page_size, wl.num_pages,
+                            wl.q_seq[t:t + 1], wl.q_pos[t:t + 1])
+        sc1, idx1, out1, lse1 = oracle.sparse_index_attention(
+            one, wl.q_I[t:t + 1], wl.w[t:t + 1], wl.k_I, wl.q[t:t + 1], wl.kv, wl.K, wl.D_v,
+            wl.softmax_scale)
+        assert np.array_equal(idx1[0], idx[t])
+        np.testing.assert_array_equal(sc1[0, :p + 1], sc[t, :p + 1])
+        np.testing.assert_array_equal(out1[0], out[t])
+        np.testing.assert_array_equal(lse1[0], lse[t])
+    assert not np.array_equal(out[0], out[1])
