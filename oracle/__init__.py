@@ -6,7 +6,8 @@ imports it, and it imports nothing from the product.  The arithmetic lives in ``
 (plain C, float64, OpenMP over query rows); this module only marshals numpy arrays.
 
 Inputs are widened exactly: bf16/fp32 tensors become float64 arrays, FP8 E4M3 codes are
-decoded by the oracle's own codec (``e4m3_decode``) and multiplied by their fp32 scale.
+decoded by the oracle's own codec (``e4m3_decode``) and multiplied by their fp32 scale, or, for
+MXFP8 blocks, by 2^(E - 127) of their shared E8M0 scale byte (``mx_dequantize_rows``).
 
 Page citations (title, section) are in ``oracle.c`` beside each function.  The end-to-end
 composition ``sparse_index_attention`` follows the pipeline of "Day 0 Inference Adaptation and
@@ -60,12 +61,15 @@ def _load():
             lib.oracle_e4m3_encode.restype = ctypes.c_uint8
             lib.oracle_quantize_rows.argtypes = [P, i64, i32, i32, P, P]
             lib.oracle_dequantize_rows.argtypes = [P, P, i64, i32, i32, P]
+            lib.oracle_mx_quantize_rows.argtypes = [P, i64, i32, P, P]
+            lib.oracle_mx_dequantize_rows.argtypes = [P, P, i64, i32, P]
             paging = [i32, P, P, i64, i32, i32, i32, P, P]
             lib.oracle_index_score.argtypes = paging + [i32, i32, P, P, P, P, i64]
             lib.oracle_topk.argtypes = [i32, P, P, i64, i32, P]
             lib.oracle_sparse_mla.argtypes = paging + [i32, i32, i32, P, P, P, i32, f64, P, P]
             lib.oracle_dense_attn.argtypes = paging + [i32, i32, i32, P, P, f64, P, P]
-            for f in ("oracle_quantize_rows", "oracle_dequantize_rows", "oracle_index_score",
+            for f in ("oracle_quantize_rows", "oracle_dequantize_rows", "oracle_mx_quantize_rows",
+                      "oracle_mx_dequantize_rows", "oracle_index_score",
                       "oracle_topk", "oracle_sparse_mla", "oracle_dense_attn"):
                 getattr(lib, f).restype = ctypes.c_int
             lib.oracle_num_threads.restype = ctypes.c_int
@@ -141,6 +145,29 @@ def dequantize_rows(codes, scales, group: int) -> np.ndarray:
     out = np.zeros((n, D), dtype=np.float64)
     _check(_load().oracle_dequantize_rows(_ptr(c), _ptr(s), n, D, group, _ptr(out)),
            "dequantize_rows")
+    return out
+
+
+def mx_quantize_rows(x):
+    """MXFP8: rows [n, D] (fp32-representable, D a multiple of 32) -> (E4M3 codes uint8 [n, D],
+    E8M0 scale bytes uint8 [n, D/32]); the rule is in ``oracle.c``."""
+    xf = np.ascontiguousarray(_f64(x).astype(np.float32))
+    n, D = xf.shape
+    codes = np.zeros((n, D), dtype=np.uint8)
+    scales = np.zeros((n, D // 32), dtype=np.uint8)
+    _check(_load().oracle_mx_quantize_rows(_ptr(xf), n, D, _ptr(codes), _ptr(scales)),
+           "mx_quantize_rows")
+    return codes, scales
+
+
+def mx_dequantize_rows(codes, scales) -> np.ndarray:
+    """decode(code) * 2^(E - 127) per 32-element block, float64 (exact)."""
+    c = np.ascontiguousarray(np.asarray(codes, dtype=np.uint8))
+    s = np.ascontiguousarray(np.asarray(scales, dtype=np.uint8))
+    n, D = c.shape
+    out = np.zeros((n, D), dtype=np.float64)
+    _check(_load().oracle_mx_dequantize_rows(_ptr(c), _ptr(s), n, D, _ptr(out)),
+           "mx_dequantize_rows")
     return out
 
 

@@ -151,6 +151,65 @@ int oracle_dequantize_rows(const uint8_t* codes, const float* scales, int64_t n_
 }
 
 /* ------------------------------------------------------------------------------------------
+ * MXFP8 (OCP Microscaling formats, FP8 E4M3 elements): every block of 32 consecutive elements
+ * shares one E8M0 scale byte E meaning 2^(E - 127) (E = 255 is NaN and never produced).  The
+ * pages store the index Q/K this way: dynamic per-group quantization, group size 32, a shared
+ * exponent ([P1] "Hierarchical Quantization"; [P2] 4.1; [P5] section 4 table).  The pages do
+ * not spell out how the shared exponent is chosen; the reading taken is the MX rule:
+ *     X = floor(log2(amax)) - 8        (8 = exponent of the top E4M3 binade: 448 = 1.75 * 2^8)
+ * clamped to [-127, 127], E = X + 127, and each element becomes the E4M3 code of x / 2^X
+ * (round to nearest even, finite overflow saturating to +-448).  An all-zero block gets E = 0
+ * and zero codes.  x / 2^X is a power-of-two rescaling, exact in double, and exact as a float
+ * whenever it is at least 2^-126; below that every candidate rounds to code 0 either way.
+ *   x: [n_rows, D] fp32-representable, D a multiple of 32; codes [n_rows, D]; scales
+ *   [n_rows, D / 32] (one byte each).
+ * ------------------------------------------------------------------------------------------ */
+int oracle_mx_quantize_rows(const float* x, int64_t n_rows, int32_t D, uint8_t* codes,
+                            uint8_t* scales) {
+    if (n_rows < 0 || D <= 0 || D % 32 != 0) return ORACLE_BAD_ARG;
+    const int32_t nb = D / 32;
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < n_rows; ++r) {
+        for (int32_t b = 0; b < nb; ++b) {
+            const float* xs = x + r * D + (int64_t)b * 32;
+            uint8_t* cs = codes + r * D + (int64_t)b * 32;
+            double amax = 0.0;
+            for (int i = 0; i < 32; ++i) {
+                double a = fabs((double)xs[i]);
+                if (a > amax) amax = a;
+            }
+            if (amax == 0.0) {
+                scales[r * nb + b] = 0;
+                for (int i = 0; i < 32; ++i) cs[i] = 0;
+                continue;
+            }
+            int e2;
+            frexp(amax, &e2);               /* amax = m * 2^e2, m in [0.5, 1) */
+            int X = (e2 - 1) - 8;           /* floor(log2(amax)) - 8 */
+            if (X < -127) X = -127;
+            if (X > 127) X = 127;
+            scales[r * nb + b] = (uint8_t)(X + 127);
+            for (int i = 0; i < 32; ++i)
+                cs[i] = oracle_e4m3_encode((float)ldexp((double)xs[i], -X));
+        }
+    }
+    return ORACLE_OK;
+}
+
+/* value = decode(code) * 2^(E - 127), into double (exact). */
+int oracle_mx_dequantize_rows(const uint8_t* codes, const uint8_t* scales, int64_t n_rows,
+                              int32_t D, double* out) {
+    if (n_rows < 0 || D <= 0 || D % 32 != 0) return ORACLE_BAD_ARG;
+    const int32_t nb = D / 32;
+    for (int64_t r = 0; r < n_rows; ++r)
+        for (int32_t i = 0; i < D; ++i) {
+            const uint8_t E = scales[r * nb + i / 32];
+            out[r * D + i] = E == 255 ? NAN : ldexp(oracle_e4m3_decode(codes[r * D + i]), (int)E - 127);
+        }
+    return ORACLE_OK;
+}
+
+/* ------------------------------------------------------------------------------------------
  * Paged cache addressing.  A sequence b stores position s in physical slot
  *     block_table[b][s / page_size] * page_size + s % page_size
  * ([P1]: the indexer reads keys straight out of the paged cache; [P3] 3.1 gather).  Returns -1 for an address outside

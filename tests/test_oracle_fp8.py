@@ -161,3 +161,105 @@ def test_pages_quantization_table_and_storage_claim():
     for group in (D, rows["index_qk"][1]):
         ratio = (D + 4 * (D // group)) / (2 * D)
         assert abs(ratio - claim) < 0.07, ratio
+
+
+# ------------------------------------------------------------------------------ MXFP8 blocks
+def _golden_mx_blocks():
+    blocks = {}
+    for line in open(os.path.join(GOLDEN, "mxfp8_blocks.txt")):
+        line = line.split("#")[0].strip()
+        if not line:
+            continue
+        name, E, i, x, code = line.split()
+        if x.lstrip("-").startswith("2^"):
+            v = math.ldexp(1.0, int(x.lstrip("-")[2:])) * (-1.0 if x.startswith("-") else 1.0)
+        else:
+            v = float(x)
+        b = blocks.setdefault(name, {"E": int(E), "x": np.zeros(32), "code": np.zeros(32, np.uint8)})
+        assert b["E"] == int(E)
+        b["x"][int(i)] = v
+        b["code"][int(i)] = int(code, 16)
+    return blocks
+
+
+def test_mx_golden_blocks():
+    """Blocks worked by hand from the MX definition, one per case: plain rounding, ties to even
+    at subnormal and normal midpoints, saturation, a negative shared exponent, an all-zero
+    block, the lower clamp of the shared exponent and a block near the float32 maximum."""
+    blocks = _golden_mx_blocks()
+    assert len(blocks) == 6
+    x = np.stack([b["x"] for b in blocks.values()]).astype(np.float32)
+    assert np.array_equal(x.astype(np.float64), np.stack([b["x"] for b in blocks.values()]))
+    codes, scales = oracle.mx_quantize_rows(x)
+    for r, (name, b) in enumerate(blocks.items()):
+        assert scales[r, 0] == b["E"], name
+        assert np.array_equal(codes[r], b["code"]), (name, codes[r], b["code"])
+
+
+def _mx_data(n, D, seed):
+    rng = np.random.default_rng(seed)
+    x = rng.standard_normal((n, D)) * np.exp2(rng.integers(-20, 20, (n, 1)))
+    x[0, :32] = 0.0                                   # an all-zero block
+    x[1, 32:64] *= 1e-30                              # a block near the bottom of float32
+    return x.astype(np.float32)
+
+
+def test_mx_scale_rule_and_error_bound():
+    """For every block: the block maximum lands in the top E4M3 binade [256, 448] after the
+    division by 2^X (so X is the largest exponent that keeps it finite within E4M3's range,
+    rounding aside), and every element is within half an E4M3 spacing of x / 2^X, or saturated
+    at +-448 when it rounds past it."""
+    x = _mx_data(64, 128, 5)
+    codes, scales = oracle.mx_quantize_rows(x)
+    deq = oracle.mx_dequantize_rows(codes, scales)
+    for r in range(x.shape[0]):
+        for blk in range(4):
+            xs = x[r, 32 * blk:32 * blk + 32].astype(np.float64)
+            E = int(scales[r, blk])
+            amax = np.abs(xs).max()
+            if amax == 0:
+                assert E == 0 and not codes[r, 32 * blk:32 * blk + 32].any()
+                continue
+            X = E - 127
+            y = xs / 2.0 ** X
+            top = np.abs(oracle.e4m3_decode(codes[r, 32 * blk + np.argmax(np.abs(xs))]))
+            if X > -127:
+                assert 256 <= np.abs(y).max() < 512 and 256 <= top <= 448
+            else:
+                assert np.abs(y).max() < 512
+            d = deq[r, 32 * blk:32 * blk + 32] / 2.0 ** X
+            for yi, di in zip(y, d):
+                a = abs(yi)
+                if a >= 2.0 ** -6:
+                    spacing = 2.0 ** (math.floor(math.log2(a)) - 3)
+                else:
+                    spacing = 2.0 ** -9
+                assert abs(di - yi) <= spacing / 2 or (abs(di) == 448 and a > 448), (r, blk, yi, di)
+
+
+def test_mx_power_of_two_rescaling_moves_only_the_scale():
+    """Multiplying a block by 2^k leaves its codes unchanged and adds k to the scale byte (away
+    from the exponent clamps): the shared exponent carries the whole magnitude."""
+    x = _mx_data(32, 64, 6)[2:]
+    c0, s0 = oracle.mx_quantize_rows(x)
+    for k in (-9, -1, 1, 13):
+        c1, s1 = oracle.mx_quantize_rows(x * np.float32(2.0 ** k))
+        assert np.array_equal(c0, c1)
+        assert np.array_equal(s0.astype(int) + k, s1.astype(int))
+
+
+def test_mx_values_on_the_grid_are_fixed_points():
+    """A block whose values already are E4M3 codes times 2^X, with one code in the top binade,
+    quantizes back to exactly those codes and E = X + 127."""
+    rng = np.random.default_rng(7)
+    finite = _all_finite_codes()
+    top = finite[(oracle.e4m3_decode(finite) >= 256)]
+    for X in (-30, -8, 0, 17):
+        codes = rng.choice(finite, (8, 32))
+        codes[:, 5] = rng.choice(top, 8)
+        vals = oracle.e4m3_decode(codes) * 2.0 ** X
+        got_c, got_s = oracle.mx_quantize_rows(vals.astype(np.float32))
+        assert np.all(got_s == X + 127)
+        same = oracle.e4m3_decode(got_c) == oracle.e4m3_decode(codes)   # +0 and -0 both decode to 0
+        assert same.all()
+        assert np.array_equal(oracle.mx_dequantize_rows(got_c, got_s), vals)
