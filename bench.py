@@ -236,8 +236,8 @@ def _timed(fn, reps, flush_l2, main):
 
 def secondary(dev, flush_l2, main, peaks, reps):
     """The path's other workloads, each measured once per bench run (rank 0, one GPU): the FP8
-    decode batch, the draft-verify decode batch, the bf16 causal prefill and the KV-cache
-    quantizer.  Each entry gives tokens/s and the fraction of the bound that applies to it (HBM
+    decode batch (fp32 and MXFP8 index scales), the draft-verify decode batch, the bf16 causal
+    prefill and the KV-cache quantizer.  Each entry gives tokens/s and the fraction of the bound that applies to it (HBM
     bytes, or bf16 tensor flops for prefill; algorithmic counts from the shapes)."""
     import sparse_index_attention_b200 as hsa
     out = {}
@@ -272,6 +272,30 @@ def secondary(dev, flush_l2, main, peaks, reps):
                          "ms_per_step": round(ms, 4), "value": wl.T_q / (ms * 1e-3), "unit": UNIT,
                          "bound": "hbm", "bytes": byt,
                          "frac": round(byt / (ms * 1e-3) / hbm, 4)}
+    # the same batch with the index queries and keys in MXFP8 (one E8M0 byte per 32 dims): the
+    # step rounds q_I onto the MX grid (two small kernels) and scores the MX key cache
+    kmx, kmx_e = hsa.hsa_quantize_mx(wl.k_I)
+    qI_flat = wl.q_I.view(-1, wl.D_I)
+    q_codes = torch.empty(qI_flat.shape, dtype=torch.uint8, device=dev)
+    q_e = torch.empty((qI_flat.shape[0], wl.D_I // 32), dtype=torch.uint8, device=dev)
+    q_mx = torch.empty_like(wl.q_I)
+
+    def mx_step():
+        hsa.hsa_quantize_mx(qI_flat, codes=q_codes, scales=q_e, stream=main)
+        hsa.hsa_dequantize_mx(q_codes, q_e, out=q_mx.view(-1, wl.D_I), stream=main)
+        hsa.hsa_fused_decode(seq, q_mx, wl.w, kmx, kmx_e, wl.q, kv8, kvs, rope, wl.K, wl.D_v,
+                             wl.softmax_scale, scores=sc, idx=idx, out=o, lse=lse, ws=ws, stream=main)
+    for _ in range(3):
+        mx_step()
+    ms = _timed(mx_step, reps, flush_l2, main)
+    # plus the rounding of q_I: read bf16, write and re-read the codes and scale bytes, write bf16
+    byt_mx = byt + wl.T_q * wl.H_I * wl.D_I * (2 + 1 + 1 + 2) + 2 * wl.T_q * wl.H_I * (wl.D_I // 32)
+    out["decode_mxfp8"] = {"workload": "the FP8 decode batch with MXFP8 index queries and keys "
+                                       "(E8M0 scale per 32 dims), rounding of q_I included",
+                           "ms_per_step": round(ms, 4), "value": wl.T_q / (ms * 1e-3), "unit": UNIT,
+                           "bound": "hbm", "bytes": byt_mx,
+                           "frac": round(byt_mx / (ms * 1e-3) / hbm, 4)}
+    del kmx, kmx_e, q_codes, q_e, q_mx
     # KV-cache quantizer on the same cache (8.4 M rows): read 1152 B, write 512 + 4 + 128 B per row
     nrow = wl.kv.shape[0]
 

@@ -61,7 +61,9 @@ typedef enum hsa_status {
 typedef enum hsa_dtype {
     HSA_F32 = 0,   /* IEEE binary32 */
     HSA_BF16 = 1,  /* bfloat16 */
-    HSA_E4M3 = 2   /* OCP FP8 E4M3 code, one byte; paired with fp32 scales */
+    HSA_E4M3 = 2,  /* OCP FP8 E4M3 code, one byte; paired with fp32 scales */
+    HSA_MXE4M3 = 3 /* MXFP8 (OCP Microscaling): E4M3 codes, and one E8M0 scale byte E, meaning
+                      2^(E - 127), shared by each block of 32 consecutive elements */
 } hsa_dtype_t;
 
 /* device status bits (OR-ed into *hsa_paged_seq_t.status) */
@@ -100,17 +102,20 @@ typedef struct hsa_paged_seq {
  * for 0 <= s <= q_pos[t]; entries s > q_pos[t] are not written.
  *   q_I      device [T_q, H_I, D_I], q_dtype F32 or BF16
  *   w        device fp32 [T_q, H_I] (head weights)
- *   k_cache  device [num_pages * page_size, D_I] of k_dtype F32, BF16 or E4M3
- *   k_scale  device fp32 [num_pages * page_size] when k_dtype == E4M3 (key = code * scale),
+ *   k_cache  device [num_pages * page_size, D_I] of k_dtype F32, BF16, E4M3 or MXE4M3 (codes)
+ *   k_scale  k_dtype E4M3: device fp32 [num_pages * page_size] (key = code * scale);
+ *            k_dtype MXE4M3: device uint8 [num_pages * page_size, D_I / 32] E8M0 bytes, 16-byte
+ *            aligned (key element d = code * 2^(E[d / 32] - 127), D_I a multiple of 32);
  *            else NULL
  *   scores   device fp32 [T_q, ld_scores], ld_scores >= max_seq_len
  * Pages: first page "Sparse Attention Pipeline Optimization" (per-head scores over the paged K
  * cache, summed with per-head weights); fifth page 3.1 (LI); BF16 and
- * quantized index paths, second page 3.1.  The tensor-core kernel serves q BF16, k BF16/E4M3,
- * H_I = 64, D_I = 128, page_size a multiple of 8; other shapes use a CUDA-core kernel. */
+ * quantized index paths, second page 3.1; MXFP8 index keys, fifth page 4 (table).  The
+ * tensor-core kernel serves q BF16, k BF16/E4M3/MXE4M3, H_I = 64, D_I = 128, page_size a
+ * multiple of 8; other shapes use a CUDA-core kernel. */
 HSA_API hsa_status_t hsa_index_score(const hsa_paged_seq_t* seq, const void* q_I, hsa_dtype_t q_dtype,
                              const float* w, int32_t H_I, int32_t D_I, const void* k_cache,
-                             hsa_dtype_t k_dtype, const float* k_scale, float* scores,
+                             hsa_dtype_t k_dtype, const void* k_scale, float* scores,
                              int64_t ld_scores, void* stream);
 
 /* ---- 2. Top-K -----------------------------------------------------------------------------
@@ -170,7 +175,7 @@ HSA_API hsa_status_t hsa_sparse_mla_attn(const hsa_paged_seq_t* seq, const void*
  * synchronization). */
 typedef struct hsa_index_args {
     const void* q_I; hsa_dtype_t q_dtype; const float* w; int32_t H_I; int32_t D_I;
-    const void* k_cache; hsa_dtype_t k_dtype; const float* k_scale;
+    const void* k_cache; hsa_dtype_t k_dtype; const void* k_scale;
 } hsa_index_args_t;
 
 typedef struct hsa_attn_args {
@@ -208,6 +213,29 @@ HSA_API hsa_status_t hsa_quantize_kv(const void* src, hsa_dtype_t src_dtype, int
                              int32_t D_rope, int32_t group, const int64_t* slot_mapping,
                              int64_t num_slots, uint8_t* codes, float* scales, void* rope_cache,
                              void* stream);
+
+/* ---- 6. MXFP8 block quantizer ------------------------------------------------------------
+ * Per row r and block b of 32 consecutive elements (D a multiple of 32):
+ *   amax = max |x|;  X = floor(log2(amax)) - 8, clamped to [-127, 127];  E = X + 127;
+ *   code = E4M3(round-to-nearest-even, saturating, of x * 2^-X);   amax == 0: E = 0, codes 0.
+ * (8 is the exponent of E4M3's top binade, 448 = 1.75 * 2^8, so the block maximum lands in
+ * [256, 448] before rounding; the OCP Microscaling rule for the shared exponent.)  From finite
+ * fp32 or bf16 data E never exceeds 246.
+ * hsa_quantize_mx: src [n_rows, D] F32/BF16 -> codes uint8 [slots, D], scales uint8
+ *   [slots, D / 32]; row r goes to slot slot_mapping[r] (NULL: slot r).  With D = 128 this
+ *   writes the MXE4M3 index key cache hsa_index_score reads; applied to q_I (slot_mapping
+ *   NULL) it quantizes the index queries.
+ * hsa_dequantize_mx: codes [n_rows, D] + scales [n_rows, D / 32] -> dst [n_rows, D] of
+ *   dst_dtype F32 or BF16, value code * 2^(E - 127): exact in F32 for every E <= 246; exact in
+ *   BF16 for E >= 3 (below that, values under the bf16 range round to nearest).  Writing MXFP8
+ *   index queries back as bf16 lets the bf16-query index kernels consume them unchanged.
+ * Pages: first page "Hierarchical Quantization" (index Q/K in MXFP8, group 32, shared
+ * exponent); second page 4.1; fifth page 4 (table). */
+HSA_API hsa_status_t hsa_quantize_mx(const void* src, hsa_dtype_t src_dtype, int64_t n_rows, int32_t D,
+                             const int64_t* slot_mapping, int64_t num_slots, uint8_t* codes,
+                             uint8_t* scales, void* stream);
+HSA_API hsa_status_t hsa_dequantize_mx(const uint8_t* codes, const uint8_t* scales, int64_t n_rows,
+                               int32_t D, void* dst, hsa_dtype_t dst_dtype, void* stream);
 
 /* ---- diagnostics -------------------------------------------------------------------------- */
 HSA_API const char* hsa_status_string(hsa_status_t s);

@@ -21,7 +21,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libhsa.so")
 
 HSA_OK, HSA_ERR_INVALID_ARG, HSA_ERR_UNSUPPORTED, HSA_ERR_CUDA, HSA_ERR_WORKSPACE = 0, 1, 2, 3, 4
-HSA_F32, HSA_BF16, HSA_E4M3 = 0, 1, 2
+HSA_F32, HSA_BF16, HSA_E4M3, HSA_MXE4M3 = 0, 1, 2, 3
 HSA_DEV_BAD_PAGE, HSA_DEV_BAD_POS, HSA_DEV_BAD_GROUP, HSA_DEV_TIMEOUT = 1, 2, 4, 8
 
 _P = ctypes.c_void_p
@@ -59,6 +59,8 @@ SYMBOLS = {
     "hsa_quantize_index": (ctypes.c_int, [_P, ctypes.c_int, _i64, _i32, _i32, _P, _i64, _P, _P, _P]),
     "hsa_quantize_kv": (ctypes.c_int, [_P, ctypes.c_int, _i64, _i32, _i32, _i32, _P, _i64, _P, _P,
                                        _P, _P]),
+    "hsa_quantize_mx": (ctypes.c_int, [_P, ctypes.c_int, _i64, _i32, _P, _i64, _P, _P, _P]),
+    "hsa_dequantize_mx": (ctypes.c_int, [_P, _P, _i64, _i32, _P, ctypes.c_int, _P]),
     "hsa_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "hsa_last_error_message": (ctypes.c_char_p, []),
     "hsa_version": (_i32, []),
@@ -118,6 +120,14 @@ def _dtype(t: torch.Tensor) -> int:
     raise TypeError(f"unsupported dtype {t.dtype}")
 
 
+def _key_dtype(k_cache: torch.Tensor, k_scale: Optional[torch.Tensor]) -> int:
+    """Index keys: 8-bit codes with uint8 (E8M0) scales are MXFP8, with fp32 scales E4M3."""
+    d = _dtype(k_cache)
+    if d == HSA_E4M3 and k_scale is not None and k_scale.dtype == torch.uint8:
+        return HSA_MXE4M3
+    return d
+
+
 def _stream(s) -> ctypes.c_void_p:
     if s is None:
         s = torch.cuda.current_stream()
@@ -163,7 +173,8 @@ def hsa_index_score(seq: PagedSeq, q_I, w, k_cache, k_scale=None, scores=None, l
         scores = torch.empty((T_q, ld), dtype=torch.float32, device=q_I.device)
     ld = scores.shape[1]
     _check(lib().hsa_index_score(seq.ref, _ptr(q_I), _dtype(q_I), _ptr(w), H_I, D_I, _ptr(k_cache),
-                                 _dtype(k_cache), _ptr(k_scale), _ptr(scores), ld, _stream(stream)),
+                                 _key_dtype(k_cache, k_scale), _ptr(k_scale), _ptr(scores), ld,
+                                 _stream(stream)),
            "hsa_index_score")
     return scores
 
@@ -252,8 +263,8 @@ def hsa_fused_decode(seq: PagedSeq, q_I, w, k_cache, k_scale, q, kv, kv_scale, k
     elif lse is False:
         lse = None
     ws = _workspace(hsa_fused_decode_workspace_size(seq, q, kv, D_v, K), dev, ws)
-    ia = hsa_index_args_t(_ptr(q_I), _dtype(q_I), _ptr(w), H_I, D_I, _ptr(k_cache), _dtype(k_cache),
-                          _ptr(k_scale))
+    ia = hsa_index_args_t(_ptr(q_I), _dtype(q_I), _ptr(w), H_I, D_I, _ptr(k_cache),
+                          _key_dtype(k_cache, k_scale), _ptr(k_scale))
     at = _attn_struct(q, kv, D_v, softmax_scale, kv_scale, kv_rope, out, lse)
     _check(lib().hsa_fused_decode(seq.ref, ctypes.byref(ia), ctypes.byref(at), K, _ptr(scores),
                                   scores.shape[1], _ptr(idx), _ptr(ws), ws.numel(), _stream(stream),
@@ -333,6 +344,42 @@ def hsa_quantize_kv(src, D_v: int, group: int, slot_mapping=None, num_slots: Opt
                                  _stream(stream)),
            "hsa_quantize_kv")
     return codes, scales, rope_cache
+
+
+def hsa_quantize_mx(src, slot_mapping=None, num_slots: Optional[int] = None, codes=None,
+                    scales=None, stream=None):
+    """MXFP8: rows [n, D] (D a multiple of 32) -> (E4M3 codes uint8 [slots, D], E8M0 scale bytes
+    uint8 [slots, D/32]).  With D = 128 the pair is an MXFP8 index key cache for
+    ``hsa_index_score``."""
+    n, D = src.shape
+    num_slots = num_slots if num_slots is not None else n
+    if codes is None:
+        codes = torch.zeros((num_slots, D), dtype=torch.uint8, device=src.device)
+    if scales is None:
+        scales = torch.zeros((num_slots, D // 32), dtype=torch.uint8, device=src.device)
+    _check(lib().hsa_quantize_mx(_ptr(src), _dtype(src), n, D, _ptr(slot_mapping), num_slots,
+                                 _ptr(codes), _ptr(scales), _stream(stream)),
+           "hsa_quantize_mx")
+    return codes, scales
+
+
+def hsa_dequantize_mx(codes, scales, dtype=torch.bfloat16, out=None, stream=None):
+    """MXFP8 codes [n, D] + E8M0 bytes [n, D/32] -> values [n, D] (code * 2^(E - 127))."""
+    n, D = codes.shape
+    if out is None:
+        out = torch.empty((n, D), dtype=dtype, device=codes.device)
+    _check(lib().hsa_dequantize_mx(_ptr(codes), _ptr(scales), n, D, _ptr(out), _dtype(out),
+                                   _stream(stream)),
+           "hsa_dequantize_mx")
+    return out
+
+
+def mx_round(x, stream=None):
+    """Index queries [..., D] rounded onto the MXFP8 grid and returned as bf16 (quantize, then
+    dequantize: two library kernels).  The bf16-query index kernels then score MXFP8 queries."""
+    flat = x.reshape(-1, x.shape[-1])
+    codes, scales = hsa_quantize_mx(flat, stream=stream)
+    return hsa_dequantize_mx(codes, scales, torch.bfloat16, stream=stream).view(x.shape)
 
 
 def hsa_version() -> int:

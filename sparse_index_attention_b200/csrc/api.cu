@@ -67,7 +67,7 @@ hsa_paged_seq_t sub_rows(const hsa_paged_seq_t& s, int32_t t0, int32_t n) {
 
 hsa_status_t check_index(const hsa_paged_seq_t* seq, const void* q_I, hsa_dtype_t q_dtype,
                          const float* w, int32_t H_I, int32_t D_I, const void* k_cache,
-                         hsa_dtype_t k_dtype, const float* k_scale, const float* scores,
+                         hsa_dtype_t k_dtype, const void* k_scale, const float* scores,
                          int64_t ld) {
     hsa_status_t st = check_seq(seq);
     if (st != HSA_OK) return st;
@@ -77,14 +77,21 @@ hsa_status_t check_index(const hsa_paged_seq_t* seq, const void* q_I, hsa_dtype_
                 "H_I * D_I = %d too large", H_I * D_I);
     HSA_REQUIRE(q_dtype == HSA_F32 || q_dtype == HSA_BF16, HSA_ERR_UNSUPPORTED,
                 "q_I dtype must be F32 or BF16");
-    HSA_REQUIRE(k_dtype == HSA_F32 || k_dtype == HSA_BF16 || k_dtype == HSA_E4M3,
-                HSA_ERR_UNSUPPORTED, "k dtype must be F32, BF16 or E4M3");
+    HSA_REQUIRE(k_dtype == HSA_F32 || k_dtype == HSA_BF16 || k_dtype == HSA_E4M3 ||
+                    k_dtype == HSA_MXE4M3,
+                HSA_ERR_UNSUPPORTED, "k dtype must be F32, BF16, E4M3 or MXE4M3");
+    HSA_REQUIRE(k_dtype != HSA_MXE4M3 || D_I % 32 == 0, HSA_ERR_INVALID_ARG,
+                "MXE4M3 keys need D_I a multiple of 32 (D_I = %d)", D_I);
     HSA_REQUIRE(ld >= seq->max_seq_len, HSA_ERR_INVALID_ARG, "ld_scores = %lld < max_seq_len",
                 (long long)ld);
     if (seq->T_q > 0) {
         HSA_REQUIRE(q_I && w && k_cache && scores, HSA_ERR_INVALID_ARG, "NULL tensor pointer");
-        HSA_REQUIRE(k_dtype != HSA_E4M3 || k_scale, HSA_ERR_INVALID_ARG,
-                    "E4M3 keys need k_scale");
+        HSA_REQUIRE((k_dtype != HSA_E4M3 && k_dtype != HSA_MXE4M3) || k_scale,
+                    HSA_ERR_INVALID_ARG, "E4M3 and MXE4M3 keys need k_scale");
+        HSA_REQUIRE(k_dtype != HSA_E4M3 || aligned(k_scale, 4), HSA_ERR_INVALID_ARG,
+                    "misaligned k_scale");
+        HSA_REQUIRE(k_dtype != HSA_MXE4M3 || aligned(k_scale, 16), HSA_ERR_INVALID_ARG,
+                    "MXE4M3 k_scale must be 16-byte aligned");
         HSA_REQUIRE(aligned(q_I, dtype_size(q_dtype)) && aligned(w, 4) && aligned(scores, 4) &&
                         aligned(k_cache, dtype_size(k_dtype)),
                     HSA_ERR_INVALID_ARG, "misaligned tensor pointer");
@@ -130,7 +137,7 @@ hsa_status_t check_attn(const hsa_paged_seq_t* seq, const void* q, hsa_dtype_t q
 
 hsa::IndexScoreArgs index_args(const hsa_paged_seq_t* seq, const void* q_I, hsa_dtype_t q_dtype,
                                const float* w, int32_t H_I, int32_t D_I, const void* k_cache,
-                               hsa_dtype_t k_dtype, const float* k_scale, float* scores,
+                               hsa_dtype_t k_dtype, const void* k_scale, float* scores,
                                int64_t ld) {
     hsa::IndexScoreArgs a;
     a.seq = view(seq);
@@ -244,11 +251,11 @@ const char* hsa_status_string(hsa_status_t s) {
 
 const char* hsa_last_error_message(void) { return g_last_error.c_str(); }
 
-int32_t hsa_version(void) { return 200; }
+int32_t hsa_version(void) { return 300; }
 
 hsa_status_t hsa_index_score(const hsa_paged_seq_t* seq, const void* q_I, hsa_dtype_t q_dtype,
                              const float* w, int32_t H_I, int32_t D_I, const void* k_cache,
-                             hsa_dtype_t k_dtype, const float* k_scale, float* scores,
+                             hsa_dtype_t k_dtype, const void* k_scale, float* scores,
                              int64_t ld_scores, void* stream) {
     g_last_error.clear();
     hsa_status_t st = check_index(seq, q_I, q_dtype, w, H_I, D_I, k_cache, k_dtype, k_scale,
@@ -424,6 +431,41 @@ hsa_status_t hsa_quantize_kv(const void* src, hsa_dtype_t src_dtype, int64_t n_r
                                                  slot_mapping, num_slots, codes, scales, D_rope,
                                                  rope_cache, (cudaStream_t)stream),
                        "quantize_kv");
+}
+
+hsa_status_t hsa_quantize_mx(const void* src, hsa_dtype_t src_dtype, int64_t n_rows, int32_t D,
+                             const int64_t* slot_mapping, int64_t num_slots, uint8_t* codes,
+                             uint8_t* scales, void* stream) {
+    g_last_error.clear();
+    HSA_REQUIRE(src_dtype == HSA_F32 || src_dtype == HSA_BF16, HSA_ERR_UNSUPPORTED,
+                "source dtype must be F32 or BF16");
+    HSA_REQUIRE(n_rows >= 0 && D >= 32 && D % 32 == 0, HSA_ERR_INVALID_ARG,
+                "need n_rows >= 0 and D a positive multiple of 32 (n_rows=%lld D=%d)",
+                (long long)n_rows, D);
+    HSA_REQUIRE(num_slots >= 0 && (slot_mapping || n_rows <= num_slots), HSA_ERR_INVALID_ARG,
+                "identity slot mapping needs n_rows <= num_slots");
+    if (n_rows == 0) return HSA_OK;
+    HSA_REQUIRE(src && codes && scales, HSA_ERR_INVALID_ARG, "NULL tensor pointer");
+    HSA_REQUIRE(aligned(src, dtype_size(src_dtype)), HSA_ERR_INVALID_ARG, "misaligned source");
+    return cuda_status(hsa::launch_quantize_mx(src, src_dtype, n_rows, D, slot_mapping, num_slots,
+                                               codes, scales, (cudaStream_t)stream),
+                       "quantize_mx");
+}
+
+hsa_status_t hsa_dequantize_mx(const uint8_t* codes, const uint8_t* scales, int64_t n_rows,
+                               int32_t D, void* dst, hsa_dtype_t dst_dtype, void* stream) {
+    g_last_error.clear();
+    HSA_REQUIRE(dst_dtype == HSA_F32 || dst_dtype == HSA_BF16, HSA_ERR_UNSUPPORTED,
+                "destination dtype must be F32 or BF16");
+    HSA_REQUIRE(n_rows >= 0 && D >= 32 && D % 32 == 0, HSA_ERR_INVALID_ARG,
+                "need n_rows >= 0 and D a positive multiple of 32 (n_rows=%lld D=%d)",
+                (long long)n_rows, D);
+    if (n_rows == 0) return HSA_OK;
+    HSA_REQUIRE(codes && scales && dst, HSA_ERR_INVALID_ARG, "NULL tensor pointer");
+    HSA_REQUIRE(aligned(dst, dtype_size(dst_dtype)), HSA_ERR_INVALID_ARG, "misaligned destination");
+    return cuda_status(hsa::launch_dequantize_mx(codes, scales, n_rows, D, dst, dst_dtype,
+                                                 (cudaStream_t)stream),
+                       "dequantize_mx");
 }
 
 }  // extern "C"

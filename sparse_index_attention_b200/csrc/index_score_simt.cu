@@ -13,11 +13,13 @@ namespace {
 
 constexpr int kThreads = 128;
 
-template <typename QT, int KT>  // KT: 0 fp32 keys, 1 bf16 keys, 2 e4m3 keys + per-key scale
+// KT: 0 fp32 keys, 1 bf16 keys, 2 e4m3 keys + per-key fp32 scale, 3 MXFP8 keys (e4m3 codes,
+// one E8M0 byte per 32 dims, applied to each element: the scale varies along the dot product)
+template <typename QT, int KT>
 __global__ void __launch_bounds__(kThreads)
 index_score_simt_kernel(SeqView v, const QT* __restrict__ q_I, const float* __restrict__ w,
                         int H_I, int D_I, const void* __restrict__ k_cache,
-                        const float* __restrict__ k_scale, float* __restrict__ scores, int64_t ld) {
+                        const void* __restrict__ k_scale, float* __restrict__ scores, int64_t ld) {
     extern __shared__ float smem[];
     float* sq = smem;                 // [H_I * D_I]
     float* sw = smem + H_I * D_I;     // [H_I]
@@ -42,13 +44,17 @@ index_score_simt_kernel(SeqView v, const QT* __restrict__ q_I, const float* __re
                 kd = reinterpret_cast<const float*>(k_cache)[slot * D_I + d];
             else if (KT == 1)
                 kd = __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(k_cache)[slot * D_I + d]);
-            else
+            else if (KT == 2)
                 kd = e4m3_to_f32(reinterpret_cast<const uint8_t*>(k_cache)[slot * D_I + d]);
+            else
+                kd = e4m3_to_f32(reinterpret_cast<const uint8_t*>(k_cache)[slot * D_I + d]) *
+                     e8m0_to_f32(reinterpret_cast<const uint8_t*>(k_scale)[slot * (D_I / 32) + d / 32]);
             dot = fmaf(qj[d], kd, dot);
         }
         acc = fmaf(sw[j], fmaxf(dot, 0.f), acc);
     }
-    if (KT == 2) acc *= k_scale[slot];  // positive per-key scale factors out of the ReLU sum
+    if (KT == 2) acc *= reinterpret_cast<const float*>(k_scale)[slot];  // positive per-key scale
+                                                                        // factors out of the ReLU sum
     scores[(int64_t)t * ld + s] = acc;
 }
 
@@ -73,10 +79,12 @@ cudaError_t launch_index_score_simt(const IndexScoreArgs& a, cudaStream_t st) {
     if (a.q_dtype == HSA_F32) {
         if (a.k_dtype == HSA_F32) return launch_t<float, 0>(a, st);
         if (a.k_dtype == HSA_BF16) return launch_t<float, 1>(a, st);
+        if (a.k_dtype == HSA_MXE4M3) return launch_t<float, 3>(a, st);
         return launch_t<float, 2>(a, st);
     }
     if (a.k_dtype == HSA_F32) return launch_t<__nv_bfloat16, 0>(a, st);
     if (a.k_dtype == HSA_BF16) return launch_t<__nv_bfloat16, 1>(a, st);
+    if (a.k_dtype == HSA_MXE4M3) return launch_t<__nv_bfloat16, 3>(a, st);
     return launch_t<__nv_bfloat16, 2>(a, st);
 }
 

@@ -20,6 +20,11 @@
 // swizzle, two 64-column halves per page); FP8 keys are loaded raw and widened to bf16 in
 // shared memory by four converter warps (e4m3 -> bf16 is exact), and the per-key fp32 scale
 // multiplies the finished score (the scale is positive, so it commutes with the ReLU sum).
+// MXFP8 keys (one E8M0 byte per 32 dims; "Inference Adaptation and Performance Optimization for
+// a Domestically Developed LLM's New Architecture", section 4 table) take the same path: the
+// producer bulk-copies each box's scale words beside its codes, the converters scale each
+// 32-dim block by 2^(E_block - E_max) while widening (exact), and the epilogue multiplies the
+// score by 2^(E_max - 127), the key's largest block scale.
 //
 // Warp roles: 0 TMA producer, 1 MMA issuer (one elected thread each), 2-5 epilogue
 // (TMEM lane quarters 2,3,0,1), 6-9 FP8 converters (FP8 variant only).
@@ -38,17 +43,19 @@ constexpr int kHI = 64;                  // index heads
 constexpr int kHalfBytes = kBM * 128;    // one 64-column swizzled half of a key tile: 16 KB
 constexpr int kTileBytes = 2 * kHalfBytes;
 
-template <int G, bool kFp8>
+template <int G, bool kFp8, bool kMx = false>
 struct Cfg {
     static constexpr int N = G * kHI;
     static constexpr int kQBytes = N * kDI * 2;
     static constexpr int kStages = kFp8 ? (G == 1 ? 4 : (G == 2 ? 3 : 2)) : (G == 1 ? 6 : (G == 2 ? 5 : 4));
     static constexpr int kRawStages = kFp8 ? 4 : 0;          // FP8 staging tiles (16 KB each)
+    static constexpr int kScaleStageBytes = kMx ? kBM * 4 : 0;  // MXFP8: 4 E8M0 bytes per key
     static constexpr int kMaxGroups = G == 1 ? 2048 : 4096;
     static constexpr int kTmemCols = 2 * N;                   // 128, 256 or 512
     static constexpr int kThreads = kFp8 ? 320 : 192;
     static constexpr size_t kSmem = 1024 + (size_t)kStages * kTileBytes + (size_t)kRawStages * (kBM * kDI) +
-                                    kQBytes + 4 * (kMaxGroups + 1) + 4 * N + 256;
+                                    (size_t)kRawStages * kScaleStageBytes + kQBytes +
+                                    4 * (kMaxGroups + 1) + 4 * N + 256;
     static_assert(kSmem <= 232448, "shared memory budget");
 };
 
@@ -89,13 +96,14 @@ __device__ __forceinline__ int first_group(const int32_t* prefix, int n_groups, 
     return lo;
 }
 
-template <int G, bool kFp8>
-__global__ void __launch_bounds__(Cfg<G, kFp8>::kThreads, 1)
+template <int G, bool kFp8, bool kMx>
+__global__ void __launch_bounds__(Cfg<G, kFp8, kMx>::kThreads, 1)
 index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_q,
                       SeqView v, int32_t q_row0, const float* __restrict__ w,
-                      const float* __restrict__ k_scale, float* __restrict__ scores, int64_t ld,
+                      const void* __restrict__ k_scale, float* __restrict__ scores, int64_t ld,
                       int32_t box_rows) {
-    using C = Cfg<G, kFp8>;
+    using C = Cfg<G, kFp8, kMx>;
+    static_assert(!kMx || kFp8, "MXFP8 keys go through the FP8 staging path");
     constexpr int N = C::N;
     constexpr int S = C::kStages;
     constexpr uint32_t kIdesc = tc::idesc_bf16_f32(kBM, N, 0, 0);
@@ -104,7 +112,8 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
     uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* tiles = base;                                          // S x 32 KB (bf16, swizzled)
     uint8_t* raw = tiles + (size_t)S * kTileBytes;                  // FP8 staging
-    uint8_t* qbuf = raw + (size_t)C::kRawStages * (kBM * kDI);      // N x 128 bf16, swizzled
+    uint8_t* kscl = raw + (size_t)C::kRawStages * (kBM * kDI);      // MXFP8 scale words [4][128]
+    uint8_t* qbuf = kscl + (size_t)C::kRawStages * C::kScaleStageBytes;  // N x 128 bf16, swizzled
     // barriers first (8-byte alignment), then the variable-size arrays
     uint64_t* bars = reinterpret_cast<uint64_t*>(qbuf + C::kQBytes);
     uint64_t* full = bars;                 // [S]  keys landed (bf16 tile ready)
@@ -212,13 +221,17 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
                     } else {
                         if (!tc::mbar_wait(&empty[stage], phase ^ 1, abort_flag)) break;
                     }
-                    tc::mbar_arrive_expect_tx(bar, (uint32_t)(n_boxes * box_rows * (kFp8 ? 128 : 256)));
+                    tc::mbar_arrive_expect_tx(bar, (uint32_t)(n_boxes * box_rows * (kFp8 ? (kMx ? 132 : 128) : 256)));
                     for (int j = 0; j < n_boxes; ++j) {
                         const int s = s0 + j * box_rows;
                         const int32_t row = (int32_t)paged_slot(v, gi.b, s);
                         if (kFp8) {
                             uint8_t* dst = raw + (size_t)(stage & 3) * (kBM * kDI) + (size_t)j * box_rows * 128;
                             tc::tma_load_2d(dst, &tmap_k, bar, 0, row);
+                            if (kMx)   // the box's E8M0 words: box_rows x 4 bytes, 32-byte aligned
+                                tc::bulk_load(kscl + (size_t)(stage & 3) * C::kScaleStageBytes + (size_t)j * box_rows * 4,
+                                              static_cast<const uint8_t*>(k_scale) + (int64_t)row * 4,
+                                              (uint32_t)box_rows * 4, bar);
                         } else {
                             uint8_t* dst = tiles + (size_t)stage * kTileBytes + (size_t)j * box_rows * 128;
                             tc::tma_load_2d(dst, &tmap_k, bar, 0, row);
@@ -314,7 +327,19 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
                     int pmax = -1;
 #pragma unroll
                     for (int j = 0; j < G; ++j) pmax = max(pmax, row_pos[j]);
-                    if (s <= pmax) kscale = __ldg(k_scale + paged_slot(v, seq_b, s));
+                    if (s <= pmax) {
+                        const int64_t slot = paged_slot(v, seq_b, s);
+                        if (kMx) {
+                            // the largest of the key's four block exponents; the converters
+                            // scaled every block relative to it
+                            const uint32_t wd = __ldg(static_cast<const uint32_t*>(k_scale) + slot);
+                            const uint32_t emax = max(max(wd & 0xFFu, (wd >> 8) & 0xFFu),
+                                                      max((wd >> 16) & 0xFFu, wd >> 24));
+                            kscale = e8m0_to_f32(emax);
+                        } else {
+                            kscale = __ldg(static_cast<const float*>(k_scale) + slot);
+                        }
+                    }
                 }
 #pragma unroll
                 for (int j = 0; j < G; ++j) {
@@ -357,6 +382,17 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
                     const int r = 32 * cw + 4 * i + (lane >> 3);
                     const uint4 in = *reinterpret_cast<const uint4*>(src + r * 128 + c * 16);
                     const uint32_t words[4] = {in.x, in.y, in.z, in.w};
+                    float fct = 1.f;
+                    if (kMx) {
+                        // MXFP8: this lane's 16 codes lie in block c / 2 of the key; scale them
+                        // by 2^(E_block - E_max) (exact: a code has 4 significant bits) and
+                        // leave 2^(E_max - 127) to the epilogue
+                        const uint32_t wd = reinterpret_cast<const uint32_t*>(
+                            kscl + (size_t)(n & 3) * C::kScaleStageBytes)[r];
+                        const int emax = (int)max(max(wd & 0xFFu, (wd >> 8) & 0xFFu),
+                                                  max((wd >> 16) & 0xFFu, wd >> 24));
+                        fct = pow2_nonpos((int)((wd >> (8 * (c >> 1))) & 0xFFu) - emax);
+                    }
                     uint32_t outw[8];
 #pragma unroll
                     for (int q = 0; q < 4; ++q) {
@@ -364,7 +400,11 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
                         for (int hlf = 0; hlf < 2; ++hlf) {
                             const __nv_fp8x2_storage_t pair = (__nv_fp8x2_storage_t)(words[q] >> (16 * hlf));
                             const __half2_raw h2 = __nv_cvt_fp8x2_to_halfraw2(pair, __NV_E4M3);
-                            const float2 f2 = __half22float2(__half2(h2));
+                            float2 f2 = __half22float2(__half2(h2));
+                            if (kMx) {
+                                f2.x *= fct;
+                                f2.y *= fct;
+                            }
                             const __nv_bfloat162 b2 = __floats2bfloat162_rn(f2.x, f2.y);
                             outw[q * 2 + hlf] = *reinterpret_cast<const uint32_t*>(&b2);
                         }
@@ -404,9 +444,9 @@ int num_sms() {
     return n;
 }
 
-template <int G, bool kFp8>
+template <int G, bool kFp8, bool kMx>
 cudaError_t launch_g(const IndexScoreArgs& a, cudaStream_t st) {
-    using C = Cfg<G, kFp8>;
+    using C = Cfg<G, kFp8, kMx>;
     const int box_rows = a.seq.page_size <= kBM ? a.seq.page_size : kBM;
     const uint64_t slots = (uint64_t)a.seq.num_pages * a.seq.page_size;
     CUtensorMap tk, tq;
@@ -418,7 +458,7 @@ cudaError_t launch_g(const IndexScoreArgs& a, cudaStream_t st) {
                                   (uint64_t)a.seq.T_q * kHI, kDI, kDI * 2, 64, C::N,
                                   CU_TENSOR_MAP_SWIZZLE_128B);
     if (!ok) return cudaErrorInvalidValue;
-    auto kern = index_score_tc_kernel<G, kFp8>;
+    auto kern = index_score_tc_kernel<G, kFp8, kMx>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::kSmem);
     if (e != cudaSuccess) return e;
     const int rows_per_launch = C::kMaxGroups * G;
@@ -440,8 +480,11 @@ cudaError_t launch_g(const IndexScoreArgs& a, cudaStream_t st) {
 }  // namespace
 
 bool index_score_tc_supported(const IndexScoreArgs& a) {
-    if (a.q_dtype != HSA_BF16 || (a.k_dtype != HSA_BF16 && a.k_dtype != HSA_E4M3)) return false;
-    if (a.k_dtype == HSA_E4M3 && a.k_scale == nullptr) return false;
+    if (a.q_dtype != HSA_BF16 ||
+        (a.k_dtype != HSA_BF16 && a.k_dtype != HSA_E4M3 && a.k_dtype != HSA_MXE4M3))
+        return false;
+    if ((a.k_dtype == HSA_E4M3 || a.k_dtype == HSA_MXE4M3) && a.k_scale == nullptr) return false;
+    if (a.k_dtype == HSA_MXE4M3 && (reinterpret_cast<uintptr_t>(a.k_scale) & 15)) return false;
     if (a.H_I != kHI || a.D_I != kDI) return false;
     const int p = a.seq.page_size;
     if (p % 8 != 0) return false;
@@ -452,10 +495,12 @@ bool index_score_tc_supported(const IndexScoreArgs& a) {
 }
 
 cudaError_t launch_index_score_tc(const IndexScoreArgs& a, cudaStream_t st) {
-    const bool fp8 = a.k_dtype == HSA_E4M3;
-    if (a.q_run % 4 == 0) return fp8 ? launch_g<4, true>(a, st) : launch_g<4, false>(a, st);
-    if (a.q_run % 2 == 0) return fp8 ? launch_g<2, true>(a, st) : launch_g<2, false>(a, st);
-    return fp8 ? launch_g<1, true>(a, st) : launch_g<1, false>(a, st);
+    const bool fp8 = a.k_dtype == HSA_E4M3, mx = a.k_dtype == HSA_MXE4M3;
+    if (a.q_run % 4 == 0)
+        return mx ? launch_g<4, true, true>(a, st) : fp8 ? launch_g<4, true, false>(a, st) : launch_g<4, false, false>(a, st);
+    if (a.q_run % 2 == 0)
+        return mx ? launch_g<2, true, true>(a, st) : fp8 ? launch_g<2, true, false>(a, st) : launch_g<2, false, false>(a, st);
+    return mx ? launch_g<1, true, true>(a, st) : fp8 ? launch_g<1, true, false>(a, st) : launch_g<1, false, false>(a, st);
 }
 
 }  // namespace hsa

@@ -19,7 +19,7 @@ struct IndexScoreArgs {
     int32_t H_I, D_I;
     const void* k_cache;
     hsa_dtype_t k_dtype;
-    const float* k_scale;
+    const void* k_scale;   // E4M3: fp32 per key; MXE4M3: E8M0 bytes, D_I / 32 per key
     float* scores;
     int64_t ld;
 };
@@ -64,5 +64,11 @@ cudaError_t launch_quantize_rows(const void* src, hsa_dtype_t src_dtype, int64_t
                                  const int64_t* slot_mapping, int64_t num_slots, uint8_t* codes,
                                  float* scales, int32_t copy_cols, void* copy_dst,
                                  cudaStream_t st);
+// MXFP8: 32-element blocks, E8M0 scale bytes, E4M3 codes (rule in hsa.h).
+cudaError_t launch_quantize_mx(const void* src, hsa_dtype_t src_dtype, int64_t n_rows, int32_t D,
+                               const int64_t* slot_mapping, int64_t num_slots, uint8_t* codes,
+                               uint8_t* scales, cudaStream_t st);
+cudaError_t launch_dequantize_mx(const uint8_t* codes, const uint8_t* scales, int64_t n_rows,
+                                 int32_t D, void* dst, hsa_dtype_t dst_dtype, cudaStream_t st);
 
 }  // namespace hsa

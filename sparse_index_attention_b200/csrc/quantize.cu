@@ -7,6 +7,9 @@
 // Scale rule (dynamic max-abs): scale = amax / 448, inv = 448 / amax, both IEEE fp32 round to
 // nearest (this file is built without fast-math, so `/` is the correctly rounded division);
 // code = cvt.rn.satfinite to E4M3 of x * inv.  An all-zero group gets scale 1 and code 0.
+//
+// MXFP8 (the pages' format for the index Q/K): 32-element blocks share one E8M0 byte E = X + 127,
+// X = floor(log2(amax)) - 8 clamped to [-127, 127]; the codes are E4M3 of x * 2^-X.
 #include "kernels.h"
 
 namespace hsa {
@@ -80,7 +83,97 @@ cudaError_t launch_t(const void* src, int64_t n_rows, int32_t src_stride, int32_
     return cudaGetLastError();
 }
 
+// floor(log2(a)) of a positive finite float, from its bits (subnormals included).
+__device__ __forceinline__ int floor_log2(float a) {
+    const uint32_t bits = __float_as_uint(a);
+    const int e = (int)(bits >> 23);
+    if (e) return e - 127;
+    return (31 - __clz((int)(bits & 0x7FFFFFu))) - 149;
+}
+
+// MXFP8 ("Day 0 Inference Adaptation and Optimization for Hybrid Attention Models",
+// "Hierarchical Quantization": index Q/K in blocks of 32 sharing one exponent).
+// One warp per 32-element block, one element per lane.  X = floor(log2(amax)) - 8
+// clamped to [-127, 127]; the element is x * 2^-X (a power-of-two rescale, exact whenever the
+// result is at least 2^-126, and below that every candidate rounds to code 0) rounded to E4M3.
+template <typename T>
+__global__ void __launch_bounds__(kThreads)
+quantize_mx_kernel(const T* __restrict__ src, int64_t n_rows, int D,
+                   const int64_t* __restrict__ slot_mapping, int64_t num_slots,
+                   uint8_t* __restrict__ codes, uint8_t* __restrict__ scales) {
+    const int64_t warp = ((int64_t)blockIdx.x * kThreads + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    const int nb = D / 32;
+    if (warp >= n_rows * nb) return;
+    const int64_t r = warp / nb;
+    const int b = (int)(warp % nb);
+    const int64_t slot = slot_mapping ? slot_mapping[r] : r;
+    if (slot < 0 || slot >= num_slots) return;
+    const float x = to_f32(src[r * D + (int64_t)b * 32 + lane]);
+    float amax = fabsf(x);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    uint8_t code = 0;
+    int E = 0;
+    if (amax > 0.f) {
+        const int X = min(127, max(-127, floor_log2(amax) - 8));
+        E = X + 127;
+        // 2^-X: X lies in [-127, 119] (amax <= FLT_MAX), so the exponent field 127 - X lies in
+        // [8, 254] and the power of two is a normal float
+        const float inv = __uint_as_float((uint32_t)(127 - X) << 23);
+        code = (uint8_t)__nv_cvt_float_to_fp8(__fmul_rn(x, inv), __NV_SATFINITE, __NV_E4M3);
+    }
+    codes[slot * D + (int64_t)b * 32 + lane] = code;
+    if (lane == 0) scales[slot * nb + b] = (uint8_t)E;
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kThreads)
+dequantize_mx_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ scales,
+                     int64_t n, int D, T* __restrict__ dst) {
+    const int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x;
+    if (i >= n) return;
+    const int64_t r = i / D;
+    const int d = (int)(i % D);
+    const float v = e4m3_to_f32(codes[i]) * e8m0_to_f32(scales[r * (D / 32) + d / 32]);
+    if constexpr (sizeof(T) == 4)
+        dst[i] = v;
+    else
+        dst[i] = __float2bfloat16_rn(v);
+}
+
 }  // namespace
+
+cudaError_t launch_quantize_mx(const void* src, hsa_dtype_t src_dtype, int64_t n_rows, int32_t D,
+                               const int64_t* slot_mapping, int64_t num_slots, uint8_t* codes,
+                               uint8_t* scales, cudaStream_t st) {
+    if (n_rows == 0) return cudaSuccess;
+    const int64_t blocks = ceil_div(n_rows * (D / 32) * 32, kThreads);
+    if (src_dtype == HSA_F32)
+        quantize_mx_kernel<float><<<(unsigned)blocks, kThreads, 0, st>>>(
+            reinterpret_cast<const float*>(src), n_rows, D, slot_mapping, num_slots, codes, scales);
+    else
+        quantize_mx_kernel<__nv_bfloat16><<<(unsigned)blocks, kThreads, 0, st>>>(
+            reinterpret_cast<const __nv_bfloat16*>(src), n_rows, D, slot_mapping, num_slots, codes,
+            scales);
+    count_launch();
+    return cudaGetLastError();
+}
+
+cudaError_t launch_dequantize_mx(const uint8_t* codes, const uint8_t* scales, int64_t n_rows,
+                                 int32_t D, void* dst, hsa_dtype_t dst_dtype, cudaStream_t st) {
+    if (n_rows == 0) return cudaSuccess;
+    const int64_t n = n_rows * D;
+    const unsigned blocks = (unsigned)ceil_div(n, kThreads);
+    if (dst_dtype == HSA_F32)
+        dequantize_mx_kernel<float><<<blocks, kThreads, 0, st>>>(codes, scales, n, D,
+                                                                 reinterpret_cast<float*>(dst));
+    else
+        dequantize_mx_kernel<__nv_bfloat16><<<blocks, kThreads, 0, st>>>(
+            codes, scales, n, D, reinterpret_cast<__nv_bfloat16*>(dst));
+    count_launch();
+    return cudaGetLastError();
+}
 
 cudaError_t launch_quantize_rows(const void* src, hsa_dtype_t src_dtype, int64_t n_rows,
                                  int32_t src_stride, int32_t D, int32_t group,

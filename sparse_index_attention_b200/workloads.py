@@ -69,6 +69,7 @@ class Workload:
     K: int
     softmax_scale: float
     chunks: Optional[List[Tuple[int, int]]] = None   # query-row ranges in issue order
+    index_mx: bool = False          # index keys and queries in MXFP8 (E8M0 per 32 dims)
 
     @property
     def num_slots(self) -> int:
@@ -180,6 +181,16 @@ def decode_fp8(device="cpu", seed=3, B=128, L=65536, page_size=64, H_I=64, D_I=1
                   1.0 / math.sqrt(D_qk), True, True)
 
 
+def decode_mxfp8(device="cpu", seed=3, **kw):
+    """decode_fp8 (same seed, so the same draws) with the index queries and keys in MXFP8: blocks
+    of 32 dims sharing one power-of-two scale ("Inference Adaptation and Performance Optimization
+    for a Domestically Developed LLM's New Architecture", section 4 table; "Day 0 Inference
+    Adaptation and Optimization for Hybrid Attention Models", "Hierarchical Quantization").
+    The latent cache stays FP8 with an fp32 scale per token."""
+    wl = decode_fp8(device=device, seed=seed, **kw)
+    return dataclasses.replace(wl, name="decode_mxfp8", index_mx=True)
+
+
 def decode_draft_bf16(device="cpu", seed=5, B=64, n_draft=4, L_min=8192, L_max=32768,
                       page_size=64, H_I=64, D_I=128, H=128, D_v=512, D_rope=64, K=2048):
     """Draft-verify decode: each sequence checks n_draft drafted tokens in one step, so it has
@@ -224,6 +235,7 @@ RECIPES = {
     "prefill_bf16": prefill_bf16,
     "decode_fp8": decode_fp8,
     "decode_draft_bf16": decode_draft_bf16,
+    "decode_mxfp8": decode_mxfp8,
     "prefill_long_zigzag": prefill_long_zigzag,
 }
 

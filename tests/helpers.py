@@ -42,7 +42,11 @@ class GpuCaches:
         self.k_scale = None
         self.kv_scale = None
         self.kv_rope = None
-        if wl.index_fp8:
+        self.q_I = wl.q_I
+        if wl.index_mx:
+            self.k, self.k_scale = hsa.hsa_quantize_mx(wl.k_I)
+            self.q_I = hsa.mx_round(wl.q_I)
+        elif wl.index_fp8:
             self.k, sc = hsa.hsa_quantize_index(wl.k_I, wl.D_I)
             self.k_scale = sc.view(-1)
         else:
@@ -55,10 +59,16 @@ class GpuCaches:
 
 
 class OracleCaches:
-    """Exact values of the caches as the oracle reads them (its own quantizer for FP8)."""
+    """Exact values of the caches (and of the index queries) as the oracle reads them: its own
+    quantizers for FP8 and MXFP8."""
 
     def __init__(self, wl: workloads.Workload, need_kv: bool = True, kv_group=None):
-        if wl.index_fp8:
+        self.q_I = wl.q_I.cpu()
+        if wl.index_mx:
+            self.k = oracle.mx_dequantize_rows(*oracle.mx_quantize_rows(wl.k_I.float().cpu()))
+            q = wl.q_I.float().cpu().reshape(-1, wl.D_I)
+            self.q_I = oracle.mx_dequantize_rows(*oracle.mx_quantize_rows(q)).reshape(wl.q_I.shape)
+        elif wl.index_fp8:
             codes, sc = oracle.quantize_rows(wl.k_I.float().cpu(), wl.D_I)
             self.k = oracle.dequantize_rows(codes, sc, wl.D_I)
         else:

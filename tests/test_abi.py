@@ -19,7 +19,7 @@ def _declared():
 def test_header_declares_the_path():
     names = _declared()
     for n in ("hsa_index_score", "hsa_topk", "hsa_sparse_mla_attn", "hsa_fused_decode",
-              "hsa_quantize_index", "hsa_quantize_kv"):
+              "hsa_quantize_index", "hsa_quantize_kv", "hsa_quantize_mx", "hsa_dequantize_mx"):
         assert n in names
 
 
@@ -59,6 +59,23 @@ def test_validation_without_gpu():
                                    None)
         assert rc == want, group
         assert b"kv_scale_group" in L.hsa_last_error_message()
+    # MXFP8 keys: scales required and 16-byte aligned, D_I a multiple of 32
+    rc = L.hsa_index_score(ctypes.byref(seq), fake, hsa.HSA_BF16, fake, 4, 32, fake, hsa.HSA_MXE4M3,
+                           None, fake, 64, None)
+    assert rc == hsa.HSA_ERR_INVALID_ARG and b"k_scale" in L.hsa_last_error_message()
+    rc = L.hsa_index_score(ctypes.byref(seq), fake, hsa.HSA_BF16, fake, 4, 48, fake, hsa.HSA_MXE4M3,
+                           fake, fake, 64, None)
+    assert rc == hsa.HSA_ERR_INVALID_ARG and b"multiple of 32" in L.hsa_last_error_message()
+    rc = L.hsa_index_score(ctypes.byref(seq), fake, hsa.HSA_BF16, fake, 4, 32, fake, hsa.HSA_MXE4M3,
+                           ctypes.c_void_p(0x1004), fake, 64, None)
+    assert rc == hsa.HSA_ERR_INVALID_ARG and b"aligned" in L.hsa_last_error_message()
+    # MXFP8 quantizer: blocks of 32, F32/BF16 sources
+    assert L.hsa_quantize_mx(fake, hsa.HSA_BF16, 10, 48, None, 10, fake, fake, None) == hsa.HSA_ERR_INVALID_ARG
+    assert L.hsa_quantize_mx(fake, hsa.HSA_E4M3, 10, 64, None, 10, fake, fake, None) == hsa.HSA_ERR_UNSUPPORTED
+    assert L.hsa_quantize_mx(fake, hsa.HSA_BF16, 11, 64, None, 10, fake, fake, None) == hsa.HSA_ERR_INVALID_ARG
+    assert L.hsa_dequantize_mx(fake, fake, 10, 40, fake, hsa.HSA_BF16, None) == hsa.HSA_ERR_INVALID_ARG
+    assert L.hsa_dequantize_mx(fake, fake, 10, 64, fake, hsa.HSA_E4M3, None) == hsa.HSA_ERR_UNSUPPORTED
+    assert L.hsa_quantize_mx(None, hsa.HSA_BF16, 0, 64, None, 0, None, None, None) == hsa.HSA_OK
     # zero rows is a no-op, not an error
     empty = hsa.hsa_paged_seq_t(1, fake, fake, 4, 16, 4, 64, 0, None, None, 1, None)
     assert L.hsa_topk(ctypes.byref(empty), None, 64, 8, None, None) == hsa.HSA_OK

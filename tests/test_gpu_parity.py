@@ -23,12 +23,12 @@ DEV = "cuda"
 def _index_vs_oracle(wl, rows=None):
     gc = GpuCaches(wl)
     seq = paged_seq(wl)
-    sc = hsa.hsa_index_score(seq, wl.q_I, wl.w, gc.k, gc.k_scale)
+    sc = hsa.hsa_index_score(seq, gc.q_I, wl.w, gc.k, gc.k_scale)
     check_status(seq)
     rows = list(range(wl.T_q)) if rows is None else rows
     oc = OracleCaches(wl, need_kv=False)
     pg = oracle_paging(wl, rows)
-    qI, w = wl.q_I[rows].cpu(), wl.w[rows].cpu()
+    qI, w = oc.q_I[rows], wl.w[rows].cpu()
     ref = oracle.index_score(pg, qI, w, oc.k, ld=sc.shape[1])
     mag = oracle.index_score(pg, qI, w.abs(), oc.k, ld=sc.shape[1])
     got = sc[rows].cpu().numpy()
@@ -48,6 +48,19 @@ def _index_vs_oracle(wl, rows=None):
 ])
 def test_index_score_vs_oracle(name, kw):
     _index_vs_oracle(workloads.make(name, DEV, **kw))
+
+
+@pytest.mark.parametrize("name,kw", [
+    ("tiny_decode_fp32", {}),                       # CUDA-core kernel (4 x 32 indexer)
+    ("decode_bf16", dict(B=5, L_min=100, L_max=1500)),   # tensor-core kernel, one row per tile
+    ("prefill_bf16", dict(T=700)),                  # tensor-core kernel, four rows per tile
+])
+def test_index_score_mxfp8_vs_oracle(name, kw):
+    """MXFP8 index queries and keys (E8M0 scale per 32 dims) on both index kernels, against the
+    oracle's own MX quantizer and the float64 score of the dequantized values."""
+    wl = workloads.make(name, DEV, **kw)
+    wl.index_fp8 = wl.index_mx = True
+    _index_vs_oracle(wl)
 
 
 @pytest.mark.parametrize("q_run,T", [(1, 2500), (2, 600), (4, 300)])
@@ -108,6 +121,74 @@ def test_index_score_fp8_every_code_bit_exact():
     ref = (oracle.e4m3_decode(codes) * scale.cpu()[slot].double().numpy()).astype(np.float32)
     assert len(set(codes.tolist())) == 254                   # every finite code is exercised
     assert np.array_equal(sc[0, :n].cpu().numpy(), ref)
+
+
+def test_index_score_mxfp8_every_code_bit_exact():
+    """Every finite E4M3 code through the MXFP8 key path of the tensor-core kernel, with the four
+    block exponents of a key all different and the largest one in any of the four blocks.  Key s
+    holds one code in all 128 dims; index heads 0-3 read dim 32b of block b with q = +1 and heads
+    4-7 with q = -1, weights +1 and -1, so the score is exactly sum_b decode(code) 2^(E_b - 127):
+    the converters' per-block rescale and the epilogue's 2^(E_max - 127) must recombine bit for
+    bit, down to scale byte 0 (2^-127) and up to 2^117."""
+    wl = workloads.make("decode_fp8", DEV, B=1, L=1536)
+    slots = wl.num_pages * wl.page_size
+    code_of_slot = torch.arange(slots, dtype=torch.int64) % 256
+    code_of_slot[(code_of_slot & 0x7F) == 0x7F] = 0
+    k8 = code_of_slot.to(torch.uint8)[:, None].expand(slots, wl.D_I).contiguous().to(DEV)
+    bases = torch.tensor([0, 1, 60, 127, 200, 240])
+    sl = torch.arange(slots)
+    base = bases[(sl // 256) % len(bases)]
+    E = torch.stack([base + (sl + 3 * b) % 4 for b in range(4)], dim=1).to(torch.uint8)
+    q = torch.zeros((1, wl.H_I, wl.D_I), dtype=torch.bfloat16)
+    w = torch.zeros((1, wl.H_I), dtype=torch.float32)
+    for b in range(4):
+        q[0, b, 32 * b], q[0, 4 + b, 32 * b] = 1.0, -1.0
+        w[0, b], w[0, 4 + b] = 1.0, -1.0
+    seq = hsa.PagedSeq(wl.seq_lens, wl.block_table, wl.page_size, wl.num_pages,
+                       wl.q_seq[:1], wl.q_pos[:1], max_seq_len=int(wl.seq_lens.max()),
+                       status=torch.zeros(1, dtype=torch.int32, device=DEV))
+    sc = hsa.hsa_index_score(seq, q.to(DEV), w.to(DEV), k8, E.contiguous().to(DEV))
+    check_status(seq)
+    n = int(wl.q_pos[0]) + 1
+    bt = wl.block_table[0].cpu().long()
+    pos = torch.arange(n)
+    slot = bt[pos // wl.page_size] * wl.page_size + pos % wl.page_size
+    codes = code_of_slot[slot].numpy().astype(np.uint8)
+    vals = oracle.e4m3_decode(codes)
+    ref = sum(vals * np.exp2(E[slot, b].double().numpy() - 127) for b in range(4))
+    assert len(set(codes.tolist())) == 254
+    assert np.array_equal(sc[0, :n].cpu().numpy().astype(np.float64), ref)
+
+
+@pytest.mark.parametrize("src_dtype", [torch.bfloat16, torch.float32])
+def test_quantize_mx_bit_exact(src_dtype):
+    """hsa_quantize_mx against the oracle's MX quantizer, scattered through a slot permutation:
+    N(0,1) keys scaled per row by 2^-40..2^40, the hand-worked golden blocks, every E4M3
+    midpoint at the top binade's scale, all-zero and sub-2^-119 blocks."""
+    g = torch.Generator().manual_seed(21)
+    x = torch.randn((4096, 128), generator=g) * torch.exp2(torch.randint(-40, 41, (4096, 1), generator=g).float())
+    vals = oracle.e4m3_decode(np.arange(0, 0x7F, dtype=np.uint8))
+    mids = torch.from_numpy(((vals[:-1] + vals[1:]) / 2).astype(np.float32))
+    mid_rows = torch.cat([mids, -mids, torch.zeros((-2 * mids.numel()) % 127)]).view(-1, 127)
+    mid_rows = torch.cat([torch.full((mid_rows.shape[0], 1), 448.0), mid_rows], 1)   # E = 127
+    edge = torch.zeros((3, 128))
+    edge[1, :32] = 2.0 ** -130
+    edge[1, 40] = -(2.0 ** -140)
+    edge[2, 64:96] = torch.linspace(-3e38, 3e38, 32)
+    x = torch.cat([x, mid_rows, edge]).to(src_dtype)
+    n = x.shape[0]
+    perm = torch.randperm(n, generator=g)
+    codes, scales = hsa.hsa_quantize_mx(x.to(DEV), slot_mapping=perm.to(DEV), num_slots=n)
+    rc, rs = oracle.mx_quantize_rows(x.float())
+    assert np.array_equal(codes.cpu()[perm].numpy(), rc)
+    assert np.array_equal(scales.cpu()[perm].numpy(), rs)
+    # dequantized values are exact in fp32; in bf16 for every block with E >= 3
+    ref = oracle.mx_dequantize_rows(rc, rs)
+    d32 = hsa.hsa_dequantize_mx(torch.from_numpy(rc).to(DEV), torch.from_numpy(rs).to(DEV), torch.float32)
+    assert np.array_equal(d32.cpu().numpy().astype(np.float64), ref)
+    d16 = hsa.hsa_dequantize_mx(torch.from_numpy(rc).to(DEV), torch.from_numpy(rs).to(DEV))
+    big = np.repeat(rs >= 3, 32, axis=1)
+    assert np.array_equal(d16.float().cpu().numpy().astype(np.float64)[big], ref[big])
 
 
 def test_index_score_paging_invariance_bitwise():

@@ -18,8 +18,8 @@ import oracle
 import sparse_index_attention_b200 as hsa
 from sparse_index_attention_b200 import workloads
 
-from helpers import (GpuCaches, OracleCaches, attn_close, check_status, index_tolerance_ok,
-                     oracle_paging, paged_seq, stable_topk_reference)
+from helpers import (GpuCaches, OracleCaches, attn_close, check_status, compact_workload,
+                     index_tolerance_ok, oracle_paging, paged_seq, stable_topk_reference)
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -29,7 +29,7 @@ TOL = {"f32": 1e-4, "bf16": 2e-2}
 def run_fused(wl, gc, aux=False):
     seq = paged_seq(wl)
     aux_stream = torch.cuda.Stream() if aux else None
-    out, lse, idx, sc = hsa.hsa_fused_decode(seq, wl.q_I, wl.w, gc.k, gc.k_scale, wl.q, gc.kv,
+    out, lse, idx, sc = hsa.hsa_fused_decode(seq, gc.q_I, wl.w, gc.k, gc.k_scale, wl.q, gc.kv,
                                              gc.kv_scale, gc.kv_rope, wl.K, wl.D_v,
                                              wl.softmax_scale, aux_stream=aux_stream)
     check_status(seq)
@@ -43,7 +43,7 @@ def check_against_oracle(wl, rows, sc, idx, out):
     assert torch.equal(idx[rows], ref_sel), "Top-K differs from the stable-sort selection"
     oc = OracleCaches(wl)
     pg = oracle_paging(wl, rows)
-    qI, w = wl.q_I[rows].cpu(), wl.w[rows].cpu()
+    qI, w = oc.q_I[rows], wl.w[rows].cpu()
     ld = sc.shape[1]
     ref_sc = oracle.index_score(pg, qI, w, oc.k, ld=ld)
     mag = oracle.index_score(pg, qI, w.abs(), oc.k, ld=ld)
@@ -78,6 +78,7 @@ def check_against_oracle(wl, rows, sc, idx, out):
     ("tiny_decode_fp32", {}),
     ("decode_bf16", dict(B=8, L_min=1500, L_max=5000)),
     ("decode_fp8", dict(B=4, L=4500)),
+    ("decode_mxfp8", dict(B=4, L=4500)),
     ("decode_draft_bf16", dict(B=5, L_min=1500, L_max=5000)),
     ("decode_draft_bf16", dict(B=3, n_draft=2, L_min=2040, L_max=2052)),
 ])
@@ -94,6 +95,7 @@ def test_pipeline_vs_oracle_small(name, kw):
     ("decode_fp8", dict(B=6, L=3000), None),
     ("decode_fp8", dict(B=6, L=3000), 128),
     ("decode_draft_bf16", dict(B=6, L_min=1500, L_max=5000), None),
+    ("decode_mxfp8", dict(B=6, L=3000), 128),
 ])
 def test_fused_equals_unfused_and_two_streams(name, kw, kv_group):
     wl = workloads.make(name, DEV, **kw)
@@ -101,7 +103,7 @@ def test_fused_equals_unfused_and_two_streams(name, kw, kv_group):
     out1, lse1, idx1, sc1 = run_fused(wl, gc, aux=False)
     out2, lse2, idx2, sc2 = run_fused(wl, gc, aux=True)
     seq = paged_seq(wl)
-    sc3 = hsa.hsa_index_score(seq, wl.q_I, wl.w, gc.k, gc.k_scale)
+    sc3 = hsa.hsa_index_score(seq, gc.q_I, wl.w, gc.k, gc.k_scale)
     idx3 = hsa.hsa_topk(seq, sc3, wl.K)
     out3, lse3 = hsa.hsa_sparse_mla_attn(seq, wl.q, gc.kv, idx3, wl.D_v, wl.softmax_scale,
                                          kv_scale=gc.kv_scale, kv_rope=gc.kv_rope)
@@ -139,6 +141,21 @@ def test_decode_draft_full_size_sampled():
     assert torch.equal(idx, ref_sel)
     rows = [r for b in (0, 29, 63) for r in range(4 * b, 4 * b + 4)]
     check_against_oracle(wl, rows, sc, idx, out)
+
+
+def test_decode_mxfp8_full_size_sampled():
+    """The tiered-quantization decode at full size (128 sequences x 65536 keys, Top-2048) with
+    the index queries and keys in MXFP8 and the latent cache in FP8: Top-K bit-exact on every
+    row, oracle checks on three rows."""
+    wl = workloads.make("decode_mxfp8", DEV)
+    gc = GpuCaches(wl)
+    out, lse, idx, sc = run_fused(wl, gc)
+    ref_sel = stable_topk_reference(sc, wl.q_pos, wl.K)
+    assert torch.equal(idx, ref_sel)
+    rows = [0, 77, 127]
+    small = compact_workload(wl, rows)    # the oracle quantizes only these rows' pages
+    del gc
+    check_against_oracle(small, list(range(len(rows))), sc[rows], idx[rows], out[rows])
 
 
 @pytest.mark.parametrize("aux", [False, True])
