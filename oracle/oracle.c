@@ -168,6 +168,8 @@ int oracle_mx_quantize_rows(const float* x, int64_t n_rows, int32_t D, uint8_t* 
                             uint8_t* scales) {
     if (n_rows < 0 || D <= 0 || D % 32 != 0) return ORACLE_BAD_ARG;
     const int32_t nb = D / 32;
+    for (int64_t i = 0; i < n_rows * (int64_t)D; ++i)   /* the MX rule is defined on finite data */
+        if (!isfinite(x[i])) return ORACLE_NOT_FINITE;
 #pragma omp parallel for schedule(static)
     for (int64_t r = 0; r < n_rows; ++r) {
         for (int32_t b = 0; b < nb; ++b) {

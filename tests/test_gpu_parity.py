@@ -174,8 +174,9 @@ def test_quantize_mx_bit_exact(src_dtype):
     edge = torch.zeros((3, 128))
     edge[1, :32] = 2.0 ** -130
     edge[1, 40] = -(2.0 ** -140)
-    edge[2, 64:96] = torch.linspace(-3e38, 3e38, 32)
+    edge[2, 64:96] = torch.linspace(-1.0, 1.0, 32) * 3e38          # finite, near the float32 top
     x = torch.cat([x, mid_rows, edge]).to(src_dtype)
+    assert torch.isfinite(x).all()
     n = x.shape[0]
     perm = torch.randperm(n, generator=g)
     codes, scales = hsa.hsa_quantize_mx(x.to(DEV), slot_mapping=perm.to(DEV), num_slots=n)

@@ -263,3 +263,10 @@ def test_mx_values_on_the_grid_are_fixed_points():
         same = oracle.e4m3_decode(got_c) == oracle.e4m3_decode(codes)   # +0 and -0 both decode to 0
         assert same.all()
         assert np.array_equal(oracle.mx_dequantize_rows(got_c, got_s), vals)
+
+
+def test_mx_rejects_non_finite_input():
+    x = np.zeros((1, 32), dtype=np.float32)
+    x[0, 3] = np.inf
+    with pytest.raises(oracle.OracleError):
+        oracle.mx_quantize_rows(x)
