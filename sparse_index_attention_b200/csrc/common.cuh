@@ -99,13 +99,6 @@ __device__ __forceinline__ float e8m0_to_f32(uint32_t E) {
     return E ? __uint_as_float(E << 23) : __uint_as_float(1u << 22);
 }
 
-// 2^k for k <= 0 as a float: normal down to 2^-126, subnormal down to 2^-149, 0 below.
-__device__ __forceinline__ float pow2_nonpos(int k) {
-    if (k >= -126) return __uint_as_float((uint32_t)(127 + k) << 23);
-    if (k >= -149) return __uint_as_float(1u << (149 + k));
-    return 0.f;
-}
-
 template <typename T>
 __device__ __forceinline__ float load_f32(const void* p, int64_t i) {
     return to_f32(reinterpret_cast<const T*>(p)[i]);

@@ -22,9 +22,10 @@
 // multiplies the finished score (the scale is positive, so it commutes with the ReLU sum).
 // MXFP8 keys (one E8M0 byte per 32 dims; "Inference Adaptation and Performance Optimization for
 // a Domestically Developed LLM's New Architecture", section 4 table) take the same path: the
-// producer bulk-copies each box's scale words beside its codes, the converters scale each
-// 32-dim block by 2^(E_block - E_max) while widening (exact), and the epilogue multiplies the
-// score by 2^(E_max - 127), the key's largest block scale.
+// producer bulk-copies each box's scale words beside its codes, the converters widen the codes
+// by placing their bits in bf16s and scale each 32-dim block by 2^(E_block - E_max) with one
+// packed multiply (exact), and the epilogue multiplies the score by 2^(E_max - 127), the key's
+// largest block scale.
 //
 // Warp roles: 0 TMA producer, 1 MMA issuer (one elected thread each), 2-5 epilogue
 // (TMEM lane quarters 2,3,0,1), 6-9 FP8 converters (FP8 variant only).
@@ -382,31 +383,45 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
                     const int r = 32 * cw + 4 * i + (lane >> 3);
                     const uint4 in = *reinterpret_cast<const uint4*>(src + r * 128 + c * 16);
                     const uint32_t words[4] = {in.x, in.y, in.z, in.w};
-                    float fct = 1.f;
+                    uint32_t outw[8];
                     if (kMx) {
-                        // MXFP8: this lane's 16 codes lie in block c / 2 of the key; scale them
-                        // by 2^(E_block - E_max) (exact: a code has 4 significant bits) and
-                        // leave 2^(E_max - 127) to the epilogue
+                        // MXFP8: this lane's 16 codes lie in block c / 2 of the key.  Each code's
+                        // sign, exponent and mantissa bits are placed in a bf16 (2^-120 times the
+                        // code's value; a subnormal code becomes a bf16 subnormal), and one packed
+                        // multiply by 2^(120 + E_block - E_max) gives code x 2^(E_block - E_max)
+                        // exactly; 2^(E_max - 127) is left to the epilogue.  A block more than
+                        // 2^246 below the key's largest is flushed to zero.
                         const uint32_t wd = reinterpret_cast<const uint32_t*>(
                             kscl + (size_t)(n & 3) * C::kScaleStageBytes)[r];
                         const int emax = (int)max(max(wd & 0xFFu, (wd >> 8) & 0xFFu),
                                                   max((wd >> 16) & 0xFFu, wd >> 24));
-                        fct = pow2_nonpos((int)((wd >> (8 * (c >> 1))) & 0xFFu) - emax);
-                    }
-                    uint32_t outw[8];
+                        const int fe = 247 + (int)((wd >> (8 * (c >> 1))) & 0xFFu) - emax;
+                        const uint32_t fb = fe > 0 ? (uint32_t)fe << 7 : 0u;
+                        const uint32_t fb2 = fb | (fb << 16);
+                        const __nv_bfloat162 f2 = *reinterpret_cast<const __nv_bfloat162*>(&fb2);
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) {
+                        for (int q = 0; q < 4; ++q) {
 #pragma unroll
-                        for (int hlf = 0; hlf < 2; ++hlf) {
-                            const __nv_fp8x2_storage_t pair = (__nv_fp8x2_storage_t)(words[q] >> (16 * hlf));
-                            const __half2_raw h2 = __nv_cvt_fp8x2_to_halfraw2(pair, __NV_E4M3);
-                            float2 f2 = __half22float2(__half2(h2));
-                            if (kMx) {
-                                f2.x *= fct;
-                                f2.y *= fct;
+                            for (int hlf = 0; hlf < 2; ++hlf) {
+                                // codes 2*hlf and 2*hlf+1 of the word into the low and high bf16
+                                const uint32_t t = __byte_perm(words[q], 0u, hlf ? 0x4342u : 0x4140u);
+                                const uint32_t bits = ((t & 0x00800080u) << 8) | ((t & 0x007F007Fu) << 4);
+                                const __nv_bfloat162 v2 =
+                                    __hmul2(*reinterpret_cast<const __nv_bfloat162*>(&bits), f2);
+                                outw[q * 2 + hlf] = *reinterpret_cast<const uint32_t*>(&v2);
                             }
-                            const __nv_bfloat162 b2 = __floats2bfloat162_rn(f2.x, f2.y);
-                            outw[q * 2 + hlf] = *reinterpret_cast<const uint32_t*>(&b2);
+                        }
+                    } else {
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+#pragma unroll
+                            for (int hlf = 0; hlf < 2; ++hlf) {
+                                const __nv_fp8x2_storage_t pair = (__nv_fp8x2_storage_t)(words[q] >> (16 * hlf));
+                                const __half2_raw h2 = __nv_cvt_fp8x2_to_halfraw2(pair, __NV_E4M3);
+                                const float2 f2 = __half22float2(__half2(h2));
+                                const __nv_bfloat162 b2 = __floats2bfloat162_rn(f2.x, f2.y);
+                                outw[q * 2 + hlf] = *reinterpret_cast<const uint32_t*>(&b2);
+                            }
                         }
                     }
                     uint8_t* rbase = dst + r * 128;
