@@ -130,3 +130,30 @@ def test_decode_fp8_full_size_sampled():
     assert torch.equal(idx, stable_topk_batched(sc, wl.q_pos, wl.K))
     rows = [0, 77, 127]
     check_rows(wl, rows, sc[rows], idx[rows], out[rows], 6e-2)
+
+
+def test_zigzag_cp_single_rank_equals_chunked_prefill():
+    """The context-parallel prefill on one NCCL rank (segments 0 and 1 of 2, the cache gathered
+    from itself and read through the rebuilt block table) gives the same bits as the chunked
+    prefill over the workload's own paging: the whole host path down to the library kernels."""
+    import datetime
+    import socket
+    import torch.distributed as dist
+    from sparse_index_attention_b200 import cp
+    wl = workloads.make("prefill_bf16", DEV, T=2048)
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{port}", rank=0, world_size=1,
+                            timeout=datetime.timedelta(seconds=60), device_id=torch.device(DEV, 0))
+    try:
+        pos = cp.rank_positions(wl.T_q, 1, 0).to(DEV).long()
+        slot = wl.block_table[0].long()[pos // wl.page_size] * wl.page_size + pos % wl.page_size
+        out_c, lse_c, idx_c = cp.prefill_zigzag_cp(
+            wl.T_q, wl.page_size, wl.q_I[pos], wl.w[pos], wl.q[pos], wl.k_I[slot], wl.kv[slot], wl.K,
+            wl.D_v, wl.softmax_scale, gather_outputs=True)
+        torch.cuda.synchronize()
+    finally:
+        dist.destroy_process_group()
+    _, _, out, lse, idx = run_prefill(wl, [(0, 1024), (1024, 2048)])
+    assert torch.equal(idx_c, idx) and torch.equal(out_c, out) and torch.equal(lse_c, lse)
