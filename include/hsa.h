@@ -12,7 +12,8 @@
  *   3. sparse MLA attention reads only the selected rows of the paged latent KV cache
  *      (latent c_kv || rope part per position, shared by every head) and attends over them.
  * FP8 storage of index keys and latent KV ("Hierarchical Quantization" on the first page;
- * the table of section 4 on the fifth) is written by hsa_quantize_index / hsa_quantize_kv.
+ * the table of section 4 on the fifth) is written by hsa_quantize_index / hsa_quantize_kv
+ * (E4M3 with fp32 scales) and hsa_quantize_mx (MXFP8: E8M0 scale per 32 elements).
  *
  * Conventions shared by every call
  *  - Memory: every tensor is caller-owned device memory, row-major and contiguous unless a

@@ -86,3 +86,21 @@ def test_missing_library_fails_loudly(monkeypatch):
     monkeypatch.setattr(hsa, "LIB_PATH", "/nonexistent/libhsa.so")
     with pytest.raises(RuntimeError, match="no fallback"):
         hsa.lib()
+
+
+def test_plain_c_program_links_and_validates(tmp_path):
+    """The header compiles as C99 with warnings as errors, and a C program linked against
+    libhsa.so gets the documented status codes from the host-side checks."""
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    assert gcc, "gcc is needed to build the C ABI check"
+    hsa.lib()                                   # the library is built
+    libdir = os.path.dirname(hsa.LIB_PATH)
+    exe = str(tmp_path / "c_abi_check")
+    subprocess.run([gcc, "-std=c99", "-Wall", "-Wextra", "-Werror", "-pedantic",
+                    "-I", os.path.join(ROOT, "include"), os.path.join(ROOT, "tests", "c_abi_check.c"),
+                    "-L", libdir, "-lhsa", "-Wl,-rpath," + libdir, "-o", exe], check=True)
+    r = subprocess.run([exe], capture_output=True, text=True, timeout=60)
+    assert r.returncode == 0, r.stderr
+    assert r.stdout.strip() == "c abi ok"
