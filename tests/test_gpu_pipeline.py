@@ -158,6 +158,23 @@ def test_decode_mxfp8_full_size_sampled():
     check_against_oracle(small, list(range(len(rows))), sc[rows], idx[rows], out[rows])
 
 
+def test_draft_verify_with_mxfp8_index_and_fp8_latent():
+    """Draft-verify rows (four per sequence, scored four to an MMA tile) over the tiered caches:
+    MXFP8 index queries and keys, FP8 latent cache with a scale per token; all rows against the
+    oracle, and the fused call equal to the three calls in sequence."""
+    wl = workloads.make("decode_draft_bf16", DEV, B=6, L_min=1500, L_max=5000)
+    wl.index_fp8 = wl.index_mx = wl.kv_fp8 = True
+    gc = GpuCaches(wl)
+    out, lse, idx, sc = run_fused(wl, gc)
+    check_against_oracle(wl, list(range(wl.T_q)), sc, idx, out)
+    seq = paged_seq(wl)
+    sc3 = hsa.hsa_index_score(seq, gc.q_I, wl.w, gc.k, gc.k_scale)
+    idx3 = hsa.hsa_topk(seq, sc3, wl.K)
+    out3, lse3 = hsa.hsa_sparse_mla_attn(seq, wl.q, gc.kv, idx3, wl.D_v, wl.softmax_scale,
+                                         kv_scale=gc.kv_scale, kv_rope=gc.kv_rope)
+    assert torch.equal(idx, idx3) and torch.equal(out, out3) and torch.equal(lse, lse3)
+
+
 @pytest.mark.parametrize("aux", [False, True])
 def test_decode_graph_replays_bitwise(aux):
     """The fused decode step captured as a CUDA graph equals the direct call bitwise, and a
