@@ -382,6 +382,52 @@ def mx_round(x, stream=None):
     return hsa_dequantize_mx(codes, scales, torch.bfloat16, stream=stream).view(x.shape)
 
 
+def hsa_decode_prolog(new_k, new_kv, slot_mapping, k_cache, k_scale, kv_cache, kv_scale, kv_rope,
+                      q_I, q_I_out, D_v: int, kv_group: Optional[int] = None, streams=None,
+                      stream=None):
+    """The writes that precede a decode step, on three streams: the new tokens' index keys into
+    the index key cache, their latent rows into the FP8 latent cache, and the index queries
+    rounded onto the MXFP8 grid into ``q_I_out`` ("Day 0 Inference Adaptation and Optimization
+    for Hybrid Attention Models", "Sparse Attention Pipeline Optimization": independent
+    prolog operators on concurrent streams; "Inference Adaptation and Performance Optimization
+    for a Domestically Developed LLM's New Architecture", 3.3).  ``stream`` (default: current)
+    waits for all three, so a decode step issued on it next sees the new rows.
+
+    new_k [n, D_I] and new_kv [n, D_v + D_rope] (F32/BF16) go to physical slots
+    ``slot_mapping`` [n] (int64).  The index key cache is MXFP8 when ``k_scale`` is uint8
+    (E8M0 bytes, [slots, D_I/32]) and E4M3 with one fp32 scale per key otherwise.  The latent
+    cache is E4M3 with one fp32 scale per ``kv_group`` dims (default D_v) plus bf16 rope.
+    Results equal the same calls issued one after another on one stream."""
+    main = torch.cuda.current_stream() if stream is None else stream
+    if streams is None:
+        streams = (torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream())
+    start = torch.cuda.Event()
+    start.record(main)
+    for st in streams:
+        st.wait_event(start)
+    num_slots = k_cache.shape[0]
+    s_k, s_kv, s_q = streams
+    if k_scale.dtype == torch.uint8:
+        hsa_quantize_mx(new_k, slot_mapping, num_slots, codes=k_cache, scales=k_scale, stream=s_k)
+    else:
+        hsa_quantize_index(new_k, new_k.shape[1], slot_mapping, num_slots, codes=k_cache,
+                           scales=k_scale.view(num_slots, 1), stream=s_k)
+    grp = kv_group or D_v
+    hsa_quantize_kv(new_kv, D_v, grp, slot_mapping, kv_cache.shape[0], codes=kv_cache,
+                    scales=kv_scale.view(kv_cache.shape[0], D_v // grp), rope_cache=kv_rope,
+                    stream=s_kv)
+    flat = q_I.reshape(-1, q_I.shape[-1])
+    codes = torch.empty(flat.shape, dtype=torch.uint8, device=flat.device)
+    scales = torch.empty((flat.shape[0], flat.shape[1] // 32), dtype=torch.uint8, device=flat.device)
+    hsa_quantize_mx(flat, codes=codes, scales=scales, stream=s_q)
+    hsa_dequantize_mx(codes, scales, out=q_I_out.view(flat.shape), stream=s_q)
+    for st in streams:
+        done = torch.cuda.Event()
+        done.record(st)
+        main.wait_event(done)
+    return q_I_out
+
+
 def hsa_version() -> int:
     return int(lib().hsa_version())
 

@@ -175,6 +175,42 @@ def test_draft_verify_with_mxfp8_index_and_fp8_latent():
     assert torch.equal(idx, idx3) and torch.equal(out, out3) and torch.equal(lse, lse3)
 
 
+@pytest.mark.parametrize("mx", [True, False])
+def test_decode_prolog_three_streams_equals_one_shot_caches(mx):
+    """The decode prolog writes the newest token of every sequence into caches that hold the
+    rest (index keys MXFP8 or E4M3, latent FP8 per token, rope bf16) and rounds q_I onto the
+    MX grid, on three streams.  Caches and queries must equal, bit for bit, those written by
+    one quantizer call over all rows, and so must the decode step that follows."""
+    wl = workloads.make("decode_fp8", DEV, B=4, L=3000)
+    n = wl.num_slots
+    last = torch.tensor([int(wl.block_table[b, (int(wl.seq_lens[b]) - 1) // wl.page_size]) * wl.page_size
+                         + (int(wl.seq_lens[b]) - 1) % wl.page_size for b in range(wl.B)],
+                        dtype=torch.int64, device=DEV)
+    if mx:
+        k_ref, ks_ref = hsa.hsa_quantize_mx(wl.k_I)
+    else:
+        k_ref, ks_ref = hsa.hsa_quantize_index(wl.k_I, wl.D_I)
+        ks_ref = ks_ref.view(-1)
+    kv_ref, kvs_ref, rope_ref = hsa.hsa_quantize_kv(wl.kv, wl.D_v, wl.D_v)
+    kvs_ref = kvs_ref.view(-1)
+    k, ks, kv, kvs, rope = (t.clone() for t in (k_ref, ks_ref, kv_ref, kvs_ref, rope_ref))
+    for t in (k, ks, kv, kvs, rope):
+        t[last] = 0
+    q_out = torch.empty_like(wl.q_I)
+    hsa.hsa_decode_prolog(wl.k_I[last], wl.kv[last], last, k, ks, kv, kvs, rope, wl.q_I, q_out, wl.D_v)
+    torch.cuda.synchronize()
+    for got, ref in ((k, k_ref), (ks, ks_ref), (kv, kv_ref), (kvs, kvs_ref), (rope, rope_ref)):
+        assert torch.equal(got, ref)
+    assert torch.equal(q_out, hsa.mx_round(wl.q_I))
+    seq = paged_seq(wl)
+    a = hsa.hsa_fused_decode(seq, q_out, wl.w, k, ks, wl.q, kv, kvs, rope, wl.K, wl.D_v,
+                             wl.softmax_scale)
+    b = hsa.hsa_fused_decode(seq, hsa.mx_round(wl.q_I), wl.w, k_ref, ks_ref, wl.q, kv_ref, kvs_ref,
+                             rope_ref, wl.K, wl.D_v, wl.softmax_scale)
+    for x, y in zip(a, b):
+        assert torch.equal(x, y)
+
+
 @pytest.mark.parametrize("aux", [False, True])
 def test_decode_graph_replays_bitwise(aux):
     """The fused decode step captured as a CUDA graph equals the direct call bitwise, and a
