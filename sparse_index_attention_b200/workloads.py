@@ -21,6 +21,9 @@ contexts with Top-2048 selection over an MLA latent cache of 512 + 64 dims, 128 
                             KV (one scale per token) with a bf16 rope part.
 * ``prefill_long_zigzag``   one sequence of 131072 tokens in 32 query chunks of 4096, issued
                             as pairs (i, 31-i); FP8 index keys, bf16 KV.
+* ``decode_mxfp8``          ``decode_fp8``'s draws with the index queries and keys in MXFP8.
+* ``decode_draft_bf16``     as ``decode_bf16`` but four query rows per sequence at its last
+                            four positions (draft-verify decode).
 """
 from __future__ import annotations
 
