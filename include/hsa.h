@@ -173,7 +173,9 @@ HSA_API hsa_status_t hsa_sparse_mla_attn(const hsa_paged_seq_t* seq, const void*
  * the caller).  Pages: first page "Sparse Attention Pipeline Optimization" (fusing the decode
  * operators and running independent ones concurrently: indexer, then the sparse attention
  * kernel; several streams); fifth page 3.3 (operators on independent streams with event
- * synchronization). */
+ * synchronization).  The members of hsa_index_args_t and hsa_attn_args_t have the meaning of
+ * the same-named arguments of hsa_index_score and hsa_sparse_mla_attn (k_scale: fp32 per key
+ * for E4M3 keys, E8M0 bytes for MXE4M3 keys). */
 typedef struct hsa_index_args {
     const void* q_I; hsa_dtype_t q_dtype; const float* w; int32_t H_I; int32_t D_I;
     const void* k_cache; hsa_dtype_t k_dtype; const void* k_scale;
