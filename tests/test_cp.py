@@ -126,3 +126,11 @@ def test_zigzag_cp_prefill_equals_one_process(world, fp8):
     for rank, out, lse, idx, pos in got:
         assert np.array_equal(out, ref_out.numpy()) and np.array_equal(lse, ref_lse.numpy()), rank
         assert np.array_equal(idx, ref_idx.numpy()[pos]), rank
+
+
+@pytest.mark.parametrize("world", [1, 2, 3])
+def test_outputs_return_to_position_order(world):
+    """Rows stacked in rank order (each rank: its two segments) come back in position order."""
+    T = 2 * world * 5
+    stacked = torch.cat([cp.rank_positions(T, world, r) for r in range(world)])
+    assert torch.equal(cp._to_position_order(stacked, T, world), torch.arange(T, dtype=torch.int32))
