@@ -24,11 +24,13 @@ from a second timed loop that issues the three C-ABI calls separately on one str
 end-to-end throughput through the C ABI with host buffers (H2D of the step's query inputs and
 D2H of its output inside the timed region), the oracle timed on a bounded sample on the host
 cores, the SM clocks sampled during the timed region, and (one GPU) "other_workloads": the FP8
-decode batch, the bf16 causal prefill and the KV quantizer, each with its roofline fraction.
+and MXFP8 decode batches, the draft-verify batch, the KV quantizer, the bf16 causal prefill of
+16384 tokens and the 131072-token zigzag prefill with FP8 index keys (each prefill with its
+per-kernel times), each with its roofline fraction.
 
 --impl reference runs the float64 CPU oracle (the only reference implementation of this path)
-on the same workload, one query row per step, and prints the same JSON line with
-"impl": "reference".
+on the same workload, as many query rows per step as the oracle has threads (--ref-rows), and
+prints the same JSON line with "impl": "reference".
 """
 from __future__ import annotations
 
@@ -162,7 +164,7 @@ def cpu_baseline(wl, rows, timer_label="oracle"):
     t0 = time.perf_counter()
     oracle.sparse_index_attention(pg.subset(rows), qI, w, k, q, kv, wl.K, wl.D_v, wl.softmax_scale)
     dt = time.perf_counter() - t0
-    return len(rows) / dt, dt, oracle.num_threads()
+    return len(rows) / dt, dt, min(oracle.num_threads(), len(rows))
 
 
 def run_reference(args, rank, world):
@@ -174,10 +176,13 @@ def run_reference(args, rank, world):
     k = wl.k_I.float().numpy().astype(np.float64)
     kv = wl.kv.float().numpy().astype(np.float64)
 
+    rows_per_step = args.ref_rows or max(1, oracle.num_threads())
+
     def step(i):
-        r = i % wl.T_q
-        oracle.sparse_index_attention(pg.subset([r]), wl.q_I[r:r + 1], wl.w[r:r + 1], k,
-                                      wl.q[r:r + 1], kv, wl.K, wl.D_v, wl.softmax_scale)
+        r0 = (i * rows_per_step) % wl.T_q
+        rows = [(r0 + j) % wl.T_q for j in range(rows_per_step)]
+        oracle.sparse_index_attention(pg.subset(rows), wl.q_I[rows], wl.w[rows], k, wl.q[rows], kv,
+                                      wl.K, wl.D_v, wl.softmax_scale)
 
     for i in range(args.warmup):
         step(i)
@@ -185,15 +190,16 @@ def run_reference(args, rank, world):
     for i in range(args.steps):
         step(args.warmup + i)
     dt = time.perf_counter() - t0
-    value = args.steps / dt
-    threads = oracle.num_threads()
+    value = args.steps * rows_per_step / dt
+    threads = min(oracle.num_threads(), rows_per_step)   # OpenMP spreads a step's rows
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "config": workload_config(wl),
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
-                             "sample": "one query row per step (index score over its whole "
-                                       "context, Top-2048, 128-head sparse MLA), rows in turn"},
+                             "sample": f"{rows_per_step} query rows per step (index score over "
+                                       "each whole context, Top-2048, 128-head sparse MLA), the "
+                                       "batch's rows in turn"},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -348,34 +354,86 @@ def secondary(dev, flush_l2, main, peaks, reps):
     del wl, sc, idx, o, lse, ws, seq
     torch.cuda.empty_cache()
 
-    # bf16 causal prefill: one sequence of 16384 tokens, every token a query, 4 query chunks of
-    # 4096 issued in zigzag pairs on two streams
-    wl = workloads.make("prefill_bf16", dev)
+    # causal prefill: the bf16 16384-token workload (4 chunks of 4096 in zigzag pairs) and the
+    # 131072-token workload with FP8 index keys (32 chunks of 4096 in zigzag pairs)
+    out["prefill_bf16"] = prefill_measure("prefill_bf16", dev, flush_l2, main, peaks, 4, reps)
+    out["prefill_long_zigzag"] = prefill_measure("prefill_long_zigzag", dev, flush_l2, main, peaks,
+                                                 None, 2)
+    return out
+
+
+def prefill_measure(name, dev, flush_l2, main, peaks, n_chunks, reps):
+    """One causal prefill workload: the whole pass (hsa_prefill_chunked, chunk pairs on two
+    streams, caller-owned score buffers) timed with CUDA events, plus the time of each kernel
+    (index score, Top-K, sparse MLA) from a second pass that issues every chunk's three calls on
+    one stream with events between them.  Fractions are of the burst bf16 tensor peak (the calls
+    are sub-second, not the seconds-long loop the sustained figure describes)."""
+    import sparse_index_attention_b200 as hsa
+    wl = workloads.make(name, dev)
+    chunks = wl.chunks if n_chunks is None else workloads.zigzag_chunks(wl.T_q, n_chunks)
+    k, ks = wl.k_I, None
+    if wl.index_fp8:
+        k, ks = hsa.hsa_quantize_index(wl.k_I, wl.D_I)
+        ks = ks.view(-1)
     seq = hsa.PagedSeq(wl.seq_lens, wl.block_table, wl.page_size, wl.num_pages, wl.q_seq, wl.q_pos,
                        q_run=wl.q_run)
-    chunks = workloads.zigzag_chunks(wl.T_q, 4)
     o = torch.empty((wl.T_q, wl.H, wl.D_v), dtype=torch.bfloat16, device=dev)
     idx = torch.empty((wl.T_q, wl.K), dtype=torch.int32, device=dev)
     streams = (torch.cuda.Stream(), torch.cuda.Stream())
+    bufs = hsa.prefill_score_buffers(seq, chunks, dev)
 
     def prefill():
-        hsa.hsa_prefill_chunked(seq, wl.q_I, wl.w, wl.k_I, None, wl.q, wl.kv, None, None, wl.K,
+        hsa.hsa_prefill_chunked(seq, wl.q_I, wl.w, k, ks, wl.q, wl.kv, None, None, wl.K,
                                 wl.D_v, wl.softmax_scale, chunks, out=o, lse=False, idx=idx,
-                                streams=streams)
+                                streams=streams, score_bufs=bufs)
     prefill()
-    ms = _timed(prefill, max(2, reps // 4), flush_l2, main)
+    ms = _timed(prefill, max(2, reps), flush_l2, main)
+    # per-kernel times: every chunk's calls on `main`, events around each call
+    names = ["index_score", "topk", "sparse_mla"]
+    tot = {n: 0.0 for n in names}
+    flush_l2()
+    evs = []
+    for r0, r1 in chunks:
+        part = seq.rows(r0, r1, q_run=min(seq.q_run, r1 - r0))
+        sc = bufs[0][:r1 - r0]
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+        e[0].record(main)
+        hsa.hsa_index_score(part, wl.q_I[r0:r1], wl.w[r0:r1], k, ks, scores=sc, stream=main)
+        e[1].record(main)
+        hsa.hsa_topk(part, sc, wl.K, idx=idx[r0:r1], stream=main)
+        e[2].record(main)
+        hsa.hsa_sparse_mla_attn(part, wl.q[r0:r1], wl.kv, idx[r0:r1], wl.D_v, wl.softmax_scale,
+                                out=o[r0:r1], lse=False, stream=main)
+        e[3].record(main)
+        evs.append(e)
+    torch.cuda.synchronize()
+    for e in evs:
+        for j, n in enumerate(names):
+            tot[n] += e[j].elapsed_time(e[j + 1])
     n = (wl.q_pos.long() + 1).cpu()
-    flops = int(n.sum()) * wl.H_I * wl.D_I * 2 + int(torch.clamp(n, max=wl.K).sum()) * wl.H * (wl.D_qk + wl.D_v) * 2
-    peak = peaks["bf16_tflops_sustained"] * 1e12
-    out["prefill_bf16"] = {"workload": "one sequence of 16384 tokens, every token a query, Top-2048, "
-                                       "4 chunks of 4096 in zigzag pairs",
-                           "ms_per_step": round(ms, 3), "value": wl.T_q / (ms * 1e-3), "unit": UNIT,
-                           "bound": "tensor", "flops": flops,
-                           "frac": round(flops / (ms * 1e-3) / peak, 4),
-                           "peak": "bf16_tflops_sustained (MEASURED_PEAKS.json)"}
-    del wl, seq, o, idx
+    idx_flops = int(n.sum()) * wl.H_I * wl.D_I * 2
+    attn_flops = int(torch.clamp(n, max=wl.K).sum()) * wl.H * (wl.D_qk + wl.D_v) * 2
+    flops = idx_flops + attn_flops
+    peak = peaks["bf16_tflops"] * 1e12
+    stage = {
+        "index_score": {"ms": round(tot["index_score"], 3), "flops": idx_flops,
+                        "TFLOP/s": round(idx_flops / (tot["index_score"] * 1e-3) / 1e12, 1),
+                        "frac": round(idx_flops / (tot["index_score"] * 1e-3) / peak, 4)},
+        "topk": {"ms": round(tot["topk"], 3)},
+        "sparse_mla": {"ms": round(tot["sparse_mla"], 3), "flops": attn_flops,
+                       "TFLOP/s": round(attn_flops / (tot["sparse_mla"] * 1e-3) / 1e12, 1),
+                       "frac": round(attn_flops / (tot["sparse_mla"] * 1e-3) / peak, 4)},
+    }
+    desc = (f"one sequence of {wl.T_q} tokens, every token a query, Top-{wl.K}, "
+            f"{len(chunks)} chunks of {chunks[0][1] - chunks[0][0]} in zigzag pairs on two streams"
+            + (", FP8 index keys (fp32 scale per key)" if wl.index_fp8 else ", bf16 caches"))
+    res = {"workload": desc, "ms_per_step": round(ms, 3), "value": wl.T_q / (ms * 1e-3), "unit": UNIT,
+           "bound": "tensor", "flops": flops, "frac": round(flops / (ms * 1e-3) / peak, 4),
+           "peak": f"bf16_tflops {peaks['bf16_tflops']} (burst, MEASURED_PEAKS.json)",
+           "stages_one_stream": stage}
+    del wl, seq, o, idx, bufs, k, ks
     torch.cuda.empty_cache()
-    return out
+    return res
 
 
 def run_ours(args, rank, world, local_rank):
@@ -584,6 +642,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-rows", type=int, default=16, help="query rows for the oracle baseline")
+    ap.add_argument("--ref-rows", type=int, default=0,
+                    help="query rows per step of the reference arm (default: the oracle's threads)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-secondary", action="store_true",
                     help="skip the FP8 decode, prefill and quantizer measurements")

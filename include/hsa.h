@@ -199,6 +199,10 @@ HSA_API hsa_status_t hsa_fused_decode(const hsa_paged_seq_t* seq, const hsa_inde
  * Per row r and group g of `group` consecutive elements:
  *   amax = max |x|; scale = amax / 448 (fp32, round to nearest); inv = 448 / amax (fp32);
  *   code = E4M3(round-to-nearest-even, saturating, of x * inv);   amax == 0: scale 1, codes 0.
+ *   A group with amax < 2^-64 is multiplied by 2^64 (exactly) before inv and the products are
+ *   formed, so that inv cannot overflow float32; this changes no code where 448 / amax is
+ *   finite.  scale is still amax / 448 (it may be subnormal, or 0 for an fp32 amax of a few
+ *   times 2^-149).
  * Row r is written to physical slot slot_mapping[r] (slot_mapping NULL: slot r).
  * hsa_quantize_index: src [n_rows, D] F32/BF16 -> codes uint8 [slots, D], scales fp32
  *   [slots, D / group].  group = D gives one scale per key (the layout hsa_index_score reads);
@@ -221,9 +225,10 @@ HSA_API hsa_status_t hsa_quantize_kv(const void* src, hsa_dtype_t src_dtype, int
  * Per row r and block b of 32 consecutive elements (D a multiple of 32):
  *   amax = max |x|;  X = floor(log2(amax)) - 8, clamped to [-127, 127];  E = X + 127;
  *   code = E4M3(round-to-nearest-even, saturating, of x * 2^-X);   amax == 0: E = 0, codes 0.
- * (8 is the exponent of E4M3's top binade, 448 = 1.75 * 2^8, so the block maximum lands in
- * [256, 448] before rounding; the OCP Microscaling rule for the shared exponent.)  From finite
- * fp32 or bf16 data E never exceeds 246.
+ * (8 is the exponent of E4M3's top binade, 448 = 1.75 * 2^8, so the block maximum times 2^-X
+ * lies in [256, 512); a value there above 448 saturates to 448, an error of up to 12.5 % that
+ * the OCP Microscaling rule for the shared exponent accepts.)  From finite fp32 or bf16 data E
+ * never exceeds 246.
  * hsa_quantize_mx: src [n_rows, D] F32/BF16 -> codes uint8 [slots, D], scales uint8
  *   [slots, D / 32]; row r goes to slot slot_mapping[r] (NULL: slot r).  With D = 128 this
  *   writes the MXE4M3 index key cache hsa_index_score reads; applied to q_I (slot_mapping
@@ -239,6 +244,48 @@ HSA_API hsa_status_t hsa_quantize_mx(const void* src, hsa_dtype_t src_dtype, int
                              uint8_t* scales, void* stream);
 HSA_API hsa_status_t hsa_dequantize_mx(const uint8_t* codes, const uint8_t* scales, int64_t n_rows,
                                int32_t D, void* dst, hsa_dtype_t dst_dtype, void* stream);
+
+/* hsa_mx_round: src [n_rows, D] F32/BF16 -> dst [n_rows, D] F32/BF16 holding the MXFP8 values
+ * (hsa_quantize_mx followed by hsa_dequantize_mx, bit for bit, in one kernel with no code or
+ * scale bytes written to memory).  Index queries rounded this way let the bf16-query index
+ * kernels score MXFP8 queries.  src and dst may not overlap partially (dst == src is allowed). */
+HSA_API hsa_status_t hsa_mx_round(const void* src, hsa_dtype_t src_dtype, int64_t n_rows, int32_t D,
+                          void* dst, hsa_dtype_t dst_dtype, void* stream);
+
+/* ---- 7. decode prolog ---------------------------------------------------------------------
+ * The writes that precede a decode step, as three independent operators on three streams:
+ *   stream_k : the new tokens' index keys into the index key cache
+ *              (k_dtype MXE4M3: hsa_quantize_mx, k_scale E8M0 bytes [num_slots, D_I / 32];
+ *               k_dtype E4M3: hsa_quantize_index with one fp32 scale per key, k_scale
+ *               [num_slots]);
+ *   stream_kv: their latent rows into the FP8 latent cache (hsa_quantize_kv: codes
+ *              [num_slots, D_v], fp32 scales [num_slots, D_v / kv_group], bf16 rope
+ *              [num_slots, D_rope]);
+ *   stream_q : the index queries q_I [q_rows, D_I] rounded onto the MXFP8 grid into q_I_out
+ *              (bf16, hsa_mx_round; skipped when q_I_out is NULL).
+ * Each side stream first waits for the work already enqueued on `stream`, and `stream` then
+ * waits for all three, so a decode step enqueued on `stream` next sees every write.  A NULL side
+ * stream means `stream` itself.  Results equal the same calls issued one after another on one
+ * stream.  new_k [n_new, D_I] and new_kv [n_new, D_v + D_rope] are F32 or BF16; token r goes to
+ * physical slot slot_mapping[r] (int64, device).  Pages: first page "Sparse Attention Pipeline
+ * Optimization" (the indexer's preparatory operators run on concurrent streams); fifth page
+ * 3.2 and 3.3 (independent operators on separate streams, synchronized by events); the Q / K
+ * projections and the K normalization themselves need model weights and are not part of this
+ * library. */
+typedef struct hsa_prolog_args {
+    int64_t n_new;                /* new tokens, >= 0 */
+    const int64_t* slot_mapping;  /* device [n_new] */
+    int64_t num_slots;            /* slots of every paged cache */
+    const void* new_k; hsa_dtype_t new_k_dtype; int32_t D_I;
+    uint8_t* k_cache; void* k_scale; hsa_dtype_t k_dtype;
+    const void* new_kv; hsa_dtype_t new_kv_dtype; int32_t D_v; int32_t D_rope; int32_t kv_group;
+    uint8_t* kv_cache; float* kv_scale; void* kv_rope;
+    const void* q_I; hsa_dtype_t q_I_dtype; int64_t q_rows;
+    void* q_I_out;                /* bf16 [q_rows, D_I], or NULL */
+} hsa_prolog_args_t;
+
+HSA_API hsa_status_t hsa_decode_prolog(const hsa_prolog_args_t* args, void* stream, void* stream_k,
+                               void* stream_kv, void* stream_q);
 
 /* ---- diagnostics -------------------------------------------------------------------------- */
 HSA_API const char* hsa_status_string(hsa_status_t s);

@@ -104,8 +104,8 @@ uint8_t oracle_e4m3_encode(float xf) {
  * [P1] "Hierarchical Quantization", [P2] 4.1/4.2, [P5] s4 table: the scale is computed from the
  * data at write time ("dynamic").  The pages do not print the scale rule; the reading taken is
  * the max-abs rule: scale = amax / 448 (fp32, round to nearest), the values are multiplied by
- * inv = 448 / amax (fp32, round to nearest) and rounded to E4M3.  amax == 0 gives scale 1 and
- * all-zero codes.  fp32 division and multiplication are reproduced exactly by doing them in
+ * inv = 448 / amax (fp32, round to nearest) and rounded to E4M3 (for amax < 2^-64 both amax and
+ * the values are first lifted by 2^64, see below).  amax == 0 gives scale 1 and all-zero codes.  fp32 division and multiplication are reproduced exactly by doing them in
  * double and rounding once to float (double carries more than 2*24+2 bits).
  *   x: [n_rows, D] (fp32-representable values), codes: [n_rows, D], scales: [n_rows, D/group]. */
 int oracle_quantize_rows(const float* x, int64_t n_rows, int32_t D, int32_t group,
@@ -121,17 +121,24 @@ int oracle_quantize_rows(const float* x, int64_t n_rows, int32_t D, int32_t grou
                 double a = fabs((double)xs[i]);
                 if (a > amax) amax = a;
             }
+            /* A group maximum below 2^-64 is multiplied by 2^64 (exact) before 448/amax is
+             * formed, and so are the group's values before they are multiplied by it: 448/amax
+             * itself would overflow float32 for amax < 448/FLT_MAX, and a zero of the group
+             * would then become 0 * inf = NaN.  Where 448/amax is finite both the reciprocal
+             * and the products only move by an exact power of two, so the codes are the same
+             * as without the lift. */
+            const double lift = amax < 0x1p-64 ? 0x1p64 : 1.0;
             float scale, inv;
             if (amax == 0.0) {
                 scale = 1.0f;
                 inv = 0.0f;
             } else {
                 scale = (float)(amax / 448.0);
-                inv = (float)(448.0 / amax);
+                inv = (float)(448.0 / (amax * lift));
             }
             scales[r * ng + g] = scale;
             for (int32_t i = 0; i < group; ++i) {
-                float y = (float)((double)xs[i] * (double)inv);
+                float y = (float)((double)xs[i] * lift * (double)inv);
                 codes[r * D + (int64_t)g * group + i] = amax == 0.0 ? 0 : oracle_e4m3_encode(y);
             }
         }

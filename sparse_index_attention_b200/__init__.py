@@ -46,6 +46,15 @@ class hsa_attn_args_t(ctypes.Structure):
                 ("softmax_scale", _f32), ("out", _P), ("out_dtype", ctypes.c_int), ("lse", _P)]
 
 
+class hsa_prolog_args_t(ctypes.Structure):
+    _fields_ = [("n_new", _i64), ("slot_mapping", _P), ("num_slots", _i64),
+                ("new_k", _P), ("new_k_dtype", ctypes.c_int), ("D_I", _i32),
+                ("k_cache", _P), ("k_scale", _P), ("k_dtype", ctypes.c_int),
+                ("new_kv", _P), ("new_kv_dtype", ctypes.c_int), ("D_v", _i32), ("D_rope", _i32),
+                ("kv_group", _i32), ("kv_cache", _P), ("kv_scale", _P), ("kv_rope", _P),
+                ("q_I", _P), ("q_I_dtype", ctypes.c_int), ("q_rows", _i64), ("q_I_out", _P)]
+
+
 SYMBOLS = {
     "hsa_index_score": (ctypes.c_int, [_P, _P, ctypes.c_int, _P, _i32, _i32, _P, ctypes.c_int, _P,
                                        _P, _i64, _P]),
@@ -61,6 +70,8 @@ SYMBOLS = {
                                        _P, _P]),
     "hsa_quantize_mx": (ctypes.c_int, [_P, ctypes.c_int, _i64, _i32, _P, _i64, _P, _P, _P]),
     "hsa_dequantize_mx": (ctypes.c_int, [_P, _P, _i64, _i32, _P, ctypes.c_int, _P]),
+    "hsa_mx_round": (ctypes.c_int, [_P, ctypes.c_int, _i64, _i32, _P, ctypes.c_int, _P]),
+    "hsa_decode_prolog": (ctypes.c_int, [_P, _P, _P, _P, _P]),
     "hsa_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "hsa_last_error_message": (ctypes.c_char_p, []),
     "hsa_version": (_i32, []),
@@ -374,57 +385,74 @@ def hsa_dequantize_mx(codes, scales, dtype=torch.bfloat16, out=None, stream=None
     return out
 
 
-def mx_round(x, stream=None):
-    """Index queries [..., D] rounded onto the MXFP8 grid and returned as bf16 (quantize, then
-    dequantize: two library kernels).  The bf16-query index kernels then score MXFP8 queries."""
+def mx_round(x, out=None, stream=None):
+    """Index queries [..., D] rounded onto the MXFP8 grid and returned as bf16 (hsa_mx_round: the
+    quantize-then-dequantize result of the MX rule in one kernel).  The bf16-query index kernels
+    then score MXFP8 queries."""
     flat = x.reshape(-1, x.shape[-1])
-    codes, scales = hsa_quantize_mx(flat, stream=stream)
-    return hsa_dequantize_mx(codes, scales, torch.bfloat16, stream=stream).view(x.shape)
+    if out is None:
+        out = torch.empty(x.shape, dtype=torch.bfloat16, device=x.device)
+    _check(lib().hsa_mx_round(_ptr(flat), _dtype(flat), flat.shape[0], flat.shape[1], _ptr(out),
+                              _dtype(out), _stream(stream)),
+           "hsa_mx_round")
+    return out
+
+
+def _cache_rows(t, name: str, width: int, dtype) -> int:
+    """Slots of a flat paged cache tensor [slots, width] (a paged [P, page, width] view is
+    accepted and flattened): a mismatch is an error, not a silently dropped row."""
+    if t.dtype != dtype:
+        raise TypeError(f"{name}: dtype {t.dtype}, expected {dtype}")
+    if width == 1 and t.dim() == 1:
+        return t.numel()
+    if t.dim() < 1 or t.shape[-1] != width or t.numel() % width:
+        raise ValueError(f"{name}: shape {tuple(t.shape)} is not [slots, {width}]")
+    return t.numel() // width
 
 
 def hsa_decode_prolog(new_k, new_kv, slot_mapping, k_cache, k_scale, kv_cache, kv_scale, kv_rope,
                       q_I, q_I_out, D_v: int, kv_group: Optional[int] = None, streams=None,
                       stream=None):
-    """The writes that precede a decode step, on three streams: the new tokens' index keys into
-    the index key cache, their latent rows into the FP8 latent cache, and the index queries
-    rounded onto the MXFP8 grid into ``q_I_out`` ("Day 0 Inference Adaptation and Optimization
-    for Hybrid Attention Models", "Sparse Attention Pipeline Optimization": independent
-    prolog operators on concurrent streams; "Inference Adaptation and Performance Optimization
-    for a Domestically Developed LLM's New Architecture", 3.3).  ``stream`` (default: current)
-    waits for all three, so a decode step issued on it next sees the new rows.
+    """The writes that precede a decode step, on three streams (hsa_decode_prolog): the new
+    tokens' index keys into the index key cache, their latent rows into the FP8 latent cache,
+    and the index queries rounded onto the MXFP8 grid into ``q_I_out`` ("Day 0 Inference
+    Adaptation and Optimization for Hybrid Attention Models", "Sparse Attention Pipeline
+    Optimization": independent prolog operators on concurrent streams; "Inference Adaptation and
+    Performance Optimization for a Domestically Developed LLM's New Architecture", 3.3).
+    ``stream`` (default: current) waits for all three, so a decode step issued on it next sees
+    the new rows.
 
     new_k [n, D_I] and new_kv [n, D_v + D_rope] (F32/BF16) go to physical slots
     ``slot_mapping`` [n] (int64).  The index key cache is MXFP8 when ``k_scale`` is uint8
     (E8M0 bytes, [slots, D_I/32]) and E4M3 with one fp32 scale per key otherwise.  The latent
     cache is E4M3 with one fp32 scale per ``kv_group`` dims (default D_v) plus bf16 rope.
     Results equal the same calls issued one after another on one stream."""
-    main = torch.cuda.current_stream() if stream is None else stream
+    n, D_I = new_k.shape
+    D_rope = new_kv.shape[1] - D_v
+    grp = kv_group or D_v
+    mx = k_scale.dtype == torch.uint8
+    slots = _cache_rows(k_cache, "k_cache", D_I, torch.uint8)
+    if _cache_rows(k_scale, "k_scale", D_I // 32 if mx else 1, torch.uint8 if mx else torch.float32) != slots:
+        raise ValueError("k_scale does not cover the key cache's slots")
+    if _cache_rows(kv_cache, "kv_cache", D_v, torch.uint8) != slots or \
+            _cache_rows(kv_scale, "kv_scale", D_v // grp, torch.float32) != slots or \
+            _cache_rows(kv_rope, "kv_rope", D_rope, torch.bfloat16) != slots:
+        raise ValueError("the latent cache tensors do not cover the key cache's slots")
+    if slot_mapping.dtype != torch.int64 or slot_mapping.numel() != n:
+        raise ValueError("slot_mapping must be int64 [n]")
+    if q_I_out is not None and (q_I_out.dtype != torch.bfloat16 or q_I_out.numel() != q_I.numel()):
+        raise ValueError("q_I_out must be bf16 with q_I's size")
     if streams is None:
         streams = (torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream())
-    start = torch.cuda.Event()
-    start.record(main)
-    for st in streams:
-        st.wait_event(start)
-    num_slots = k_cache.shape[0]
-    s_k, s_kv, s_q = streams
-    if k_scale.dtype == torch.uint8:
-        hsa_quantize_mx(new_k, slot_mapping, num_slots, codes=k_cache, scales=k_scale, stream=s_k)
-    else:
-        hsa_quantize_index(new_k, new_k.shape[1], slot_mapping, num_slots, codes=k_cache,
-                           scales=k_scale.view(num_slots, 1), stream=s_k)
-    grp = kv_group or D_v
-    hsa_quantize_kv(new_kv, D_v, grp, slot_mapping, kv_cache.shape[0], codes=kv_cache,
-                    scales=kv_scale.view(kv_cache.shape[0], D_v // grp), rope_cache=kv_rope,
-                    stream=s_kv)
-    flat = q_I.reshape(-1, q_I.shape[-1])
-    codes = torch.empty(flat.shape, dtype=torch.uint8, device=flat.device)
-    scales = torch.empty((flat.shape[0], flat.shape[1] // 32), dtype=torch.uint8, device=flat.device)
-    hsa_quantize_mx(flat, codes=codes, scales=scales, stream=s_q)
-    hsa_dequantize_mx(codes, scales, out=q_I_out.view(flat.shape), stream=s_q)
-    for st in streams:
-        done = torch.cuda.Event()
-        done.record(st)
-        main.wait_event(done)
+    flat_q = q_I.reshape(-1, D_I)
+    a = hsa_prolog_args_t(n, _ptr(slot_mapping), slots, _ptr(new_k), _dtype(new_k), D_I,
+                          _ptr(k_cache), _ptr(k_scale), HSA_MXE4M3 if mx else HSA_E4M3,
+                          _ptr(new_kv), _dtype(new_kv), D_v, D_rope, grp, _ptr(kv_cache),
+                          _ptr(kv_scale), _ptr(kv_rope), _ptr(flat_q), _dtype(flat_q),
+                          flat_q.shape[0], _ptr(q_I_out))
+    _check(lib().hsa_decode_prolog(ctypes.byref(a), _stream(stream), _stream(streams[0]),
+                                   _stream(streams[1]), _stream(streams[2])),
+           "hsa_decode_prolog")
     return q_I_out
 
 
@@ -437,9 +465,17 @@ def hsa_launch_count() -> int:
     return int(lib().hsa_launch_count())
 
 
+def prefill_score_buffers(seq: PagedSeq, chunks, device, n: int = 2):
+    """Caller-owned fp32 score buffers for hsa_prefill_chunked: one [max chunk rows, max_seq_len]
+    buffer per stream, allocated once and reused by every call."""
+    rows_max = max(r1 - r0 for r0, r1 in chunks)
+    return tuple(torch.empty((rows_max, seq.max_seq_len), dtype=torch.float32, device=device)
+                 for _ in range(n))
+
+
 def hsa_prefill_chunked(seq: PagedSeq, q_I, w, k_cache, k_scale, q, kv, kv_scale, kv_rope, K: int,
                         D_v: int, softmax_scale: float, chunks, out=None, lse=True, idx=None,
-                        streams=None):
+                        streams=None, score_bufs=None):
     """Causal prefill over query-row windows issued in the order of `chunks` [(r0, r1), ...].
 
     Consecutive chunks form pairs that run concurrently, one on each of two streams; with the
@@ -447,7 +483,9 @@ def hsa_prefill_chunked(seq: PagedSeq, q_I, w, k_cache, k_scale, q, kv, kv_scale
     Optimization for Hybrid Attention LLMs", 5.2) every pair carries the same causal index work.
     Each chunk is hsa_index_score -> hsa_topk -> hsa_sparse_mla_attn on its rows, so its outputs
     land at the rows' own offsets and no restore step exists; the issue order cannot change any
-    result.  This function only slices tensors and issues C-ABI calls.  Returns (out, lse, idx).
+    result.  This function only slices tensors and issues C-ABI calls.  ``score_bufs`` (one per
+    stream, from prefill_score_buffers) holds the chunks' scores; when it is not given, buffers
+    are allocated for this call.  Returns (out, lse, idx).
     """
     T_q = q.shape[0]
     dev = q.device
@@ -464,11 +502,13 @@ def hsa_prefill_chunked(seq: PagedSeq, q_I, w, k_cache, k_scale, q, kv, kv_scale
         streams = (torch.cuda.Stream(), torch.cuda.Stream())
     start = torch.cuda.Event()
     start.record(main)
+    own = score_bufs is None
+    bufs = list(prefill_score_buffers(seq, chunks, dev, len(streams)) if own else score_bufs)
     rows_max = max(r1 - r0 for r0, r1 in chunks)
-    bufs = []
+    if len(bufs) < len(streams) or any(b.shape[0] < rows_max or b.shape[1] < seq.max_seq_len for b in bufs):
+        raise ValueError("score buffers smaller than [max chunk rows, max_seq_len]")
     for s in streams:
         s.wait_event(start)
-        bufs.append(torch.empty((rows_max, seq.max_seq_len), dtype=torch.float32, device=dev))
     for i, (r0, r1) in enumerate(chunks):
         s = streams[i % 2]
         part = seq.rows(r0, r1, q_run=min(seq.q_run, r1 - r0))
@@ -482,6 +522,7 @@ def hsa_prefill_chunked(seq: PagedSeq, q_I, w, k_cache, k_scale, q, kv, kv_scale
         done = torch.cuda.Event()
         done.record(s)
         main.wait_event(done)
-    for b, s in zip(bufs, streams):
-        b.record_stream(s)
+    if own:
+        for b, s in zip(bufs, streams):
+            b.record_stream(s)
     return out, lse, idx

@@ -227,6 +227,68 @@ hsa_attn_args_t make_attn(const void* q, hsa_dtype_t q_dtype, int32_t H, int32_t
     return a;
 }
 
+// Host-side checks of the cache-write quantizers (shared by their entry points and the prolog,
+// which checks every operator before it enqueues any).  D_rope = 0 and rope = NULL for index
+// keys.
+hsa_status_t check_quantize_rows(const void* src, hsa_dtype_t src_dtype, int64_t n_rows, int32_t D,
+                                 int32_t D_rope, int32_t group, const int64_t* slot_mapping,
+                                 int64_t num_slots, const uint8_t* codes, const float* scales,
+                                 const void* rope) {
+    HSA_REQUIRE(src_dtype == HSA_F32 || src_dtype == HSA_BF16, HSA_ERR_UNSUPPORTED,
+                "source dtype must be F32 or BF16");
+    HSA_REQUIRE(n_rows >= 0 && D >= 1 && D_rope >= 0 && group >= 1 && D % group == 0,
+                HSA_ERR_INVALID_ARG, "need n_rows >= 0, D >= 1, D_rope >= 0, group | D "
+                "(n_rows=%lld D=%d group=%d)", (long long)n_rows, D, group);
+    HSA_REQUIRE(num_slots >= 0 && (slot_mapping || n_rows <= num_slots), HSA_ERR_INVALID_ARG,
+                "identity slot mapping needs n_rows <= num_slots");
+    if (n_rows == 0) return HSA_OK;
+    HSA_REQUIRE(src && codes && scales && (D_rope == 0 || rope), HSA_ERR_INVALID_ARG,
+                "NULL tensor pointer");
+    HSA_REQUIRE(aligned(src, dtype_size(src_dtype)) && aligned(scales, 4) &&
+                    (D_rope == 0 || aligned(rope, 2)) &&
+                    (slot_mapping == nullptr || aligned(slot_mapping, 8)),
+                HSA_ERR_INVALID_ARG, "misaligned source, scales, rope cache or slot mapping");
+    return HSA_OK;
+}
+
+hsa_status_t check_quantize_mx(const void* src, hsa_dtype_t src_dtype, int64_t n_rows, int32_t D,
+                               const int64_t* slot_mapping, int64_t num_slots, const uint8_t* codes,
+                               const uint8_t* scales) {
+    HSA_REQUIRE(src_dtype == HSA_F32 || src_dtype == HSA_BF16, HSA_ERR_UNSUPPORTED,
+                "source dtype must be F32 or BF16");
+    HSA_REQUIRE(n_rows >= 0 && D >= 32 && D % 32 == 0, HSA_ERR_INVALID_ARG,
+                "need n_rows >= 0 and D a positive multiple of 32 (n_rows=%lld D=%d)",
+                (long long)n_rows, D);
+    HSA_REQUIRE(num_slots >= 0 && (slot_mapping || n_rows <= num_slots), HSA_ERR_INVALID_ARG,
+                "identity slot mapping needs n_rows <= num_slots");
+    if (n_rows == 0) return HSA_OK;
+    HSA_REQUIRE(src && codes && scales, HSA_ERR_INVALID_ARG, "NULL tensor pointer");
+    HSA_REQUIRE(aligned(src, dtype_size(src_dtype)) &&
+                    (slot_mapping == nullptr || aligned(slot_mapping, 8)),
+                HSA_ERR_INVALID_ARG, "misaligned source or slot mapping");
+    return HSA_OK;
+}
+
+hsa_status_t check_mx_round(const void* src, hsa_dtype_t src_dtype, int64_t n_rows, int32_t D,
+                            const void* dst, hsa_dtype_t dst_dtype) {
+    HSA_REQUIRE((src_dtype == HSA_F32 || src_dtype == HSA_BF16) &&
+                    (dst_dtype == HSA_F32 || dst_dtype == HSA_BF16),
+                HSA_ERR_UNSUPPORTED, "source and destination dtypes must be F32 or BF16");
+    HSA_REQUIRE(n_rows >= 0 && D >= 32 && D % 32 == 0, HSA_ERR_INVALID_ARG,
+                "need n_rows >= 0 and D a positive multiple of 32 (n_rows=%lld D=%d)",
+                (long long)n_rows, D);
+    if (n_rows == 0) return HSA_OK;
+    HSA_REQUIRE(src && dst, HSA_ERR_INVALID_ARG, "NULL tensor pointer");
+    HSA_REQUIRE(aligned(src, dtype_size(src_dtype)) && aligned(dst, dtype_size(dst_dtype)),
+                HSA_ERR_INVALID_ARG, "misaligned source or destination");
+    const uintptr_t s0 = reinterpret_cast<uintptr_t>(src), d0 = reinterpret_cast<uintptr_t>(dst);
+    const uintptr_t s1 = s0 + (uintptr_t)n_rows * D * dtype_size(src_dtype);
+    const uintptr_t d1 = d0 + (uintptr_t)n_rows * D * dtype_size(dst_dtype);
+    HSA_REQUIRE(s0 == d0 ? src_dtype == dst_dtype : (d1 <= s0 || s1 <= d0), HSA_ERR_INVALID_ARG,
+                "source and destination overlap");
+    return HSA_OK;
+}
+
 }  // namespace
 
 uint64_t& hsa::launch_counter() {
@@ -398,15 +460,9 @@ hsa_status_t hsa_quantize_index(const void* src, hsa_dtype_t src_dtype, int64_t 
                                 int32_t D, int32_t group, const int64_t* slot_mapping,
                                 int64_t num_slots, uint8_t* codes, float* scales, void* stream) {
     g_last_error.clear();
-    HSA_REQUIRE(src_dtype == HSA_F32 || src_dtype == HSA_BF16, HSA_ERR_UNSUPPORTED,
-                "source dtype must be F32 or BF16");
-    HSA_REQUIRE(n_rows >= 0 && D >= 1 && group >= 1 && D % group == 0, HSA_ERR_INVALID_ARG,
-                "need n_rows >= 0, D >= 1, group | D (n_rows=%lld D=%d group=%d)",
-                (long long)n_rows, D, group);
-    HSA_REQUIRE(num_slots >= 0 && (slot_mapping || n_rows <= num_slots), HSA_ERR_INVALID_ARG,
-                "identity slot mapping needs n_rows <= num_slots");
-    if (n_rows == 0) return HSA_OK;
-    HSA_REQUIRE(src && codes && scales, HSA_ERR_INVALID_ARG, "NULL tensor pointer");
+    hsa_status_t st = check_quantize_rows(src, src_dtype, n_rows, D, 0, group, slot_mapping,
+                                          num_slots, codes, scales, nullptr);
+    if (st != HSA_OK || n_rows == 0) return st;
     return cuda_status(hsa::launch_quantize_rows(src, src_dtype, n_rows, D, D, group, slot_mapping,
                                                  num_slots, codes, scales, 0, nullptr,
                                                  (cudaStream_t)stream),
@@ -418,15 +474,9 @@ hsa_status_t hsa_quantize_kv(const void* src, hsa_dtype_t src_dtype, int64_t n_r
                              int64_t num_slots, uint8_t* codes, float* scales, void* rope_cache,
                              void* stream) {
     g_last_error.clear();
-    HSA_REQUIRE(src_dtype == HSA_F32 || src_dtype == HSA_BF16, HSA_ERR_UNSUPPORTED,
-                "source dtype must be F32 or BF16");
-    HSA_REQUIRE(n_rows >= 0 && D_v >= 1 && D_rope >= 0 && group >= 1 && D_v % group == 0,
-                HSA_ERR_INVALID_ARG, "need n_rows >= 0, D_v >= 1, D_rope >= 0, group | D_v");
-    HSA_REQUIRE(num_slots >= 0 && (slot_mapping || n_rows <= num_slots), HSA_ERR_INVALID_ARG,
-                "identity slot mapping needs n_rows <= num_slots");
-    if (n_rows == 0) return HSA_OK;
-    HSA_REQUIRE(src && codes && scales && (D_rope == 0 || rope_cache), HSA_ERR_INVALID_ARG,
-                "NULL tensor pointer");
+    hsa_status_t st = check_quantize_rows(src, src_dtype, n_rows, D_v, D_rope, group, slot_mapping,
+                                          num_slots, codes, scales, rope_cache);
+    if (st != HSA_OK || n_rows == 0) return st;
     return cuda_status(hsa::launch_quantize_rows(src, src_dtype, n_rows, D_v + D_rope, D_v, group,
                                                  slot_mapping, num_slots, codes, scales, D_rope,
                                                  rope_cache, (cudaStream_t)stream),
@@ -437,16 +487,9 @@ hsa_status_t hsa_quantize_mx(const void* src, hsa_dtype_t src_dtype, int64_t n_r
                              const int64_t* slot_mapping, int64_t num_slots, uint8_t* codes,
                              uint8_t* scales, void* stream) {
     g_last_error.clear();
-    HSA_REQUIRE(src_dtype == HSA_F32 || src_dtype == HSA_BF16, HSA_ERR_UNSUPPORTED,
-                "source dtype must be F32 or BF16");
-    HSA_REQUIRE(n_rows >= 0 && D >= 32 && D % 32 == 0, HSA_ERR_INVALID_ARG,
-                "need n_rows >= 0 and D a positive multiple of 32 (n_rows=%lld D=%d)",
-                (long long)n_rows, D);
-    HSA_REQUIRE(num_slots >= 0 && (slot_mapping || n_rows <= num_slots), HSA_ERR_INVALID_ARG,
-                "identity slot mapping needs n_rows <= num_slots");
-    if (n_rows == 0) return HSA_OK;
-    HSA_REQUIRE(src && codes && scales, HSA_ERR_INVALID_ARG, "NULL tensor pointer");
-    HSA_REQUIRE(aligned(src, dtype_size(src_dtype)), HSA_ERR_INVALID_ARG, "misaligned source");
+    hsa_status_t st = check_quantize_mx(src, src_dtype, n_rows, D, slot_mapping, num_slots, codes,
+                                        scales);
+    if (st != HSA_OK || n_rows == 0) return st;
     return cuda_status(hsa::launch_quantize_mx(src, src_dtype, n_rows, D, slot_mapping, num_slots,
                                                codes, scales, (cudaStream_t)stream),
                        "quantize_mx");
@@ -466,6 +509,89 @@ hsa_status_t hsa_dequantize_mx(const uint8_t* codes, const uint8_t* scales, int6
     return cuda_status(hsa::launch_dequantize_mx(codes, scales, n_rows, D, dst, dst_dtype,
                                                  (cudaStream_t)stream),
                        "dequantize_mx");
+}
+
+hsa_status_t hsa_mx_round(const void* src, hsa_dtype_t src_dtype, int64_t n_rows, int32_t D,
+                          void* dst, hsa_dtype_t dst_dtype, void* stream) {
+    g_last_error.clear();
+    hsa_status_t st = check_mx_round(src, src_dtype, n_rows, D, dst, dst_dtype);
+    if (st != HSA_OK || n_rows == 0) return st;
+    return cuda_status(hsa::launch_mx_round(src, src_dtype, n_rows, D, dst, dst_dtype,
+                                            (cudaStream_t)stream),
+                       "mx_round");
+}
+
+hsa_status_t hsa_decode_prolog(const hsa_prolog_args_t* a, void* stream, void* stream_k,
+                               void* stream_kv, void* stream_q) {
+    g_last_error.clear();
+    HSA_REQUIRE(a != nullptr, HSA_ERR_INVALID_ARG, "prolog args NULL");
+    HSA_REQUIRE(a->n_new >= 0 && a->q_rows >= 0, HSA_ERR_INVALID_ARG, "need n_new >= 0, q_rows >= 0");
+    HSA_REQUIRE(a->k_dtype == HSA_MXE4M3 || a->k_dtype == HSA_E4M3, HSA_ERR_UNSUPPORTED,
+                "index key cache must be MXE4M3 or E4M3");
+    HSA_REQUIRE(a->n_new == 0 || a->slot_mapping, HSA_ERR_INVALID_ARG, "slot_mapping NULL");
+    // every operator's arguments are checked before anything is enqueued or any stream forked
+    hsa_status_t st = HSA_OK;
+    if (a->k_dtype == HSA_MXE4M3)
+        st = check_quantize_mx(a->new_k, a->new_k_dtype, a->n_new, a->D_I, a->slot_mapping,
+                               a->num_slots, a->k_cache, static_cast<uint8_t*>(a->k_scale));
+    else
+        st = check_quantize_rows(a->new_k, a->new_k_dtype, a->n_new, a->D_I, 0, a->D_I,
+                                 a->slot_mapping, a->num_slots, a->k_cache,
+                                 static_cast<float*>(a->k_scale), nullptr);
+    if (st != HSA_OK) return st;
+    st = check_quantize_rows(a->new_kv, a->new_kv_dtype, a->n_new, a->D_v, a->D_rope, a->kv_group,
+                             a->slot_mapping, a->num_slots, a->kv_cache, a->kv_scale, a->kv_rope);
+    if (st != HSA_OK) return st;
+    const bool want_q = a->q_I_out != nullptr && a->q_rows > 0;
+    if (want_q) {
+        st = check_mx_round(a->q_I, a->q_I_dtype, a->q_rows, a->D_I, a->q_I_out, HSA_BF16);
+        if (st != HSA_OK) return st;
+    }
+    cudaStream_t s0 = (cudaStream_t)stream;
+    const cudaStream_t side[3] = {stream_k ? (cudaStream_t)stream_k : s0,
+                                  stream_kv ? (cudaStream_t)stream_kv : s0,
+                                  stream_q ? (cudaStream_t)stream_q : s0};
+    cudaEvent_t ev[4] = {nullptr, nullptr, nullptr, nullptr};
+    hsa_status_t r = HSA_OK;
+    for (int i = 0; i < 4 && r == HSA_OK; ++i)
+        r = cuda_status(cudaEventCreateWithFlags(&ev[i], cudaEventDisableTiming), "cudaEventCreate");
+    // fork: each side stream starts after the work already on the main stream
+    if (r == HSA_OK) r = cuda_status(cudaEventRecord(ev[0], s0), "cudaEventRecord");
+    for (int i = 0; i < 3 && r == HSA_OK; ++i)
+        if (side[i] != s0) r = cuda_status(cudaStreamWaitEvent(side[i], ev[0], 0), "cudaStreamWaitEvent");
+    if (r == HSA_OK && a->n_new > 0) {
+        if (a->k_dtype == HSA_MXE4M3)
+            r = cuda_status(hsa::launch_quantize_mx(a->new_k, a->new_k_dtype, a->n_new, a->D_I,
+                                                    a->slot_mapping, a->num_slots, a->k_cache,
+                                                    static_cast<uint8_t*>(a->k_scale), side[0]),
+                            "quantize_mx");
+        else
+            r = cuda_status(hsa::launch_quantize_rows(a->new_k, a->new_k_dtype, a->n_new, a->D_I,
+                                                      a->D_I, a->D_I, a->slot_mapping, a->num_slots,
+                                                      a->k_cache, static_cast<float*>(a->k_scale),
+                                                      0, nullptr, side[0]),
+                            "quantize_index");
+        if (r == HSA_OK)
+            r = cuda_status(hsa::launch_quantize_rows(a->new_kv, a->new_kv_dtype, a->n_new,
+                                                      a->D_v + a->D_rope, a->D_v, a->kv_group,
+                                                      a->slot_mapping, a->num_slots, a->kv_cache,
+                                                      a->kv_scale, a->D_rope, a->kv_rope, side[1]),
+                            "quantize_kv");
+    }
+    if (r == HSA_OK && want_q)
+        r = cuda_status(hsa::launch_mx_round(a->q_I, a->q_I_dtype, a->q_rows, a->D_I, a->q_I_out,
+                                             HSA_BF16, side[2]),
+                        "mx_round");
+    // join (also after a failed launch, so that nothing enqueued is left unordered)
+    for (int i = 0; i < 3; ++i) {
+        if (side[i] == s0 || ev[1 + i] == nullptr || ev[0] == nullptr) continue;
+        hsa_status_t e = cuda_status(cudaEventRecord(ev[1 + i], side[i]), "cudaEventRecord");
+        if (e == HSA_OK) e = cuda_status(cudaStreamWaitEvent(s0, ev[1 + i], 0), "cudaStreamWaitEvent");
+        if (r == HSA_OK) r = e;
+    }
+    for (int i = 0; i < 4; ++i)
+        if (ev[i]) cudaEventDestroy(ev[i]);
+    return r;
 }
 
 }  // extern "C"

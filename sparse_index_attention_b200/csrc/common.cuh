@@ -118,9 +118,10 @@ inline void count_launch(int n = 1) { launch_counter() += (uint64_t)n; }
 
 // Programmatic dependent launch.  The tensor-core path's kernels (index score, Top-K, sparse MLA)
 // are launched so that a kernel may start while the previous kernel on the stream is still
-// running.  Such a kernel reads only the row descriptors (which no kernel of this library
-// writes) before pdl_wait(), which returns once every earlier kernel on the stream has finished
-// and its writes are visible; it touches nothing else until then.  Right after its own
+// running.  Such a kernel reads no global memory before pdl_wait() (not even the row
+// descriptors: a decode loop may advance q_pos, seq_lens and the block table on the device just
+// before the call), which returns once every earlier kernel on the stream has finished and its
+// writes are visible; only barrier set-up and the TMEM allocation run before it.  Right after its own
 // pdl_wait() it calls pdl_trigger(), which lets the next kernel launch: so when a kernel starts,
 // everything before its predecessor has finished.  Without the launch attribute both are no-ops.
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }

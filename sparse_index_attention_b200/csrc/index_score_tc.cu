@@ -158,6 +158,11 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
         tc::tmem_alloc(tmem_holder, C::kTmemCols);
         tc::tmem_relinquish();
     }
+    // the row descriptors and the queries, weights and keys may all be written by the previous
+    // kernel on the stream (a decode loop advances q_pos and seq_lens on the device), so nothing
+    // of them is read before this wait
+    pdl_wait();
+    pdl_trigger();
     // tiles per group, then an exclusive prefix sum (warp 0)
     for (int g = tid; g < n_groups; g += blockDim.x) {
         const GroupInfo gi = group_info(v, g, G, blockIdx.x == 0);
@@ -183,8 +188,6 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
     tc::tc_fence_before();
     __syncthreads();
     tc::tc_fence_after();
-    pdl_wait();              // queries, weights and keys may be the previous kernel's output
-    pdl_trigger();
     const uint32_t tmem_base = *tmem_holder;
     const int64_t total = n_groups > 0 ? prefix[n_groups] : 0;
     const int64_t f_begin = total * blockIdx.x / gridDim.x;

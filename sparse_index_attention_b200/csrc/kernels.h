@@ -68,6 +68,9 @@ cudaError_t launch_quantize_rows(const void* src, hsa_dtype_t src_dtype, int64_t
 cudaError_t launch_quantize_mx(const void* src, hsa_dtype_t src_dtype, int64_t n_rows, int32_t D,
                                const int64_t* slot_mapping, int64_t num_slots, uint8_t* codes,
                                uint8_t* scales, cudaStream_t st);
+// quantize_mx followed by dequantize_mx in one kernel (rows contiguous, no slot mapping).
+cudaError_t launch_mx_round(const void* src, hsa_dtype_t src_dtype, int64_t n_rows, int32_t D,
+                            void* dst, hsa_dtype_t dst_dtype, cudaStream_t st);
 cudaError_t launch_dequantize_mx(const uint8_t* codes, const uint8_t* scales, int64_t n_rows,
                                  int32_t D, void* dst, hsa_dtype_t dst_dtype, cudaStream_t st);
 

@@ -6,7 +6,9 @@
 //
 // Scale rule (dynamic max-abs): scale = amax / 448, inv = 448 / amax, both IEEE fp32 round to
 // nearest (this file is built without fast-math, so `/` is the correctly rounded division);
-// code = cvt.rn.satfinite to E4M3 of x * inv.  An all-zero group gets scale 1 and code 0.
+// code = cvt.rn.satfinite to E4M3 of x * inv.  An all-zero group gets scale 1 and code 0.  A
+// group maximum below 2^-64 is lifted by 2^64 together with the values before inv and the
+// products are formed, so inv stays finite.
 //
 // MXFP8 (the pages' format for the index Q/K): 32-element blocks share one E8M0 byte E = X + 127,
 // X = floor(log2(amax)) - 8 clamped to [-127, 127]; the codes are E4M3 of x * 2^-X.
@@ -36,15 +38,19 @@ quantize_groups_kernel(const T* __restrict__ src, int64_t n_rows, int src_stride
     for (int i = lane; i < group; i += 32) amax = fmaxf(amax, fabsf(to_f32(x[i])));
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    // below 2^-64 the maximum and the values are lifted by 2^64 (exact) first: 448 / amax would
+    // overflow for amax < 448 / FLT_MAX and turn the group's zeros into 0 * inf = NaN; where it
+    // is finite the lift changes no code (reciprocal and products move by a power of two)
+    const float lift = amax < 0x1p-64f ? 0x1p64f : 1.f;
     float scale = 1.f, inv = 0.f;
     if (amax > 0.f) {
         scale = amax / 448.0f;
-        inv = 448.0f / amax;
+        inv = 448.0f / (amax * lift);
     }
     if (lane == 0) scales[slot * ng + g] = scale;
     uint8_t* c = codes + slot * D + (int64_t)g * group;
     for (int i = lane; i < group; i += 32) {
-        const float y = __fmul_rn(to_f32(x[i]), inv);
+        const float y = __fmul_rn(__fmul_rn(to_f32(x[i]), lift), inv);
         c[i] = amax > 0.f ? (uint8_t)__nv_cvt_float_to_fp8(y, __NV_SATFINITE, __NV_E4M3) : (uint8_t)0;
     }
 }
@@ -127,6 +133,34 @@ quantize_mx_kernel(const T* __restrict__ src, int64_t n_rows, int D,
     if (lane == 0) scales[slot * nb + b] = (uint8_t)E;
 }
 
+// Queries rounded onto the MXFP8 grid in one pass: the block exponent and code of
+// quantize_mx_kernel, written back as code * 2^(E - 127) in the destination type (the two-kernel
+// quantize-then-dequantize result, bit for bit, without the round trip through memory).
+template <typename T, typename U>
+__global__ void __launch_bounds__(kThreads)
+mx_round_kernel(const T* __restrict__ src, int64_t n_rows, int D, U* __restrict__ dst) {
+    const int64_t warp = ((int64_t)blockIdx.x * kThreads + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    const int nb = D / 32;
+    if (warp >= n_rows * nb) return;
+    const int64_t i = warp * 32 + lane;            // rows are contiguous: block b of row r
+    const float x = to_f32(src[i]);
+    float amax = fabsf(x);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    float v = 0.f;
+    if (amax > 0.f) {
+        const int X = min(127, max(-127, floor_log2(amax) - 8));
+        const float inv = __uint_as_float((uint32_t)(127 - X) << 23);
+        const uint8_t code = (uint8_t)__nv_cvt_float_to_fp8(__fmul_rn(x, inv), __NV_SATFINITE, __NV_E4M3);
+        v = e4m3_to_f32(code) * e8m0_to_f32((uint32_t)(X + 127));
+    }
+    if constexpr (sizeof(U) == 4)
+        dst[i] = v;
+    else
+        dst[i] = __float2bfloat16_rn(v);
+}
+
 template <typename T>
 __global__ void __launch_bounds__(kThreads)
 dequantize_mx_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ scales,
@@ -156,6 +190,28 @@ cudaError_t launch_quantize_mx(const void* src, hsa_dtype_t src_dtype, int64_t n
         quantize_mx_kernel<__nv_bfloat16><<<(unsigned)blocks, kThreads, 0, st>>>(
             reinterpret_cast<const __nv_bfloat16*>(src), n_rows, D, slot_mapping, num_slots, codes,
             scales);
+    count_launch();
+    return cudaGetLastError();
+}
+
+cudaError_t launch_mx_round(const void* src, hsa_dtype_t src_dtype, int64_t n_rows, int32_t D,
+                            void* dst, hsa_dtype_t dst_dtype, cudaStream_t st) {
+    if (n_rows == 0) return cudaSuccess;
+    const unsigned blocks = (unsigned)ceil_div(n_rows * (D / 32) * 32, kThreads);
+    const bool f32_in = src_dtype == HSA_F32, f32_out = dst_dtype == HSA_F32;
+    using bf = __nv_bfloat16;
+    if (f32_in && f32_out)
+        mx_round_kernel<float, float><<<blocks, kThreads, 0, st>>>(
+            reinterpret_cast<const float*>(src), n_rows, D, reinterpret_cast<float*>(dst));
+    else if (f32_in)
+        mx_round_kernel<float, bf><<<blocks, kThreads, 0, st>>>(
+            reinterpret_cast<const float*>(src), n_rows, D, reinterpret_cast<bf*>(dst));
+    else if (f32_out)
+        mx_round_kernel<bf, float><<<blocks, kThreads, 0, st>>>(
+            reinterpret_cast<const bf*>(src), n_rows, D, reinterpret_cast<float*>(dst));
+    else
+        mx_round_kernel<bf, bf><<<blocks, kThreads, 0, st>>>(
+            reinterpret_cast<const bf*>(src), n_rows, D, reinterpret_cast<bf*>(dst));
     count_launch();
     return cudaGetLastError();
 }

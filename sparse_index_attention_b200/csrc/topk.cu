@@ -181,9 +181,9 @@ topk_kernel(SeqView v, const float* __restrict__ scores, int64_t ld, int K, int 
     uint32_t* keys = keys_raw;           // staged keys: key i of the row at keys[i]
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int t = blockIdx.x;
-    const RowInfo r = load_row(v, t);
-    pdl_wait();                          // the scores are the previous kernel's output
+    pdl_wait();                          // scores and row descriptors may be earlier kernels' output
     pdl_trigger();
+    const RowInfo r = load_row(v, t);
     int32_t* out = idx + (int64_t)t * K;
     const int n = r.pos + 1;             // 0 for an invalid row: all -1
     if (n <= K) {

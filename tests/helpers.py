@@ -97,6 +97,48 @@ def attn_close(gpu, ref, tol):
     return bool(np.all(ok)), float(err.max())
 
 
+def check_selection_vs_oracle(ref_sc, mag, gidx, n_valid, K, labels=None, rel=1e-3):
+    """Oracle-score agreement of the GPU selection, per the path's contract: the float64-score
+    selection (oracle Top-K) agrees on >= 99.9 % of positions summed over the rows, and every
+    position in the symmetric difference of a row is a near tie of the oracle's K-th score,
+    |I_ref(s) - I_ref(kth)| <= rel (|I_ref(kth)| + M) with M the larger magnitude sum of the two
+    positions.  Rows with n <= K must agree exactly.  Returns the oracle selection."""
+    ref_idx = oracle.topk(ref_sc, n_valid, K)
+    agree = total = 0
+    for i in range(len(gidx)):
+        a = set(gidx[i][gidx[i] >= 0].tolist())
+        b = set(ref_idx[i][ref_idx[i] >= 0].tolist())
+        total += len(b)
+        agree += len(a & b)
+        n = int(n_valid[i])
+        label = labels[i] if labels is not None else i
+        if n <= K:
+            assert a == b, ("short row selects every position", label)
+            continue
+        row = ref_sc[i, :n]
+        kth = -np.partition(-row, K - 1)[K - 1]
+        m_kth = mag[i, :n][row == kth].max()
+        for s in a ^ b:
+            m = max(mag[i, s], m_kth)
+            assert abs(row[s] - kth) <= rel * (abs(kth) + m), ("not a near tie", label, s)
+    assert agree >= 0.999 * total, (agree, total)
+    return ref_idx
+
+
+def attention_vs_oracle(pg, q, kv, gidx, ref_idx, D_v, scale, out, tol):
+    """Attention of the GPU's own selection against the oracle's attention over that same
+    selection (gated at `tol`), so that a near-tie swap in the index is not charged to the
+    attention kernel.  The end-to-end comparison (oracle attention over the oracle's own
+    selection) is returned as a reported number: a swapped near tie of the index score may carry
+    any attention weight."""
+    ref_out, _ = oracle.sparse_mla(pg, q, kv, gidx, D_v, scale)
+    got = out.float().cpu().numpy()
+    ok, worst = attn_close(got, ref_out, tol)
+    assert ok, ("attention on the GPU's selection", worst)
+    e2e_out, _ = oracle.sparse_mla(pg, q, kv, ref_idx, D_v, scale)
+    return float(np.abs(got - e2e_out).max())
+
+
 def stable_topk_reference(scores: torch.Tensor, q_pos: torch.Tensor, K: int) -> torch.Tensor:
     """Selection from the same fp32 scores with torch's stable sort (descending score, ties by
     position), re-sorted ascending: the reference for the bit-exact Top-K check."""

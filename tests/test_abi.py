@@ -19,7 +19,8 @@ def _declared():
 def test_header_declares_the_path():
     names = _declared()
     for n in ("hsa_index_score", "hsa_topk", "hsa_sparse_mla_attn", "hsa_fused_decode",
-              "hsa_quantize_index", "hsa_quantize_kv", "hsa_quantize_mx", "hsa_dequantize_mx"):
+              "hsa_quantize_index", "hsa_quantize_kv", "hsa_quantize_mx", "hsa_dequantize_mx",
+              "hsa_mx_round", "hsa_decode_prolog"):
         assert n in names
 
 
@@ -76,6 +77,40 @@ def test_validation_without_gpu():
     assert L.hsa_dequantize_mx(fake, fake, 10, 40, fake, hsa.HSA_BF16, None) == hsa.HSA_ERR_INVALID_ARG
     assert L.hsa_dequantize_mx(fake, fake, 10, 64, fake, hsa.HSA_E4M3, None) == hsa.HSA_ERR_UNSUPPORTED
     assert L.hsa_quantize_mx(None, hsa.HSA_BF16, 0, 64, None, 0, None, None, None) == hsa.HSA_OK
+    # cache-write quantizers: misaligned sources, scales, rope cache or slot mapping are refused
+    odd = ctypes.c_void_p(0x1001)
+    rc = L.hsa_quantize_index(odd, hsa.HSA_BF16, 10, 128, 128, None, 10, fake, fake, None)
+    assert rc == hsa.HSA_ERR_INVALID_ARG and b"misaligned" in L.hsa_last_error_message()
+    rc = L.hsa_quantize_index(fake, hsa.HSA_F32, 10, 128, 128, None, 10, fake, odd, None)
+    assert rc == hsa.HSA_ERR_INVALID_ARG
+    rc = L.hsa_quantize_kv(fake, hsa.HSA_BF16, 10, 512, 64, 512, odd, 10, fake, fake, fake, None)
+    assert rc == hsa.HSA_ERR_INVALID_ARG
+    rc = L.hsa_quantize_kv(fake, hsa.HSA_BF16, 10, 512, 64, 512, None, 10, fake, fake, odd, None)
+    assert rc == hsa.HSA_ERR_INVALID_ARG
+    rc = L.hsa_quantize_kv(odd, hsa.HSA_F32, 10, 512, 64, 512, None, 10, fake, fake, fake, None)
+    assert rc == hsa.HSA_ERR_INVALID_ARG
+    rc = L.hsa_quantize_mx(fake, hsa.HSA_BF16, 10, 64, odd, 10, fake, fake, None)
+    assert rc == hsa.HSA_ERR_INVALID_ARG
+    # MX rounding of queries: blocks of 32, partial overlap refused, in place allowed
+    assert L.hsa_mx_round(fake, hsa.HSA_BF16, 4, 48, fake, hsa.HSA_BF16, None) == hsa.HSA_ERR_INVALID_ARG
+    assert L.hsa_mx_round(fake, hsa.HSA_E4M3, 4, 64, fake, hsa.HSA_BF16, None) == hsa.HSA_ERR_UNSUPPORTED
+    rc = L.hsa_mx_round(ctypes.c_void_p(0x1000), hsa.HSA_BF16, 4, 64, ctypes.c_void_p(0x1040),
+                        hsa.HSA_BF16, None)
+    assert rc == hsa.HSA_ERR_INVALID_ARG and b"overlap" in L.hsa_last_error_message()
+    # decode prolog: every operator is checked before anything is enqueued
+    pa = hsa.hsa_prolog_args_t(4, fake, 64, fake, hsa.HSA_BF16, 128, fake, fake, hsa.HSA_MXE4M3,
+                               fake, hsa.HSA_BF16, 512, 64, 48, fake, fake, fake, fake, hsa.HSA_BF16,
+                               8, fake)
+    assert L.hsa_decode_prolog(ctypes.byref(pa), None, None, None, None) == hsa.HSA_ERR_INVALID_ARG
+    pa.kv_group = 512
+    pa.k_dtype = hsa.HSA_BF16
+    assert L.hsa_decode_prolog(ctypes.byref(pa), None, None, None, None) == hsa.HSA_ERR_UNSUPPORTED
+    pa.k_dtype = hsa.HSA_MXE4M3
+    pa.slot_mapping = None
+    assert L.hsa_decode_prolog(ctypes.byref(pa), None, None, None, None) == hsa.HSA_ERR_INVALID_ARG
+    pa.slot_mapping = odd
+    assert L.hsa_decode_prolog(ctypes.byref(pa), None, None, None, None) == hsa.HSA_ERR_INVALID_ARG
+    assert L.hsa_decode_prolog(None, None, None, None, None) == hsa.HSA_ERR_INVALID_ARG
     # zero rows is a no-op, not an error
     empty = hsa.hsa_paged_seq_t(1, fake, fake, 4, 16, 4, 64, 0, None, None, 1, None)
     assert L.hsa_topk(ctypes.byref(empty), None, 64, 8, None, None) == hsa.HSA_OK

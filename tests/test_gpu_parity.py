@@ -356,6 +356,32 @@ def test_quantize_kv_bit_exact_and_rounding_ties():
     assert np.array_equal(gcodes.cpu().numpy(), ref)
 
 
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_quantize_tiny_group_maxima_bit_exact(dtype):
+    """Groups whose maximum is far below 448 / FLT_MAX (1e-37, 1e-40, 2^-64, 2^-65, 2^-140)
+    and which hold zeros: codes and scales equal the oracle's bit for bit, and no NaN code
+    appears.  The same rows through the KV quantizer (latent part) agree as well."""
+    rng = np.random.default_rng(21)
+    rows = []
+    for amax in (1e-37, 1e-40, 2.0 ** -64, 2.0 ** -65, 2.0 ** -140, 1.0):
+        base = rng.standard_normal(128)
+        base[rng.random(128) < 0.25] = 0.0
+        base = base / np.abs(base).max() * amax
+        rows.append(base)
+    x = torch.tensor(np.stack(rows), dtype=torch.float32).to(dtype)
+    xf = x.float()
+    for grp in (128, 32):
+        codes, scales = hsa.hsa_quantize_index(x.to(DEV), grp)
+        rc, rs = oracle.quantize_rows(xf, grp)
+        assert np.array_equal(codes.cpu().numpy(), rc), grp
+        assert np.array_equal(scales.cpu().numpy(), rs), grp
+        assert not np.any((rc & 0x7F) == 0x7F)
+    kv = torch.cat([x, torch.zeros((x.shape[0], 64), dtype=dtype)], dim=1).contiguous()
+    kcodes, kscales, _ = hsa.hsa_quantize_kv(kv.to(DEV), 128, 128)
+    rc, rs = oracle.quantize_rows(xf, 128)
+    assert np.array_equal(kcodes.cpu().numpy(), rc) and np.array_equal(kscales.cpu().numpy(), rs)
+
+
 def test_device_checks_flag_instead_of_faulting():
     wl = workloads.make("decode_bf16", DEV, B=3, L_min=200, L_max=600)
     status = torch.zeros(1, dtype=torch.int32, device=DEV)

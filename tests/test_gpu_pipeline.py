@@ -7,7 +7,8 @@ Checks per the path's contract:
         the symmetric difference is a near tie of the oracle's K-th score within the index-score
         tolerance;
   (iii) index scores within 1e-3 (|I_ref| + M); attention outputs within 2e-2 abs/rel (bf16),
-        6e-2 (FP8 caches), 1e-4 (fp32) of the oracle's end-to-end output;
+        6e-2 (FP8 caches), 1e-4 (fp32) of the oracle's attention over the GPU's own selection
+        (the end-to-end difference, over the oracle's own selection, is printed);
   (iv)  fused == unfused and two-stream == one-stream, bitwise.
 """
 import numpy as np
@@ -18,8 +19,9 @@ import oracle
 import sparse_index_attention_b200 as hsa
 from sparse_index_attention_b200 import workloads
 
-from helpers import (GpuCaches, OracleCaches, attn_close, check_status, compact_workload,
-                     index_tolerance_ok, oracle_paging, paged_seq, stable_topk_reference)
+from helpers import (GpuCaches, OracleCaches, attention_vs_oracle, check_selection_vs_oracle,
+                     check_status, compact_workload, index_tolerance_ok, oracle_paging, paged_seq,
+                     stable_topk_reference)
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -53,25 +55,12 @@ def check_against_oracle(wl, rows, sc, idx, out):
         n = n_valid[i]
         ok, worst = index_tolerance_ok(got_sc[i, :n], ref_sc[i, :n], mag[i, :n])
         assert ok, ("index score", rows[i], worst)
-    ref_idx = oracle.topk(ref_sc, n_valid, K)
     gidx = idx[rows].cpu().numpy()
-    agree = total = 0
-    for i in range(len(rows)):
-        a = set(gidx[i][gidx[i] >= 0].tolist())
-        b = set(ref_idx[i][ref_idx[i] >= 0].tolist())
-        total += len(b)
-        agree += len(a & b)
-        n = n_valid[i]
-        if n > K:
-            kth = np.sort(ref_sc[i, :n])[::-1][K - 1]
-            for s in a ^ b:
-                m = max(mag[i, s], mag[i, :n][ref_sc[i, :n] == kth].max())
-                assert abs(ref_sc[i, s] - kth) <= 1e-3 * (abs(kth) + m), ("not a near tie", rows[i], s)
-    assert agree >= 0.999 * total, (agree, total)
-    ref_out, _ = oracle.sparse_mla(pg, wl.q[rows].cpu(), oc.kv, ref_idx, wl.D_v, wl.softmax_scale)
+    ref_idx = check_selection_vs_oracle(ref_sc, mag, gidx, n_valid, K, rows)
     tol = 6e-2 if (wl.kv_fp8 or wl.index_fp8) else TOL[wl.dtype]
-    ok, worst = attn_close(out[rows].float().cpu().numpy(), ref_out, tol)
-    assert ok, ("attention", worst)
+    e2e = attention_vs_oracle(pg, wl.q[rows].cpu(), oc.kv, gidx, ref_idx, wl.D_v, wl.softmax_scale,
+                              out[rows], tol)
+    print(f"{wl.name}: end-to-end attention difference over {len(rows)} rows {e2e:.3g}")
 
 
 @pytest.mark.parametrize("name,kw", [
@@ -202,6 +191,23 @@ def test_decode_prolog_three_streams_equals_one_shot_caches(mx):
     for got, ref in ((k, k_ref), (ks, ks_ref), (kv, kv_ref), (kvs, kvs_ref), (rope, rope_ref)):
         assert torch.equal(got, ref)
     assert torch.equal(q_out, hsa.mx_round(wl.q_I))
+    # the rows the prolog wrote, against the oracle's own quantizers of the same source rows
+    src_k = wl.k_I[last].float().cpu()
+    if mx:
+        rc, rs = oracle.mx_quantize_rows(src_k)
+        assert np.array_equal(k[last].cpu().numpy(), rc) and np.array_equal(ks[last].cpu().numpy(), rs)
+    else:
+        rc, rs = oracle.quantize_rows(src_k, wl.D_I)
+        assert np.array_equal(k[last].cpu().numpy(), rc)
+        assert np.array_equal(ks[last].cpu().numpy(), rs[:, 0])
+    rc, rs = oracle.quantize_rows(wl.kv[last][:, :wl.D_v].float().cpu(), wl.D_v)
+    assert np.array_equal(kv[last].cpu().numpy(), rc) and np.array_equal(kvs[last].cpu().numpy(), rs[:, 0])
+    assert torch.equal(rope[last], wl.kv[last][:, wl.D_v:])
+    # q_I on the MX grid: the oracle's quantize-then-dequantize, rounded to bf16 (exact here:
+    # every block exponent of N(0, 1) data is far above the bf16 subnormal range)
+    qf = wl.q_I.float().cpu().reshape(-1, wl.D_I)
+    q_ref = oracle.mx_dequantize_rows(*oracle.mx_quantize_rows(qf))
+    assert np.array_equal(q_out.float().cpu().numpy().reshape(q_ref.shape), q_ref)
     seq = paged_seq(wl)
     a = hsa.hsa_fused_decode(seq, q_out, wl.w, k, ks, wl.q, kv, kvs, rope, wl.K, wl.D_v,
                              wl.softmax_scale)
@@ -231,4 +237,88 @@ def test_decode_graph_replays_bitwise(aux):
                                                       wl.softmax_scale)
         torch.cuda.synchronize()
         assert torch.equal(idx_g, idx_d) and torch.equal(out_g, out_d) and torch.equal(lse_g, lse_d)
+        # the replayed step against the oracle on this step's inputs
+        check_against_oracle(wl, [0, 3, 7], g.scores, idx_g, out_g)
     check_status(seq)
+
+
+def _growing_decode(wl, steps):
+    """A decode loop's state before its first step: every sequence holds `steps` tokens fewer
+    than the workload, each crosses into a new cache page during the loop, the caches hold no
+    rows for the missing tokens yet (zeroed slots) and the block table has no entries for the
+    pages still to come (an out-of-range page id, which a kernel would report as a bad page if
+    it read one)."""
+    P = wl.page_size
+    final = wl.seq_lens.tolist()
+    len0 = []
+    for b, L in enumerate(final):
+        m = (L - steps + 1) // P
+        len0.append(P * m - 1 - (b % 2))
+    len0_t = torch.tensor(len0, dtype=torch.int32, device=DEV)
+    bt_true = wl.block_table.clone()
+    bt = bt_true.clone()
+    for b, n0 in enumerate(len0):
+        bt[b, (n0 + P - 1) // P:] = wl.num_pages + 7
+    return len0, len0_t, bt_true, bt
+
+
+def _slot_of(bt_true, P, b, pos):
+    return int(bt_true[b, pos // P]) * P + pos % P
+
+
+@pytest.mark.parametrize("graph", [False, True])
+def test_decode_loop_descriptors_advanced_on_device(graph):
+    """A decode loop that advances the row descriptors on the device, on the launching stream,
+    right before each step: seq_lens and q_pos grow by one, the block table gains the page of
+    the new position when it starts one, and the decode prolog writes the new token's MXFP8
+    index key, FP8 latent row and rope into the caches and rounds q_I onto the MX grid.  Each
+    step (the fused call, or a replay of the captured step) must see all of it: it is compared
+    with the oracle on the state of that step, and no device check may fire."""
+    steps = 3
+    wl = workloads.make("decode_mxfp8", DEV, B=4, L=2600)
+    P = wl.page_size
+    len0, _, bt_true, bt = _growing_decode(wl, steps)
+    k_full, ks_full = hsa.hsa_quantize_mx(wl.k_I)
+    kv_full, kvs_full, rope_full = hsa.hsa_quantize_kv(wl.kv, wl.D_v, wl.D_v)
+    k, ks, kv, kvs, rope = (t.clone() for t in (k_full, ks_full, kv_full, kvs_full.view(-1), rope_full))
+    for b, n0 in enumerate(len0):
+        for pos in range(n0, int(wl.seq_lens[b])):
+            s = _slot_of(bt_true, P, b, pos)
+            for t in (k, ks, kv, kvs, rope):
+                t[s] = 0
+    seq_lens = torch.tensor(len0, dtype=torch.int32, device=DEV)
+    q_pos = seq_lens - 1
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    seq = hsa.PagedSeq(seq_lens, bt, P, wl.num_pages, wl.q_seq, q_pos,
+                       max_seq_len=int(wl.seq_lens.max()), q_run=1, status=status)
+    assert seq.seq_lens.data_ptr() == seq_lens.data_ptr() and seq.block_table.data_ptr() == bt.data_ptr()
+    q_out = hsa.mx_round(wl.q_I)
+    g = None
+    if graph:
+        g = hsa.DecodeGraph(seq, q_out, wl.w, k, ks, wl.q, kv, kvs, rope, wl.K, wl.D_v,
+                            wl.softmax_scale, aux=True)
+    main = torch.cuda.current_stream()
+    rows = list(range(wl.T_q))
+    ar = torch.arange(wl.B, device=DEV)
+    for i in range(steps):
+        # ---- the loop's own device work, on the launching stream, before the step
+        pos = [n0 + i for n0 in len0]
+        slots = torch.tensor([_slot_of(bt_true, P, b, p) for b, p in enumerate(pos)], dtype=torch.int64,
+                             device=DEV)
+        seq_lens.add_(1)
+        q_pos.add_(1)
+        lp = (q_pos // P).long()
+        bt[ar, lp] = bt_true[ar, lp]
+        hsa.hsa_decode_prolog(wl.k_I[slots], wl.kv[slots], slots, k, ks, kv, kvs, rope, wl.q_I,
+                              q_out, wl.D_v, stream=main)
+        if graph:
+            out, lse, idx, sc = (t.clone() for t in g.replay())
+        else:
+            out, lse, idx, sc = hsa.hsa_fused_decode(seq, q_out, wl.w, k, ks, wl.q, kv, kvs, rope,
+                                                     wl.K, wl.D_v, wl.softmax_scale, stream=main)
+        torch.cuda.synchronize()
+        assert int(status.item()) == 0, f"device status {int(status.item()):#x} at step {i}"
+        import dataclasses
+        state = dataclasses.replace(wl, seq_lens=seq_lens.clone(), q_pos=q_pos.clone(),
+                                    block_table=bt_true)
+        check_against_oracle(state, rows, sc, idx, out)

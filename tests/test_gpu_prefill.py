@@ -11,8 +11,8 @@ import oracle
 import sparse_index_attention_b200 as hsa
 from sparse_index_attention_b200 import workloads
 
-from helpers import (GpuCaches, OracleCaches, attn_close, check_status, compact_workload,
-                     index_tolerance_ok, oracle_paging, paged_seq)
+from helpers import (GpuCaches, OracleCaches, attention_vs_oracle, check_selection_vs_oracle,
+                     check_status, compact_workload, index_tolerance_ok, oracle_paging, paged_seq)
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -38,13 +38,15 @@ def stable_topk_batched(scores, q_pos, K):
 
 
 def check_rows(wl_full, rows, sc, idx, out, tol):
-    """Index tolerance, oracle-selection agreement and attention tolerance on the sampled rows
-    (sc / idx / out hold those rows' GPU results, in order)."""
+    """Index tolerance, oracle-selection agreement with the near-tie check on every mismatch,
+    and attention tolerance on the GPU's own selection, for the sampled rows (sc / idx / out
+    hold those rows' GPU results, in order)."""
     wl = compact_workload(wl_full, rows)
+    labels = list(rows)
     rows = list(range(wl.T_q))
     oc = OracleCaches(wl)
     pg = oracle_paging(wl)
-    qI, w = wl.q_I, wl.w
+    qI, w = oc.q_I, wl.w
     ld = sc.shape[1]
     ref_sc = oracle.index_score(pg, qI, w, oc.k, ld=ld)
     mag = oracle.index_score(pg, qI, w.abs(), oc.k, ld=ld)
@@ -53,15 +55,11 @@ def check_rows(wl_full, rows, sc, idx, out, tol):
     for i in range(len(rows)):
         n = n_valid[i]
         ok, worst = index_tolerance_ok(got[i, :n], ref_sc[i, :n], mag[i, :n])
-        assert ok, ("index", rows[i], worst)
-    ref_idx = oracle.topk(ref_sc, n_valid, wl.K)
+        assert ok, ("index", labels[i], worst)
     gidx = idx.cpu().numpy()
-    agree = sum(len(set(a[a >= 0]) & set(b[b >= 0])) for a, b in zip(gidx, ref_idx))
-    total = int((ref_idx >= 0).sum())
-    assert agree >= 0.999 * total, (agree, total)
-    ref_out, _ = oracle.sparse_mla(pg, wl.q, oc.kv, ref_idx, wl.D_v, wl.softmax_scale)
-    ok, worst = attn_close(out.float().cpu().numpy(), ref_out, tol)
-    assert ok, ("attention", worst)
+    ref_idx = check_selection_vs_oracle(ref_sc, mag, gidx, n_valid, wl.K, labels)
+    e2e = attention_vs_oracle(pg, wl.q, oc.kv, gidx, ref_idx, wl.D_v, wl.softmax_scale, out, tol)
+    print(f"{wl.name}: end-to-end attention difference over {len(rows)} rows {e2e:.3g}")
 
 
 def run_prefill(wl, chunks=None):
@@ -155,5 +153,10 @@ def test_zigzag_cp_single_rank_equals_chunked_prefill():
         torch.cuda.synchronize()
     finally:
         dist.destroy_process_group()
-    _, _, out, lse, idx = run_prefill(wl, [(0, 1024), (1024, 2048)])
+    gc, seq, out, lse, idx = run_prefill(wl, [(0, 1024), (1024, 2048)])
     assert torch.equal(idx_c, idx) and torch.equal(out_c, out) and torch.equal(lse_c, lse)
+    # the context-parallel result against the oracle on sampled rows (scores recomputed per row)
+    rows = workloads.sample_rows(wl.T_q, 256, extra=(1023, 1024, 2047))
+    sc_rows = torch.cat([hsa.hsa_index_score(seq.rows(r, r + 1, q_run=1), wl.q_I[r:r + 1],
+                                             wl.w[r:r + 1], gc.k) for r in rows])
+    check_rows(wl, rows, sc_rows, idx_c[rows], out_c[rows], 2e-2)

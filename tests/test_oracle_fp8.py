@@ -129,6 +129,46 @@ def test_quantize_scale_rule_and_error_bound():
     assert np.all(np.abs(deq - x) <= bound + np.abs(x) * 1e-6)
 
 
+@pytest.mark.parametrize("amax", [1e-37, 1e-40, 2.0 ** -64, 2.0 ** -65, 2.0 ** -140])
+def test_quantize_tiny_group_maximum(amax):
+    """A group whose maximum is so small that 448 / amax overflows float32 (below about
+    1.3e-36): no NaN or saturated code appears, the group's zeros stay code 0, its maximum
+    takes the top code, and every value dequantizes within half a spacing (times the scale)."""
+    amax = np.float32(amax)
+    x = np.zeros((2, 32), dtype=np.float32)
+    x[0, 3] = amax
+    x[0, 9] = -amax / np.float32(2)
+    x[0, 17] = amax * np.float32(0.3)
+    x[1] = x[0] * np.float32(-1)
+    codes, scales = oracle.quantize_rows(x, 32)
+    assert not np.any((codes & 0x7F) == 0x7F)                 # no NaN code
+    for r in range(2):
+        zero = x[r] == 0
+        assert np.all((codes[r][zero] & 0x7F) == 0)                # +0 or -0
+        assert (int(codes[r, 3]) & 0x7F) == 0x7E                # the maximum -> 448
+        assert int(codes[r, 9]) & 0x7F == 0x76                   # half of it -> 224 = 1.75 * 2^7
+        assert scales[r, 0] == np.float32(np.float64(amax) / 448.0)
+    deq = oracle.dequantize_rows(codes, scales, 32)
+    # half the top binade's spacing (16) times the scale, plus what the stored scale lost by
+    # rounding (it is subnormal, or 0, for the smallest maxima) times the largest code
+    s_exact = np.float64(amax) / 448.0
+    s = np.float64(scales[0, 0])
+    assert np.all(np.abs(deq - x) <= 16 * s * (1 + 1e-6) + 448 * abs(s - s_exact) * (1 + 1e-6))
+
+
+def test_quantize_lift_changes_no_code_where_the_reciprocal_is_finite():
+    """Groups above and below the 2^-64 lift threshold but with a finite 448 / amax get exactly
+    the codes of the same group scaled up by a power of two (the scale rule is homogeneous
+    under exact power-of-two scaling)."""
+    rng = np.random.default_rng(11)
+    base = rng.standard_normal((16, 32)).astype(np.float32)
+    c_ref, s_ref = oracle.quantize_rows(base, 32)
+    for k in (-60, -64, -66, -90, -110):
+        c, s = oracle.quantize_rows(base * np.float32(2.0 ** k), 32)
+        assert np.array_equal(c, c_ref), k
+        assert np.array_equal(s.astype(np.float64), s_ref.astype(np.float64) * 2.0 ** k), k
+
+
 def test_group_32_variant_shares_scales_per_group():
     rng = np.random.default_rng(8)
     x = rng.standard_normal((4, 128)).astype(np.float32)
@@ -205,10 +245,10 @@ def _mx_data(n, D, seed):
 
 
 def test_mx_scale_rule_and_error_bound():
-    """For every block: the block maximum lands in the top E4M3 binade [256, 448] after the
-    division by 2^X (so X is the largest exponent that keeps it finite within E4M3's range,
-    rounding aside), and every element is within half an E4M3 spacing of x / 2^X, or saturated
-    at +-448 when it rounds past it."""
+    """For every block: the block maximum lies in [256, 512) after the division by 2^X (the top
+    E4M3 binade and the range above it that saturates to 448), its code decodes into
+    [256, 448], and every element is within half an E4M3 spacing of x / 2^X, or saturated at
+    +-448 when it rounds past it."""
     x = _mx_data(64, 128, 5)
     codes, scales = oracle.mx_quantize_rows(x)
     deq = oracle.mx_dequantize_rows(codes, scales)
