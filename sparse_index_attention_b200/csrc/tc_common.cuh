@@ -263,6 +263,23 @@ __device__ __forceinline__ void st_async_v4(uint32_t remote_addr, uint32_t remot
         : "memory");
 }
 
+// 4-byte store into another CTA's shared memory that counts 4 bytes against that CTA's mbarrier
+// transaction count.
+__device__ __forceinline__ void st_async_b32(uint32_t remote_addr, uint32_t remote_bar, uint32_t v) {
+    asm volatile(
+        "st.async.shared::cluster.mbarrier::complete_tx::bytes.b32 [%0], %1, [%2];"
+        ::"r"(remote_addr), "r"(v), "r"(remote_bar)
+        : "memory");
+}
+
+// Arrive (release, cluster scope) on an mbarrier in another CTA of the cluster (a shared::cluster
+// address from mapa_shared): this thread's earlier shared-memory reads and writes are ordered
+// before the arrival.
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t remote_bar) {
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(remote_bar)
+                 : "memory");
+}
+
 // Commit that arrives on the mbarrier at the same shared-memory offset in every CTA of
 // `cta_mask` once this thread's prior tcgen05 operations complete.
 __device__ __forceinline__ void mma_commit_multicast(uint64_t* bar, uint16_t cta_mask) {
