@@ -60,6 +60,14 @@ struct Cfg {
     static_assert(kSmem <= 232448, "shared memory budget");
 };
 
+// floor(log2(a)) of a positive finite float, from its bits (subnormals included).
+__device__ __forceinline__ int floor_log2_f(float a) {
+    const uint32_t bits = __float_as_uint(a);
+    const int e = (int)(bits >> 23);
+    if (e) return e - 127;
+    return (31 - __clz((int)(bits & 0x7FFFFFu))) - 149;
+}
+
 struct GroupInfo {
     int32_t b;        // sequence (of the group's first valid row)
     int32_t pos_max;  // largest valid position in the group, -1 if none
@@ -105,9 +113,13 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
                       int32_t box_rows) {
     using C = Cfg<G, kFp8, kMx>;
     static_assert(!kMx || kFp8, "MXFP8 keys go through the FP8 staging path");
+    // E4M3 keys with fp32 scales run the MMA in f16: a code widens to f16 in one conversion
+    // (exact), and the queries are rescaled per head by a power of two into f16's range, the
+    // inverse power folded into the head weight, which leaves every product and sum as in bf16.
+    constexpr bool kF16 = kFp8 && !kMx;
     constexpr int N = C::N;
     constexpr int S = C::kStages;
-    constexpr uint32_t kIdesc = tc::idesc_bf16_f32(kBM, N, 0, 0);
+    constexpr uint32_t kIdesc = kF16 ? tc::idesc_f16_f32(kBM, N) : tc::idesc_bf16_f32(kBM, N, 0, 0);
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -126,9 +138,10 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
     uint64_t* raw_full = q_empty + 1;      // [4] FP8 bytes landed
     uint64_t* raw_empty = raw_full + 4;    // [4] converters done with the staging tile
     uint64_t* epi_bar = raw_empty + 4;     // the four epilogue warps
-    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(epi_bar + 1);
+    uint64_t* q_ready = epi_bar + 1;       // f16 MMA: the group's queries converted (4 warps)
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(q_ready + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
-    static_assert((2 * S + 2 + 2 + 2 + 8 + 1) * 8 + 8 <= 256, "barrier block");
+    static_assert((2 * S + 2 + 2 + 2 + 8 + 2) * 8 + 8 <= 256, "barrier block");
     int32_t* prefix = reinterpret_cast<int32_t*>(reinterpret_cast<uint8_t*>(bars) + 256);
     float* w_s = reinterpret_cast<float*>(prefix + C::kMaxGroups + 1);
 
@@ -151,6 +164,7 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
             tc::mbar_init(&raw_empty[i], 128);
         }
         tc::mbar_init(epi_bar, 4);
+        tc::mbar_init(q_ready, 4);
         *abort_flag = 0;
         tc::fence_barrier_init();
     }
@@ -260,7 +274,7 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
                 for (int64_t f = f_begin; f < f_end; ++f) {
                     locate(prefix, n_groups, f, g, kt);
                     if (g != cur) {
-                        if (!tc::mbar_wait(q_full, q_phase, abort_flag)) break;
+                        if (!tc::mbar_wait(kF16 ? q_ready : q_full, q_phase, abort_flag)) break;
                         q_phase ^= 1;
                         cur = g;
                     }
@@ -299,14 +313,61 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
             uint32_t acc = 0, acc_phase = 0;
             int32_t row_pos[G];
             int32_t seq_b = 0;
+            uint32_t qf_phase = 0;
             tc::WarpSetSync epi_sync{epi_bar, 0};
             for (int64_t f = f_begin; f < f_end; ++f) {
                 locate(prefix, n_groups, f, g, kt);
                 if (g != cur) {
                     if (!epi_sync.sync(abort_flag)) break;   // everyone is done with the old weights
-                    for (int i = et; i < N; i += 128) {
-                        const int t = g * G + i / kHI;
-                        w_s[i] = t < v.T_q ? w[(int64_t)t * kHI + (i % kHI)] : 0.f;
+                    if (kF16) {
+                        // the group's queries (TMA-landed bf16, two 64-dim swizzled halves) become
+                        // f16 in place: row i (query row x head) is scaled by 2^-e so that its
+                        // largest magnitude lies in [2^14, 2^15), and its weight by 2^e; two
+                        // threads per row, one per half
+                        if (!tc::mbar_wait(q_full, qf_phase, abort_flag)) break;
+                        qf_phase ^= 1;
+                        const int hf = et & 1;
+                        for (int i = et >> 1; i < N; i += 64) {
+                            uint4* rowp = reinterpret_cast<uint4*>(qbuf + (size_t)hf * (N * 128) + (size_t)i * 128);
+                            uint4 x[8];
+                            float mx = 0.f;
+#pragma unroll
+                            for (int c = 0; c < 8; ++c) {
+                                x[c] = rowp[c];
+                                const uint32_t wv[4] = {x[c].x, x[c].y, x[c].z, x[c].w};
+#pragma unroll
+                                for (int qq = 0; qq < 4; ++qq) {
+                                    const float2 f2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&wv[qq]));
+                                    mx = fmaxf(mx, fmaxf(fabsf(f2.x), fabsf(f2.y)));
+                                }
+                            }
+                            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+                            const int e = mx > 0.f ? min(100, max(-100, floor_log2_f(mx) - 14)) : 0;
+                            const float f = __uint_as_float((uint32_t)(127 - e) << 23);
+#pragma unroll
+                            for (int c = 0; c < 8; ++c) {
+                                uint32_t wv[4] = {x[c].x, x[c].y, x[c].z, x[c].w};
+#pragma unroll
+                                for (int qq = 0; qq < 4; ++qq) {
+                                    const float2 f2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&wv[qq]));
+                                    const __half2 h2 = __floats2half2_rn(f2.x * f, f2.y * f);
+                                    wv[qq] = *reinterpret_cast<const uint32_t*>(&h2);
+                                }
+                                rowp[c] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+                            }
+                            if (hf == 0) {
+                                const int t = g * G + i / kHI;
+                                w_s[i] = t < v.T_q ? w[(int64_t)t * kHI + (i % kHI)] *
+                                                         __uint_as_float((uint32_t)(127 + e) << 23)
+                                                   : 0.f;
+                            }
+                        }
+                        tc::fence_async_smem();   // the f16 queries -> the tensor core
+                    } else {
+                        for (int i = et; i < N; i += 128) {
+                            const int t = g * G + i / kHI;
+                            w_s[i] = t < v.T_q ? w[(int64_t)t * kHI + (i % kHI)] : 0.f;
+                        }
                     }
                     const GroupInfo gi = group_info(v, g, G, false);
                     seq_b = gi.b < 0 ? 0 : gi.b;
@@ -320,6 +381,7 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
                         }
                     }
                     if (!epi_sync.sync(abort_flag)) break;   // the new weights are in place
+                    if (kF16 && lane == 0) tc::mbar_arrive(q_ready);
                     cur = g;
                 }
                 if (!tc::mbar_wait(&acc_full[acc], acc_phase, abort_flag)) break;
@@ -419,11 +481,10 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
                         for (int q = 0; q < 4; ++q) {
 #pragma unroll
                             for (int hlf = 0; hlf < 2; ++hlf) {
+                                // one conversion per code pair, straight to the f16 the MMA reads
                                 const __nv_fp8x2_storage_t pair = (__nv_fp8x2_storage_t)(words[q] >> (16 * hlf));
                                 const __half2_raw h2 = __nv_cvt_fp8x2_to_halfraw2(pair, __NV_E4M3);
-                                const float2 f2 = __half22float2(__half2(h2));
-                                const __nv_bfloat162 b2 = __floats2bfloat162_rn(f2.x, f2.y);
-                                outw[q * 2 + hlf] = *reinterpret_cast<const uint32_t*>(&b2);
+                                outw[q * 2 + hlf] = (uint32_t)h2.x | ((uint32_t)h2.y << 16);
                             }
                         }
                     }

@@ -15,33 +15,29 @@
 // The fp32 output accumulator O (128 x 512) alone fills the 512 TMEM columns of an SM, so a
 // cluster of two CTAs splits the latent dims: CTA r owns value dims [256r, 256r + 256) and, for
 // S, the matching 256 latent dims plus rope dims [512 + 32r, 544 + 32r).  Each CTA computes a
-// partial S over its 288 dims and the pair swaps partial S through distributed shared memory
-// (st.async, which also completes the receiver's mbarrier transaction count).  No gathered byte
-// and no MMA is duplicated between the two CTAs.
-//
-// The exchanged partial S travels as fp16 with a power-of-two scale per head and 32 columns
-// (the scale keeps the largest magnitude below 2^15, so nothing overflows; the rounding is
-// 2^-11 relative, some 20 times finer than the bf16 rounding P gets before P.V).  Each CTA
-// rounds its own partial in exactly the same way before adding the peer's, so both CTAs hold
-// the bitwise identical S, take identical softmax decisions and produce the two halves of one
-// consistent output.
+// partial S over its 288 dims, the pair swaps partial S through distributed shared memory
+// (st.async that also completes the receiver's mbarrier transaction count), and both add the
+// halves (fp32 addition commutes, so both hold the identical S and take identical softmax
+// decisions).  Each CTA then accumulates its half of O.  No gathered byte and no MMA is
+// duplicated between the two CTAs.
 //
 // Shared memory per CTA: the rope part of Q (8 KB, 64-byte swizzle), four KV stages of 64
 // gathered rows (36 KB each: four 64-dim 128-byte-swizzled blocks + one 32-dim 64-byte-swizzled
 // rope block; the stage is the K-major B operand of Q.KV^T and, read MN-major, the B operand of
-// P.V), two P buffers (bf16, 128 heads x 64 rows, 128-byte swizzled: the A operand of P.V), two
-// exchange buffers for the peer's partial S (16 KB of fp16 laid out [8-column chunk][head][8]
-// so that every warp-wide store and load covers 512 contiguous bytes, plus 512 bytes of scale
-// exponents), and the physical slots of the next 1024 selected entries.  Tensor memory: O (256
-// columns), two partial-S buffers (2 x 64 columns) and the latent part of Q (128 columns, the A
-// operand of Q.KV^T).
+// P.V), two 32 KB exchange buffers that receive the peer's partial S (fp32, laid out
+// [4-column chunk][head][4] so that every warp-wide store and load covers 512 contiguous bytes),
+// and the physical slots of the next 1024 selected entries.  Tensor memory: O (256 columns), two
+// partial-S buffers (2 x 64 columns; P, bf16 pairs, overwrites the first half of its S buffer and
+// is the TMEM A operand of P.V) and the latent part of Q (128 columns, the A operand of Q.KV^T).
 //
-// Pipeline.  An S buffer is released as soon as the softmax and sender warps have loaded it (P
-// goes to shared memory, not over S), and the MMA warp issues Q.KV^T(n) ahead of P.V(n-2), so
-// the tensor core computes the next tiles' S while the exchange and softmax of the previous
-// ones run.  Measured on B200: one tcgen05.mma issues in about 60 cycles whatever its N, so
-// Q.KV^T (18 MMAs of N = 64) costs more issue time than its flops; the cluster network moves
-// 512 contiguous bytes per warp store about twice as fast as one row per thread.
+// Pipeline per tile n: sender warps push partial S(n) to the peer as soon as Q.KV^T(n) is done,
+// independent of the softmax, so the distributed-shared-memory hop overlaps the softmax of the
+// previous tile, and the tensor core runs Q.KV^T(n+1) and P.V(n-1) while softmax(n) runs.  The
+// peer may overwrite an exchange buffer only after this CTA's P.V of the tile that used it (MMA
+// commit multicast to the peer), which is also what makes receiving tile n prove that P.V(n-2)
+// has finished.  Measured on B200: one tcgen05.mma issues in about 60 cycles whatever its N, so
+// Q.KV^T (18 MMAs of N = 64) costs more issue time than its flops; the cluster network moves the
+// 32 KB exchange in about 1 us when warp stores are contiguous (1.8 us with one row per thread).
 //
 // (A TMA tile::gather4 version of the gather -- four 128-byte rows per instruction, 80 per tile
 // and CTA -- delivered only about 0.75 TB/s here: the MMA warp waited on the gathered tiles for
@@ -73,15 +69,10 @@ constexpr int kQRopeBytes = kH * 64;               // 128 heads x 32 dims bf16, 
 constexpr int kKvBlk = kBN * 128;                  // 64 rows x 64 dims
 constexpr int kKvRope = kBN * 64;                  // 64 rows x 32 dims
 constexpr int kStageBytes = 4 * kKvBlk + kKvRope;  // 36 KB
-constexpr int kPBytes = kH * kBN * 2;              // 16 KB of bf16 P
-constexpr int kRecvHBytes = kH * kBN * 2;          // 16 KB of fp16 partial S
-constexpr int kRecvEBytes = kH * 4;                // one word of two scale exponents per head
-constexpr int kRecvBytes = kRecvHBytes + kRecvEBytes;
+constexpr int kRecvBytes = kH * kBN * 4;           // 32 KB of fp32 partial S
 constexpr int kOffStages = kQRopeBytes;
-constexpr int kOffP = kOffStages + kStages * kStageBytes;
-constexpr int kOffRecvH = kOffP + 2 * kPBytes;
-constexpr int kOffRecvE = kOffRecvH + 2 * kRecvHBytes;
-constexpr int kOffSlots = kOffRecvE + 2 * kRecvEBytes;
+constexpr int kOffRecv = kOffStages + kStages * kStageBytes;
+constexpr int kOffSlots = kOffRecv + 2 * kRecvBytes;
 constexpr int kOffMasks = kOffSlots + 4 * kSlotWin;
 constexpr int kOffXmax = kOffMasks + 8 * kStages;              // [2 tiles][2 halves][128] fp32
 constexpr int kOffXsum = kOffXmax + 4 * 512;                   // [2 halves][128] fp32
@@ -91,8 +82,7 @@ constexpr int kKv8RowBytes = kDv;       // 512: e4m3 latent codes (FP8 cache)
 constexpr int kRopeRowBytes = 128;      // bf16 rope of the FP8 cache
 constexpr size_t kSmem = 1024 + kOffBars + 256;
 static_assert(kSmem <= 232448, "shared memory budget");
-static_assert(kOffStages % 1024 == 0 && kStageBytes % 1024 == 0 && kOffP % 1024 == 0, "swizzle alignment");
-static_assert(kOffRecvH % 16 == 0 && kOffXmax % 16 == 0 && kOffBars % 8 == 0, "alignment");
+static_assert(kOffStages % 1024 == 0 && kStageBytes % 1024 == 0 && kOffRecv % 1024 == 0, "swizzle alignment");
 
 constexpr uint32_t kTmemO = 0;       // 256 columns: this CTA's half of O
 constexpr uint32_t kTmemS = 256;     // 2 x 64 columns: partial S, double-buffered
@@ -104,16 +94,15 @@ constexpr uint32_t kIdescPV = tc::idesc_bf16_f32(kH, 256, 0, 1);
 constexpr float kRescaleLog2 = 8.f;  // rescale O only when the running max grows by > 2^8
 
 struct Bars {
-    uint64_t q_full;      // Q of the row in place: latent part in TMEM, rope part in smem (8 warps)
+    uint64_t q_full;      // Q of the row in place: latent part in TMEM, rope part in smem (4 warps)
     uint64_t q_empty;     // last Q.KV^T of the row done
     uint64_t kv_full[kStages], kv_empty[kStages];
-    uint64_t s_full[2];     // Q.KV^T of the tile in S buffer b committed
-    uint64_t s_free[2];     // softmax (8 warps) and senders (4 warps) have loaded S buffer b
-    uint64_t p_full[2];     // softmax wrote P buffer b (8 warps)
-    uint64_t p_free[2];     // P.V of the tile in P buffer b completed
+    uint64_t s_full[2], s_empty[2];
+    uint64_t s_sent[2];     // the senders have read partial S of the buffer (P may overwrite it)
+    uint64_t p_full;
     uint64_t pv_done;     // this CTA's P.V of a tile completed
-    uint64_t recv_full[2];  // the peer's partial S of the tile in exchange buffer b has landed
-    uint64_t recv_free[2];  // the peer's softmax (8 warps) has read its exchange buffer b
+    uint64_t peer_free[2];  // the peer's P.V of a tile of parity b completed (its buffer b is free)
+    uint64_t recv_full[2];
     uint64_t o_ready, o_free;
     uint64_t pair_sync[4];  // the two softmax warps of a head quarter (maxima / row sums posted)
     uint32_t tmem;
@@ -139,33 +128,6 @@ __device__ __forceinline__ int row_tiles(const SeqView& v, const int32_t* __rest
     return (int)ceil_div(row_extent(idx + (int64_t)t * K, K, lane), kBN);
 }
 
-// Scale exponent e >= 0 of the exchanged partial S: 2^-e brings every magnitude up to `mx` below
-// 2^15, inside fp16's range (e = 0 unless |S| >= 2^15).
-__device__ __forceinline__ int exch_exp(float mx) {
-    return max(0, (int)((__float_as_uint(mx) >> 23) & 0xFFu) - 141);
-}
-__device__ __forceinline__ float pow2i(int e) { return __uint_as_float((uint32_t)(127 + e) << 23); }
-
-// 32 partial-S values of one head -> 16 words of fp16 pairs at scale 2^-e; returns e.  The same
-// function rounds a CTA's own partial (so both CTAs add identically rounded halves).
-__device__ __forceinline__ int pack_exchange(const float* v, uint32_t* w) {
-    float mx = 0.f;
-#pragma unroll
-    for (int i = 0; i < 32; ++i) mx = fmaxf(mx, fabsf(v[i]));
-    const int e = exch_exp(mx);
-    const float f = pow2i(-e);
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-        const __half2 h2 = __floats2half2_rn(v[2 * i] * f, v[2 * i + 1] * f);
-        w[i] = *reinterpret_cast<const uint32_t*>(&h2);
-    }
-    return e;
-}
-
-__device__ __forceinline__ float2 unpack_half2(uint32_t w) {
-    return __half22float2(*reinterpret_cast<const __half2*>(&w));
-}
-
 // kFp8Kv: the latent part of the cache is e4m3 codes with one fp32 scale per row and the rope part
 // a separate bf16 array; the producers widen code x scale to bf16 on the way into the stage.
 template <bool kFp8Kv>
@@ -179,9 +141,7 @@ sparse_mla_tc_kernel(SeqView v,
     uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* q_rope = base;
     uint8_t* stages = base + kOffStages;
-    uint8_t* pbuf = base + kOffP;
-    uint8_t* recv_h = base + kOffRecvH;
-    uint32_t* recv_e = reinterpret_cast<uint32_t*>(base + kOffRecvE);
+    uint8_t* recv = base + kOffRecv;
     int32_t* slots = reinterpret_cast<int32_t*>(base + kOffSlots);
     volatile uint64_t* masks = reinterpret_cast<volatile uint64_t*>(base + kOffMasks);
     float* xmax = reinterpret_cast<float*>(base + kOffXmax);
@@ -205,13 +165,14 @@ sparse_mla_tc_kernel(SeqView v,
         }
         for (int i = 0; i < 2; ++i) {
             tc::mbar_init(&bars->s_full[i], 1);
-            tc::mbar_init(&bars->s_free[i], 8 + 4);
-            tc::mbar_init(&bars->p_full[i], 8);
-            tc::mbar_init(&bars->p_free[i], 1);
+            tc::mbar_init(&bars->s_empty[i], 1);    // P.V of the tile whose P sits in the buffer
+            tc::mbar_init(&bars->s_sent[i], 4);     // 4 sender warps
             tc::mbar_init(&bars->recv_full[i], 1);
-            tc::mbar_init(&bars->recv_free[i], 8);
         }
+        tc::mbar_init(&bars->p_full, 8);
         tc::mbar_init(&bars->pv_done, 1);
+        tc::mbar_init(&bars->peer_free[0], 1);
+        tc::mbar_init(&bars->peer_free[1], 1);
         tc::mbar_init(&bars->o_ready, 1);
         tc::mbar_init(&bars->o_free, 8);
         for (int i = 0; i < 4; ++i) tc::mbar_init(&bars->pair_sync[i], 2);
@@ -227,7 +188,7 @@ sparse_mla_tc_kernel(SeqView v,
     tc::cluster_sync_all();  // the peer's barriers exist before anything remote touches them
     tc::tc_fence_after();
     const uint32_t tmem_base = bars->tmem;
-    pdl_wait();              // the selection and the row descriptors may be earlier kernels' output
+    pdl_wait();              // the selection is the previous kernel's output
     pdl_trigger();
 
     if (warp < 4) {
@@ -345,28 +306,25 @@ sparse_mla_tc_kernel(SeqView v,
         tc::cp_async_wait<0>();   // nothing of this thread still in flight when the CTA leaves
     } else if (warp == 4) {
         // ---------------------------------------------------------------- MMA issuer
-        // Per tile n of a row: Q.KV^T(n) as soon as its stage has landed and its S buffer is free
-        // (softmax and senders of tile n-2 have loaded it), then P.V(n-2); the row's last two
-        // P.V follow its last Q.KV^T.
         const uint32_t qr_addr = tc::smem_u32(q_rope);
         uint32_t n = 0, qr = 0, rows_done = 0;
         bool stop = false;
         auto pv = [&](uint32_t m, bool first) -> bool {
-            if (!tc::mbar_wait(&bars->p_full[m & 1], (m >> 1) & 1, abort_flag)) return false;
+            if (!tc::mbar_wait(&bars->p_full, m & 1, abort_flag)) return false;
             if (first && !tc::mbar_wait(&bars->o_free, (rows_done & 1) ^ 1, abort_flag)) return false;
-            tc::fence_async_smem();   // P written by the softmax threads -> tensor core
             tc::tc_fence_after();
             if (lane == 0) {
-                const uint32_t p_addr = tc::smem_u32(pbuf + (m & 1) * kPBytes);
+                const uint32_t p_tmem = tmem_base + kTmemS + (m & 1) * kBN;   // P (bf16 pairs) over S
                 const uint32_t v_addr = tc::smem_u32(stages + (m % kStages) * kStageBytes);
 #pragma unroll
                 for (int kk = 0; kk < kBN / 16; ++kk)
-                    tc::mma_bf16(tmem_base + kTmemO, tc::sw128_desc(p_addr + kk * 32, 16, 1024),
-                                 tc::sw128_desc(v_addr + kk * 2048, kKvBlk, 1024), kIdescPV,
-                                 (first && kk == 0) ? 0u : 1u);
+                    tc::mma_bf16_tmem_a(tmem_base + kTmemO, p_tmem + 8 * kk,
+                                        tc::sw128_desc(v_addr + kk * 2048, kKvBlk, 1024), kIdescPV,
+                                        (first && kk == 0) ? 0u : 1u);
                 tc::mma_commit(&bars->kv_empty[m % kStages]);
-                tc::mma_commit(&bars->p_free[m & 1]);
+                tc::mma_commit(&bars->s_empty[m & 1]);
                 tc::mma_commit(&bars->pv_done);
+                tc::mma_commit_multicast(&bars->peer_free[m & 1], (uint16_t)(1u << peer));
             }
             __syncwarp();
             return true;
@@ -377,11 +335,10 @@ sparse_mla_tc_kernel(SeqView v,
             if (ntiles == 0) continue;
             if (!tc::mbar_wait(&bars->q_full, qr & 1, abort_flag)) break;
             ++qr;
-            const uint32_t n0 = n;
             for (int j = 0; j < ntiles; ++j, ++n) {
                 const uint32_t st = n % kStages, sb = n & 1;
                 if (!tc::mbar_wait(&bars->kv_full[st], (n / kStages) & 1, abort_flag) ||
-                    (n >= 2 && !tc::mbar_wait(&bars->s_free[sb], ((n - 2) >> 1) & 1, abort_flag))) {
+                    !tc::mbar_wait(&bars->s_empty[sb], ((n >> 1) & 1) ^ 1, abort_flag)) {
                     stop = true;
                     break;
                 }
@@ -403,14 +360,12 @@ sparse_mla_tc_kernel(SeqView v,
                     if (j == ntiles - 1) tc::mma_commit(&bars->q_empty);
                 }
                 __syncwarp();
-                if (j >= 2 && !pv(n - 2, n - 2 == n0)) {
+                if (j > 0 && !pv(n - 1, j == 1)) {
                     stop = true;
                     break;
                 }
             }
-            if (stop) break;
-            if (ntiles >= 2 && !pv(n - 2, n - 2 == n0)) break;
-            if (!pv(n - 1, n - 1 == n0)) break;
+            if (stop || !pv(n - 1, ntiles == 1)) break;
             if (lane == 0) tc::mma_commit(&bars->o_ready);
             __syncwarp();
             ++rows_done;
@@ -425,8 +380,6 @@ sparse_mla_tc_kernel(SeqView v,
         const int half = (warp - 5) >> 2;              // which 32 columns / 128 output dims
         const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
         const uint32_t col = (uint32_t)(32 * half);
-        const uint32_t peer_recv_free[2] = {tc::mapa_shared(tc::smem_u32(&bars->recv_free[0]), peer),
-                                            tc::mapa_shared(tc::smem_u32(&bars->recv_free[1]), peer)};
         uint32_t n = 0, rows_done = 0;
         bool stop = false;
         tc::WarpSetSync pair_sync{&bars->pair_sync[(warp - 5) & 3], 0};   // warps w and w + 4
@@ -482,8 +435,10 @@ sparse_mla_tc_kernel(SeqView v,
             for (int j = 0; j < ntiles; ++j, ++n) {
                 const uint32_t b = n & 1, st = n % kStages;
                 // ---- softmax(n), columns [col, col + 32)
+                // own partial S(n) is complete once the senders have read it (s_sent), which
+                // also frees its columns for P; it is loaded while the peer's half is in flight
                 if (!tc::mbar_wait(&bars->kv_full[st], (n / kStages) & 1, abort_flag) ||
-                    !tc::mbar_wait(&bars->s_full[b], (n >> 1) & 1, abort_flag)) {
+                    !tc::mbar_wait(&bars->s_sent[b], (n >> 1) & 1, abort_flag)) {
                     stop = true;
                     break;
                 }
@@ -492,44 +447,19 @@ sparse_mla_tc_kernel(SeqView v,
                 float s[32];
                 tc::tmem_ld32(tmem_base + lane_off + kTmemS + b * kBN + col, s);
                 tc::tmem_ld_wait();
-                tc::tc_fence_before();
-                __syncwarp();
-                if (lane == 0) tc::mbar_arrive(&bars->s_free[b]);    // own partial S loaded
-                // own partial rounded exactly as the senders round it for the peer
-                {
-                    uint32_t w[16];
-                    const float f = pow2i(pack_exchange(s, w));
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        const float2 x = unpack_half2(w[i]);
-                        s[2 * i] = x.x * f;
-                        s[2 * i + 1] = x.y * f;
-                    }
-                }
                 if (!tc::mbar_wait_cluster(&bars->recv_full[b], (n >> 1) & 1, abort_flag)) {
                     stop = true;
                     break;
                 }
-                {
-                    const uint4* other = reinterpret_cast<const uint4*>(recv_h + b * kRecvHBytes) + h;
-                    const float f = pow2i((int)((recv_e[b * kH + h] >> (8 * half)) & 0xFFu));
-                    uint4 o4[4];
+                const float4* other = reinterpret_cast<const float4*>(recv + b * kRecvBytes) + h;
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) o4[i] = other[(4 * half + i) * kH];
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const uint32_t wv[4] = {o4[i].x, o4[i].y, o4[i].z, o4[i].w};
-#pragma unroll
-                        for (int qq = 0; qq < 4; ++qq) {
-                            const float2 x = unpack_half2(wv[qq]);
-                            s[8 * i + 2 * qq] += x.x * f;
-                            s[8 * i + 2 * qq + 1] += x.y * f;
-                        }
-                    }
+                for (int i = 0; i < 8; ++i) {
+                    const float4 o = other[(8 * half + i) * kH];
+                    s[4 * i] += o.x;
+                    s[4 * i + 1] += o.y;
+                    s[4 * i + 2] += o.z;
+                    s[4 * i + 3] += o.w;
                 }
-                // the peer may refill this exchange buffer (the values are in registers)
-                __syncwarp();
-                if (lane == 0) tc::mbar_arrive_remote(peer_recv_free[b]);
                 if (__any_sync(0xffffffffu, valid != 0xffffffffu)) {
 #pragma unroll
                     for (int i = 0; i < 32; ++i)
@@ -545,12 +475,6 @@ sparse_mla_tc_kernel(SeqView v,
                     break;
                 }
                 mt = fmaxf(mt, xmax[(n & 1) * 256 + (half ^ 1) * 128 + h]);
-                // P buffer b is free once P.V of tile n-2 has completed; that also makes the
-                // pv_done parity below unambiguous (P.V(n-2) done, P.V(n) not yet issued)
-                if (n >= 2 && !tc::mbar_wait(&bars->p_free[b], ((n - 2) >> 1) & 1, abort_flag)) {
-                    stop = true;
-                    break;
-                }
                 // lazy rescale: a head whose running max grew by more than 2^8 rescales O and l
                 // to the new max (both threads of the head take the same decision; the TMEM
                 // accesses are warp-wide)
@@ -579,7 +503,6 @@ sparse_mla_tc_kernel(SeqView v,
                         tc::tmem_st32(tmem_base + lane_off + kTmemO + c, o);
                     }
                     tc::tmem_st_wait();
-                    tc::tc_fence_before();
                 }
                 // p = 2^(s * scale_log2 - m): one FFMA per element (masked entries are -inf -> 0);
                 // a head with nothing valid so far (m = -inf) contributes zeros
@@ -596,18 +519,14 @@ sparse_mla_tc_kernel(SeqView v,
                     pk[i / 2] = *reinterpret_cast<const uint32_t*>(&b2);
                 }
                 l += (ps[0] + ps[1]) + (ps[2] + ps[3]);
-                // P (bf16) of this thread's 32 columns into P buffer b: row h, 16-byte chunks
-                // 4*half..4*half+3, 128-byte swizzle (chunk c at c ^ (h & 7))
-                {
-                    uint8_t* prow = pbuf + b * kPBytes + h * 128;
-#pragma unroll
-                    for (int i = 0; i < 4; ++i)
-                        *reinterpret_cast<uint4*>(prow + ((((4 * half + i) ^ (h & 7))) * 16)) =
-                            make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
-                }
-                tc::fence_async_smem();
+                // P over this thread's 32 columns of the S buffer: rows 32*half.. -> 16 columns of
+                // bf16 pairs (the senders have read partial S, and the other half of the head read
+                // its columns before the maxima were exchanged)
+                tc::tmem_st16_u(tmem_base + lane_off + kTmemS + b * kBN + 16 * half, pk);
+                tc::tmem_st_wait();
+                tc::tc_fence_before();
                 __syncwarp();
-                if (lane == 0) tc::mbar_arrive(&bars->p_full[b]);
+                if (lane == 0) tc::mbar_arrive(&bars->p_full);
                 // ---- last tile of the row: put the next row's Q in place
                 if (j + 1 == ntiles) {
                     t_next = next_row(t + n_clusters, ntiles_next, r_next);
@@ -662,10 +581,9 @@ sparse_mla_tc_kernel(SeqView v,
         // hop never waits behind a softmax.
         const int h = (warp & 3) * 32 + lane;
         const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
-        uint32_t peer_h[2], peer_e[2], peer_bar[2];
+        uint32_t peer_recv[2], peer_bar[2];
         for (int b = 0; b < 2; ++b) {
-            peer_h[b] = tc::mapa_shared(tc::smem_u32(recv_h + b * kRecvHBytes), peer);
-            peer_e[b] = tc::mapa_shared(tc::smem_u32(recv_e + b * kH), peer);
+            peer_recv[b] = tc::mapa_shared(tc::smem_u32(recv + b * kRecvBytes), peer);
             peer_bar[b] = tc::mapa_shared(tc::smem_u32(&bars->recv_full[b]), peer);
         }
         uint32_t m = 0;
@@ -686,28 +604,32 @@ sparse_mla_tc_kernel(SeqView v,
                 tc::tmem_ld_wait();
                 tc::tc_fence_before();
                 __syncwarp();
-                if (lane == 0) tc::mbar_arrive(&bars->s_free[b]);
-                uint32_t hw[32];
-                const int e0 = pack_exchange(sv, hw);
-                const int e1 = pack_exchange(sv + 32, hw + 16);
-                // the peer's softmax has read its exchange buffer b (tile m - 2).  One barrier
-                // per buffer: the peer cannot read tile m before it is sent, so the barrier is
-                // never two phases ahead of this wait.
-                if (m >= 2 && !tc::mbar_wait(&bars->recv_free[b], ((m - 2) >> 1) & 1, abort_flag)) {
+                if (lane == 0) tc::mbar_arrive(&bars->s_sent[b]);
+                // the peer's P.V(m-2) has released its buffer b.  One barrier per buffer: the
+                // peer cannot complete P.V(m) before it receives this tile, so the barrier is
+                // never two phases ahead of this wait (with a single barrier for both buffers it
+                // could be, since the peer may finish P.V(m-1) first, and a parity wait would
+                // then alias).
+                if (m >= 2 && !tc::mbar_wait(&bars->peer_free[b], ((m - 2) >> 1) & 1, abort_flag)) {
                     stop = true;
                     break;
                 }
-                // this CTA's own exchange buffer b receives the peer's tile m: expect its bytes
                 if (warp == 13 && lane == 0) tc::mbar_arrive_expect_tx(&bars->recv_full[b], kRecvBytes);
-                // chunk i (columns 8i..8i+7) of every head lies at [i][head]: each warp instruction
-                // writes 512 contiguous bytes
-                const uint32_t dst = peer_h[b] + h * 16;
+                // chunk i (columns 4i..4i+3) of every head lies at [i][head]: each warp instruction
+                // writes 512 contiguous bytes, which the cluster network moves about twice as fast
+                // as one row per thread
+                const uint32_t dst = peer_recv[b] + h * 16;
 #pragma unroll
-                for (int i = 0; i < kBN / 8; ++i)
-                    tc::st_async_v4(dst + i * (kH * 16), peer_bar[b], hw[4 * i], hw[4 * i + 1],
-                                    hw[4 * i + 2], hw[4 * i + 3]);
-                tc::st_async_b32(peer_e[b] + h * 4, peer_bar[b], (uint32_t)e0 | ((uint32_t)e1 << 8));
+                for (int i = 0; i < kBN / 4; ++i)
+                    tc::st_async_v4(dst + i * (kH * 16), peer_bar[b], __float_as_uint(sv[4 * i]),
+                                    __float_as_uint(sv[4 * i + 1]), __float_as_uint(sv[4 * i + 2]),
+                                    __float_as_uint(sv[4 * i + 3]));
             }
+        }
+        // the peer's last two P.V commits arrive here; take them before leaving
+        if (!stop) {
+            if (m >= 2) tc::mbar_wait(&bars->peer_free[(m - 2) & 1], ((m - 2) >> 1) & 1, abort_flag);
+            if (m >= 1) tc::mbar_wait(&bars->peer_free[(m - 1) & 1], ((m - 1) >> 1) & 1, abort_flag);
         }
     }
     __syncwarp();

@@ -62,6 +62,19 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     return ok != 0;
 }
 
+// Non-blocking test of the same condition (mbarrier.test_wait never suspends the thread, unlike
+// try_wait): for a thread that polls several barriers in turn.
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+        " selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
 // Wait for the phase with the given parity to complete.  Gives up after `limit_ns` of wall time
 // (a pipeline partner that never arrives): sets *abort and returns false so that every role
 // can leave its loop and the CTA can release its TMEM and exit.
@@ -175,6 +188,13 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, int a_mn, in
            | ((uint32_t)(M >> 4) << 24); // M / 16
 }
 
+// Instruction descriptor for kind::f16 with f16 A and B (both K-major), fp32 D, M x N tile.
+__host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N) {
+    return (1u << 4)                     // D format: f32
+           | ((uint32_t)(N >> 3) << 17)  // N / 8 (A and B format 0: f16)
+           | ((uint32_t)(M >> 4) << 24); // M / 16
+}
+
 // Shared memory matrix descriptor, 128-byte swizzle.  `lbo` / `sbo` in bytes: for a K-major
 // operand sbo is the distance between groups of 8 rows (1024 for densely packed 128-byte rows)
 // and lbo is unused; for an MN-major operand lbo is the distance between 64-element column
@@ -272,11 +292,12 @@ __device__ __forceinline__ void st_async_b32(uint32_t remote_addr, uint32_t remo
         : "memory");
 }
 
-// Arrive (release, cluster scope) on an mbarrier in another CTA of the cluster (a shared::cluster
-// address from mapa_shared): this thread's earlier shared-memory reads and writes are ordered
-// before the arrival.
-__device__ __forceinline__ void mbar_arrive_remote(uint32_t remote_bar) {
-    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(remote_bar)
+// Arrive on an mbarrier in another CTA of the cluster (a shared::cluster address from
+// mapa_shared) with relaxed ordering: no fence, so the arrival does not wait for this thread's
+// (or its SM's) outstanding memory operations.  Use it only to signal that loads whose values
+// this thread has already consumed are complete.
+__device__ __forceinline__ void mbar_arrive_remote_relaxed(uint32_t remote_bar) {
+    asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(remote_bar)
                  : "memory");
 }
 
