@@ -66,11 +66,12 @@ def _load():
             paging = [i32, P, P, i64, i32, i32, i32, P, P]
             lib.oracle_index_score.argtypes = paging + [i32, i32, P, P, P, P, i64]
             lib.oracle_topk.argtypes = [i32, P, P, i64, i32, P]
+            lib.oracle_topk_blocks.argtypes = [i32, P, P, i64, i32, i32, P]
             lib.oracle_sparse_mla.argtypes = paging + [i32, i32, i32, P, P, P, i32, f64, P, P]
             lib.oracle_dense_attn.argtypes = paging + [i32, i32, i32, P, P, f64, P, P]
             for f in ("oracle_quantize_rows", "oracle_dequantize_rows", "oracle_mx_quantize_rows",
                       "oracle_mx_dequantize_rows", "oracle_index_score",
-                      "oracle_topk", "oracle_sparse_mla", "oracle_dense_attn"):
+                      "oracle_topk", "oracle_topk_blocks", "oracle_sparse_mla", "oracle_dense_attn"):
                 getattr(lib, f).restype = ctypes.c_int
             lib.oracle_num_threads.restype = ctypes.c_int
             _lib = lib
@@ -218,6 +219,19 @@ def topk(scores, n_valid, K: int) -> np.ndarray:
     T_q, ld = sc.shape
     idx = np.zeros((T_q, K), dtype=np.int32)
     _check(_load().oracle_topk(T_q, _ptr(nv), _ptr(sc), ld, K, _ptr(idx)), "topk")
+    return idx
+
+
+def topk_blocks(scores, n_valid, K: int, block: int) -> np.ndarray:
+    """[T_q, K] int32: block-aligned selection (the K / block blocks of `block` positions with the
+    highest block maximum, ties to the lower block; all their causal positions), ascending, -1
+    padded; rows with n <= K select all."""
+    sc = _f64(scores)
+    nv = _i32(n_valid)
+    T_q, ld = sc.shape
+    idx = np.zeros((T_q, K), dtype=np.int32)
+    _check(_load().oracle_topk_blocks(T_q, _ptr(nv), _ptr(sc), ld, K, block, _ptr(idx)),
+           "topk_blocks")
     return idx
 
 

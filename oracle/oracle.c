@@ -322,6 +322,70 @@ int oracle_topk(int32_t T_q, const int32_t* n_valid, const double* scores, int64
     return ORACLE_OK;
 }
 
+/* Block-aligned selection, [P3] 3.1 (the selection is aligned to cache blocks so that the sparse
+ * attention that follows reads the cache in contiguous blocks).  The page does not spell out the
+ * rule; the reading taken: row t's causal positions [0, n_t) fall into blocks of `block`
+ * consecutive positions (the last one possibly partial); a block scores the maximum of its
+ * positions' scores; rows with n_t <= K select every position as in oracle_topk; otherwise the
+ * K / block blocks first in the order (block score descending, block index ascending) are
+ * selected and every causal position of a selected block is kept.  Output: the kept positions
+ * ascending, then -1 padding to K (a partial block can leave fewer than K).  block must divide K.
+ * Algorithm: block maxima, then the same full-sort threshold rule as oracle_topk applied to the
+ * blocks. */
+int oracle_topk_blocks(int32_t T_q, const int32_t* n_valid, const double* scores, int64_t ld,
+                       int32_t K, int32_t block, int32_t* idx) {
+    if (K <= 0 || block <= 0 || K % block != 0) return ORACLE_BAD_ARG;
+    for (int32_t t = 0; t < T_q; ++t) {
+        if (n_valid[t] < 0 || n_valid[t] > ld) return ORACLE_BAD_ARG;
+        for (int64_t s = 0; s < n_valid[t]; ++s)
+            if (!isfinite(scores[(int64_t)t * ld + s])) return ORACLE_NOT_FINITE;
+    }
+    const int32_t kb = K / block;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int32_t t = 0; t < T_q; ++t) {
+        const double* row = scores + (int64_t)t * ld;
+        int32_t* out = idx + (int64_t)t * K;
+        const int64_t n = n_valid[t];
+        if (n <= K) {
+            for (int64_t i = 0; i < K; ++i) out[i] = i < n ? (int32_t)i : -1;
+            continue;
+        }
+        const int64_t nb = (n + block - 1) / block;
+        double* bmax = (double*)malloc(sizeof(double) * (size_t)nb);
+        double* tmp = (double*)malloc(sizeof(double) * (size_t)nb);
+        char* keep = (char*)calloc((size_t)nb, 1);
+        for (int64_t b = 0; b < nb; ++b) {
+            double m = -INFINITY;
+            for (int64_t s = b * block; s < (b + 1) * block && s < n; ++s)
+                if (row[s] > m) m = row[s];
+            bmax[b] = m;
+        }
+        memcpy(tmp, bmax, sizeof(double) * (size_t)nb);
+        qsort(tmp, (size_t)nb, sizeof(double), cmp_desc);
+        const double v = tmp[kb - 1];
+        int64_t greater = 0;
+        for (int64_t b = 0; b < nb; ++b) greater += bmax[b] > v;
+        int64_t ties_wanted = kb - greater;
+        for (int64_t b = 0; b < nb; ++b) {
+            if (bmax[b] > v) {
+                keep[b] = 1;
+            } else if (bmax[b] == v && ties_wanted > 0) {
+                keep[b] = 1;
+                --ties_wanted;
+            }
+        }
+        int64_t taken = 0;
+        for (int64_t b = 0; b < nb; ++b)
+            if (keep[b])
+                for (int64_t s = b * block; s < (b + 1) * block && s < n; ++s) out[taken++] = (int32_t)s;
+        for (; taken < K; ++taken) out[taken] = -1;
+        free(bmax);
+        free(tmp);
+        free(keep);
+    }
+    return ORACLE_OK;
+}
+
 /* Sparse MLA attention over the selected latent rows, [P1] "Sparse Attention Pipeline
  * Optimization" ("reads only the selected entries ... block-wise fused attention"),
  * [P3] 3.2, [P5] s3 (SFA).  Each cache row holds the compressed latent c_kv (D_v values)

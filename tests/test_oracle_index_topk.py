@@ -161,3 +161,82 @@ def test_topk_constructed_rows():
 def test_topk_rejects_non_finite():
     with pytest.raises(oracle.OracleError):
         oracle.topk(np.array([[1.0, np.nan, 2.0]]), [3], 1)
+
+
+# ----------------------------------------------------------------- block-aligned selection
+def _blocks_brute(row, n, K, B):
+    """Independent restatement: block maxima over the causal prefix, blocks ordered by (max
+    descending, block ascending) with numpy's lexsort, the first K / B blocks kept whole."""
+    if n <= K:
+        return [i for i in range(n)] + [-1] * (K - n)
+    nb = -(-n // B)
+    bmax = np.full(nb, -np.inf)
+    for b in range(nb):
+        bmax[b] = np.max(row[b * B:min(n, (b + 1) * B)])
+    order = np.lexsort((np.arange(nb), -bmax))[:K // B]
+    keep = sorted(order.tolist())
+    out = [s for b in keep for s in range(b * B, min(n, (b + 1) * B))]
+    return out + [-1] * (K - len(out))
+
+
+@pytest.mark.parametrize("B", [1, 4, 16, 64])
+def test_topk_blocks_matches_brute_force(B):
+    rng = np.random.default_rng(31 + B)
+    K = 64
+    T, ld = 40, 700
+    sc = rng.integers(-6, 7, size=(T, ld)).astype(np.float64)      # heavy ties
+    sc[::3] = rng.standard_normal((len(sc[::3]), ld))
+    n_valid = rng.integers(1, ld + 1, size=T).astype(np.int32)
+    n_valid[:3] = [K, K + 1, 1]
+    got = oracle.topk_blocks(sc, n_valid, K, B)
+    for t in range(T):
+        assert got[t].tolist() == _blocks_brute(sc[t], int(n_valid[t]), K, B), (t, B)
+
+
+def test_topk_blocks_with_unit_blocks_is_topk():
+    rng = np.random.default_rng(5)
+    sc = rng.integers(-3, 4, size=(25, 300)).astype(np.float64)
+    n_valid = rng.integers(1, 301, size=25).astype(np.int32)
+    assert np.array_equal(oracle.topk_blocks(sc, n_valid, 32, 1), oracle.topk(sc, n_valid, 32))
+
+
+def test_topk_blocks_constructed_row():
+    """Block 3 holds one very high score among low ones: it is kept whole, and the block of the
+    next-highest maxima follow; a position Top-K would instead take scattered positions."""
+    B, K = 8, 16
+    row = np.zeros(100)
+    row[:] = -np.arange(100) / 1000.0          # decreasing: block 0 has the best maximum
+    row[27] = 50.0                              # block 3 (positions 24..31)
+    got = oracle.topk_blocks(row[None], np.array([100], np.int32), K, B)[0].tolist()
+    assert got == list(range(0, 8)) + list(range(24, 32))
+    # a partial last block counts with its causal positions only
+    row2 = np.zeros(20)
+    row2[17] = 9.0                              # block 2 = positions 16..19 (n = 20)
+    got2 = oracle.topk_blocks(row2[None], np.array([20], np.int32), 8, 4)[0].tolist()
+    assert got2 == [0, 1, 2, 3, 16, 17, 18, 19]
+
+
+def test_topk_blocks_invariants():
+    rng = np.random.default_rng(9)
+    B, K = 16, 128
+    sc = rng.standard_normal((30, 2000))
+    n_valid = rng.integers(129, 2001, size=30).astype(np.int32)
+    got = oracle.topk_blocks(sc, n_valid, K, B)
+    for t in range(30):
+        n = int(n_valid[t])
+        sel = got[t][got[t] >= 0]
+        assert np.all(np.diff(sel) > 0)                          # ascending, distinct
+        blocks = sorted(set((sel // B).tolist()))
+        assert len(blocks) == K // B
+        for b in blocks:                                          # whole causal blocks
+            assert set(range(b * B, min(n, (b + 1) * B))) <= set(sel.tolist())
+        bmax = np.array([sc[t, b * B:min(n, (b + 1) * B)].max() for b in range(-(-n // B))])
+        kept = np.array(blocks)
+        dropped = np.setdiff1d(np.arange(len(bmax)), kept)
+        if len(dropped):
+            assert bmax[kept].min() >= bmax[dropped].max()       # no dropped block beats a kept one
+
+
+def test_topk_blocks_rejects_bad_arguments():
+    with pytest.raises(oracle.OracleError):
+        oracle.topk_blocks(np.zeros((1, 10)), np.array([10], np.int32), 12, 8)   # 8 does not divide 12
