@@ -260,7 +260,7 @@ def secondary(dev, flush_l2, main, peaks, reps):
     idx = torch.empty((wl.T_q, wl.K), dtype=torch.int32, device=dev)
     o = torch.empty((wl.T_q, wl.H, wl.D_v), dtype=torch.bfloat16, device=dev)
     lse = torch.empty((wl.T_q, wl.H), dtype=torch.float32, device=dev)
-    ws = torch.empty(max(1, hsa.hsa_fused_decode_workspace_size(seq, wl.q, kv8, wl.D_v, wl.K)),
+    ws = torch.zeros(max(1, hsa.hsa_fused_decode_workspace_size(seq, wl.q, kv8, wl.D_v, wl.K)),
                      dtype=torch.uint8, device=dev)
 
     def fp8_step():
@@ -328,7 +328,7 @@ def secondary(dev, flush_l2, main, peaks, reps):
     idx = torch.empty((wl.T_q, wl.K), dtype=torch.int32, device=dev)
     o = torch.empty((wl.T_q, wl.H, wl.D_v), dtype=torch.bfloat16, device=dev)
     lse = torch.empty((wl.T_q, wl.H), dtype=torch.float32, device=dev)
-    ws = torch.empty(max(1, hsa.hsa_fused_decode_workspace_size(seq, wl.q, wl.kv, wl.D_v, wl.K)),
+    ws = torch.zeros(max(1, hsa.hsa_fused_decode_workspace_size(seq, wl.q, wl.kv, wl.D_v, wl.K)),
                      dtype=torch.uint8, device=dev)
 
     def draft_step():
@@ -454,7 +454,7 @@ def run_ours(args, rank, world, local_rank):
     idx = torch.empty((wl.T_q, wl.K), dtype=torch.int32, device=dev)
     out = torch.empty((wl.T_q, wl.H, wl.D_v), dtype=torch.bfloat16, device=dev)
     lse = torch.empty((wl.T_q, wl.H), dtype=torch.float32, device=dev)
-    ws = torch.empty(max(1, hsa.hsa_fused_decode_workspace_size(seq, wl.q, wl.kv, wl.D_v, wl.K)),
+    ws = torch.zeros(max(1, hsa.hsa_fused_decode_workspace_size(seq, wl.q, wl.kv, wl.D_v, wl.K)),
                      dtype=torch.uint8, device=dev)
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
 

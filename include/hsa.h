@@ -132,6 +132,20 @@ HSA_API hsa_status_t hsa_index_score(const hsa_paged_seq_t* seq, const void* q_I
 HSA_API hsa_status_t hsa_topk(const hsa_paged_seq_t* seq, const float* scores, int64_t ld_scores,
                       int32_t K, int32_t* idx, void* stream);
 
+/* Block-aligned selection (third page, 3.1: the selection is aligned to cache blocks so that
+ * the attention reads the cache in contiguous pieces).  For row t with n = q_pos[t] + 1:
+ *   n <= K : as hsa_topk;
+ *   n >  K : positions fall into blocks [b * block, (b + 1) * block) (the last one cut at n); a
+ *            block scores the largest score of its positions; the K / block blocks first in the
+ *            order (block score descending, block index ascending) are kept, and every position
+ *            of a kept block is written, ascending, then -1 up to K (a kept partial last block
+ *            leaves fewer than K).
+ * block >= 8 and divides K; ceil(max_seq_len / block) may not exceed about 56000.  With block =
+ * page_size each kept block is one whole cache page. */
+HSA_API hsa_status_t hsa_topk_blocks(const hsa_paged_seq_t* seq, const float* scores,
+                             int64_t ld_scores, int32_t K, int32_t block, int32_t* idx,
+                             void* stream);
+
 /* ---- 3. sparse MLA attention -----------------------------------------------------------
  * For row t, head h, over S_t = { idx[t,k] != -1 }:
  *   z_n = softmax_scale * sum_{d<D_qk} q[t,h,d] * key(n, d)
@@ -149,7 +163,13 @@ HSA_API hsa_status_t hsa_topk(const hsa_paged_seq_t* seq, const float* scores, i
  *   idx      device int32 [T_q, K]: positions in [0, q_pos[t]] or -1
  *   out      device [T_q, H, D_v] of out_dtype (F32 or BF16)
  *   lse      device fp32 [T_q, H] or NULL
- *   ws       workspace of at least hsa_sparse_mla_workspace_size() bytes, 256-byte aligned
+ *   ws       workspace of at least hsa_sparse_mla_workspace_size() bytes, 256-byte aligned and
+ *            zero-filled before its first use (with few query rows -- at most 256 -- the
+ *            tensor-core kernel spreads the rows' tiles evenly over all clusters and merges a row
+ *            cut between clusters through this workspace; it keeps one counter per row there,
+ *            which every call returns to zero.  After a call that set HSA_DEV_TIMEOUT, zero it
+ *            again.  A workspace smaller than the size reported, or NULL, makes the kernel take
+ *            whole rows per cluster instead; the results agree within rounding.)
  * Pages: first page "Sparse Attention Pipeline Optimization" (indexed reads, block-wise fused
  * attention); third page 3.2 (partition by query, aggregate over the selected positions,
  * stage them in shared memory); fifth page 3 (SFA).  The tensor-core kernel serves q BF16,
@@ -170,7 +190,10 @@ HSA_API hsa_status_t hsa_sparse_mla_attn(const hsa_paged_seq_t* seq, const void*
  * caller buffers that hold the intermediate results afterwards.  With stream_aux != NULL the
  * rows are split in two halves; the second half runs on stream_aux, overlapping the first
  * half's attention (event-ordered; stream_main waits for stream_aux before returning work to
- * the caller).  Pages: first page "Sparse Attention Pipeline Optimization" (fusing the decode
+ * the caller).  Scores and selections are then bitwise the same; the attention of a row that
+ * the few-rows schedule cuts between clusters may differ in the last bit, since the halves
+ * cut their rows at other places.  ws: zero-filled before first use, as for
+ * hsa_sparse_mla_attn.  Pages: first page "Sparse Attention Pipeline Optimization" (fusing the decode
  * operators and running independent ones concurrently: indexer, then the sparse attention
  * kernel; several streams); fifth page 3.3 (operators on independent streams with event
  * synchronization).  The members of hsa_index_args_t and hsa_attn_args_t have the meaning of

@@ -59,6 +59,7 @@ SYMBOLS = {
     "hsa_index_score": (ctypes.c_int, [_P, _P, ctypes.c_int, _P, _i32, _i32, _P, ctypes.c_int, _P,
                                        _P, _i64, _P]),
     "hsa_topk": (ctypes.c_int, [_P, _P, _i64, _i32, _P, _P]),
+    "hsa_topk_blocks": (ctypes.c_int, [_P, _P, _i64, _i32, _i32, _P, _P]),
     "hsa_sparse_mla_workspace_size": (_sz, [_P, _i32, _i32, _i32, _i32]),
     "hsa_sparse_mla_attn": (ctypes.c_int, [_P, _P, ctypes.c_int, _i32, _i32, _i32, _P, ctypes.c_int,
                                            _P, _i32, _P, _P, _i32, _f32, _P, ctypes.c_int, _P, _P, _sz,
@@ -198,14 +199,27 @@ def hsa_topk(seq: PagedSeq, scores, K: int, idx=None, stream=None):
     return idx
 
 
+def hsa_topk_blocks(seq: PagedSeq, scores, K: int, block: int, idx=None, stream=None):
+    """Block-aligned selection: the K / block blocks of `block` positions with the highest block
+    maximum, all their causal positions ascending, -1 padded (rows with n <= K select all)."""
+    if idx is None:
+        idx = torch.empty((seq.T_q, K), dtype=torch.int32, device=scores.device)
+    _check(lib().hsa_topk_blocks(seq.ref, _ptr(scores), scores.shape[1], K, block, _ptr(idx),
+                                 _stream(stream)),
+           "hsa_topk_blocks")
+    return idx
+
+
 def hsa_sparse_mla_workspace_size(seq: PagedSeq, H: int, D_qk: int, D_v: int, K: int) -> int:
     return int(lib().hsa_sparse_mla_workspace_size(seq.ref, H, D_qk, D_v, K))
 
 
 def _workspace(nbytes: int, device, ws):
+    """Workspace of nbytes (zero-filled: the attention's split schedule keeps row counters there,
+    which must start at zero and which every call leaves at zero)."""
     if ws is not None:
         return ws
-    return torch.empty(max(nbytes, 1), dtype=torch.uint8, device=device)
+    return torch.zeros(max(nbytes, 1), dtype=torch.uint8, device=device)
 
 
 def _kv_group(kv, kv_scale, D_v: int) -> int:

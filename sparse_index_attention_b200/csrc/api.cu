@@ -196,10 +196,10 @@ size_t attn_ws_bytes(const hsa::SparseMlaArgs& a) {
 hsa_status_t run_attn(const hsa::SparseMlaArgs& a, cudaStream_t st) {
     if (a.seq.T_q == 0) return HSA_OK;
     if (hsa::sparse_mla_tc_supported(a)) {
-        const size_t need = hsa::sparse_mla_tc_workspace(a.seq.T_q, a.K);
-        HSA_REQUIRE(a.ws_bytes >= need && (need == 0 || (a.ws && aligned(a.ws, 256))),
-                    HSA_ERR_WORKSPACE, "workspace of %zu bytes needed (256-byte aligned), got %zu",
-                    need, a.ws_bytes);
+        // a workspace smaller than the split schedule needs (or none) selects whole rows per
+        // cluster; a given workspace must be 256-byte aligned
+        HSA_REQUIRE(a.ws == nullptr || a.ws_bytes == 0 || aligned(a.ws, 256), HSA_ERR_WORKSPACE,
+                    "workspace must be 256-byte aligned");
         return cuda_status(hsa::launch_sparse_mla_tc(a, st), "sparse_mla_attn (tensor core)");
     }
     return cuda_status(hsa::launch_sparse_mla_simt(a, st), "sparse_mla_attn");
@@ -343,6 +343,25 @@ hsa_status_t hsa_topk(const hsa_paged_seq_t* seq, const float* scores, int64_t l
                        "topk");
 }
 
+hsa_status_t hsa_topk_blocks(const hsa_paged_seq_t* seq, const float* scores, int64_t ld_scores,
+                             int32_t K, int32_t block, int32_t* idx, void* stream) {
+    g_last_error.clear();
+    hsa_status_t st = check_seq(seq);
+    if (st != HSA_OK) return st;
+    HSA_REQUIRE(K >= 1 && K <= 65536, HSA_ERR_INVALID_ARG, "K = %d out of range", K);
+    HSA_REQUIRE(block >= 8 && block <= K && K % block == 0, HSA_ERR_INVALID_ARG,
+                "block = %d must be >= 8 and divide K = %d", block, K);
+    HSA_REQUIRE(ld_scores >= seq->max_seq_len, HSA_ERR_INVALID_ARG, "ld_scores < max_seq_len");
+    HSA_REQUIRE(hsa::topk_blocks_smem(seq->max_seq_len, K, block) <= 227 * 1024, HSA_ERR_UNSUPPORTED,
+                "max_seq_len / block = %d blocks per row is too many", (int)hsa::ceil_div(seq->max_seq_len, block));
+    if (seq->T_q == 0) return HSA_OK;
+    HSA_REQUIRE(scores && idx && aligned(scores, 4) && aligned(idx, 4), HSA_ERR_INVALID_ARG,
+                "NULL or misaligned scores / idx");
+    return cuda_status(hsa::launch_topk_blocks(view(seq), seq->max_seq_len, scores, ld_scores, K,
+                                               block, idx, (cudaStream_t)stream),
+                       "topk_blocks");
+}
+
 size_t hsa_sparse_mla_workspace_size(const hsa_paged_seq_t* seq, int32_t H, int32_t D_qk,
                                      int32_t D_v, int32_t K) {
     if (seq == nullptr || seq->T_q <= 0) return 0;
@@ -398,9 +417,8 @@ hsa_status_t hsa_fused_decode(const hsa_paged_seq_t* seq, const hsa_index_args_t
     HSA_REQUIRE(K >= 1 && K <= 65536, HSA_ERR_INVALID_ARG, "K = %d out of range", K);
     if (seq->T_q == 0) return HSA_OK;
     HSA_REQUIRE(idx && aligned(idx, 4), HSA_ERR_INVALID_ARG, "idx NULL or misaligned");
-    const size_t need = hsa_fused_decode_workspace_size(seq, at, K);
-    HSA_REQUIRE(ws_bytes >= need && (need == 0 || (ws && aligned(ws, 256))), HSA_ERR_WORKSPACE,
-                "workspace of %zu bytes needed (256-byte aligned), got %zu", need, ws_bytes);
+    HSA_REQUIRE(ws == nullptr || ws_bytes == 0 || aligned(ws, 256), HSA_ERR_WORKSPACE,
+                "workspace must be 256-byte aligned");
 
     cudaStream_t s0 = (cudaStream_t)stream_main, s1 = (cudaStream_t)stream_aux;
     // split point: half the rows, on a run boundary so no run is cut
@@ -445,10 +463,13 @@ hsa_status_t hsa_fused_decode(const hsa_paged_seq_t* seq, const hsa_index_args_t
     hsa_paged_seq_t first = sub_rows(*seq, 0, t1);
     size_t ws0 = attn_ws_bytes(attn_args(&first, *at, nullptr, K, nullptr, 0));
     ws0 = (ws0 + 255) / 256 * 256;
-    if (r == HSA_OK) r = one_part(0, t1, ws, ws0, s0, ev_topk);
+    // each half takes its own region; a workspace too small for a half runs it with whole rows
+    const bool ws_a = ws != nullptr && ws_bytes >= ws0;
+    if (r == HSA_OK) r = one_part(0, t1, ws_a ? ws : nullptr, ws_a ? ws0 : 0, s0, ev_topk);
     if (r == HSA_OK) r = cuda_status(cudaStreamWaitEvent(s1, ev_topk, 0), "cudaStreamWaitEvent");
     if (r == HSA_OK)
-        r = one_part(t1, seq->T_q - t1, static_cast<char*>(ws) + ws0, ws_bytes - ws0, s1, nullptr);
+        r = one_part(t1, seq->T_q - t1, ws_a ? static_cast<char*>(ws) + ws0 : nullptr,
+                     ws_a ? ws_bytes - ws0 : 0, s1, nullptr);
     if (r == HSA_OK) r = cuda_status(cudaEventRecord(ev_done, s1), "cudaEventRecord");
     if (r == HSA_OK) r = cuda_status(cudaStreamWaitEvent(s0, ev_done, 0), "cudaStreamWaitEvent");
     if (ev_topk) cudaEventDestroy(ev_topk);

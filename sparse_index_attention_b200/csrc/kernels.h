@@ -32,6 +32,12 @@ cudaError_t launch_index_score_tc(const IndexScoreArgs& a, cudaStream_t st);
 cudaError_t launch_topk(const SeqView& seq, int32_t max_seq_len, const float* scores, int64_t ld,
                         int32_t K, int32_t* idx, cudaStream_t st);
 
+// Block-aligned selection: the K / block blocks of `block` positions with the highest block
+// maximum, all their causal positions ascending (block >= 8, block | K).
+cudaError_t launch_topk_blocks(const SeqView& seq, int32_t max_seq_len, const float* scores,
+                               int64_t ld, int32_t K, int32_t block, int32_t* idx, cudaStream_t st);
+size_t topk_blocks_smem(int32_t max_seq_len, int32_t K, int32_t block);
+
 // ---- sparse MLA -------------------------------------------------------------------------------
 struct SparseMlaArgs {
     SeqView seq;

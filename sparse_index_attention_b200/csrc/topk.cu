@@ -313,7 +313,75 @@ cudaError_t launch_variant(const SeqView& seq, const float* scores, int64_t ld, 
     return e != cudaSuccess ? e : cudaGetLastError();
 }
 
+// Block-aligned selection ("Day-One Inference Adaptation for Very Large Hybrid-Attention
+// Models", 3.1: the selection is aligned to cache blocks so that the attention reads the cache in
+// contiguous pieces).  A row with n > K causal positions keeps the K / block blocks of `block`
+// positions with the highest block maximum (ties to the lower block; the last block may be
+// partial) and every causal position of each kept block, in ascending order.  One CTA per row:
+// the block maxima become keys in shared memory, the radix select above picks the blocks
+// exactly, write_selection lists them in block order, and the threads expand them to positions.
+__global__ void __launch_bounds__(kThreads, 1)
+topk_blocks_kernel(SeqView v, const float* __restrict__ scores, int64_t ld, int K, int block,
+                   int32_t* __restrict__ idx) {
+    extern __shared__ __align__(16) uint32_t sm[];
+    uint32_t* hist = sm;                                          // [kBins]
+    uint64_t* wsum = reinterpret_cast<uint64_t*>(sm + kBins);     // [kWarps]
+    uint32_t* misc = sm + kBins + 2 * kWarps;                     // [16]
+    int32_t* chosen = reinterpret_cast<int32_t*>(misc + 16);      // [K / block] kept blocks
+    uint32_t* bkey = misc + 16 + K / block;                       // [blocks of the row]
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int t = blockIdx.x;
+    pdl_wait();
+    pdl_trigger();
+    const RowInfo r = load_row(v, t);
+    int32_t* out = idx + (int64_t)t * K;
+    const int n = r.pos + 1;
+    if (n <= K) {
+        for (int i = tid; i < K; i += kThreads) out[i] = i < n ? i : -1;
+        return;
+    }
+    const float* src = scores + (int64_t)t * ld;
+    const int nb = (n + block - 1) / block, kb = K / block;
+    for (int b = warp; b < nb; b += kWarps) {
+        float m = -INFINITY;
+        const int s1 = min(n, (b + 1) * block);
+        for (int s = b * block + lane; s < s1; s += 32) m = fmaxf(m, __ldg(src + s));
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        if (lane == 0) bkey[b] = score_key(m);
+    }
+    for (int b = tid; b < kBins; b += kThreads) hist[b] = 0u;
+    __syncthreads();
+    auto get = [&](int i) { return bkey[i]; };
+    const Kth kth = radix_select<3>(get, nb, (uint32_t)kb, hist, wsum, misc);
+    write_selection(get, [](int i) { return (int32_t)i; }, nb, kth.key, kth.krem, kb, chosen, wsum);
+    __syncthreads();
+    // kept block j (ascending) fills slots [j * block, (j + 1) * block); only the last block of
+    // the row can be partial, and it is the last kept one if kept, so its missing positions are
+    // the -1 padding at the end
+    for (int i = tid; i < K; i += kThreads) {
+        const int s = chosen[i / block] * block + i % block;
+        out[i] = s < n ? s : -1;
+    }
+}
+
 }  // namespace
+
+cudaError_t launch_topk_blocks(const SeqView& seq, int32_t max_seq_len, const float* scores,
+                               int64_t ld, int32_t K, int32_t block, int32_t* idx, cudaStream_t st) {
+    if (seq.T_q == 0) return cudaSuccess;
+    const size_t smem = sizeof(uint32_t) * ((size_t)kFixedWords + (size_t)(K / block) +
+                                            (size_t)ceil_div(max_seq_len, block));
+    auto k = topk_blocks_kernel;
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    e = launch_pdl(k, dim3(seq.T_q), dim3(kThreads), smem, st, seq, scores, ld, (int)K, (int)block, idx);
+    return e != cudaSuccess ? e : cudaGetLastError();
+}
+
+size_t topk_blocks_smem(int32_t max_seq_len, int32_t K, int32_t block) {
+    return sizeof(uint32_t) * ((size_t)kFixedWords + (size_t)(K / block) + (size_t)ceil_div(max_seq_len, block));
+}
 
 cudaError_t launch_topk(const SeqView& seq, int32_t max_seq_len, const float* scores, int64_t ld,
                         int32_t K, int32_t* idx, cudaStream_t st) {

@@ -20,7 +20,7 @@ def test_header_declares_the_path():
     names = _declared()
     for n in ("hsa_index_score", "hsa_topk", "hsa_sparse_mla_attn", "hsa_fused_decode",
               "hsa_quantize_index", "hsa_quantize_kv", "hsa_quantize_mx", "hsa_dequantize_mx",
-              "hsa_mx_round", "hsa_decode_prolog"):
+              "hsa_mx_round", "hsa_decode_prolog", "hsa_topk_blocks"):
         assert n in names
 
 
@@ -111,6 +111,11 @@ def test_validation_without_gpu():
     pa.slot_mapping = odd
     assert L.hsa_decode_prolog(ctypes.byref(pa), None, None, None, None) == hsa.HSA_ERR_INVALID_ARG
     assert L.hsa_decode_prolog(None, None, None, None, None) == hsa.HSA_ERR_INVALID_ARG
+    # block-aligned selection: block >= 8 dividing K
+    for blk in (4, 48, 0):
+        rc = L.hsa_topk_blocks(ctypes.byref(seq), fake, 64, 64, blk, fake, None)
+        assert rc == hsa.HSA_ERR_INVALID_ARG, blk
+    assert L.hsa_topk_blocks(ctypes.byref(seq), fake, 32, 64, 16, fake, None) == hsa.HSA_ERR_INVALID_ARG
     # zero rows is a no-op, not an error
     empty = hsa.hsa_paged_seq_t(1, fake, fake, 4, 16, 4, 64, 0, None, None, 1, None)
     assert L.hsa_topk(ctypes.byref(empty), None, 64, 8, None, None) == hsa.HSA_OK

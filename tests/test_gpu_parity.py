@@ -292,6 +292,68 @@ def test_sparse_mla_vs_oracle(name, kw, tol):
     _attn_vs_oracle(workloads.make(name, DEV, **kw), tol)
 
 
+@pytest.mark.parametrize("name,kw,block", [
+    ("decode_bf16", dict(B=6, L_min=1500, L_max=9000), 64),
+    ("prefill_bf16", dict(T=2400), 64),
+    ("decode_bf16", dict(B=4, L_min=3000, L_max=5000), 16),
+])
+def test_topk_blocks_bit_exact_and_attention(name, kw, block):
+    """Block-aligned selection on the GPU's own fp32 scores equals the oracle's rule bit for bit
+    (rows shorter than K, partial last blocks, ties of block maxima included), keeps whole
+    cache pages when block = page size, and the attention over it matches the oracle's."""
+    wl = workloads.make(name, DEV, **kw)
+    seq = paged_seq(wl)
+    sc = hsa.hsa_index_score(seq, wl.q_I, wl.w, wl.k_I)
+    sc_t = sc.clone()
+    if wl.T_q > 3:                                  # ties between block maxima on row 2
+        n2 = int(wl.q_pos[2]) + 1
+        sc_t[2, :n2] = torch.floor(sc_t[2, :n2] * 2) / 2
+    idx = hsa.hsa_topk_blocks(seq, sc_t, wl.K, block)
+    check_status(seq)
+    n_valid = (wl.q_pos + 1).cpu().numpy().astype(np.int32)
+    ref = oracle.topk_blocks(sc_t.cpu(), n_valid, wl.K, block)
+    assert np.array_equal(idx.cpu().numpy(), ref)
+    if block == wl.page_size:                       # whole pages
+        g = idx.cpu().numpy()
+        for t in range(wl.T_q):
+            sel = g[t][g[t] >= 0]
+            if int(n_valid[t]) > wl.K:
+                assert len(set((sel // block).tolist())) == wl.K // block
+    _attn_vs_oracle(wl, 2e-2, idx.cpu())
+
+
+@pytest.mark.parametrize("B", [3, 64])
+def test_sparse_mla_rows_split_between_clusters(B):
+    """With few query rows the tensor-core kernel lays the rows' tiles end to end and gives each
+    cluster an equal run of them, so rows are cut between clusters and finished by log-sum-exp
+    (3 rows: each cut into many parts; 64 rows: the decode batch's shape).  A short row and an
+    empty row ride along.  Checked against the oracle, against the same call with whole rows per
+    cluster (no workspace), within rounding, and the workspace's row counters are back to 0."""
+    wl = workloads.make("decode_bf16", DEV, B=B, L_min=2100, L_max=6000)
+    idx = workloads.random_selection(wl.q_pos, wl.K, seed=11)
+    idx[1, 700:] = -1                     # 11 of 32 tiles
+    idx[2] = -1                           # nothing selected
+    out, lse = _attn_vs_oracle(wl, 2e-2, idx)
+    assert torch.all(out[2] == 0) and torch.all(torch.isneginf(lse[2]))
+    seq = paged_seq(wl)
+    need = hsa.hsa_sparse_mla_workspace_size(seq, wl.H, wl.D_qk, wl.D_v, wl.K)
+    assert need > 0
+    ws = torch.zeros(need, dtype=torch.uint8, device=DEV)
+    out_s, lse_s = hsa.hsa_sparse_mla_attn(seq, wl.q, wl.kv, idx.to(DEV), wl.D_v, wl.softmax_scale, ws=ws)
+    out_w, lse_w = hsa.hsa_sparse_mla_attn(seq, wl.q, wl.kv, idx.to(DEV), wl.D_v, wl.softmax_scale,
+                                           ws=torch.zeros(1, dtype=torch.uint8, device=DEV))
+    check_status(seq)
+    assert torch.equal(out_s, out)                       # same schedule, same bits
+    assert torch.allclose(out_s.float(), out_w.float(), atol=5e-3, rtol=5e-3)
+    fin = torch.isfinite(lse_w)
+    assert torch.equal(fin, torch.isfinite(lse_s))
+    assert torch.allclose(lse_s[fin], lse_w[fin], atol=1e-4, rtol=1e-4)
+    assert int(ws[:wl.T_q * 8].count_nonzero()) == 0     # counters returned to zero
+    # a second call on the same workspace gives the same bits
+    out_2, lse_2 = hsa.hsa_sparse_mla_attn(seq, wl.q, wl.kv, idx.to(DEV), wl.D_v, wl.softmax_scale, ws=ws)
+    assert torch.equal(out_2, out_s) and torch.equal(lse_2, lse_s)
+
+
 @pytest.mark.parametrize("kv_group", [512, 128, 64])
 @pytest.mark.parametrize("H", [128, 16])
 def test_sparse_mla_fp8_scale_groups(kv_group, H):

@@ -9,7 +9,8 @@ Checks per the path's contract:
   (iii) index scores within 1e-3 (|I_ref| + M); attention outputs within 2e-2 abs/rel (bf16),
         6e-2 (FP8 caches), 1e-4 (fp32) of the oracle's attention over the GPU's own selection
         (the end-to-end difference, over the oracle's own selection, is printed);
-  (iv)  fused == unfused and two-stream == one-stream, bitwise.
+  (iv)  fused == unfused bitwise; two-stream == one-stream bitwise for scores and selections,
+        and within rounding for attention (the halves cut rows between clusters elsewhere).
 """
 import numpy as np
 import pytest
@@ -101,8 +102,14 @@ def test_fused_equals_unfused_and_two_streams(name, kw, kv_group):
         n = int(wl.q_pos[t]) + 1
         assert torch.equal(sc1[t, :n], sc2[t, :n]) and torch.equal(sc1[t, :n], sc3[t, :n])
     assert torch.equal(idx1, idx2) and torch.equal(idx1, idx3)
-    assert torch.equal(out1, out2) and torch.equal(out1, out3)
-    assert torch.equal(lse1, lse2) and torch.equal(lse1, lse3)
+    assert torch.equal(out1, out3) and torch.equal(lse1, lse3)
+    # the two-stream form runs each half of the rows as its own launch, so the few-rows schedule
+    # cuts rows between clusters at other places: equal up to the rounding of the merge
+    tol = TOL[wl.dtype] if not (wl.kv_fp8 or wl.index_fp8) else 6e-2
+    assert torch.allclose(out1.float(), out2.float(), atol=tol / 4, rtol=tol / 4)
+    fin = torch.isfinite(lse1)
+    assert torch.equal(fin, torch.isfinite(lse2))
+    assert torch.allclose(lse1[fin], lse2[fin], atol=1e-4, rtol=1e-4)
 
 
 def test_decode_bf16_full_size_sampled():
