@@ -240,6 +240,58 @@ def _timed(fn, reps, flush_l2, main):
     return statistics.median(ts)
 
 
+def stage_times(calls, names, reps, flush_l2, main):
+    """Mean CUDA-event time (ms) of each call, the calls issued in turn on `main` with events
+    between them, L2 flushed before each round."""
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(calls) + 1)] for _ in range(reps)]
+    for i in range(reps):
+        flush_l2()
+        ev[i][0].record(main)
+        for j, c in enumerate(calls):
+            c()
+            ev[i][j + 1].record(main)
+    torch.cuda.synchronize()
+    return {n: {"ms": round(statistics.mean(e[j].elapsed_time(e[j + 1]) for e in ev), 4)}
+            for j, n in enumerate(names)}
+
+
+def block_aligned(dev, flush_l2, main, peaks, reps):
+    """Block-aligned selection on the bf16 decode batch (blocks of one cache page, 64 positions):
+    the selection kernel, and the attention over whole-page selections beside the attention over
+    the position selection of the same scores (both gather 2048 rows per query row)."""
+    import sparse_index_attention_b200 as hsa
+    wl = workloads.make(WORKLOAD, dev)
+    seq = hsa.PagedSeq(wl.seq_lens, wl.block_table, wl.page_size, wl.num_pages, wl.q_seq, wl.q_pos,
+                       q_run=wl.q_run)
+    sc = hsa.hsa_index_score(seq, wl.q_I, wl.w, wl.k_I)
+    idx_p = hsa.hsa_topk(seq, sc, wl.K)
+    idx_b = hsa.hsa_topk_blocks(seq, sc, wl.K, wl.page_size)
+    o = torch.empty((wl.T_q, wl.H, wl.D_v), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((wl.T_q, wl.H), dtype=torch.float32, device=dev)
+    ws = torch.zeros(max(1, hsa.hsa_sparse_mla_workspace_size(seq, wl.H, wl.D_qk, wl.D_v, wl.K)),
+                     dtype=torch.uint8, device=dev)
+    for _ in range(3):
+        hsa.hsa_sparse_mla_attn(seq, wl.q, wl.kv, idx_b, wl.D_v, wl.softmax_scale, out=o, lse=lse, ws=ws, stream=main)
+    st = stage_times(
+        [lambda: hsa.hsa_topk(seq, sc, wl.K, idx=idx_p, stream=main),
+         lambda: hsa.hsa_topk_blocks(seq, sc, wl.K, wl.page_size, idx=idx_b, stream=main),
+         lambda: hsa.hsa_sparse_mla_attn(seq, wl.q, wl.kv, idx_p, wl.D_v, wl.softmax_scale, out=o,
+                                         lse=lse, ws=ws, stream=main),
+         lambda: hsa.hsa_sparse_mla_attn(seq, wl.q, wl.kv, idx_b, wl.D_v, wl.softmax_scale, out=o,
+                                         lse=lse, ws=ws, stream=main)],
+        ["topk_positions", "topk_blocks", "sparse_mla_positions", "sparse_mla_blocks"], reps,
+        flush_l2, main)
+    rows = int((idx_b >= 0).sum())
+    byt = rows * wl.D_qk * 2 + wl.T_q * wl.H * (wl.D_qk + wl.D_v) * 2
+    res = {"workload": "the bf16 decode batch, selection of whole cache pages (64 positions): the "
+                       "32 pages with the highest page maximum per row",
+           "stages": st, "rows_gathered": rows,
+           "attention_frac_blocks": round(byt / (st["sparse_mla_blocks"]["ms"] * 1e-3) / (peaks["hbm_gbs"] * 1e9), 4)}
+    del wl, seq, sc, idx_p, idx_b, o, lse, ws
+    torch.cuda.empty_cache()
+    return res
+
+
 def secondary(dev, flush_l2, main, peaks, reps):
     """The path's other workloads, each measured once per bench run (rank 0, one GPU): the FP8
     decode batch (fp32 and MXFP8 index scales), the draft-verify decode batch, the bf16 causal
@@ -273,35 +325,55 @@ def secondary(dev, flush_l2, main, peaks, reps):
     sel = int(torch.clamp(n, max=wl.K).sum())
     byt = int(n.sum()) * (wl.D_I + 4 + 4) + sel * (wl.D_v + 4 + 2 * (wl.D_qk - wl.D_v)) + \
         wl.T_q * wl.H * (wl.D_qk + wl.D_v) * 2 + wl.T_q * wl.H_I * (wl.D_I * 2 + 4)
+    stage = stage_times(
+        [lambda: hsa.hsa_index_score(seq, wl.q_I, wl.w, k8, ks, scores=sc, stream=main),
+         lambda: hsa.hsa_topk(seq, sc, wl.K, idx=idx, stream=main),
+         lambda: hsa.hsa_sparse_mla_attn(seq, wl.q, kv8, idx, wl.D_v, wl.softmax_scale, kv_scale=kvs,
+                                         kv_rope=rope, out=o, lse=lse, ws=ws, stream=main)],
+        ["index_score", "topk", "sparse_mla"], reps, flush_l2, main)
+    idx_bytes = int(n.sum()) * (wl.D_I + 4 + 4) + wl.T_q * wl.H_I * (wl.D_I * 2 + 4)
+    attn_bytes = sel * (wl.D_v + 4 + 2 * (wl.D_qk - wl.D_v)) + wl.T_q * wl.H * (wl.D_qk + wl.D_v) * 2
+    stage["index_score"]["frac"] = round(idx_bytes / (stage["index_score"]["ms"] * 1e-3) / hbm, 4)
+    stage["sparse_mla"]["frac"] = round(attn_bytes / (stage["sparse_mla"]["ms"] * 1e-3) / hbm, 4)
     out["decode_fp8"] = {"workload": "128 sequences x 65536 keys, FP8 index keys (fp32 scale per key), "
                                      "FP8 latent (fp32 scale per token) + bf16 rope, Top-2048, 128 heads",
                          "ms_per_step": round(ms, 4), "value": wl.T_q / (ms * 1e-3), "unit": UNIT,
                          "bound": "hbm", "bytes": byt,
-                         "frac": round(byt / (ms * 1e-3) / hbm, 4)}
+                         "frac": round(byt / (ms * 1e-3) / hbm, 4), "stages": stage}
     # the same batch with the index queries and keys in MXFP8 (one E8M0 byte per 32 dims): the
-    # step rounds q_I onto the MX grid (two small kernels) and scores the MX key cache
+    # step quantizes q_I to MX codes and scales (hsa_quantize_mx, one kernel) and scores them
+    # against the MX key cache with the block-scaled MMA (hsa_index_score_mx inside the step)
     kmx, kmx_e = hsa.hsa_quantize_mx(wl.k_I)
     qI_flat = wl.q_I.view(-1, wl.D_I)
     q_codes = torch.empty(qI_flat.shape, dtype=torch.uint8, device=dev)
     q_e = torch.empty((qI_flat.shape[0], wl.D_I // 32), dtype=torch.uint8, device=dev)
-    q_mx = torch.empty_like(wl.q_I)
 
     def mx_step():
         hsa.hsa_quantize_mx(qI_flat, codes=q_codes, scales=q_e, stream=main)
-        hsa.hsa_dequantize_mx(q_codes, q_e, out=q_mx.view(-1, wl.D_I), stream=main)
-        hsa.hsa_fused_decode(seq, q_mx, wl.w, kmx, kmx_e, wl.q, kv8, kvs, rope, wl.K, wl.D_v,
-                             wl.softmax_scale, scores=sc, idx=idx, out=o, lse=lse, ws=ws, stream=main)
+        hsa.hsa_fused_decode(seq, q_codes.view(wl.q_I.shape), wl.w, kmx, kmx_e, wl.q, kv8, kvs, rope,
+                             wl.K, wl.D_v, wl.softmax_scale, scores=sc, idx=idx, out=o, lse=lse,
+                             ws=ws, stream=main, q_I_scale=q_e)
     for _ in range(3):
         mx_step()
     ms = _timed(mx_step, reps, flush_l2, main)
-    # plus the rounding of q_I: read bf16, write and re-read the codes and scale bytes, write bf16
-    byt_mx = byt + wl.T_q * wl.H_I * wl.D_I * (2 + 1 + 1 + 2) + 2 * wl.T_q * wl.H_I * (wl.D_I // 32)
+    n_q = wl.T_q * wl.H_I
+    # the index kernel reads codes + scale words instead of bf16 queries; the quantizer reads the
+    # bf16 queries and writes codes and scales
+    byt_mx = byt - n_q * wl.D_I * 2 + n_q * (wl.D_I + 4) + n_q * (wl.D_I * 2 + wl.D_I + 4)
+    stage_mx = stage_times(
+        [lambda: hsa.hsa_quantize_mx(qI_flat, codes=q_codes, scales=q_e, stream=main),
+         lambda: hsa.hsa_index_score(seq, q_codes.view(wl.q_I.shape), wl.w, kmx, kmx_e, scores=sc,
+                                     stream=main, q_scale=q_e)],
+        ["quantize_q", "index_score_mx"], reps, flush_l2, main)
+    idx_mx_bytes = int(n.sum()) * (wl.D_I + 4 + 4) + n_q * (wl.D_I + 4 + 4)
+    stage_mx["index_score_mx"]["frac"] = round(idx_mx_bytes / (stage_mx["index_score_mx"]["ms"] * 1e-3) / hbm, 4)
     out["decode_mxfp8"] = {"workload": "the FP8 decode batch with MXFP8 index queries and keys "
-                                       "(E8M0 scale per 32 dims), rounding of q_I included",
+                                       "(E8M0 scale per 32 dims, block-scaled MMA on the codes), "
+                                       "quantization of q_I included",
                            "ms_per_step": round(ms, 4), "value": wl.T_q / (ms * 1e-3), "unit": UNIT,
                            "bound": "hbm", "bytes": byt_mx,
-                           "frac": round(byt_mx / (ms * 1e-3) / hbm, 4)}
-    del kmx, kmx_e, q_codes, q_e, q_mx
+                           "frac": round(byt_mx / (ms * 1e-3) / hbm, 4), "stages": stage_mx}
+    del kmx, kmx_e, q_codes, q_e
     # KV-cache quantizer on the same cache (8.4 M rows): read 1152 B, write 512 + 4 + 128 B per row
     nrow = wl.kv.shape[0]
 
@@ -353,6 +425,8 @@ def secondary(dev, flush_l2, main, peaks, reps):
         "frac": round(byt / (ms * 1e-3) / hbm, 4)}
     del wl, sc, idx, o, lse, ws, seq
     torch.cuda.empty_cache()
+
+    out["decode_bf16_block_aligned"] = block_aligned(dev, flush_l2, main, peaks, reps)
 
     # causal prefill: the bf16 16384-token workload (4 chunks of 4096 in zigzag pairs) and the
     # 131072-token workload with FP8 index keys (32 chunks of 4096 in zigzag pairs)

@@ -119,6 +119,21 @@ HSA_API hsa_status_t hsa_index_score(const hsa_paged_seq_t* seq, const void* q_I
                              hsa_dtype_t k_dtype, const void* k_scale, float* scores,
                              int64_t ld_scores, void* stream);
 
+/* The index score with MXFP8 queries and keys: both operands are E4M3 codes with one E8M0 scale
+ * byte per 32 dims, so the product runs as a block-scaled MMA on the codes themselves (first
+ * page "Hierarchical Quantization": index Q and K in MXFP8; fifth page 4, table).
+ *   scores[t, s] = sum_j w[t,j] * max(0, sum_d qv(t,j,d) * kv(slot(t,s), d)),
+ *   qv(t,j,d) = q_codes[t,j,d] * 2^(q_scale[t,j,d/32] - 127)   (kv likewise from k_codes, k_scale)
+ *   q_codes  device uint8 [T_q, H_I, D_I];  q_scale device uint8 [T_q, H_I, D_I / 32], 16-byte
+ *            aligned (hsa_quantize_mx writes both from bf16 or fp32 queries)
+ *   k_codes, k_scale, w, scores: as hsa_index_score with k_dtype MXE4M3.
+ * D_I must be a multiple of 32.  The tensor-core kernel serves H_I = 64, D_I = 128, page_size a
+ * multiple of 8; other shapes use a CUDA-core kernel.  Same errors as hsa_index_score. */
+HSA_API hsa_status_t hsa_index_score_mx(const hsa_paged_seq_t* seq, const uint8_t* q_codes,
+                                const uint8_t* q_scale, const float* w, int32_t H_I, int32_t D_I,
+                                const uint8_t* k_codes, const uint8_t* k_scale, float* scores,
+                                int64_t ld_scores, void* stream);
+
 /* ---- 2. Top-K -----------------------------------------------------------------------------
  * For row t with n = q_pos[t] + 1 candidate positions:
  *   n <= K : idx[t] = 0, 1, ..., n-1, then -1 up to K;
@@ -163,13 +178,8 @@ HSA_API hsa_status_t hsa_topk_blocks(const hsa_paged_seq_t* seq, const float* sc
  *   idx      device int32 [T_q, K]: positions in [0, q_pos[t]] or -1
  *   out      device [T_q, H, D_v] of out_dtype (F32 or BF16)
  *   lse      device fp32 [T_q, H] or NULL
- *   ws       workspace of at least hsa_sparse_mla_workspace_size() bytes, 256-byte aligned and
- *            zero-filled before its first use (with few query rows -- at most 256 -- the
- *            tensor-core kernel spreads the rows' tiles evenly over all clusters and merges a row
- *            cut between clusters through this workspace; it keeps one counter per row there,
- *            which every call returns to zero.  After a call that set HSA_DEV_TIMEOUT, zero it
- *            again.  A workspace smaller than the size reported, or NULL, makes the kernel take
- *            whole rows per cluster instead; the results agree within rounding.)
+ *   ws       workspace of at least hsa_sparse_mla_workspace_size() bytes, 256-byte aligned
+ *            (the current kernels report 0 and need none; a call may pass NULL)
  * Pages: first page "Sparse Attention Pipeline Optimization" (indexed reads, block-wise fused
  * attention); third page 3.2 (partition by query, aggregate over the selected positions,
  * stage them in shared memory); fifth page 3 (SFA).  The tensor-core kernel serves q BF16,
@@ -190,10 +200,7 @@ HSA_API hsa_status_t hsa_sparse_mla_attn(const hsa_paged_seq_t* seq, const void*
  * caller buffers that hold the intermediate results afterwards.  With stream_aux != NULL the
  * rows are split in two halves; the second half runs on stream_aux, overlapping the first
  * half's attention (event-ordered; stream_main waits for stream_aux before returning work to
- * the caller).  Scores and selections are then bitwise the same; the attention of a row that
- * the few-rows schedule cuts between clusters may differ in the last bit, since the halves
- * cut their rows at other places.  ws: zero-filled before first use, as for
- * hsa_sparse_mla_attn.  Pages: first page "Sparse Attention Pipeline Optimization" (fusing the decode
+ * the caller); the results are bitwise the same.  ws: as for hsa_sparse_mla_attn.  Pages: first page "Sparse Attention Pipeline Optimization" (fusing the decode
  * operators and running independent ones concurrently: indexer, then the sparse attention
  * kernel; several streams); fifth page 3.3 (operators on independent streams with event
  * synchronization).  The members of hsa_index_args_t and hsa_attn_args_t have the meaning of
@@ -202,6 +209,8 @@ HSA_API hsa_status_t hsa_sparse_mla_attn(const hsa_paged_seq_t* seq, const void*
 typedef struct hsa_index_args {
     const void* q_I; hsa_dtype_t q_dtype; const float* w; int32_t H_I; int32_t D_I;
     const void* k_cache; hsa_dtype_t k_dtype; const void* k_scale;
+    const void* q_scale;   /* q_dtype MXE4M3 (keys MXE4M3 too): the queries' E8M0 bytes, as in
+                              hsa_index_score_mx; else ignored */
 } hsa_index_args_t;
 
 typedef struct hsa_attn_args {
@@ -285,7 +294,9 @@ HSA_API hsa_status_t hsa_mx_round(const void* src, hsa_dtype_t src_dtype, int64_
  *              [num_slots, D_v], fp32 scales [num_slots, D_v / kv_group], bf16 rope
  *              [num_slots, D_rope]);
  *   stream_q : the index queries q_I [q_rows, D_I] rounded onto the MXFP8 grid into q_I_out
- *              (bf16, hsa_mx_round; skipped when q_I_out is NULL).
+ *              (bf16, hsa_mx_round; skipped when q_I_out is NULL), and / or quantized to MXFP8
+ *              codes q_codes_out [q_rows, D_I] and E8M0 scales q_scale_out [q_rows, D_I / 32]
+ *              for hsa_index_score_mx (hsa_quantize_mx; skipped when q_codes_out is NULL).
  * Each side stream first waits for the work already enqueued on `stream`, and `stream` then
  * waits for all three, so a decode step enqueued on `stream` next sees every write.  A NULL side
  * stream means `stream` itself.  Results equal the same calls issued one after another on one
@@ -305,6 +316,8 @@ typedef struct hsa_prolog_args {
     uint8_t* kv_cache; float* kv_scale; void* kv_rope;
     const void* q_I; hsa_dtype_t q_I_dtype; int64_t q_rows;
     void* q_I_out;                /* bf16 [q_rows, D_I], or NULL */
+    uint8_t* q_codes_out;         /* uint8 [q_rows, D_I], or NULL */
+    uint8_t* q_scale_out;         /* uint8 [q_rows, D_I / 32] (with q_codes_out) */
 } hsa_prolog_args_t;
 
 HSA_API hsa_status_t hsa_decode_prolog(const hsa_prolog_args_t* args, void* stream, void* stream_k,

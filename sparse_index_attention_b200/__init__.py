@@ -36,7 +36,7 @@ class hsa_paged_seq_t(ctypes.Structure):
 
 class hsa_index_args_t(ctypes.Structure):
     _fields_ = [("q_I", _P), ("q_dtype", ctypes.c_int), ("w", _P), ("H_I", _i32), ("D_I", _i32),
-                ("k_cache", _P), ("k_dtype", ctypes.c_int), ("k_scale", _P)]
+                ("k_cache", _P), ("k_dtype", ctypes.c_int), ("k_scale", _P), ("q_scale", _P)]
 
 
 class hsa_attn_args_t(ctypes.Structure):
@@ -52,12 +52,14 @@ class hsa_prolog_args_t(ctypes.Structure):
                 ("k_cache", _P), ("k_scale", _P), ("k_dtype", ctypes.c_int),
                 ("new_kv", _P), ("new_kv_dtype", ctypes.c_int), ("D_v", _i32), ("D_rope", _i32),
                 ("kv_group", _i32), ("kv_cache", _P), ("kv_scale", _P), ("kv_rope", _P),
-                ("q_I", _P), ("q_I_dtype", ctypes.c_int), ("q_rows", _i64), ("q_I_out", _P)]
+                ("q_I", _P), ("q_I_dtype", ctypes.c_int), ("q_rows", _i64), ("q_I_out", _P),
+                ("q_codes_out", _P), ("q_scale_out", _P)]
 
 
 SYMBOLS = {
     "hsa_index_score": (ctypes.c_int, [_P, _P, ctypes.c_int, _P, _i32, _i32, _P, ctypes.c_int, _P,
                                        _P, _i64, _P]),
+    "hsa_index_score_mx": (ctypes.c_int, [_P, _P, _P, _P, _i32, _i32, _P, _P, _P, _i64, _P]),
     "hsa_topk": (ctypes.c_int, [_P, _P, _i64, _i32, _P, _P]),
     "hsa_topk_blocks": (ctypes.c_int, [_P, _P, _i64, _i32, _i32, _P, _P]),
     "hsa_sparse_mla_workspace_size": (_sz, [_P, _i32, _i32, _i32, _i32]),
@@ -178,12 +180,19 @@ class PagedSeq:
 
 # ------------------------------------------------------------------------------ entry points
 def hsa_index_score(seq: PagedSeq, q_I, w, k_cache, k_scale=None, scores=None, ld: Optional[int] = None,
-                    stream=None):
+                    stream=None, q_scale=None):
+    """Index scores [T_q, ld].  With q_scale (uint8 E8M0 [T_q, H_I, D_I / 32]) q_I holds MXFP8
+    codes and the keys must be MXFP8 too: hsa_index_score_mx, the block-scaled path."""
     T_q, H_I, D_I = q_I.shape
     if scores is None:
         ld = ld or seq.max_seq_len
         scores = torch.empty((T_q, ld), dtype=torch.float32, device=q_I.device)
     ld = scores.shape[1]
+    if q_scale is not None:
+        _check(lib().hsa_index_score_mx(seq.ref, _ptr(q_I), _ptr(q_scale), _ptr(w), H_I, D_I,
+                                        _ptr(k_cache), _ptr(k_scale), _ptr(scores), ld, _stream(stream)),
+               "hsa_index_score_mx")
+        return scores
     _check(lib().hsa_index_score(seq.ref, _ptr(q_I), _dtype(q_I), _ptr(w), H_I, D_I, _ptr(k_cache),
                                  _key_dtype(k_cache, k_scale), _ptr(k_scale), _ptr(scores), ld,
                                  _stream(stream)),
@@ -272,8 +281,9 @@ def hsa_fused_decode_workspace_size(seq: PagedSeq, q, kv, D_v: int, K: int) -> i
 
 def hsa_fused_decode(seq: PagedSeq, q_I, w, k_cache, k_scale, q, kv, kv_scale, kv_rope, K: int,
                      D_v: int, softmax_scale: float, scores=None, idx=None, out=None, lse=True,
-                     ws=None, stream=None, aux_stream=None):
-    """index score -> Top-K -> sparse MLA in one call.  Returns (out, lse, idx, scores)."""
+                     ws=None, stream=None, aux_stream=None, q_I_scale=None):
+    """index score -> Top-K -> sparse MLA in one call.  Returns (out, lse, idx, scores).  With
+    q_I_scale, q_I holds MXFP8 codes (keys MXFP8 too), as in hsa_index_score_mx."""
     T_q, H_I, D_I = q_I.shape
     _, H, D_qk = q.shape
     dev = q.device
@@ -288,8 +298,9 @@ def hsa_fused_decode(seq: PagedSeq, q_I, w, k_cache, k_scale, q, kv, kv_scale, k
     elif lse is False:
         lse = None
     ws = _workspace(hsa_fused_decode_workspace_size(seq, q, kv, D_v, K), dev, ws)
-    ia = hsa_index_args_t(_ptr(q_I), _dtype(q_I), _ptr(w), H_I, D_I, _ptr(k_cache),
-                          _key_dtype(k_cache, k_scale), _ptr(k_scale))
+    ia = hsa_index_args_t(_ptr(q_I), HSA_MXE4M3 if q_I_scale is not None else _dtype(q_I), _ptr(w),
+                          H_I, D_I, _ptr(k_cache), _key_dtype(k_cache, k_scale), _ptr(k_scale),
+                          _ptr(q_I_scale))
     at = _attn_struct(q, kv, D_v, softmax_scale, kv_scale, kv_rope, out, lse)
     _check(lib().hsa_fused_decode(seq.ref, ctypes.byref(ia), ctypes.byref(at), K, _ptr(scores),
                                   scores.shape[1], _ptr(idx), _ptr(ws), ws.numel(), _stream(stream),
@@ -426,7 +437,7 @@ def _cache_rows(t, name: str, width: int, dtype) -> int:
 
 def hsa_decode_prolog(new_k, new_kv, slot_mapping, k_cache, k_scale, kv_cache, kv_scale, kv_rope,
                       q_I, q_I_out, D_v: int, kv_group: Optional[int] = None, streams=None,
-                      stream=None):
+                      stream=None, q_codes_out=None, q_scale_out=None):
     """The writes that precede a decode step, on three streams (hsa_decode_prolog): the new
     tokens' index keys into the index key cache, their latent rows into the FP8 latent cache,
     and the index queries rounded onto the MXFP8 grid into ``q_I_out`` ("Day 0 Inference
@@ -440,6 +451,8 @@ def hsa_decode_prolog(new_k, new_kv, slot_mapping, k_cache, k_scale, kv_cache, k
     ``slot_mapping`` [n] (int64).  The index key cache is MXFP8 when ``k_scale`` is uint8
     (E8M0 bytes, [slots, D_I/32]) and E4M3 with one fp32 scale per key otherwise.  The latent
     cache is E4M3 with one fp32 scale per ``kv_group`` dims (default D_v) plus bf16 rope.
+    With ``q_codes_out`` (uint8, q_I's size) and ``q_scale_out`` (uint8 [rows, D_I/32]) the
+    queries are also quantized to MXFP8 codes and scales for the block-scaled index path.
     Results equal the same calls issued one after another on one stream."""
     n, D_I = new_k.shape
     D_rope = new_kv.shape[1] - D_v
@@ -456,6 +469,11 @@ def hsa_decode_prolog(new_k, new_kv, slot_mapping, k_cache, k_scale, kv_cache, k
         raise ValueError("slot_mapping must be int64 [n]")
     if q_I_out is not None and (q_I_out.dtype != torch.bfloat16 or q_I_out.numel() != q_I.numel()):
         raise ValueError("q_I_out must be bf16 with q_I's size")
+    if q_codes_out is not None and (
+            q_codes_out.dtype != torch.uint8 or q_codes_out.numel() != q_I.numel() or
+            q_scale_out is None or q_scale_out.dtype != torch.uint8 or
+            q_scale_out.numel() != q_I.numel() // 32):
+        raise ValueError("q_codes_out / q_scale_out must be uint8 codes and E8M0 scales of q_I")
     if streams is None:
         streams = (torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream())
     flat_q = q_I.reshape(-1, D_I)
@@ -463,7 +481,7 @@ def hsa_decode_prolog(new_k, new_kv, slot_mapping, k_cache, k_scale, kv_cache, k
                           _ptr(k_cache), _ptr(k_scale), HSA_MXE4M3 if mx else HSA_E4M3,
                           _ptr(new_kv), _dtype(new_kv), D_v, D_rope, grp, _ptr(kv_cache),
                           _ptr(kv_scale), _ptr(kv_rope), _ptr(flat_q), _dtype(flat_q),
-                          flat_q.shape[0], _ptr(q_I_out))
+                          flat_q.shape[0], _ptr(q_I_out), _ptr(q_codes_out), _ptr(q_scale_out))
     _check(lib().hsa_decode_prolog(ctypes.byref(a), _stream(stream), _stream(streams[0]),
                                    _stream(streams[1]), _stream(streams[2])),
            "hsa_decode_prolog")

@@ -66,17 +66,19 @@ hsa_paged_seq_t sub_rows(const hsa_paged_seq_t& s, int32_t t0, int32_t n) {
 }
 
 hsa_status_t check_index(const hsa_paged_seq_t* seq, const void* q_I, hsa_dtype_t q_dtype,
-                         const float* w, int32_t H_I, int32_t D_I, const void* k_cache,
-                         hsa_dtype_t k_dtype, const void* k_scale, const float* scores,
-                         int64_t ld) {
+                         const void* q_scale, const float* w, int32_t H_I, int32_t D_I,
+                         const void* k_cache, hsa_dtype_t k_dtype, const void* k_scale,
+                         const float* scores, int64_t ld) {
     hsa_status_t st = check_seq(seq);
     if (st != HSA_OK) return st;
     HSA_REQUIRE(H_I >= 1 && H_I <= 256 && D_I >= 1 && D_I <= 1024, HSA_ERR_INVALID_ARG,
                 "H_I = %d, D_I = %d out of range", H_I, D_I);
     HSA_REQUIRE((size_t)H_I * D_I * 4 <= 160 * 1024, HSA_ERR_UNSUPPORTED,
                 "H_I * D_I = %d too large", H_I * D_I);
-    HSA_REQUIRE(q_dtype == HSA_F32 || q_dtype == HSA_BF16, HSA_ERR_UNSUPPORTED,
-                "q_I dtype must be F32 or BF16");
+    HSA_REQUIRE(q_dtype == HSA_F32 || q_dtype == HSA_BF16 || q_dtype == HSA_MXE4M3, HSA_ERR_UNSUPPORTED,
+                "q_I dtype must be F32, BF16 or MXE4M3");
+    HSA_REQUIRE(q_dtype != HSA_MXE4M3 || k_dtype == HSA_MXE4M3, HSA_ERR_UNSUPPORTED,
+                "MXE4M3 queries need MXE4M3 keys");
     HSA_REQUIRE(k_dtype == HSA_F32 || k_dtype == HSA_BF16 || k_dtype == HSA_E4M3 ||
                     k_dtype == HSA_MXE4M3,
                 HSA_ERR_UNSUPPORTED, "k dtype must be F32, BF16, E4M3 or MXE4M3");
@@ -92,6 +94,8 @@ hsa_status_t check_index(const hsa_paged_seq_t* seq, const void* q_I, hsa_dtype_
                     "misaligned k_scale");
         HSA_REQUIRE(k_dtype != HSA_MXE4M3 || aligned(k_scale, 16), HSA_ERR_INVALID_ARG,
                     "MXE4M3 k_scale must be 16-byte aligned");
+        HSA_REQUIRE(q_dtype != HSA_MXE4M3 || (q_scale && aligned(q_scale, 16)), HSA_ERR_INVALID_ARG,
+                    "MXE4M3 queries need q_scale, 16-byte aligned");
         HSA_REQUIRE(aligned(q_I, dtype_size(q_dtype)) && aligned(w, 4) && aligned(scores, 4) &&
                         aligned(k_cache, dtype_size(k_dtype)),
                     HSA_ERR_INVALID_ARG, "misaligned tensor pointer");
@@ -136,15 +140,16 @@ hsa_status_t check_attn(const hsa_paged_seq_t* seq, const void* q, hsa_dtype_t q
 }
 
 hsa::IndexScoreArgs index_args(const hsa_paged_seq_t* seq, const void* q_I, hsa_dtype_t q_dtype,
-                               const float* w, int32_t H_I, int32_t D_I, const void* k_cache,
-                               hsa_dtype_t k_dtype, const void* k_scale, float* scores,
-                               int64_t ld) {
+                               const void* q_scale, const float* w, int32_t H_I, int32_t D_I,
+                               const void* k_cache, hsa_dtype_t k_dtype, const void* k_scale,
+                               float* scores, int64_t ld) {
     hsa::IndexScoreArgs a;
     a.seq = view(seq);
     a.max_seq_len = seq->max_seq_len;
     a.q_run = seq->q_run;
     a.q_I = q_I;
     a.q_dtype = q_dtype;
+    a.q_scale = q_dtype == HSA_MXE4M3 ? q_scale : nullptr;
     a.w = w;
     a.H_I = H_I;
     a.D_I = D_I;
@@ -313,18 +318,31 @@ const char* hsa_status_string(hsa_status_t s) {
 
 const char* hsa_last_error_message(void) { return g_last_error.c_str(); }
 
-int32_t hsa_version(void) { return 300; }
+int32_t hsa_version(void) { return 400; }
 
 hsa_status_t hsa_index_score(const hsa_paged_seq_t* seq, const void* q_I, hsa_dtype_t q_dtype,
                              const float* w, int32_t H_I, int32_t D_I, const void* k_cache,
                              hsa_dtype_t k_dtype, const void* k_scale, float* scores,
                              int64_t ld_scores, void* stream) {
     g_last_error.clear();
-    hsa_status_t st = check_index(seq, q_I, q_dtype, w, H_I, D_I, k_cache, k_dtype, k_scale,
-                                  scores, ld_scores);
+    hsa_status_t st = check_index(seq, q_I, q_dtype, nullptr, w, H_I, D_I, k_cache, k_dtype,
+                                  k_scale, scores, ld_scores);
     if (st != HSA_OK) return st;
-    return run_index(index_args(seq, q_I, q_dtype, w, H_I, D_I, k_cache, k_dtype, k_scale, scores,
-                                ld_scores),
+    return run_index(index_args(seq, q_I, q_dtype, nullptr, w, H_I, D_I, k_cache, k_dtype, k_scale,
+                                scores, ld_scores),
+                     (cudaStream_t)stream);
+}
+
+hsa_status_t hsa_index_score_mx(const hsa_paged_seq_t* seq, const uint8_t* q_codes,
+                                const uint8_t* q_scale, const float* w, int32_t H_I, int32_t D_I,
+                                const uint8_t* k_codes, const uint8_t* k_scale, float* scores,
+                                int64_t ld_scores, void* stream) {
+    g_last_error.clear();
+    hsa_status_t st = check_index(seq, q_codes, HSA_MXE4M3, q_scale, w, H_I, D_I, k_codes,
+                                  HSA_MXE4M3, k_scale, scores, ld_scores);
+    if (st != HSA_OK) return st;
+    return run_index(index_args(seq, q_codes, HSA_MXE4M3, q_scale, w, H_I, D_I, k_codes,
+                                HSA_MXE4M3, k_scale, scores, ld_scores),
                      (cudaStream_t)stream);
 }
 
@@ -408,8 +426,8 @@ hsa_status_t hsa_fused_decode(const hsa_paged_seq_t* seq, const hsa_index_args_t
                               void* stream_main, void* stream_aux) {
     g_last_error.clear();
     HSA_REQUIRE(ix && at, HSA_ERR_INVALID_ARG, "index / attn args NULL");
-    hsa_status_t st = check_index(seq, ix->q_I, ix->q_dtype, ix->w, ix->H_I, ix->D_I, ix->k_cache,
-                                  ix->k_dtype, ix->k_scale, scores, ld_scores);
+    hsa_status_t st = check_index(seq, ix->q_I, ix->q_dtype, ix->q_scale, ix->w, ix->H_I, ix->D_I,
+                                  ix->k_cache, ix->k_dtype, ix->k_scale, scores, ld_scores);
     if (st != HSA_OK) return st;
     st = check_attn(seq, at->q, at->q_dtype, at->H, at->D_qk, at->D_v, at->kv, at->kv_dtype,
                     at->kv_scale, at->kv_scale_group, at->kv_rope, idx, K, at->out, at->out_dtype);
@@ -430,8 +448,11 @@ hsa_status_t hsa_fused_decode(const hsa_paged_seq_t* seq, const hsa_index_args_t
                         cudaEvent_t after_topk) -> hsa_status_t {
         hsa_paged_seq_t part = sub_rows(*seq, r0, n);
         const size_t qI = (size_t)r0 * ix->H_I * ix->D_I * dtype_size(ix->q_dtype);
+        const void* qs = ix->q_dtype == HSA_MXE4M3
+                             ? static_cast<const char*>(ix->q_scale) + (size_t)r0 * ix->H_I * (ix->D_I / 32)
+                             : nullptr;
         hsa::IndexScoreArgs ia = index_args(
-            &part, static_cast<const char*>(ix->q_I) + qI, ix->q_dtype, ix->w + (size_t)r0 * ix->H_I,
+            &part, static_cast<const char*>(ix->q_I) + qI, ix->q_dtype, qs, ix->w + (size_t)r0 * ix->H_I,
             ix->H_I, ix->D_I, ix->k_cache, ix->k_dtype, ix->k_scale, scores + (size_t)r0 * ld_scores,
             ld_scores);
         hsa_status_t r = run_index(ia, s);
@@ -568,6 +589,12 @@ hsa_status_t hsa_decode_prolog(const hsa_prolog_args_t* a, void* stream, void* s
         st = check_mx_round(a->q_I, a->q_I_dtype, a->q_rows, a->D_I, a->q_I_out, HSA_BF16);
         if (st != HSA_OK) return st;
     }
+    const bool want_qc = a->q_codes_out != nullptr && a->q_rows > 0;
+    if (want_qc) {
+        st = check_quantize_mx(a->q_I, a->q_I_dtype, a->q_rows, a->D_I, nullptr, a->q_rows,
+                               a->q_codes_out, a->q_scale_out);
+        if (st != HSA_OK) return st;
+    }
     cudaStream_t s0 = (cudaStream_t)stream;
     const cudaStream_t side[3] = {stream_k ? (cudaStream_t)stream_k : s0,
                                   stream_kv ? (cudaStream_t)stream_kv : s0,
@@ -603,6 +630,10 @@ hsa_status_t hsa_decode_prolog(const hsa_prolog_args_t* a, void* stream, void* s
         r = cuda_status(hsa::launch_mx_round(a->q_I, a->q_I_dtype, a->q_rows, a->D_I, a->q_I_out,
                                              HSA_BF16, side[2]),
                         "mx_round");
+    if (r == HSA_OK && want_qc)
+        r = cuda_status(hsa::launch_quantize_mx(a->q_I, a->q_I_dtype, a->q_rows, a->D_I, nullptr,
+                                                a->q_rows, a->q_codes_out, a->q_scale_out, side[2]),
+                        "quantize_mx (queries)");
     // join (also after a failed launch, so that nothing enqueued is left unordered)
     for (int i = 0; i < 3; ++i) {
         if (side[i] == s0 || ev[1 + i] == nullptr || ev[0] == nullptr) continue;

@@ -14,10 +14,12 @@ namespace {
 constexpr int kThreads = 128;
 
 // KT: 0 fp32 keys, 1 bf16 keys, 2 e4m3 keys + per-key fp32 scale, 3 MXFP8 keys (e4m3 codes,
-// one E8M0 byte per 32 dims, applied to each element: the scale varies along the dot product)
+// one E8M0 byte per 32 dims, applied to each element: the scale varies along the dot product).
+// QT = uint8_t: MXFP8 queries (codes, q_scale one E8M0 byte per 32 dims), decoded on load.
 template <typename QT, int KT>
 __global__ void __launch_bounds__(kThreads)
-index_score_simt_kernel(SeqView v, const QT* __restrict__ q_I, const float* __restrict__ w,
+index_score_simt_kernel(SeqView v, const QT* __restrict__ q_I, const uint8_t* __restrict__ q_scale,
+                        const float* __restrict__ w,
                         int H_I, int D_I, const void* __restrict__ k_cache,
                         const void* __restrict__ k_scale, float* __restrict__ scores, int64_t ld) {
     extern __shared__ float smem[];
@@ -28,7 +30,12 @@ index_score_simt_kernel(SeqView v, const QT* __restrict__ q_I, const float* __re
     const int s0 = blockIdx.x * kThreads;
     if (r.pos < 0 || s0 > r.pos) return;  // uniform over the block
     const int64_t qoff = (int64_t)t * H_I * D_I;
-    for (int i = threadIdx.x; i < H_I * D_I; i += kThreads) sq[i] = to_f32(q_I[qoff + i]);
+    for (int i = threadIdx.x; i < H_I * D_I; i += kThreads) {
+        if constexpr (sizeof(QT) == 1)
+            sq[i] = e4m3_to_f32(q_I[qoff + i]) * e8m0_to_f32(q_scale[(qoff + i) / 32]);
+        else
+            sq[i] = to_f32(q_I[qoff + i]);
+    }
     for (int i = threadIdx.x; i < H_I; i += kThreads) sw[i] = w[(int64_t)t * H_I + i];
     __syncthreads();
     const int s = s0 + threadIdx.x;
@@ -67,7 +74,8 @@ cudaError_t launch_t(const IndexScoreArgs& a, cudaStream_t st) {
         cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
     }
-    k<<<grid, kThreads, smem, st>>>(a.seq, reinterpret_cast<const QT*>(a.q_I), a.w, a.H_I, a.D_I,
+    k<<<grid, kThreads, smem, st>>>(a.seq, reinterpret_cast<const QT*>(a.q_I),
+                                    static_cast<const uint8_t*>(a.q_scale), a.w, a.H_I, a.D_I,
                                     a.k_cache, a.k_scale, a.scores, a.ld);
     count_launch();
     return cudaGetLastError();
@@ -76,6 +84,7 @@ cudaError_t launch_t(const IndexScoreArgs& a, cudaStream_t st) {
 }  // namespace
 
 cudaError_t launch_index_score_simt(const IndexScoreArgs& a, cudaStream_t st) {
+    if (a.q_dtype == HSA_MXE4M3) return launch_t<uint8_t, 3>(a, st);   // MX queries need MX keys
     if (a.q_dtype == HSA_F32) {
         if (a.k_dtype == HSA_F32) return launch_t<float, 0>(a, st);
         if (a.k_dtype == HSA_BF16) return launch_t<float, 1>(a, st);

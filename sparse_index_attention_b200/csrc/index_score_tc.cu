@@ -44,19 +44,29 @@ constexpr int kHI = 64;                  // index heads
 constexpr int kHalfBytes = kBM * 128;    // one 64-column swizzled half of a key tile: 16 KB
 constexpr int kTileBytes = 2 * kHalfBytes;
 
-template <int G, bool kFp8, bool kMx = false>
+template <int G, bool kFp8, bool kMx = false, bool kBs = false>
 struct Cfg {
+    static_assert(!kBs || (G <= 2 && !kFp8 && !kMx), "block-scaled: codes straight to the MMA, G <= 2");
     static constexpr int N = G * kHI;
-    static constexpr int kQBytes = N * kDI * 2;
-    static constexpr int kStages = kFp8 ? (G == 1 ? 4 : (G == 2 ? 3 : 2)) : (G == 1 ? 6 : (G == 2 ? 5 : 4));
+    static constexpr int kTile = kBs ? kBM * kDI : kTileBytes;  // one MMA stage: 16 KB codes or 32 KB bf16
+    static constexpr int kQBytes = N * kDI * (kBs ? 1 : 2);
+    static constexpr int kStages = kBs ? (G == 1 ? 8 : 6)
+                                       : kFp8 ? (G == 1 ? 4 : (G == 2 ? 3 : 2)) : (G == 1 ? 6 : (G == 2 ? 5 : 4));
     static constexpr int kRawStages = kFp8 ? 4 : 0;          // FP8 staging tiles (16 KB each)
-    static constexpr int kScaleStageBytes = kMx ? kBM * 4 : 0;  // MXFP8: 4 E8M0 bytes per key
+    static constexpr int kScaleStageBytes = (kMx || kBs) ? kBM * 4 : 0;  // 4 E8M0 bytes per key
+    static constexpr int kScaleStages = kBs ? kStages : kRawStages;
     static constexpr int kMaxGroups = G == 1 ? 2048 : 4096;
-    static constexpr int kTmemCols = 2 * N;                   // 128, 256 or 512
-    static constexpr int kThreads = kFp8 ? 320 : 192;
-    static constexpr size_t kSmem = 1024 + (size_t)kStages * kTileBytes + (size_t)kRawStages * (kBM * kDI) +
-                                    (size_t)kRawStages * kScaleStageBytes + kQBytes +
-                                    4 * (kMaxGroups + 1) + 4 * N + 256;
+    // TMEM: two accumulators of N columns; block-scaled adds the key scales (4 columns per stage)
+    // and the query scales (N / 32 columns)
+    static constexpr int kSfaCol = 2 * N;
+    static constexpr int kSfbCol = 2 * N + 4 * kStages;
+    static constexpr int kTmemCols = kBs ? (G == 1 ? 256 : 512) : 2 * N;   // 128, 256 or 512
+    static_assert(!kBs || kSfbCol + N / 32 <= kTmemCols, "TMEM budget");
+    static constexpr int kThreads = (kFp8 || kBs) ? 320 : 192;
+    static constexpr int kBarBytes = 512;
+    static constexpr size_t kSmem = 1024 + (size_t)kStages * kTile + (size_t)kRawStages * (kBM * kDI) +
+                                    (size_t)kScaleStages * kScaleStageBytes + kQBytes +
+                                    4 * (kMaxGroups + 1) + 4 * N + kBarBytes;
     static_assert(kSmem <= 232448, "shared memory budget");
 };
 
@@ -105,13 +115,13 @@ __device__ __forceinline__ int first_group(const int32_t* prefix, int n_groups, 
     return lo;
 }
 
-template <int G, bool kFp8, bool kMx>
-__global__ void __launch_bounds__(Cfg<G, kFp8, kMx>::kThreads, 1)
+template <int G, bool kFp8, bool kMx, bool kBs = false>
+__global__ void __launch_bounds__(Cfg<G, kFp8, kMx, kBs>::kThreads, 1)
 index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_q,
                       SeqView v, int32_t q_row0, const float* __restrict__ w,
-                      const void* __restrict__ k_scale, float* __restrict__ scores, int64_t ld,
-                      int32_t box_rows) {
-    using C = Cfg<G, kFp8, kMx>;
+                      const void* __restrict__ k_scale, const uint32_t* __restrict__ q_scale,
+                      float* __restrict__ scores, int64_t ld, int32_t box_rows) {
+    using C = Cfg<G, kFp8, kMx, kBs>;
     static_assert(!kMx || kFp8, "MXFP8 keys go through the FP8 staging path");
     // E4M3 keys with fp32 scales run the MMA in f16: a code widens to f16 in one conversion
     // (exact), and the queries are rescaled per head by a power of two into f16's range, the
@@ -120,13 +130,17 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
     constexpr int N = C::N;
     constexpr int S = C::kStages;
     constexpr uint32_t kIdesc = kF16 ? tc::idesc_f16_f32(kBM, N) : tc::idesc_bf16_f32(kBM, N, 0, 0);
+    // kBs (MXFP8 queries and keys): the codes go from TMA straight to a block-scaled MMA
+    // (kind::mxf8f6f4, K = 32 per instruction, one E8M0 scale per 32 dims of every key and
+    // query row, read from TMEM); warps 6-9 place each tile's key scales in TMEM, the epilogue
+    // warps each group's query scales.
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t* tiles = base;                                          // S x 32 KB (bf16, swizzled)
-    uint8_t* raw = tiles + (size_t)S * kTileBytes;                  // FP8 staging
-    uint8_t* kscl = raw + (size_t)C::kRawStages * (kBM * kDI);      // MXFP8 scale words [4][128]
-    uint8_t* qbuf = kscl + (size_t)C::kRawStages * C::kScaleStageBytes;  // N x 128 bf16, swizzled
+    uint8_t* tiles = base;                                          // S x 32 KB bf16 (16 KB codes), swizzled
+    uint8_t* raw = tiles + (size_t)S * C::kTile;                    // FP8 staging
+    uint8_t* kscl = raw + (size_t)C::kRawStages * (kBM * kDI);      // MXFP8 scale words [4 or S][128]
+    uint8_t* qbuf = kscl + (size_t)C::kScaleStages * C::kScaleStageBytes;  // N x 128 bf16 (codes), swizzled
     // barriers first (8-byte alignment), then the variable-size arrays
     uint64_t* bars = reinterpret_cast<uint64_t*>(qbuf + C::kQBytes);
     uint64_t* full = bars;                 // [S]  keys landed (bf16 tile ready)
@@ -138,11 +152,13 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
     uint64_t* raw_full = q_empty + 1;      // [4] FP8 bytes landed
     uint64_t* raw_empty = raw_full + 4;    // [4] converters done with the staging tile
     uint64_t* epi_bar = raw_empty + 4;     // the four epilogue warps
-    uint64_t* q_ready = epi_bar + 1;       // f16 MMA: the group's queries converted (4 warps)
-    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(q_ready + 1);
+    uint64_t* q_ready = epi_bar + 1;       // f16 MMA: the group's queries converted; block-scaled:
+                                           // the group's query scales in TMEM (4 warps)
+    uint64_t* sf_full = q_ready + 1;       // [S] block-scaled: the tile's key scales in TMEM (4 warps)
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(sf_full + S);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
-    static_assert((2 * S + 2 + 2 + 2 + 8 + 2) * 8 + 8 <= 256, "barrier block");
-    int32_t* prefix = reinterpret_cast<int32_t*>(reinterpret_cast<uint8_t*>(bars) + 256);
+    static_assert((3 * S + 2 + 2 + 2 + 8 + 2) * 8 + 8 <= C::kBarBytes, "barrier block");
+    int32_t* prefix = reinterpret_cast<int32_t*>(reinterpret_cast<uint8_t*>(bars) + C::kBarBytes);
     float* w_s = reinterpret_cast<float*>(prefix + C::kMaxGroups + 1);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -152,6 +168,7 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
         for (int i = 0; i < S; ++i) {
             tc::mbar_init(&full[i], kFp8 ? 128 : 1);
             tc::mbar_init(&empty[i], 1);
+            tc::mbar_init(&sf_full[i], 4);
         }
         for (int i = 0; i < 2; ++i) {
             tc::mbar_init(&acc_full[i], 1);
@@ -226,7 +243,7 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
                         tc::mbar_arrive_expect_tx(q_full, C::kQBytes);
                         const int32_t qrow = q_row0 + g * G * kHI;
                         tc::tma_load_2d(qbuf, &tmap_q, q_full, 0, qrow);
-                        tc::tma_load_2d(qbuf + N * 128, &tmap_q, q_full, 64, qrow);
+                        if (!kBs) tc::tma_load_2d(qbuf + N * 128, &tmap_q, q_full, 64, qrow);
                         gi = group_info(v, g, G, false);
                         cur = g;
                     }
@@ -239,7 +256,8 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
                     } else {
                         if (!tc::mbar_wait(&empty[stage], phase ^ 1, abort_flag)) break;
                     }
-                    tc::mbar_arrive_expect_tx(bar, (uint32_t)(n_boxes * box_rows * (kFp8 ? (kMx ? 132 : 128) : 256)));
+                    tc::mbar_arrive_expect_tx(
+                        bar, (uint32_t)(n_boxes * box_rows * (kFp8 ? (kMx ? 132 : 128) : kBs ? 132 : 256)));
                     for (int j = 0; j < n_boxes; ++j) {
                         const int s = s0 + j * box_rows;
                         const int32_t row = (int32_t)paged_slot(v, gi.b, s);
@@ -250,6 +268,12 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
                                 tc::bulk_load(kscl + (size_t)(stage & 3) * C::kScaleStageBytes + (size_t)j * box_rows * 4,
                                               static_cast<const uint8_t*>(k_scale) + (int64_t)row * 4,
                                               (uint32_t)box_rows * 4, bar);
+                        } else if (kBs) {   // codes straight into the MMA stage, scale words beside
+                            uint8_t* dst = tiles + (size_t)stage * C::kTile + (size_t)j * box_rows * 128;
+                            tc::tma_load_2d(dst, &tmap_k, bar, 0, row);
+                            tc::bulk_load(kscl + (size_t)stage * C::kScaleStageBytes + (size_t)j * box_rows * 4,
+                                          static_cast<const uint8_t*>(k_scale) + (int64_t)row * 4,
+                                          (uint32_t)box_rows * 4, bar);
                         } else {
                             uint8_t* dst = tiles + (size_t)stage * kTileBytes + (size_t)j * box_rows * 128;
                             tc::tma_load_2d(dst, &tmap_k, bar, 0, row);
@@ -275,20 +299,36 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
                     locate(prefix, n_groups, f, g, kt);
                     if (g != cur) {
                         if (!tc::mbar_wait(kF16 ? q_ready : q_full, q_phase, abort_flag)) break;
+                        if (kBs && !tc::mbar_wait(q_ready, q_phase, abort_flag)) break;
                         q_phase ^= 1;
                         cur = g;
                     }
                     if (!tc::mbar_wait(&full[stage], phase, abort_flag)) break;
+                    if (kBs && !tc::mbar_wait(&sf_full[stage], phase, abort_flag)) break;
                     if (!tc::mbar_wait(&acc_empty[acc], acc_phase ^ 1, abort_flag)) break;
                     tc::tc_fence_after();
-                    const uint32_t a_addr = tc::smem_u32(tiles + (size_t)stage * kTileBytes);
+                    const uint32_t a_addr = tc::smem_u32(tiles + (size_t)stage * C::kTile);
                     const uint32_t d = tmem_base + acc * N;
+                    if (kBs) {
+                        // four K = 32 steps through the 128-byte code rows; step k reads byte k
+                        // of every key's and query row's scale word
 #pragma unroll
-                    for (int k = 0; k < kDI / 16; ++k) {
-                        const uint32_t koff = (uint32_t)((k >> 2) * kHalfBytes + (k & 3) * 32);
-                        const uint32_t qoff = (uint32_t)((k >> 2) * (N * 128) + (k & 3) * 32);
-                        tc::mma_bf16(d, tc::sw128_desc(a_addr + koff, 16, 1024),
-                                     tc::sw128_desc(q_addr + qoff, 16, 1024), kIdesc, k > 0 ? 1u : 0u);
+                        for (int k = 0; k < kDI / 32; ++k) {
+                            const uint32_t sel = (uint32_t)k << 30;
+                            tc::mma_mxf8(d, tc::sw128_desc(a_addr + k * 32, 16, 1024),
+                                         tc::sw128_desc(q_addr + k * 32, 16, 1024),
+                                         tc::idesc_mxf8_f32(kBM, N, k, k),
+                                         (tmem_base + C::kSfaCol + 4 * stage) | sel,
+                                         (tmem_base + C::kSfbCol) | sel, k > 0 ? 1u : 0u);
+                        }
+                    } else {
+#pragma unroll
+                        for (int k = 0; k < kDI / 16; ++k) {
+                            const uint32_t koff = (uint32_t)((k >> 2) * kHalfBytes + (k & 3) * 32);
+                            const uint32_t qoff = (uint32_t)((k >> 2) * (N * 128) + (k & 3) * 32);
+                            tc::mma_bf16(d, tc::sw128_desc(a_addr + koff, 16, 1024),
+                                         tc::sw128_desc(q_addr + qoff, 16, 1024), kIdesc, k > 0 ? 1u : 0u);
+                        }
                     }
                     tc::mma_commit(&empty[stage]);
                     tc::mma_commit(&acc_full[acc]);
@@ -369,6 +409,20 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
                             w_s[i] = t < v.T_q ? w[(int64_t)t * kHI + (i % kHI)] : 0.f;
                         }
                     }
+                    if (kBs) {
+                        // the group's query scale words into TMEM: column c, lane l holds query
+                        // row (x head) 32c + l; each warp writes the copy in its own lane quarter
+                        uint32_t qs[N / 32];
+#pragma unroll
+                        for (int c = 0; c < N / 32; ++c) {
+                            const int i = 32 * c + lane;
+                            qs[c] = g * G + i / kHI < v.T_q ? __ldg(q_scale + q_row0 + (int64_t)g * N + i) : 0u;
+                        }
+                        const uint32_t ta = tmem_base + ((uint32_t)(quarter * 32) << 16) + C::kSfbCol;
+                        if constexpr (N == 64) tc::tmem_st2_u(ta, qs[0], qs[1]);
+                        else tc::tmem_st4_u(ta, qs[0], qs[1], qs[2], qs[3]);
+                        tc::tc_fence_before();
+                    }
                     const GroupInfo gi = group_info(v, g, G, false);
                     seq_b = gi.b < 0 ? 0 : gi.b;
 #pragma unroll
@@ -381,7 +435,7 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
                         }
                     }
                     if (!epi_sync.sync(abort_flag)) break;   // the new weights are in place
-                    if (kF16 && lane == 0) tc::mbar_arrive(q_ready);
+                    if ((kF16 || kBs) && lane == 0) tc::mbar_arrive(q_ready);
                     cur = g;
                 }
                 if (!tc::mbar_wait(&acc_full[acc], acc_phase, abort_flag)) break;
@@ -425,6 +479,25 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
                 if (lane == 0) tc::mbar_arrive(&acc_empty[acc]);
                 acc ^= 1;
                 if (acc == 0) acc_phase ^= 1;
+            }
+        } else if (kBs) {
+            // ------------------------------------------------------------ key scales -> TMEM
+            // warp 6 + i fills TMEM lane quarter (6 + i) % 4: column 4 x stage + c, lane l holds
+            // the scale word of key 32c + l of the stage's tile (every quarter holds a copy)
+            const int quarter = warp & 3;
+            uint32_t stage = 0, phase = 0;
+            for (int64_t f = f_begin; f < f_end; ++f) {
+                if (!tc::mbar_wait(&full[stage], phase, abort_flag)) break;
+                const uint32_t* wsc = reinterpret_cast<const uint32_t*>(kscl + (size_t)stage * C::kScaleStageBytes);
+                tc::tmem_st4_u(tmem_base + ((uint32_t)(quarter * 32) << 16) + C::kSfaCol + 4 * stage,
+                               wsc[lane], wsc[32 + lane], wsc[64 + lane], wsc[96 + lane]);
+                tc::tc_fence_before();
+                __syncwarp();
+                if (lane == 0) tc::mbar_arrive(&sf_full[stage]);
+                if (++stage == (uint32_t)S) {
+                    stage = 0;
+                    phase ^= 1;
+                }
             }
         } else if (kFp8) {
             // ------------------------------------------------------------ FP8 -> bf16 converters
@@ -523,21 +596,29 @@ int num_sms() {
     return n;
 }
 
-template <int G, bool kFp8, bool kMx>
+template <int G, bool kFp8, bool kMx, bool kBs = false>
 cudaError_t launch_g(const IndexScoreArgs& a, cudaStream_t st) {
-    using C = Cfg<G, kFp8, kMx>;
+    using C = Cfg<G, kFp8, kMx, kBs>;
     const int box_rows = a.seq.page_size <= kBM ? a.seq.page_size : kBM;
     const uint64_t slots = (uint64_t)a.seq.num_pages * a.seq.page_size;
     CUtensorMap tk, tq;
-    bool ok = kFp8 ? make_tensor_map_2d(&tk, a.k_cache, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, slots, kDI,
-                                        kDI, kDI, box_rows, CU_TENSOR_MAP_SWIZZLE_NONE)
-                   : make_tensor_map_2d(&tk, a.k_cache, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, slots,
-                                        kDI, kDI * 2, 64, box_rows, CU_TENSOR_MAP_SWIZZLE_128B);
-    ok = ok && make_tensor_map_2d(&tq, a.q_I, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
-                                  (uint64_t)a.seq.T_q * kHI, kDI, kDI * 2, 64, C::N,
-                                  CU_TENSOR_MAP_SWIZZLE_128B);
+    bool ok;
+    if (kBs) {   // one 128-byte swizzled box per code row, for the keys and the queries
+        ok = make_tensor_map_2d(&tk, a.k_cache, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, slots, kDI, kDI,
+                                kDI, box_rows, CU_TENSOR_MAP_SWIZZLE_128B) &&
+             make_tensor_map_2d(&tq, a.q_I, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)a.seq.T_q * kHI,
+                                kDI, kDI, kDI, C::N, CU_TENSOR_MAP_SWIZZLE_128B);
+    } else {
+        ok = kFp8 ? make_tensor_map_2d(&tk, a.k_cache, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, slots, kDI,
+                                       kDI, kDI, box_rows, CU_TENSOR_MAP_SWIZZLE_NONE)
+                  : make_tensor_map_2d(&tk, a.k_cache, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, slots,
+                                       kDI, kDI * 2, 64, box_rows, CU_TENSOR_MAP_SWIZZLE_128B);
+        ok = ok && make_tensor_map_2d(&tq, a.q_I, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                                      (uint64_t)a.seq.T_q * kHI, kDI, kDI * 2, 64, C::N,
+                                      CU_TENSOR_MAP_SWIZZLE_128B);
+    }
     if (!ok) return cudaErrorInvalidValue;
-    auto kern = index_score_tc_kernel<G, kFp8, kMx>;
+    auto kern = index_score_tc_kernel<G, kFp8, kMx, kBs>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::kSmem);
     if (e != cudaSuccess) return e;
     const int rows_per_launch = C::kMaxGroups * G;
@@ -549,7 +630,8 @@ cudaError_t launch_g(const IndexScoreArgs& a, cudaStream_t st) {
         const int64_t groups = ceil_div(v.T_q, G);
         const int grid = (int)std::min<int64_t>(num_sms(), std::max<int64_t>(1, groups * 64));
         e = launch_pdl(kern, dim3(grid), dim3(C::kThreads), C::kSmem, st, tk, tq, v, t0 * kHI,
-                       a.w + (int64_t)t0 * kHI, a.k_scale, a.scores + (int64_t)t0 * a.ld, a.ld, box_rows);
+                       a.w + (int64_t)t0 * kHI, a.k_scale, static_cast<const uint32_t*>(a.q_scale),
+                       a.scores + (int64_t)t0 * a.ld, a.ld, box_rows);
         if (e == cudaSuccess) e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
@@ -559,9 +641,13 @@ cudaError_t launch_g(const IndexScoreArgs& a, cudaStream_t st) {
 }  // namespace
 
 bool index_score_tc_supported(const IndexScoreArgs& a) {
-    if (a.q_dtype != HSA_BF16 ||
-        (a.k_dtype != HSA_BF16 && a.k_dtype != HSA_E4M3 && a.k_dtype != HSA_MXE4M3))
+    if (a.q_dtype == HSA_MXE4M3) {   // block-scaled MMA: MXFP8 queries need MXFP8 keys
+        if (a.k_dtype != HSA_MXE4M3 || a.q_scale == nullptr || (reinterpret_cast<uintptr_t>(a.q_scale) & 15))
+            return false;
+    } else if (a.q_dtype != HSA_BF16 ||
+               (a.k_dtype != HSA_BF16 && a.k_dtype != HSA_E4M3 && a.k_dtype != HSA_MXE4M3)) {
         return false;
+    }
     if ((a.k_dtype == HSA_E4M3 || a.k_dtype == HSA_MXE4M3) && a.k_scale == nullptr) return false;
     if (a.k_dtype == HSA_MXE4M3 && (reinterpret_cast<uintptr_t>(a.k_scale) & 15)) return false;
     if (a.H_I != kHI || a.D_I != kDI) return false;
@@ -575,6 +661,8 @@ bool index_score_tc_supported(const IndexScoreArgs& a) {
 
 cudaError_t launch_index_score_tc(const IndexScoreArgs& a, cudaStream_t st) {
     const bool fp8 = a.k_dtype == HSA_E4M3, mx = a.k_dtype == HSA_MXE4M3;
+    if (a.q_dtype == HSA_MXE4M3)   // two query rows per tile at most (TMEM holds the scales too)
+        return a.q_run % 2 == 0 ? launch_g<2, false, false, true>(a, st) : launch_g<1, false, false, true>(a, st);
     if (a.q_run % 4 == 0)
         return mx ? launch_g<4, true, true>(a, st) : fp8 ? launch_g<4, true, false>(a, st) : launch_g<4, false, false>(a, st);
     if (a.q_run % 2 == 0)

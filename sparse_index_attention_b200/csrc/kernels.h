@@ -14,7 +14,8 @@ struct IndexScoreArgs {
     int32_t max_seq_len;
     int32_t q_run;
     const void* q_I;
-    hsa_dtype_t q_dtype;
+    hsa_dtype_t q_dtype;   // F32, BF16, or MXE4M3 (codes, with q_scale)
+    const void* q_scale;   // MXE4M3 queries: E8M0 bytes, D_I / 32 per (row, head); else NULL
     const float* w;
     int32_t H_I, D_I;
     const void* k_cache;

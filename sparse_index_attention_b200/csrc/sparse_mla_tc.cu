@@ -47,16 +47,7 @@
 // Warp roles: 0-3 producers (slot window + gather; warp w owns rows 16w..16w+15 of every tile),
 // 4 MMA issuer, 5-12 softmax / epilogue (two threads per head h = TMEM lane h, 32 columns each;
 // warps w and w + 4 share heads and swap tile maxima through a two-warp barrier), 13-16 senders
-// (partial S to the peer).
-//
-// Schedule.  Persistent clusters.  With many query rows each cluster takes whole rows (cluster,
-// cluster + n_clusters, ...).  With few rows (a decode batch: 64 rows would leave 10 of the 74
-// clusters idle, 128 rows run 1.73 waves) the (row, tile) pairs of all rows are laid end to end
-// and each cluster takes one contiguous range of them (stream-K), so every cluster gets the
-// same number of tiles.  A row cut between clusters is finished by log-sum-exp: each part
-// writes its normalised partial output (bf16), its running maximum and its softmax sum to the
-// workspace and increments the row's counter; the part that increments last merges all parts,
-// writes the row and resets the counter.  No cluster ever waits for another.
+// (partial S to the peer).  Persistent: each cluster loops over query rows.
 #include <algorithm>
 
 #include "kernels.h"
@@ -89,10 +80,7 @@ constexpr int kOffBars = kOffXsum + 4 * 256;
 constexpr int kKvRowBytes = kDqk * 2;   // 1152: bf16 latent ‖ rope
 constexpr int kKv8RowBytes = kDv;       // 512: e4m3 latent codes (FP8 cache)
 constexpr int kRopeRowBytes = 128;      // bf16 rope of the FP8 cache
-constexpr int kMaxSplitRows = 256;          // rows up to which the stream-K schedule is used
-constexpr int kMinSplitTiles = 8;           // at least this many tiles per cluster in that mode
-constexpr int kOffSched = kOffBars + 256;   // [kMaxSplitRows + 1] prefix of tiles per row, flag
-constexpr size_t kSmem = 1024 + kOffSched + 4 * (kMaxSplitRows + 2);
+constexpr size_t kSmem = 1024 + kOffBars + 256;
 static_assert(kSmem <= 232448, "shared memory budget");
 static_assert(kOffStages % 1024 == 0 && kStageBytes % 1024 == 0 && kOffRecv % 1024 == 0, "swizzle alignment");
 
@@ -117,7 +105,6 @@ struct Bars {
     uint64_t recv_full[2];
     uint64_t o_ready, o_free;
     uint64_t pair_sync[4];  // the two softmax warps of a head quarter (maxima / row sums posted)
-    uint64_t epi_sync;      // the eight softmax warps (a split row's partial written / merged)
     uint32_t tmem;
     int abort;
 };
@@ -141,73 +128,6 @@ __device__ __forceinline__ int row_tiles(const SeqView& v, const int32_t* __rest
     return (int)ceil_div(row_extent(idx + (int64_t)t * K, K, lane), kBN);
 }
 
-// One segment of a cluster's work: tiles [j0, j1) of query row t, which has ntiles tiles.
-struct Seg {
-    int t, j0, j1, ntiles;
-};
-
-// The cluster's segments in order.  Row mode: rows cluster, cluster + n_clusters, ... (rows with
-// no tiles are skipped).  Split mode: units [u0, u1) of the rows laid end to end, prefix[t] being
-// the first unit of row t (prefix[T_q] = total).
-struct Sched {
-    bool split;
-    int cluster, n_clusters, T_q;
-    const int32_t* prefix;
-    int u0, u1;   // at most 256 rows x 1024 tiles
-    // cursor
-    int t, u;
-
-    __device__ __forceinline__ void begin() {
-        if (split) {
-            u = u0;
-            t = 0;
-        } else {
-            t = cluster;
-        }
-    }
-    // next segment; row mode calls row_tiles (warp-wide)
-    __device__ __forceinline__ bool next(Seg& sg, const SeqView& v, const int32_t* __restrict__ idx,
-                                         int K, int lane, RowInfo& r) {
-        if (split) {
-            if (u >= u1) return false;
-            while (prefix[t + 1] <= u) ++t;
-            sg.t = t;
-            sg.ntiles = prefix[t + 1] - prefix[t];
-            sg.j0 = u - prefix[t];
-            sg.j1 = min(sg.ntiles, u1 - prefix[t]);
-            u = prefix[t] + sg.j1;
-            r = load_row(v, t);
-            return true;
-        }
-        for (; t < T_q; t += n_clusters) {
-            const int nt = row_tiles(v, idx, K, t, lane, r);
-            if (nt > 0) {
-                sg.t = t;
-                sg.ntiles = nt;
-                sg.j0 = 0;
-                sg.j1 = nt;
-                t += n_clusters;
-                return true;
-            }
-        }
-        return false;
-    }
-};
-
-// Cluster owning unit u when `units` units are cut into `clusters` ranges [c*units/clusters, ...).
-__device__ __forceinline__ int unit_owner(int u, int units, int clusters) {
-    return (int)(((int64_t)(u + 1) * clusters - 1) / units);
-}
-
-// Workspace of the split schedule: row counters, then one partial per (cluster, first / last
-// segment, CTA rank): bf16 output [32 chunks of 8 dims][128 heads] (this CTA's 256 dims) and
-// fp32 running maximum (log2 units) and sum per head.
-constexpr size_t kPartOBytes = 256 * kH * 2;
-constexpr size_t kPartBytes = kPartOBytes + 2 * kH * 4;
-__host__ __device__ constexpr size_t split_counter_bytes(int T_q) {
-    return ((size_t)T_q * 2 * 4 + 255) / 256 * 256;
-}
-
 // kFp8Kv: the latent part of the cache is e4m3 codes with one fp32 scale per row and the rope part
 // a separate bf16 array; the producers widen code x scale to bf16 on the way into the stage.
 template <bool kFp8Kv>
@@ -216,8 +136,7 @@ sparse_mla_tc_kernel(SeqView v,
                      const __nv_bfloat16* __restrict__ q, const uint8_t* __restrict__ kv_bytes,
                      const float* __restrict__ kv_scale, int kv_group, const uint8_t* __restrict__ rope_bytes,
                      int64_t rope_row_bytes, const int32_t* __restrict__ idx, int K,
-                     float scale_log2, __nv_bfloat16* __restrict__ out, float* __restrict__ lse,
-                     int split_clusters, uint8_t* __restrict__ ws) {
+                     float scale_log2, __nv_bfloat16* __restrict__ out, float* __restrict__ lse) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* q_rope = base;
@@ -229,8 +148,6 @@ sparse_mla_tc_kernel(SeqView v,
     float* xsum = reinterpret_cast<float*>(base + kOffXsum);
     Bars* bars = reinterpret_cast<Bars*>(base + kOffBars);
     volatile int* abort_flag = &bars->abort;
-    int32_t* prefix = reinterpret_cast<int32_t*>(base + kOffSched);
-    volatile int32_t* merge_flag = prefix + kMaxSplitRows + 1;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const uint32_t rank = tc::cluster_ctarank();
@@ -259,7 +176,6 @@ sparse_mla_tc_kernel(SeqView v,
         tc::mbar_init(&bars->o_ready, 1);
         tc::mbar_init(&bars->o_free, 8);
         for (int i = 0; i < 4; ++i) tc::mbar_init(&bars->pair_sync[i], 2);
-        tc::mbar_init(&bars->epi_sync, 8);
         bars->abort = 0;
         tc::fence_barrier_init();
     }
@@ -272,54 +188,8 @@ sparse_mla_tc_kernel(SeqView v,
     tc::cluster_sync_all();  // the peer's barriers exist before anything remote touches them
     tc::tc_fence_after();
     const uint32_t tmem_base = bars->tmem;
-    pdl_wait();              // the selection and the row descriptors may be earlier kernels' output
+    pdl_wait();              // the selection is the previous kernel's output
     pdl_trigger();
-
-    // the schedule: split mode when the launch asked for it (few rows, workspace given)
-    Sched sched;
-    sched.split = split_clusters > 0;
-    sched.cluster = cluster;
-    sched.n_clusters = n_clusters;
-    sched.T_q = v.T_q;
-    sched.prefix = prefix;
-    sched.u0 = sched.u1 = 0;
-    int units = 0;
-    if (sched.split) {
-        // tiles of every row (warps 0-3, warp-wide scans), then the prefix (warp 0)
-        if (warp < 4) {
-            for (int t = warp; t < v.T_q; t += 4) {
-                RowInfo r;
-                const int nt = row_tiles(v, idx, K, t, lane, r);
-                if (lane == 0) prefix[t + 1] = nt;
-            }
-        }
-        __syncthreads();
-        if (warp == 0) {
-            int32_t carry = 0;
-            for (int t0 = 0; t0 < v.T_q; t0 += 32) {
-                const int t = t0 + lane;
-                const int32_t x = t < v.T_q ? prefix[t + 1] : 0;
-                int32_t incl = x;
-#pragma unroll
-                for (int o = 1; o < 32; o <<= 1) {
-                    const int32_t y = __shfl_up_sync(0xffffffffu, incl, o);
-                    if (lane >= o) incl += y;
-                }
-                __syncwarp();
-                if (t < v.T_q) prefix[t + 1] = carry + incl;
-                carry += __shfl_sync(0xffffffffu, incl, 31);
-            }
-            if (lane == 0) prefix[0] = 0;
-        }
-        __syncthreads();
-        units = prefix[v.T_q];
-        // clusters beyond split_clusters get no units
-        if (cluster < split_clusters) {
-            sched.u0 = (int)((int64_t)units * cluster / split_clusters);
-            sched.u1 = (int)((int64_t)units * (cluster + 1) / split_clusters);
-        }
-    }
-    sched.begin();
 
     if (warp < 4) {
         // ---------------------------------------------------------------- producers (gather)
@@ -327,12 +197,13 @@ sparse_mla_tc_kernel(SeqView v,
         uint16_t* masks16 = reinterpret_cast<uint16_t*>(const_cast<uint64_t*>(masks));
         uint32_t n = 0;
         bool stop = false;
-        Seg sg;
-        RowInfo r;
-        while (!stop && sched.next(sg, v, idx, K, lane, r)) {
-            const int32_t* idx_row = idx + (int64_t)sg.t * K;
-            for (int j = sg.j0; j < sg.j1; ++j, ++n) {
-                if ((j - sg.j0) % (kSlotWin / kBN) == 0) {
+        for (int t = cluster; t < v.T_q && !stop; t += n_clusters) {
+            RowInfo r;
+            const int ntiles = row_tiles(v, idx, K, t, lane, r);
+            if (ntiles == 0) continue;
+            const int32_t* idx_row = idx + (int64_t)t * K;
+            for (int j = 0; j < ntiles; ++j, ++n) {
+                if (j % (kSlotWin / kBN) == 0) {
                     // physical slots of this warp's rows for the next 32 tiles (-1: none), eight
                     // independent lookups per lane in flight at a time
 #pragma unroll 1
@@ -359,7 +230,7 @@ sparse_mla_tc_kernel(SeqView v,
                     stop = true;
                     break;
                 }
-                const int32_t* ts = my_slots + ((j - sg.j0) % (kSlotWin / kBN)) * 16;
+                const int32_t* ts = my_slots + (j % (kSlotWin / kBN)) * 16;
                 uint8_t* sbase = stages + st * kStageBytes;
                 if (!kFp8Kv) {
                     // latent half: one row per warp instruction, lane = 16-byte chunk
@@ -458,12 +329,13 @@ sparse_mla_tc_kernel(SeqView v,
             __syncwarp();
             return true;
         };
-        Seg sg;
-        RowInfo r;
-        while (!stop && sched.next(sg, v, idx, K, lane, r)) {
+        for (int t = cluster; t < v.T_q && !stop; t += n_clusters) {
+            RowInfo r;
+            const int ntiles = row_tiles(v, idx, K, t, lane, r);
+            if (ntiles == 0) continue;
             if (!tc::mbar_wait(&bars->q_full, qr & 1, abort_flag)) break;
             ++qr;
-            for (int j = sg.j0; j < sg.j1; ++j, ++n) {
+            for (int j = 0; j < ntiles; ++j, ++n) {
                 const uint32_t st = n % kStages, sb = n & 1;
                 if (!tc::mbar_wait(&bars->kv_full[st], (n / kStages) & 1, abort_flag) ||
                     !tc::mbar_wait(&bars->s_empty[sb], ((n >> 1) & 1) ^ 1, abort_flag)) {
@@ -485,15 +357,15 @@ sparse_mla_tc_kernel(SeqView v,
                         tc::mma_bf16(d, tc::sw64_desc(qr_addr + kk * 32, 512),
                                      tc::sw64_desc(kv_addr + 4 * kKvBlk + kk * 32, 512), kIdescQK, 1u);
                     tc::mma_commit(&bars->s_full[sb]);
-                    if (j == sg.j1 - 1) tc::mma_commit(&bars->q_empty);
+                    if (j == ntiles - 1) tc::mma_commit(&bars->q_empty);
                 }
                 __syncwarp();
-                if (j > sg.j0 && !pv(n - 1, j == sg.j0 + 1)) {
+                if (j > 0 && !pv(n - 1, j == 1)) {
                     stop = true;
                     break;
                 }
             }
-            if (stop || !pv(n - 1, sg.j1 - sg.j0 == 1)) break;
+            if (stop || !pv(n - 1, ntiles == 1)) break;
             if (lane == 0) tc::mma_commit(&bars->o_ready);
             __syncwarp();
             ++rows_done;
@@ -512,39 +384,18 @@ sparse_mla_tc_kernel(SeqView v,
         bool stop = false;
         tc::WarpSetSync pair_sync{&bars->pair_sync[(warp - 5) & 3], 0};   // warps w and w + 4
 
-        tc::WarpSetSync epi_sync{&bars->epi_sync, 0};                       // warps 5-12
-        // a row without any selection: output 0, lse -inf
-        auto zero_row = [&](int t) {
-            __nv_bfloat16* orow = out + ((int64_t)t * kH + h) * kDv + 256 * rank + 128 * half;
-            for (int c = 0; c < 128; c += 8) *reinterpret_cast<uint4*>(orow + c) = make_uint4(0, 0, 0, 0);
-            if (lse != nullptr && rank == 0 && half == 0) lse[(int64_t)t * kH + h] = -INFINITY;
-        };
-        // the next segment; in row mode the empty rows skipped on the way are written here, in
-        // split mode each empty row is written by the cluster whose unit range holds its place
-        auto next_seg = [&](Seg& sg) -> bool {
-            RowInfo r;
-            if (sched.split) return sched.next(sg, v, idx, K, lane, r);
-            for (; sched.t < v.T_q; sched.t += n_clusters) {
-                const int nt = row_tiles(v, idx, K, sched.t, lane, r);
-                if (nt > 0) {
-                    sg.t = sched.t;
-                    sg.j0 = 0;
-                    sg.j1 = sg.ntiles = nt;
-                    sched.t += n_clusters;
-                    return true;
-                }
-                zero_row(sched.t);
+        // next row (t0, t0 + n_clusters, ...) with work; rows without any selection are written
+        // here directly (output 0, lse -inf)
+        auto next_row = [&](int t0, int& ntiles, RowInfo& r) -> int {
+            for (int t = t0; t < v.T_q; t += n_clusters) {
+                ntiles = row_tiles(v, idx, K, t, lane, r);
+                if (ntiles > 0) return t;
+                __nv_bfloat16* orow = out + ((int64_t)t * kH + h) * kDv + 256 * rank + 128 * half;
+                for (int c = 0; c < 128; c += 8) *reinterpret_cast<uint4*>(orow + c) = make_uint4(0, 0, 0, 0);
+                if (lse != nullptr && rank == 0 && half == 0) lse[(int64_t)t * kH + h] = -INFINITY;
             }
-            return false;
+            return -1;
         };
-        if (sched.split && cluster < split_clusters) {
-            for (int t = 0; t < v.T_q; ++t) {
-                if (prefix[t + 1] != prefix[t]) continue;
-                const int pos = prefix[t];
-                if ((pos >= sched.u0 && pos < sched.u1) || (pos == units && cluster == split_clusters - 1))
-                    zero_row(t);
-            }
-        }
         // Q row t: this CTA's 256 latent dims into TMEM (lane h, columns 384.. as bf16 pairs) and
         // its 32 rope dims into shared memory (64-byte swizzle: chunk c of row h at c ^ ((h>>1)&3));
         // each of the two threads of a head moves half of it
@@ -573,15 +424,15 @@ sparse_mla_tc_kernel(SeqView v,
             __syncwarp();
             if (lane == 0) tc::mbar_arrive(&bars->q_full);
         };
-        Seg sg;
-        bool have = next_seg(sg);
-        if (have) load_q(sg.t);
-        while (have && !stop) {
+        int ntiles = 0;
+        RowInfo r;
+        int t = next_row(cluster, ntiles, r);
+        if (t >= 0) load_q(t);
+        while (t >= 0 && !stop) {
             float m_used = -INFINITY, l = 0.f;
-            Seg sg_next;
-            bool have_next = false;
-            const int t = sg.t;
-            for (int j = sg.j0; j < sg.j1; ++j, ++n) {
+            int t_next = -1, ntiles_next = 0;
+            RowInfo r_next;
+            for (int j = 0; j < ntiles; ++j, ++n) {
                 const uint32_t b = n & 1, st = n % kStages;
                 // ---- softmax(n), columns [col, col + 32)
                 // own partial S(n) is complete once the senders have read it (s_sent), which
@@ -676,16 +527,16 @@ sparse_mla_tc_kernel(SeqView v,
                 tc::tc_fence_before();
                 __syncwarp();
                 if (lane == 0) tc::mbar_arrive(&bars->p_full);
-                // ---- last tile of the segment: put the next segment's Q in place
-                if (j + 1 == sg.j1) {
-                    have_next = next_seg(sg_next);
-                    if (have_next) {
+                // ---- last tile of the row: put the next row's Q in place
+                if (j + 1 == ntiles) {
+                    t_next = next_row(t + n_clusters, ntiles_next, r_next);
+                    if (t_next >= 0) {
                         if (!tc::mbar_wait(&bars->q_empty, rows_done & 1, abort_flag)) {
                             stop = true;
                             break;
                         }
                         tc::tc_fence_after();
-                        load_q(sg_next.t);
+                        load_q(t_next);
                     }
                 }
             }
@@ -695,123 +546,33 @@ sparse_mla_tc_kernel(SeqView v,
             if (!tc::mbar_wait(&bars->o_ready, rows_done & 1, abort_flag) || !pair_sync.sync(abort_flag)) break;
             tc::tc_fence_after();
             const float l_all = l + xsum[(half ^ 1) * 128 + h];
+            __nv_bfloat16* orow = out + ((int64_t)t * kH + h) * kDv + 256 * rank + 128 * half;
             const float inv_l = l_all > 0.f ? 1.f / l_all : 0.f;
-            if (sg.j0 == 0 && sg.j1 == sg.ntiles) {
-                // the whole row: O / l -> bf16 -> the output row
-                __nv_bfloat16* orow = out + ((int64_t)t * kH + h) * kDv + 256 * rank + 128 * half;
 #pragma unroll 1
-                for (int c = 0; c < 128; c += 32) {
-                    float o[32];
-                    tc::tmem_ld32(tmem_base + lane_off + kTmemO + 128 * half + c, o);
-                    tc::tmem_ld_wait();
+            for (int c = 0; c < 128; c += 32) {
+                float o[32];
+                tc::tmem_ld32(tmem_base + lane_off + kTmemO + 128 * half + c, o);
+                tc::tmem_ld_wait();
 #pragma unroll
-                    for (int i = 0; i < 32; i += 8) {
-                        uint32_t w4[4];
+                for (int i = 0; i < 32; i += 8) {
+                    uint32_t w4[4];
 #pragma unroll
-                        for (int qq = 0; qq < 4; ++qq) {
-                            const __nv_bfloat162 b2 = __floats2bfloat162_rn(o[i + 2 * qq] * inv_l, o[i + 2 * qq + 1] * inv_l);
-                            w4[qq] = *reinterpret_cast<const uint32_t*>(&b2);
-                        }
-                        *reinterpret_cast<uint4*>(orow + c + i) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+                    for (int qq = 0; qq < 4; ++qq) {
+                        const __nv_bfloat162 b2 = __floats2bfloat162_rn(o[i + 2 * qq] * inv_l, o[i + 2 * qq + 1] * inv_l);
+                        w4[qq] = *reinterpret_cast<const uint32_t*>(&b2);
                     }
-                }
-                tc::tc_fence_before();
-                __syncwarp();
-                if (lane == 0) tc::mbar_arrive(&bars->o_free);
-                if (lse != nullptr && rank == 0 && half == 0)
-                    lse[(int64_t)t * kH + h] = l_all > 0.f ? (m_used + log2f(l_all)) * 0.69314718055994531f : -INFINITY;
-            } else {
-                // a part of a row cut between clusters: its normalised output (bf16), running
-                // maximum and sum go to this cluster's partial slot (first or last segment)
-                const int slot = 2 * cluster + (sched.u0 >= prefix[t] ? 0 : 1);
-                uint8_t* part = ws + split_counter_bytes(v.T_q) + ((size_t)slot * 2 + rank) * kPartBytes;
-                uint4* po = reinterpret_cast<uint4*>(part);              // [32 chunks][128 heads]
-                float* pml = reinterpret_cast<float*>(part + kPartOBytes);  // m [128], l [128]
-#pragma unroll 1
-                for (int c = 0; c < 128; c += 32) {
-                    float o[32];
-                    tc::tmem_ld32(tmem_base + lane_off + kTmemO + 128 * half + c, o);
-                    tc::tmem_ld_wait();
-#pragma unroll
-                    for (int i = 0; i < 32; i += 8) {
-                        uint32_t w4[4];
-#pragma unroll
-                        for (int qq = 0; qq < 4; ++qq) {
-                            const __nv_bfloat162 b2 = __floats2bfloat162_rn(o[i + 2 * qq] * inv_l, o[i + 2 * qq + 1] * inv_l);
-                            w4[qq] = *reinterpret_cast<const uint32_t*>(&b2);
-                        }
-                        po[((128 * half + c + i) / 8) * kH + h] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
-                    }
-                }
-                if (half == 0) {
-                    pml[h] = m_used;
-                    pml[kH + h] = l_all;
-                }
-                tc::tc_fence_before();
-                __syncwarp();
-                if (lane == 0) tc::mbar_arrive(&bars->o_free);
-                // every softmax warp has written its share; the last part to arrive merges
-                __threadfence();
-                if (!epi_sync.sync(abort_flag)) break;
-                const int c0 = unit_owner(prefix[t], units, split_clusters);
-                const int c1 = unit_owner(prefix[t] + sg.ntiles - 1, units, split_clusters);
-                int* cnt = reinterpret_cast<int*>(ws) + 2 * t + rank;
-                if (warp == 5 && lane == 0) *merge_flag = atomicAdd(cnt, 1) == c1 - c0 ? 1 : 0;
-                if (!epi_sync.sync(abort_flag)) break;
-                if (*merge_flag) {
-                    __threadfence();
-                    float mx = -INFINITY;
-                    for (int pc = c0; pc <= c1; ++pc) {
-                        const int ps = 2 * pc + ((int)((int64_t)units * pc / split_clusters) >= prefix[t] ? 0 : 1);
-                        const float* ml = reinterpret_cast<const float*>(
-                            ws + split_counter_bytes(v.T_q) + ((size_t)ps * 2 + rank) * kPartBytes + kPartOBytes);
-                        mx = fmaxf(mx, __ldcg(ml + h));
-                    }
-                    // weight of part p: l_p 2^(m_p - max); output = sum_p weight_p o_p / sum_p weight_p
-                    auto part_of = [&](int pc) -> const uint8_t* {
-                        const int ps = 2 * pc + ((int)((int64_t)units * pc / split_clusters) >= prefix[t] ? 0 : 1);
-                        return ws + split_counter_bytes(v.T_q) + ((size_t)ps * 2 + rank) * kPartBytes;
-                    };
-                    auto weight_of = [&](const uint8_t* pp) -> float {
-                        const float* ml = reinterpret_cast<const float*>(pp + kPartOBytes);
-                        const float mp = __ldcg(ml + h), lp = __ldcg(ml + kH + h);
-                        return (mp == -INFINITY || !(lp > 0.f)) ? 0.f : lp * exp2f(mp - mx);
-                    };
-                    float L = 0.f;
-                    for (int pc = c0; pc <= c1; ++pc) L += weight_of(part_of(pc));
-                    const float invL = L > 0.f ? 1.f / L : 0.f;
-                    __nv_bfloat16* orow = out + ((int64_t)t * kH + h) * kDv + 256 * rank + 128 * half;
-#pragma unroll 1
-                    for (int i = 0; i < 16; ++i) {
-                        float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-                        for (int pc = c0; pc <= c1; ++pc) {
-                            const uint8_t* pp = part_of(pc);
-                            const float wgt = weight_of(pp);
-                            const uint4 x = __ldcg(reinterpret_cast<const uint4*>(pp) + (16 * half + i) * kH + h);
-                            const uint32_t wv[4] = {x.x, x.y, x.z, x.w};
-#pragma unroll
-                            for (int qq = 0; qq < 4; ++qq) {
-                                const float2 f2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&wv[qq]));
-                                acc[2 * qq] = fmaf(wgt, f2.x, acc[2 * qq]);
-                                acc[2 * qq + 1] = fmaf(wgt, f2.y, acc[2 * qq + 1]);
-                            }
-                        }
-                        uint32_t w4[4];
-#pragma unroll
-                        for (int qq = 0; qq < 4; ++qq) {
-                            const __nv_bfloat162 b2 = __floats2bfloat162_rn(acc[2 * qq] * invL, acc[2 * qq + 1] * invL);
-                            w4[qq] = *reinterpret_cast<const uint32_t*>(&b2);
-                        }
-                        *reinterpret_cast<uint4*>(orow + 8 * i) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
-                    }
-                    if (lse != nullptr && rank == 0 && half == 0)
-                        lse[(int64_t)t * kH + h] = L > 0.f ? (mx + log2f(L)) * 0.69314718055994531f : -INFINITY;
-                    if (warp == 5 && lane == 0) *cnt = 0;   // ready for the next launch
+                    *reinterpret_cast<uint4*>(orow + c + i) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
                 }
             }
+            tc::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(&bars->o_free);
+            if (lse != nullptr && rank == 0 && half == 0)
+                lse[(int64_t)t * kH + h] = l_all > 0.f ? (m_used + log2f(l_all)) * 0.69314718055994531f : -INFINITY;
             ++rows_done;
-            sg = sg_next;
-            have = have_next;
+            t = t_next;
+            ntiles = ntiles_next;
+            r = r_next;
         }
     } else {
         // ---------------------------------------------------------------- senders
@@ -827,10 +588,10 @@ sparse_mla_tc_kernel(SeqView v,
         }
         uint32_t m = 0;
         bool stop = false;
-        Seg sg;
-        RowInfo r;
-        while (!stop && sched.next(sg, v, idx, K, lane, r)) {
-            for (int j = sg.j0; j < sg.j1; ++j, ++m) {
+        for (int t = cluster; t < v.T_q && !stop; t += n_clusters) {
+            RowInfo r;
+            const int ntiles = row_tiles(v, idx, K, t, lane, r);
+            for (int j = 0; j < ntiles; ++j, ++m) {
                 const uint32_t b = m & 1;
                 if (!tc::mbar_wait(&bars->s_full[b], (m >> 1) & 1, abort_flag)) {
                     stop = true;
@@ -911,21 +672,7 @@ bool sparse_mla_tc_supported(const SparseMlaArgs& a) {
     return true;
 }
 
-namespace {
-// Clusters of the split (stream-K) schedule for T_q rows of at most ceil(K / 64) tiles each, 0
-// when the rows are too many for it (each cluster then takes whole rows).
-int split_clusters_for(int32_t T_q, int32_t K) {
-    if (T_q <= 0 || T_q > kMaxSplitRows) return 0;
-    const int64_t units = (int64_t)T_q * ceil_div(K, kBN);
-    return (int)std::max<int64_t>(1, std::min<int64_t>(num_sms() / 2, units / kMinSplitTiles));
-}
-}  // namespace
-
-size_t sparse_mla_tc_workspace(int32_t T_q, int32_t K) {
-    const int sc = split_clusters_for(T_q, K);
-    if (sc == 0) return 0;
-    return split_counter_bytes(T_q) + (size_t)sc * 2 * 2 * kPartBytes;
-}
+size_t sparse_mla_tc_workspace(int32_t, int32_t) { return 0; }
 
 cudaError_t launch_sparse_mla_tc(const SparseMlaArgs& a, cudaStream_t st) {
     if (a.seq.T_q == 0) return cudaSuccess;
@@ -933,10 +680,7 @@ cudaError_t launch_sparse_mla_tc(const SparseMlaArgs& a, cudaStream_t st) {
     auto kern = fp8 ? sparse_mla_tc_kernel<true> : sparse_mla_tc_kernel<false>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmem);
     if (e != cudaSuccess) return e;
-    // split schedule when the rows are few and the workspace it needs was given; else whole rows
-    int split = split_clusters_for(a.seq.T_q, a.K);
-    if (split > 0 && (a.ws == nullptr || a.ws_bytes < sparse_mla_tc_workspace(a.seq.T_q, a.K))) split = 0;
-    const int clusters = split > 0 ? split : std::max(1, std::min(a.seq.T_q, num_sms() / 2));
+    const int clusters = std::max(1, std::min(a.seq.T_q, num_sms() / 2));
     const float scale_log2 = a.softmax_scale * 1.4426950408889634f;
     const uint8_t* kv = reinterpret_cast<const uint8_t*>(a.kv);
     // the bf16 cache packs the rope dims after the latent ones in each 1152-byte row
@@ -945,8 +689,7 @@ cudaError_t launch_sparse_mla_tc(const SparseMlaArgs& a, cudaStream_t st) {
     e = launch_pdl(kern, dim3(2 * clusters), dim3(kThreads), kSmem, st, a.seq,
                    reinterpret_cast<const __nv_bfloat16*>(a.q), kv, fp8 ? a.kv_scale : nullptr,
                    fp8 ? a.kv_scale_group : kDv, rope, rope_row,
-                   a.idx, a.K, scale_log2, reinterpret_cast<__nv_bfloat16*>(a.out), a.lse, split,
-                   static_cast<uint8_t*>(a.ws));
+                   a.idx, a.K, scale_log2, reinterpret_cast<__nv_bfloat16*>(a.out), a.lse);
     return e != cudaSuccess ? e : cudaGetLastError();
 }
 

@@ -195,6 +195,46 @@ __host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N) {
            | ((uint32_t)(M >> 4) << 24); // M / 16
 }
 
+// Instruction descriptor for kind::mxf8f6f4 with block scaling: E4M3 A and B (both K-major),
+// fp32 D, E8M0 scale factors, one per 32 consecutive K elements.  One MMA covers K = 32, so it
+// reads one scale per row of A and one per row of B: byte a_sf (b_sf) of the 32-bit TMEM words
+// that hold the scales.
+__host__ __device__ constexpr uint32_t idesc_mxf8_f32(int M, int N, int a_sf, int b_sf) {
+    return ((uint32_t)b_sf << 4)          // B scale-factor byte
+                                          // A and B format 0: E4M3; both K-major
+           | ((uint32_t)(N >> 3) << 17)   // N / 8
+           | (1u << 23)                   // scale-factor format: E8M0
+           | ((uint32_t)(M >> 4) << 24)   // M / 16
+           | ((uint32_t)a_sf << 29);      // A scale-factor byte
+}
+
+// D[tmem] (+)= (A x 2^(SA - 127)) * (B x 2^(SB - 127))^T, kind::mxf8f6f4 block-scaled, one CTA.
+// sfa / sfb are TMEM addresses of the scale words (their top two bits repeat the byte the
+// instruction descriptor selects).
+__device__ __forceinline__ void mma_mxf8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                         uint32_t idesc, uint32_t sfa, uint32_t sfb,
+                                         uint32_t accumulate) {
+    asm volatile(
+        "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+        " tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n}\n" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+        : "memory");
+}
+
+// 32 lanes x 4 (x 2) columns of raw 32-bit words into TMEM (waits for the store).
+__device__ __forceinline__ void tmem_st4_u(uint32_t taddr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1, %2, %3, %4};\n"
+        "tcgen05.wait::st.sync.aligned;" ::"r"(taddr), "r"(a), "r"(b), "r"(c), "r"(d)
+        : "memory");
+}
+__device__ __forceinline__ void tmem_st2_u(uint32_t taddr, uint32_t a, uint32_t b) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x2.b32 [%0], {%1, %2};\n"
+        "tcgen05.wait::st.sync.aligned;" ::"r"(taddr), "r"(a), "r"(b)
+        : "memory");
+}
+
 // Shared memory matrix descriptor, 128-byte swizzle.  `lbo` / `sbo` in bytes: for a K-major
 // operand sbo is the distance between groups of 8 rows (1024 for densely packed 128-byte rows)
 // and lbo is unused; for an MN-major operand lbo is the distance between 64-element column

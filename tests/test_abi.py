@@ -51,6 +51,16 @@ def test_validation_without_gpu():
     rc = L.hsa_index_score(ctypes.byref(seq), fake, hsa.HSA_BF16, fake, 4, 32, fake, hsa.HSA_E4M3,
                            None, fake, 64, None)
     assert rc == hsa.HSA_ERR_INVALID_ARG                       # E4M3 keys without scales
+    rc = L.hsa_index_score(ctypes.byref(seq), fake, hsa.HSA_MXE4M3, fake, 4, 32, fake, hsa.HSA_MXE4M3,
+                           fake, fake, 64, None)
+    assert rc == hsa.HSA_ERR_INVALID_ARG                       # MX queries without their scales
+    rc = L.hsa_index_score_mx(ctypes.byref(seq), fake, None, fake, 4, 32, fake, fake, fake, 64, None)
+    assert rc == hsa.HSA_ERR_INVALID_ARG                       # q_scale NULL
+    rc = L.hsa_index_score_mx(ctypes.byref(seq), fake, ctypes.c_void_p(0x1004), fake, 4, 32, fake,
+                              fake, fake, 64, None)
+    assert rc == hsa.HSA_ERR_INVALID_ARG                       # q_scale not 16-byte aligned
+    rc = L.hsa_index_score_mx(ctypes.byref(seq), fake, fake, fake, 4, 48, fake, fake, fake, 64, None)
+    assert rc == hsa.HSA_ERR_INVALID_ARG                       # D_I not a multiple of 32
     rc = L.hsa_quantize_index(fake, hsa.HSA_BF16, 10, 128, 48, None, 10, fake, fake, None)
     assert rc == hsa.HSA_ERR_INVALID_ARG                       # group does not divide D
     # E4M3 latent cache: the scale group must be a multiple of 16 that divides D_v

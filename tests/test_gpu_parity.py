@@ -63,6 +63,80 @@ def test_index_score_mxfp8_vs_oracle(name, kw):
     _index_vs_oracle(wl)
 
 
+@pytest.mark.parametrize("name,kw", [
+    ("decode_bf16", dict(B=5, L_min=100, L_max=1500)),                   # one query row per tile
+    ("decode_draft_bf16", dict(B=4, n_draft=2, L_min=300, L_max=1400)),  # row pairs: two per tile
+    ("prefill_bf16", dict(T=700)),                                      # two rows per tile
+    ("prefill_bf16", dict(T=301)),                                      # odd run: one row per tile
+])
+def test_index_score_mx_block_scaled_vs_oracle(name, kw):
+    """MXFP8 queries and keys as codes + E8M0 scales (hsa_index_score_mx: the block-scaled MMA on
+    the codes), against the float64 score of the oracle's own MX quantization of both, and
+    against the bf16-query MX path on the same rounded queries."""
+    wl = workloads.make(name, DEV, **kw)
+    wl.index_fp8 = wl.index_mx = True
+    seq = paged_seq(wl)
+    k, ks = hsa.hsa_quantize_mx(wl.k_I)
+    qc, qs = hsa.hsa_quantize_mx(wl.q_I.reshape(-1, wl.D_I))
+    sc = hsa.hsa_index_score(seq, qc.view(wl.q_I.shape), wl.w, k, ks,
+                             q_scale=qs.view(wl.T_q, wl.H_I, wl.D_I // 32))
+    check_status(seq)
+    # the same scores through the bf16-query MX path (queries rounded onto the MX grid)
+    sc_bf = hsa.hsa_index_score(seq, hsa.mx_round(wl.q_I), wl.w, k, ks)
+    oc = OracleCaches(wl, need_kv=False)
+    rows = list(range(wl.T_q))
+    pg = oracle_paging(wl, rows)
+    ref = oracle.index_score(pg, oc.q_I, wl.w.cpu(), oc.k, ld=sc.shape[1])
+    mag = oracle.index_score(pg, oc.q_I, wl.w.cpu().abs(), oc.k, ld=sc.shape[1])
+    got, got_bf = sc.cpu().numpy(), sc_bf.cpu().numpy()
+    for t in rows:
+        n = int(wl.q_pos[t]) + 1
+        ok, worst = index_tolerance_ok(got[t, :n], ref[t, :n], mag[t, :n])
+        assert ok, (name, t, worst)
+        ok, worst = index_tolerance_ok(got[t, :n], got_bf[t, :n], mag[t, :n])
+        assert ok, (name, t, worst)
+
+
+def test_index_score_mx_block_scaled_every_code():
+    """Every finite E4M3 key code through the block-scaled MMA, with four different block
+    exponents per key (as in the MXFP8 key-path test) and MXFP8 queries +1 / -1 at dim 32b of
+    block b: the score is sum_b decode(code) 2^(E_b - 127), bit for bit wherever that is a normal
+    fp32 number; below 2^-126 the tensor core may flush to zero, which is all that is allowed."""
+    wl = workloads.make("decode_fp8", DEV, B=1, L=1536)
+    slots = wl.num_pages * wl.page_size
+    code_of_slot = torch.arange(slots, dtype=torch.int64) % 256
+    code_of_slot[(code_of_slot & 0x7F) == 0x7F] = 0
+    k8 = code_of_slot.to(torch.uint8)[:, None].expand(slots, wl.D_I).contiguous().to(DEV)
+    bases = torch.tensor([0, 1, 60, 127, 200, 240])
+    sl = torch.arange(slots)
+    base = bases[(sl // 256) % len(bases)]
+    E = torch.stack([base + (sl + 3 * b) % 4 for b in range(4)], dim=1).to(torch.uint8)
+    q = torch.zeros((1, wl.H_I, wl.D_I), dtype=torch.bfloat16)
+    w = torch.zeros((1, wl.H_I), dtype=torch.float32)
+    for b in range(4):
+        q[0, b, 32 * b], q[0, 4 + b, 32 * b] = 1.0, -1.0
+        w[0, b], w[0, 4 + b] = 1.0, -1.0
+    qc, qs = hsa.hsa_quantize_mx(q.reshape(-1, wl.D_I).to(DEV))
+    seq = hsa.PagedSeq(wl.seq_lens, wl.block_table, wl.page_size, wl.num_pages,
+                       wl.q_seq[:1], wl.q_pos[:1], max_seq_len=int(wl.seq_lens.max()),
+                       status=torch.zeros(1, dtype=torch.int32, device=DEV))
+    sc = hsa.hsa_index_score(seq, qc.view(1, wl.H_I, wl.D_I), w.to(DEV), k8, E.contiguous().to(DEV),
+                             q_scale=qs.view(1, wl.H_I, wl.D_I // 32))
+    check_status(seq)
+    n = int(wl.q_pos[0]) + 1
+    bt = wl.block_table[0].cpu().long()
+    pos = torch.arange(n)
+    slot = bt[pos // wl.page_size] * wl.page_size + pos % wl.page_size
+    codes = code_of_slot[slot].numpy().astype(np.uint8)
+    vals = oracle.e4m3_decode(codes)
+    ref = sum(vals * np.exp2(E[slot, b].double().numpy() - 127) for b in range(4))
+    assert len(set(codes.tolist())) == 254
+    got = sc[0, :n].cpu().numpy().astype(np.float64)
+    normal = np.abs(ref) >= 2.0 ** -126
+    assert np.array_equal(got[normal], ref[normal])
+    assert np.all((got[~normal] == ref[~normal]) | (got[~normal] == 0.0))
+
+
 @pytest.mark.parametrize("q_run,T", [(1, 2500), (2, 600), (4, 300)])
 def test_index_score_row_groupings(q_run, T):
     """The tensor-core kernel groups q_run-aligned rows (1, 2 or 4 per MMA tile) and splits
@@ -323,12 +397,10 @@ def test_topk_blocks_bit_exact_and_attention(name, kw, block):
 
 
 @pytest.mark.parametrize("B", [3, 64])
-def test_sparse_mla_rows_split_between_clusters(B):
-    """With few query rows the tensor-core kernel lays the rows' tiles end to end and gives each
-    cluster an equal run of them, so rows are cut between clusters and finished by log-sum-exp
-    (3 rows: each cut into many parts; 64 rows: the decode batch's shape).  A short row and an
-    empty row ride along.  Checked against the oracle, against the same call with whole rows per
-    cluster (no workspace), within rounding, and the workspace's row counters are back to 0."""
+def test_sparse_mla_short_rows_and_workspace(B):
+    """Few rows (3) and the decode batch's 64, with a short row (11 of 32 tiles) and an empty row
+    riding along, against the oracle; the workspace the library reports is not needed by the
+    current kernel, so a call with none and a repeated call give the same bits."""
     wl = workloads.make("decode_bf16", DEV, B=B, L_min=2100, L_max=6000)
     idx = workloads.random_selection(wl.q_pos, wl.K, seed=11)
     idx[1, 700:] = -1                     # 11 of 32 tiles
@@ -337,20 +409,11 @@ def test_sparse_mla_rows_split_between_clusters(B):
     assert torch.all(out[2] == 0) and torch.all(torch.isneginf(lse[2]))
     seq = paged_seq(wl)
     need = hsa.hsa_sparse_mla_workspace_size(seq, wl.H, wl.D_qk, wl.D_v, wl.K)
-    assert need > 0
-    ws = torch.zeros(need, dtype=torch.uint8, device=DEV)
+    ws = torch.zeros(max(need, 1), dtype=torch.uint8, device=DEV)
     out_s, lse_s = hsa.hsa_sparse_mla_attn(seq, wl.q, wl.kv, idx.to(DEV), wl.D_v, wl.softmax_scale, ws=ws)
-    out_w, lse_w = hsa.hsa_sparse_mla_attn(seq, wl.q, wl.kv, idx.to(DEV), wl.D_v, wl.softmax_scale,
-                                           ws=torch.zeros(1, dtype=torch.uint8, device=DEV))
-    check_status(seq)
-    assert torch.equal(out_s, out)                       # same schedule, same bits
-    assert torch.allclose(out_s.float(), out_w.float(), atol=5e-3, rtol=5e-3)
-    fin = torch.isfinite(lse_w)
-    assert torch.equal(fin, torch.isfinite(lse_s))
-    assert torch.allclose(lse_s[fin], lse_w[fin], atol=1e-4, rtol=1e-4)
-    assert int(ws[:wl.T_q * 8].count_nonzero()) == 0     # counters returned to zero
-    # a second call on the same workspace gives the same bits
     out_2, lse_2 = hsa.hsa_sparse_mla_attn(seq, wl.q, wl.kv, idx.to(DEV), wl.D_v, wl.softmax_scale, ws=ws)
+    check_status(seq)
+    assert torch.equal(out_s, out) and torch.equal(lse_s, lse)
     assert torch.equal(out_2, out_s) and torch.equal(lse_2, lse_s)
 
 

@@ -103,13 +103,7 @@ def test_fused_equals_unfused_and_two_streams(name, kw, kv_group):
         assert torch.equal(sc1[t, :n], sc2[t, :n]) and torch.equal(sc1[t, :n], sc3[t, :n])
     assert torch.equal(idx1, idx2) and torch.equal(idx1, idx3)
     assert torch.equal(out1, out3) and torch.equal(lse1, lse3)
-    # the two-stream form runs each half of the rows as its own launch, so the few-rows schedule
-    # cuts rows between clusters at other places: equal up to the rounding of the merge
-    tol = TOL[wl.dtype] if not (wl.kv_fp8 or wl.index_fp8) else 6e-2
-    assert torch.allclose(out1.float(), out2.float(), atol=tol / 4, rtol=tol / 4)
-    fin = torch.isfinite(lse1)
-    assert torch.equal(fin, torch.isfinite(lse2))
-    assert torch.allclose(lse1[fin], lse2[fin], atol=1e-4, rtol=1e-4)
+    assert torch.equal(out1, out2) and torch.equal(lse1, lse2)
 
 
 def test_decode_bf16_full_size_sampled():
@@ -193,7 +187,10 @@ def test_decode_prolog_three_streams_equals_one_shot_caches(mx):
     for t in (k, ks, kv, kvs, rope):
         t[last] = 0
     q_out = torch.empty_like(wl.q_I)
-    hsa.hsa_decode_prolog(wl.k_I[last], wl.kv[last], last, k, ks, kv, kvs, rope, wl.q_I, q_out, wl.D_v)
+    q_codes = torch.empty(wl.q_I.shape, dtype=torch.uint8, device=DEV) if mx else None
+    q_sc = torch.empty((wl.T_q, wl.H_I, wl.D_I // 32), dtype=torch.uint8, device=DEV) if mx else None
+    hsa.hsa_decode_prolog(wl.k_I[last], wl.kv[last], last, k, ks, kv, kvs, rope, wl.q_I, q_out, wl.D_v,
+                          q_codes_out=q_codes, q_scale_out=q_sc)
     torch.cuda.synchronize()
     for got, ref in ((k, k_ref), (ks, ks_ref), (kv, kv_ref), (kvs, kvs_ref), (rope, rope_ref)):
         assert torch.equal(got, ref)
@@ -213,8 +210,12 @@ def test_decode_prolog_three_streams_equals_one_shot_caches(mx):
     # q_I on the MX grid: the oracle's quantize-then-dequantize, rounded to bf16 (exact here:
     # every block exponent of N(0, 1) data is far above the bf16 subnormal range)
     qf = wl.q_I.float().cpu().reshape(-1, wl.D_I)
-    q_ref = oracle.mx_dequantize_rows(*oracle.mx_quantize_rows(qf))
+    qc_ref, qs_ref = oracle.mx_quantize_rows(qf)
+    q_ref = oracle.mx_dequantize_rows(qc_ref, qs_ref)
     assert np.array_equal(q_out.float().cpu().numpy().reshape(q_ref.shape), q_ref)
+    if mx:   # the queries' MXFP8 codes and scales for the block-scaled index path
+        assert np.array_equal(q_codes.cpu().numpy().reshape(qc_ref.shape), qc_ref)
+        assert np.array_equal(q_sc.cpu().numpy().reshape(qs_ref.shape), qs_ref)
     seq = paged_seq(wl)
     a = hsa.hsa_fused_decode(seq, q_out, wl.w, k, ks, wl.q, kv, kvs, rope, wl.K, wl.D_v,
                              wl.softmax_scale)
@@ -222,6 +223,16 @@ def test_decode_prolog_three_streams_equals_one_shot_caches(mx):
                              rope_ref, wl.K, wl.D_v, wl.softmax_scale)
     for x, y in zip(a, b):
         assert torch.equal(x, y)
+    if mx:
+        # the step on the codes (block-scaled MMA): same scores up to the index tolerance
+        c = hsa.hsa_fused_decode(seq, q_codes, wl.w, k, ks, wl.q, kv, kvs, rope, wl.K, wl.D_v,
+                                 wl.softmax_scale, q_I_scale=q_sc)
+        mag = hsa.hsa_index_score(seq, q_out, wl.w.abs(), k, ks)
+        for t in range(wl.T_q):
+            n = int(wl.q_pos[t]) + 1
+            ok, worst = index_tolerance_ok(c[3][t, :n].cpu().numpy(), a[3][t, :n].cpu().numpy().astype(np.float64),
+                                           mag[t, :n].cpu().numpy().astype(np.float64))
+            assert ok, (t, worst)
 
 
 @pytest.mark.parametrize("aux", [False, True])
