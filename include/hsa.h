@@ -227,6 +227,27 @@ HSA_API hsa_status_t hsa_fused_decode(const hsa_paged_seq_t* seq, const hsa_inde
                               int64_t ld_scores, int32_t* idx, void* ws, size_t ws_bytes,
                               void* stream_main, void* stream_aux);
 
+/* The fused decode step for callers that may not allocate device memory: code that runs while
+ * a CUDA graph is being captured (an allocation cannot be captured), and engines or plug-ins
+ * whose device memory all belongs to a pool they do not manage.  hsa_fused_decode needs scores
+ * and idx buffers from its caller; this variant keeps both in a scratch array that the library
+ * itself declares, 40 MiB, held on every GPU where the library's kernels are loaded until the
+ * process exits.  It calls no cudaMalloc or cudaFree and no allocating routine, runs on one
+ * stream, and gives the same out and lse as hsa_fused_decode on that stream (the paper has no
+ * counterpart: this is an interface for such callers, not a step of the method).
+ *   The step's scores [T_q, ld] fp32, ld = max_seq_len rounded up to a multiple of 4, and its
+ *   selections [T_q, K] int32, each rounded up to 256 bytes, must fit in the 40 MiB: a larger
+ *   call returns HSA_ERR_WORKSPACE and enqueues nothing (the FP8 decode batch, 128 rows of 65536
+ *   positions with K = 2048, needs 33 MiB).
+ *   The first call on a device looks up the scratch's address there (with that device current);
+ *   make that first call outside any stream capture.
+ *   Every call on a device uses the same scratch, which keeps the last call's scores and
+ *   selections (nothing in it needs to start at zero): calls that overlap on the GPU -- on
+ *   different streams without ordering between them -- race on it and must not be made.
+ * Arguments as for hsa_fused_decode; other errors as there. */
+HSA_API hsa_status_t hsa_fused_decode_noalloc(const hsa_paged_seq_t* seq, const hsa_index_args_t* index,
+                                      const hsa_attn_args_t* attn, int32_t K, void* stream);
+
 /* ---- 5. FP8 quantizers (cache write) --------------------------------------------------------
  * Per row r and group g of `group` consecutive elements:
  *   amax = max |x|; scale = amax / 448 (fp32, round to nearest); inv = 448 / amax (fp32);

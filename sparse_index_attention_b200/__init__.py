@@ -68,6 +68,7 @@ SYMBOLS = {
                                            _P]),
     "hsa_fused_decode_workspace_size": (_sz, [_P, _P, _i32]),
     "hsa_fused_decode": (ctypes.c_int, [_P, _P, _P, _i32, _P, _i64, _P, _P, _sz, _P, _P]),
+    "hsa_fused_decode_noalloc": (ctypes.c_int, [_P, _P, _P, _i32, _P]),
     "hsa_quantize_index": (ctypes.c_int, [_P, ctypes.c_int, _i64, _i32, _i32, _P, _i64, _P, _P, _P]),
     "hsa_quantize_kv": (ctypes.c_int, [_P, ctypes.c_int, _i64, _i32, _i32, _i32, _P, _i64, _P, _P,
                                        _P, _P]),
@@ -307,6 +308,21 @@ def hsa_fused_decode(seq: PagedSeq, q_I, w, k_cache, k_scale, q, kv, kv_scale, k
                                   None if aux_stream is None else ctypes.c_void_p(aux_stream.cuda_stream)),
            "hsa_fused_decode")
     return out, lse, idx, scores
+
+def hsa_fused_decode_noalloc(seq: PagedSeq, q_I, w, k_cache, k_scale, q, kv, kv_scale, kv_rope, K: int,
+                             D_v: int, softmax_scale: float, out, lse=None, stream=None, q_I_scale=None):
+    """The fused decode step with its scores and selections in the library's own scratch
+    (hsa_fused_decode_noalloc: for callers that may not allocate device memory).  ``out``
+    [T_q, H, D_v] and ``lse`` [T_q, H] fp32 (or None) are the caller's; returns (out, lse)."""
+    T_q, H_I, D_I = q_I.shape
+    ia = hsa_index_args_t(_ptr(q_I), HSA_MXE4M3 if q_I_scale is not None else _dtype(q_I), _ptr(w),
+                          H_I, D_I, _ptr(k_cache), _key_dtype(k_cache, k_scale), _ptr(k_scale),
+                          _ptr(q_I_scale))
+    at = _attn_struct(q, kv, D_v, softmax_scale, kv_scale, kv_rope, out, lse)
+    _check(lib().hsa_fused_decode_noalloc(seq.ref, ctypes.byref(ia), ctypes.byref(at), K,
+                                          _stream(stream)),
+           "hsa_fused_decode_noalloc")
+    return out, lse
 
 
 class DecodeGraph:

@@ -4,6 +4,7 @@
 #include <stdarg.h>
 #include <stdio.h>
 
+#include <mutex>
 #include <string>
 
 #include "kernels.h"
@@ -644,6 +645,66 @@ hsa_status_t hsa_decode_prolog(const hsa_prolog_args_t* a, void* stream, void* s
     for (int i = 0; i < 4; ++i)
         if (ev[i]) cudaEventDestroy(ev[i]);
     return r;
+}
+
+}  // extern "C"
+
+// ---- the fused decode step without allocation -------------------------------------------------
+// Scratch of hsa_fused_decode_noalloc: the step's scores, then its selections.  Every GPU on which
+// the library's kernels are loaded holds these 40 MiB from then until the process exits.
+constexpr size_t kNoAllocScratchBytes = size_t(40) << 20;
+static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
+
+namespace {
+
+constexpr int kNoAllocMaxDevices = 64;
+std::mutex g_noalloc_mutex;
+uint8_t* g_noalloc_ptr[kNoAllocMaxDevices];   // the scratch's address on each device, once known
+
+// The scratch's device address on the current device; the first call on a device looks it up
+// (with that device current) and keeps it.
+hsa_status_t noalloc_scratch(uint8_t** p) {
+    int dev = -1;
+    hsa_status_t r = cuda_status(cudaGetDevice(&dev), "cudaGetDevice");
+    if (r != HSA_OK) return r;
+    HSA_REQUIRE(dev >= 0 && dev < kNoAllocMaxDevices, HSA_ERR_UNSUPPORTED,
+                "device %d: the no-allocation entry serves devices 0..%d", dev, kNoAllocMaxDevices - 1);
+    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+    if (g_noalloc_ptr[dev] == nullptr) {
+        void* q = nullptr;
+        r = cuda_status(cudaGetSymbolAddress(&q, g_noalloc_scratch), "cudaGetSymbolAddress (scratch)");
+        if (r != HSA_OK) return r;
+        g_noalloc_ptr[dev] = static_cast<uint8_t*>(q);
+    }
+    *p = g_noalloc_ptr[dev];
+    return HSA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+hsa_status_t hsa_fused_decode_noalloc(const hsa_paged_seq_t* seq, const hsa_index_args_t* ix,
+                                      const hsa_attn_args_t* at, int32_t K, void* stream) {
+    g_last_error.clear();
+    HSA_REQUIRE(seq && ix && at, HSA_ERR_INVALID_ARG, "seq / index / attn args NULL");
+    HSA_REQUIRE(seq->T_q >= 0 && seq->max_seq_len >= 1, HSA_ERR_INVALID_ARG,
+                "T_q = %d, max_seq_len = %d", seq->T_q, seq->max_seq_len);
+    HSA_REQUIRE(K >= 1 && K <= 65536, HSA_ERR_INVALID_ARG, "K = %d out of range", K);
+    // scores [T_q, ld] fp32 (rows 16-byte aligned), then idx [T_q, K] int32
+    const int64_t ld = ((int64_t)seq->max_seq_len + 3) / 4 * 4;
+    const size_t score_bytes = ((size_t)seq->T_q * ld * 4 + 255) / 256 * 256;
+    const size_t idx_bytes = ((size_t)seq->T_q * K * 4 + 255) / 256 * 256;
+    HSA_REQUIRE(score_bytes + idx_bytes <= kNoAllocScratchBytes, HSA_ERR_WORKSPACE,
+                "T_q = %d rows, max_seq_len = %d and K = %d need %zu bytes of scratch; the "
+                "no-allocation entry holds %zu",
+                seq->T_q, seq->max_seq_len, K, score_bytes + idx_bytes, kNoAllocScratchBytes);
+    uint8_t* scratch = nullptr;
+    hsa_status_t r = noalloc_scratch(&scratch);
+    if (r != HSA_OK) return r;
+    return hsa_fused_decode(seq, ix, at, K, reinterpret_cast<float*>(scratch), ld,
+                            reinterpret_cast<int32_t*>(scratch + score_bytes), nullptr, 0, stream,
+                            nullptr);
 }
 
 }  // extern "C"

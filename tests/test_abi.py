@@ -61,6 +61,14 @@ def test_validation_without_gpu():
     assert rc == hsa.HSA_ERR_INVALID_ARG                       # q_scale not 16-byte aligned
     rc = L.hsa_index_score_mx(ctypes.byref(seq), fake, fake, fake, 4, 48, fake, fake, fake, 64, None)
     assert rc == hsa.HSA_ERR_INVALID_ARG                       # D_I not a multiple of 32
+    # the no-allocation decode step rejects a step whose scores and selections exceed its
+    # scratch before anything touches the device
+    big = hsa.hsa_paged_seq_t(1, fake, fake, 2048, 64, 2048, 131072, 128, fake, fake, 1, None)
+    ia = hsa.hsa_index_args_t(fake, hsa.HSA_BF16, fake, 64, 128, fake, hsa.HSA_BF16, None, None)
+    at = hsa.hsa_attn_args_t(fake, hsa.HSA_BF16, 128, 576, 512, fake, hsa.HSA_BF16, None, 512, None,
+                             0.04, fake, hsa.HSA_BF16, None)
+    rc = L.hsa_fused_decode_noalloc(ctypes.byref(big), ctypes.byref(ia), ctypes.byref(at), 2048, None)
+    assert rc == hsa.HSA_ERR_WORKSPACE and b"scratch" in L.hsa_last_error_message()
     rc = L.hsa_quantize_index(fake, hsa.HSA_BF16, 10, 128, 48, None, 10, fake, fake, None)
     assert rc == hsa.HSA_ERR_INVALID_ARG                       # group does not divide D
     # E4M3 latent cache: the scale group must be a multiple of 16 that divides D_v
