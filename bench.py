@@ -709,6 +709,26 @@ def run_ours(args, rank, world, local_rank):
         dist.destroy_process_group()
 
 
+def run_profile_case(args):
+    """A small causal prefill (prefill_bf16 shapes, --profile-rows query rows of one sequence):
+    index score, Top-K and sparse MLA, each called three times on one stream, nothing timed.
+    For one-kernel ncu captures of the prefill kernels at a size whose capture ends quickly."""
+    import sparse_index_attention_b200 as hsa
+    dev = "cuda"
+    wl = workloads.make("prefill_bf16", dev, T=args.profile_rows)
+    seq = hsa.PagedSeq(wl.seq_lens, wl.block_table, wl.page_size, wl.num_pages, wl.q_seq, wl.q_pos,
+                       q_run=wl.q_run)
+    sc = hsa.hsa_index_score(seq, wl.q_I, wl.w, wl.k_I)
+    idx = hsa.hsa_topk(seq, sc, wl.K)
+    out, _ = hsa.hsa_sparse_mla_attn(seq, wl.q, wl.kv, idx, wl.D_v, wl.softmax_scale, lse=False)
+    for _ in range(2):
+        hsa.hsa_index_score(seq, wl.q_I, wl.w, wl.k_I, scores=sc)
+        hsa.hsa_topk(seq, sc, wl.K, idx=idx)
+        hsa.hsa_sparse_mla_attn(seq, wl.q, wl.kv, idx, wl.D_v, wl.softmax_scale, out=out, lse=False)
+    torch.cuda.synchronize()
+    print(json.dumps({"profile_case": "prefill_bf16", "rows": wl.T_q, "launches_per_kernel": 3}))
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -721,7 +741,13 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-secondary", action="store_true",
                     help="skip the FP8 decode, prefill and quantizer measurements")
+    ap.add_argument("--profile-rows", type=int, default=0,
+                    help="only run a small prefill of this many rows (three calls of each kernel, "
+                         "for ncu captures) and exit")
     args = ap.parse_args()
+    if args.profile_rows > 0:
+        run_profile_case(args)
+        return
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     rank = int(os.environ.get("RANK", "0"))

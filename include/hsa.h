@@ -227,6 +227,27 @@ HSA_API hsa_status_t hsa_fused_decode(const hsa_paged_seq_t* seq, const hsa_inde
                               int64_t ld_scores, int32_t* idx, void* ws, size_t ws_bytes,
                               void* stream_main, void* stream_aux);
 
+/* Causal prefill over query-row chunks (Python: hsa_prefill_chunked).  Chunk i covers rows
+ * [chunks[2i], chunks[2i+1]) (host int32 array, non-empty, inside [0, T_q); with q_run > 1 its
+ * bounds should be multiples of q_run) and runs hsa_index_score -> hsa_topk ->
+ * hsa_sparse_mla_attn on those rows, on stream_a for even i and stream_b for odd i (NULL: the
+ * calling stream), so consecutive chunks form pairs that run concurrently.  With the zigzag order
+ * (chunk i of 2N paired with chunk 2N-1-i) every pair carries the same causal work ("Efficient
+ * Inference Deployment and Optimization for Hybrid Attention LLMs", 5.2: zigzag load balancing;
+ * its multi-GPU form is the same chunks on several ranks).  Outputs land at the rows' own
+ * offsets of out / lse / idx ([T_q, ...]), so the order of the chunks changes no result.  Both
+ * side streams first wait for the work already on `stream`, which then waits for both.
+ *   score_bufs  host array of two device fp32 buffers [score_rows, ld_scores], one per side
+ *               stream, reused chunk after chunk (score_rows >= the largest chunk's rows;
+ *               ld_scores >= max_seq_len); they hold scores of the last chunks afterwards
+ *   idx         device int32 [T_q, K]: every row's selection afterwards
+ * index / attn as for hsa_fused_decode.  Needs no workspace. */
+HSA_API hsa_status_t hsa_prefill_chunked(const hsa_paged_seq_t* seq, const hsa_index_args_t* index,
+                                 const hsa_attn_args_t* attn, int32_t K, const int32_t* chunks,
+                                 int32_t n_chunks, float* const* score_bufs, int32_t score_rows,
+                                 int64_t ld_scores, int32_t* idx, void* stream, void* stream_a,
+                                 void* stream_b);
+
 /* The fused decode step for callers that may not allocate device memory: code that runs while
  * a CUDA graph is being captured (an allocation cannot be captured), and engines or plug-ins
  * whose device memory all belongs to a pool they do not manage.  hsa_fused_decode needs scores

@@ -69,6 +69,7 @@ SYMBOLS = {
     "hsa_fused_decode_workspace_size": (_sz, [_P, _P, _i32]),
     "hsa_fused_decode": (ctypes.c_int, [_P, _P, _P, _i32, _P, _i64, _P, _P, _sz, _P, _P]),
     "hsa_fused_decode_noalloc": (ctypes.c_int, [_P, _P, _P, _i32, _P]),
+    "hsa_prefill_chunked": (ctypes.c_int, [_P, _P, _P, _i32, _P, _i32, _P, _i32, _i64, _P, _P, _P, _P]),
     "hsa_quantize_index": (ctypes.c_int, [_P, ctypes.c_int, _i64, _i32, _i32, _P, _i64, _P, _P, _P]),
     "hsa_quantize_kv": (ctypes.c_int, [_P, ctypes.c_int, _i64, _i32, _i32, _i32, _P, _i64, _P, _P,
                                        _P, _P]),
@@ -531,7 +532,8 @@ def hsa_prefill_chunked(seq: PagedSeq, q_I, w, k_cache, k_scale, q, kv, kv_scale
     Optimization for Hybrid Attention LLMs", 5.2) every pair carries the same causal index work.
     Each chunk is hsa_index_score -> hsa_topk -> hsa_sparse_mla_attn on its rows, so its outputs
     land at the rows' own offsets and no restore step exists; the issue order cannot change any
-    result.  This function only slices tensors and issues C-ABI calls.  ``score_bufs`` (one per
+    result.  This function marshals its arguments into one C-ABI call (hsa_prefill_chunked,
+    which issues the chunks and orders the streams).  ``score_bufs`` (one per
     stream, from prefill_score_buffers) holds the chunks' scores; when it is not given, buffers
     are allocated for this call.  Returns (out, lse, idx).
     """
@@ -548,28 +550,23 @@ def hsa_prefill_chunked(seq: PagedSeq, q_I, w, k_cache, k_scale, q, kv, kv_scale
     main = torch.cuda.current_stream()
     if streams is None:
         streams = (torch.cuda.Stream(), torch.cuda.Stream())
-    start = torch.cuda.Event()
-    start.record(main)
     own = score_bufs is None
-    bufs = list(prefill_score_buffers(seq, chunks, dev, len(streams)) if own else score_bufs)
+    bufs = list(prefill_score_buffers(seq, chunks, dev, 2) if own else score_bufs)
     rows_max = max(r1 - r0 for r0, r1 in chunks)
-    if len(bufs) < len(streams) or any(b.shape[0] < rows_max or b.shape[1] < seq.max_seq_len for b in bufs):
-        raise ValueError("score buffers smaller than [max chunk rows, max_seq_len]")
-    for s in streams:
-        s.wait_event(start)
-    for i, (r0, r1) in enumerate(chunks):
-        s = streams[i % 2]
-        part = seq.rows(r0, r1, q_run=min(seq.q_run, r1 - r0))
-        sc = bufs[i % 2][:r1 - r0]
-        hsa_index_score(part, q_I[r0:r1], w[r0:r1], k_cache, k_scale, scores=sc, stream=s)
-        hsa_topk(part, sc, K, idx=idx[r0:r1], stream=s)
-        hsa_sparse_mla_attn(part, q[r0:r1], kv, idx[r0:r1], D_v, softmax_scale, kv_scale=kv_scale,
-                            kv_rope=kv_rope, out=out[r0:r1], lse=None if lse is None else lse[r0:r1],
-                            stream=s)
-    for s in streams:
-        done = torch.cuda.Event()
-        done.record(s)
-        main.wait_event(done)
+    if len(bufs) < 2 or bufs[0].shape != bufs[1].shape or bufs[0].shape[0] < rows_max or \
+            bufs[0].shape[1] < seq.max_seq_len or not all(b.is_contiguous() for b in bufs[:2]):
+        raise ValueError("two contiguous score buffers of at least [max chunk rows, max_seq_len]")
+    T_qI, H_I, D_I = q_I.shape
+    ia = hsa_index_args_t(_ptr(q_I), _dtype(q_I), _ptr(w), H_I, D_I, _ptr(k_cache),
+                          _key_dtype(k_cache, k_scale), _ptr(k_scale), None)
+    at = _attn_struct(q, kv, D_v, softmax_scale, kv_scale, kv_rope, out, lse)
+    flat = [x for rr in chunks for x in rr]
+    arr = (ctypes.c_int32 * len(flat))(*flat)
+    bp = (ctypes.c_void_p * 2)(bufs[0].data_ptr(), bufs[1].data_ptr())
+    _check(lib().hsa_prefill_chunked(seq.ref, ctypes.byref(ia), ctypes.byref(at), K, arr, len(chunks),
+                                     bp, bufs[0].shape[0], bufs[0].shape[1], _ptr(idx),
+                                     _stream(main), _stream(streams[0]), _stream(streams[1])),
+           "hsa_prefill_chunked")
     if own:
         for b, s in zip(bufs, streams):
             b.record_stream(s)

@@ -499,6 +499,81 @@ hsa_status_t hsa_fused_decode(const hsa_paged_seq_t* seq, const hsa_index_args_t
     return r;
 }
 
+hsa_status_t hsa_prefill_chunked(const hsa_paged_seq_t* seq, const hsa_index_args_t* ix,
+                                 const hsa_attn_args_t* at, int32_t K, const int32_t* chunks,
+                                 int32_t n_chunks, float* const* score_bufs, int32_t score_rows,
+                                 int64_t ld_scores, int32_t* idx, void* stream, void* stream_a,
+                                 void* stream_b) {
+    g_last_error.clear();
+    HSA_REQUIRE(ix && at, HSA_ERR_INVALID_ARG, "index / attn args NULL");
+    HSA_REQUIRE(n_chunks >= 0 && (n_chunks == 0 || chunks), HSA_ERR_INVALID_ARG, "chunks NULL");
+    HSA_REQUIRE(score_bufs && score_bufs[0] && score_bufs[1], HSA_ERR_INVALID_ARG,
+                "two score buffers are needed");
+    hsa_status_t st = check_index(seq, ix->q_I, ix->q_dtype, ix->q_scale, ix->w, ix->H_I, ix->D_I,
+                                  ix->k_cache, ix->k_dtype, ix->k_scale, score_bufs[0], ld_scores);
+    if (st != HSA_OK) return st;
+    st = check_attn(seq, at->q, at->q_dtype, at->H, at->D_qk, at->D_v, at->kv, at->kv_dtype,
+                    at->kv_scale, at->kv_scale_group, at->kv_rope, idx, K, at->out, at->out_dtype);
+    if (st != HSA_OK) return st;
+    HSA_REQUIRE(idx && aligned(idx, 4) && aligned(score_bufs[1], 4), HSA_ERR_INVALID_ARG,
+                "idx NULL or a buffer misaligned");
+    for (int32_t i = 0; i < n_chunks; ++i) {
+        const int32_t r0 = chunks[2 * i], r1 = chunks[2 * i + 1];
+        HSA_REQUIRE(0 <= r0 && r0 < r1 && r1 <= seq->T_q, HSA_ERR_INVALID_ARG,
+                    "chunk %d = [%d, %d) outside [0, T_q = %d) or empty", i, r0, r1, seq->T_q);
+        HSA_REQUIRE(r1 - r0 <= score_rows, HSA_ERR_INVALID_ARG,
+                    "chunk %d has %d rows; the score buffers hold %d", i, r1 - r0, score_rows);
+    }
+    if (n_chunks == 0 || seq->T_q == 0) return HSA_OK;
+
+    cudaStream_t s0 = (cudaStream_t)stream;
+    const cudaStream_t side[2] = {stream_a ? (cudaStream_t)stream_a : s0,
+                                  stream_b ? (cudaStream_t)stream_b : s0};
+    cudaEvent_t ev[3] = {nullptr, nullptr, nullptr};
+    hsa_status_t r = HSA_OK;
+    for (int i = 0; i < 3 && r == HSA_OK; ++i)
+        r = cuda_status(cudaEventCreateWithFlags(&ev[i], cudaEventDisableTiming), "cudaEventCreate");
+    // fork: both side streams start after the work already on `stream`
+    if (r == HSA_OK) r = cuda_status(cudaEventRecord(ev[0], s0), "cudaEventRecord");
+    for (int i = 0; i < 2 && r == HSA_OK; ++i)
+        if (side[i] != s0) r = cuda_status(cudaStreamWaitEvent(side[i], ev[0], 0), "cudaStreamWaitEvent");
+    const size_t qsz = dtype_size(ix->q_dtype), asz = dtype_size(at->q_dtype), osz = dtype_size(at->out_dtype);
+    for (int32_t i = 0; i < n_chunks && r == HSA_OK; ++i) {
+        const int32_t r0 = chunks[2 * i], n = chunks[2 * i + 1] - r0;
+        cudaStream_t s = side[i & 1];
+        hsa_paged_seq_t part = sub_rows(*seq, r0, n);
+        part.q_run = seq->q_run < n ? seq->q_run : n;
+        float* sc = score_bufs[i & 1];
+        const void* qs = ix->q_dtype == HSA_MXE4M3
+                             ? static_cast<const char*>(ix->q_scale) + (size_t)r0 * ix->H_I * (ix->D_I / 32)
+                             : nullptr;
+        r = run_index(index_args(&part, static_cast<const char*>(ix->q_I) + (size_t)r0 * ix->H_I * ix->D_I * qsz,
+                                 ix->q_dtype, qs, ix->w + (size_t)r0 * ix->H_I, ix->H_I, ix->D_I,
+                                 ix->k_cache, ix->k_dtype, ix->k_scale, sc, ld_scores),
+                      s);
+        if (r != HSA_OK) break;
+        r = cuda_status(hsa::launch_topk(view(&part), part.max_seq_len, sc, ld_scores, K,
+                                         idx + (size_t)r0 * K, s),
+                        "topk");
+        if (r != HSA_OK) break;
+        hsa_attn_args_t pa = *at;
+        pa.q = static_cast<const char*>(at->q) + (size_t)r0 * at->H * at->D_qk * asz;
+        pa.out = static_cast<char*>(at->out) + (size_t)r0 * at->H * at->D_v * osz;
+        pa.lse = at->lse ? at->lse + (size_t)r0 * at->H : nullptr;
+        r = run_attn(attn_args(&part, pa, idx + (size_t)r0 * K, K, nullptr, 0), s);
+    }
+    // join (also after a failed launch, so that nothing enqueued is left unordered)
+    for (int i = 0; i < 2; ++i) {
+        if (side[i] == s0 || ev[1 + i] == nullptr || ev[0] == nullptr) continue;
+        hsa_status_t e = cuda_status(cudaEventRecord(ev[1 + i], side[i]), "cudaEventRecord");
+        if (e == HSA_OK) e = cuda_status(cudaStreamWaitEvent(s0, ev[1 + i], 0), "cudaStreamWaitEvent");
+        if (r == HSA_OK) r = e;
+    }
+    for (int i = 0; i < 3; ++i)
+        if (ev[i]) cudaEventDestroy(ev[i]);
+    return r;
+}
+
 hsa_status_t hsa_quantize_index(const void* src, hsa_dtype_t src_dtype, int64_t n_rows,
                                 int32_t D, int32_t group, const int64_t* slot_mapping,
                                 int64_t num_slots, uint8_t* codes, float* scales, void* stream) {

@@ -7,8 +7,8 @@
 // Mapping.  One tcgen05 MMA tile is D[128 keys x G*64] = K_tile[128 x 128] . Q_group^T, with the
 // keys on M (TMEM lanes) and G query rows x 64 index heads on N (TMEM columns).  The epilogue
 // thread that owns TMEM lane r owns key s = tile*128 + r and reduces its 64 head columns per
-// query row in registers: no cross-thread reduction.  Accumulators are double-buffered in TMEM
-// so the epilogue of tile i overlaps the MMA of tile i+1.
+// query row in registers: no cross-thread reduction.  Accumulators are multi-buffered in TMEM
+// (four for N <= 128, two for N = 256) so the epilogue of tile i overlaps the MMAs of the next.
 //
 // Schedule.  Work is the flat list of (query group, key tile) pairs, where a group is G
 // consecutive rows of one sequence and its key range is [0, max position of the group].  Each
@@ -17,18 +17,21 @@
 // changes.  Every CTA derives the list itself from q_pos (prefix sum in shared memory).
 //
 // Data movement.  Keys come through the block table page by page with 2D TMA loads (128-byte
-// swizzle, two 64-column halves per page); FP8 keys are loaded raw and widened to bf16 in
-// shared memory by four converter warps (e4m3 -> bf16 is exact), and the per-key fp32 scale
-// multiplies the finished score (the scale is positive, so it commutes with the ReLU sum).
-// MXFP8 keys (one E8M0 byte per 32 dims; "Inference Adaptation and Performance Optimization for
-// a Domestically Developed LLM's New Architecture", section 4 table) take the same path: the
-// producer bulk-copies each box's scale words beside its codes, the converters widen the codes
-// by placing their bits in bf16s and scale each 32-dim block by 2^(E_block - E_max) with one
-// packed multiply (exact), and the epilogue multiplies the score by 2^(E_max - 127), the key's
-// largest block scale.
+// swizzle, two 64-column halves per page); FP8 keys are loaded raw and widened in shared memory
+// by four converter warps (E4M3 -> f16 in one conversion, exact; the MMA then runs in f16, the
+// queries rescaled into f16's range per head), and the per-key fp32 scale multiplies the
+// finished score (the scale is positive, so it commutes with the ReLU sum).  MXFP8 keys (one
+// E8M0 byte per 32 dims; "Inference Adaptation and Performance Optimization for a Domestically
+// Developed LLM's New Architecture", section 4 table) with bf16 queries take the same path: the
+// producer bulk-copies each box's scale words beside its codes, the converters place the codes'
+// bits in bf16s and scale each 32-dim block by 2^(E_block - E_max) with one packed multiply
+// (exact), and the epilogue multiplies the score by 2^(E_max - 127), the key's largest block
+// scale.  MXFP8 keys with MXFP8 queries skip the converters: the codes go straight to a
+// block-scaled MMA (kind::mxf8f6f4) that reads the E8M0 scales from TMEM.
 //
 // Warp roles: 0 TMA producer, 1 MMA issuer (one elected thread each), 2-5 epilogue
-// (TMEM lane quarters 2,3,0,1), 6-9 FP8 converters (FP8 variant only).
+// (TMEM lane quarters 2,3,0,1), 6-9 FP8 converters (FP8 keys) or key-scale writers
+// (block-scaled MMA).
 #include <algorithm>
 
 #include "kernels.h"
@@ -53,15 +56,19 @@ struct Cfg {
     static constexpr int kStages = kBs ? (G == 1 ? 8 : 6)
                                        : kFp8 ? (G == 1 ? 4 : (G == 2 ? 3 : 2)) : (G == 1 ? 6 : (G == 2 ? 5 : 4));
     static constexpr int kRawStages = kFp8 ? 4 : 0;          // FP8 staging tiles (16 KB each)
+    static constexpr int kR = kRawStages > 0 ? kRawStages : 1;
     static constexpr int kScaleStageBytes = (kMx || kBs) ? kBM * 4 : 0;  // 4 E8M0 bytes per key
     static constexpr int kScaleStages = kBs ? kStages : kRawStages;
     static constexpr int kMaxGroups = G == 1 ? 2048 : 4096;
-    // TMEM: two accumulators of N columns; block-scaled adds the key scales (4 columns per stage)
-    // and the query scales (N / 32 columns)
-    static constexpr int kSfaCol = 2 * N;
-    static constexpr int kSfbCol = 2 * N + 4 * kStages;
-    static constexpr int kTmemCols = kBs ? (G == 1 ? 256 : 512) : 2 * N;   // 128, 256 or 512
+    // TMEM: kAcc accumulators of N columns (four for N <= 128, so the MMA may run up to four
+    // tiles ahead of the epilogue; two for N = 256); block-scaled adds the key scales (4 columns
+    // per stage) and the query scales (N / 32 columns) after them
+    static constexpr int kAcc = (N <= 64 || (N == 128 && !kBs)) ? 4 : 2;
+    static constexpr int kSfaCol = kAcc * N;
+    static constexpr int kSfbCol = kSfaCol + 4 * kStages;
+    static constexpr int kTmemCols = kBs ? 512 : kAcc * N;   // 256 or 512
     static_assert(!kBs || kSfbCol + N / 32 <= kTmemCols, "TMEM budget");
+    static_assert(kAcc * N <= kTmemCols, "TMEM budget");
     static constexpr int kThreads = (kFp8 || kBs) ? 320 : 192;
     static constexpr int kBarBytes = 512;
     static constexpr size_t kSmem = 1024 + (size_t)kStages * kTile + (size_t)kRawStages * (kBM * kDI) +
@@ -145,19 +152,19 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
     uint64_t* bars = reinterpret_cast<uint64_t*>(qbuf + C::kQBytes);
     uint64_t* full = bars;                 // [S]  keys landed (bf16 tile ready)
     uint64_t* empty = full + S;            // [S]  MMA done with the tile
-    uint64_t* acc_full = empty + S;        // [2]
-    uint64_t* acc_empty = acc_full + 2;    // [2]
-    uint64_t* q_full = acc_empty + 2;
+    uint64_t* acc_full = empty + S;        // [kAcc]
+    uint64_t* acc_empty = acc_full + 4;    // [kAcc]
+    uint64_t* q_full = acc_empty + 4;
     uint64_t* q_empty = q_full + 1;
-    uint64_t* raw_full = q_empty + 1;      // [4] FP8 bytes landed
-    uint64_t* raw_empty = raw_full + 4;    // [4] converters done with the staging tile
-    uint64_t* epi_bar = raw_empty + 4;     // the four epilogue warps
+    uint64_t* raw_full = q_empty + 1;      // [kR] FP8 bytes landed
+    uint64_t* raw_empty = raw_full + 8;    // [kR] converters done with the staging tile
+    uint64_t* epi_bar = raw_empty + 8;     // the four epilogue warps
     uint64_t* q_ready = epi_bar + 1;       // f16 MMA: the group's queries converted; block-scaled:
                                            // the group's query scales in TMEM (4 warps)
     uint64_t* sf_full = q_ready + 1;       // [S] block-scaled: the tile's key scales in TMEM (4 warps)
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(sf_full + S);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
-    static_assert((3 * S + 2 + 2 + 2 + 8 + 2) * 8 + 8 <= C::kBarBytes, "barrier block");
+    static_assert((3 * S + 4 + 4 + 2 + 16 + 2) * 8 + 8 <= C::kBarBytes && C::kR <= 8 && C::kAcc <= 4, "barrier block");
     int32_t* prefix = reinterpret_cast<int32_t*>(reinterpret_cast<uint8_t*>(bars) + C::kBarBytes);
     float* w_s = reinterpret_cast<float*>(prefix + C::kMaxGroups + 1);
 
@@ -170,13 +177,13 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
             tc::mbar_init(&empty[i], 1);
             tc::mbar_init(&sf_full[i], 4);
         }
-        for (int i = 0; i < 2; ++i) {
+        for (int i = 0; i < C::kAcc; ++i) {
             tc::mbar_init(&acc_full[i], 1);
             tc::mbar_init(&acc_empty[i], 4);
         }
         tc::mbar_init(q_full, 1);
         tc::mbar_init(q_empty, 1);
-        for (int i = 0; i < 4; ++i) {
+        for (int i = 0; i < C::kR; ++i) {
             tc::mbar_init(&raw_full[i], 1);
             tc::mbar_init(&raw_empty[i], 128);
         }
@@ -250,9 +257,9 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
                     const int s0 = kt * kBM;
                     const int n_keys = min(kBM, gi.pos_max + 1 - s0);
                     const int n_boxes = (int)ceil_div(n_keys, box_rows);
-                    uint64_t* bar = kFp8 ? &raw_full[stage & 3] : &full[stage];
+                    uint64_t* bar = kFp8 ? &raw_full[stage % C::kR] : &full[stage];
                     if (kFp8) {
-                        if (!tc::mbar_wait(&raw_empty[stage & 3], ((stage >> 2) & 1) ^ 1, abort_flag)) break;
+                        if (!tc::mbar_wait(&raw_empty[stage % C::kR], ((stage / C::kR) & 1) ^ 1, abort_flag)) break;
                     } else {
                         if (!tc::mbar_wait(&empty[stage], phase ^ 1, abort_flag)) break;
                     }
@@ -262,10 +269,10 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
                         const int s = s0 + j * box_rows;
                         const int32_t row = (int32_t)paged_slot(v, gi.b, s);
                         if (kFp8) {
-                            uint8_t* dst = raw + (size_t)(stage & 3) * (kBM * kDI) + (size_t)j * box_rows * 128;
+                            uint8_t* dst = raw + (size_t)(stage % C::kR) * (kBM * kDI) + (size_t)j * box_rows * 128;
                             tc::tma_load_2d(dst, &tmap_k, bar, 0, row);
                             if (kMx)   // the box's E8M0 words: box_rows x 4 bytes, 32-byte aligned
-                                tc::bulk_load(kscl + (size_t)(stage & 3) * C::kScaleStageBytes + (size_t)j * box_rows * 4,
+                                tc::bulk_load(kscl + (size_t)(stage % C::kR) * C::kScaleStageBytes + (size_t)j * box_rows * 4,
                                               static_cast<const uint8_t*>(k_scale) + (int64_t)row * 4,
                                               (uint32_t)box_rows * 4, bar);
                         } else if (kBs) {   // codes straight into the MMA stage, scale words beside
@@ -281,7 +288,7 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
                         }
                     }
                     if (kFp8) {
-                        ++stage;   // staging ring of 4; the bf16 ring is advanced by the converters
+                        ++stage;   // staging ring of kR; the MMA ring is advanced by the converters
                     } else if (++stage == (uint32_t)S) {
                         stage = 0;
                         phase ^= 1;
@@ -339,8 +346,10 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
                         stage = 0;
                         phase ^= 1;
                     }
-                    acc ^= 1;
-                    if (acc == 0) acc_phase ^= 1;
+                    if (++acc == (uint32_t)C::kAcc) {
+                        acc = 0;
+                        acc_phase ^= 1;
+                    }
                 }
             }
             __syncwarp();
@@ -464,21 +473,37 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
 #pragma unroll
                 for (int j = 0; j < G; ++j) {
                     float a[64];
-                    tc::tmem_ld32(taddr + j * kHI, a);
-                    tc::tmem_ld32(taddr + j * kHI + 32, a + 32);
-                    tc::tmem_ld_wait();
-                    float sc = 0.f;
                     const float* wj = w_s + j * kHI;
+                    float sc = 0.f;
+                    if constexpr (G == 1) {
+                        tc::tmem_ld32(taddr, a);
+                        tc::tmem_ld32(taddr + 32, a + 32);
 #pragma unroll
-                    for (int h = 0; h < kHI; ++h) sc = fmaf(wj[h], fmaxf(a[h], 0.f), sc);
+                        for (int h = 0; h < kHI; ++h) sc = fmaf(wj[h], fmaxf(a[h], 0.f), sc);
+                    } else {
+                        // several rows per tile: the epilogue bounds the kernel; one 64-column
+                        // load and four partial sums (no 64-long dependent chain)
+                        tc::tmem_ld64(taddr + j * kHI, a);
+                        float p0 = 0.f, p1 = 0.f, p2 = 0.f, p3 = 0.f;
+#pragma unroll
+                        for (int h = 0; h < kHI; h += 4) {
+                            p0 = fmaf(wj[h], fmaxf(a[h], 0.f), p0);
+                            p1 = fmaf(wj[h + 1], fmaxf(a[h + 1], 0.f), p1);
+                            p2 = fmaf(wj[h + 2], fmaxf(a[h + 2], 0.f), p2);
+                            p3 = fmaf(wj[h + 3], fmaxf(a[h + 3], 0.f), p3);
+                        }
+                        sc = (p0 + p1) + (p2 + p3);
+                    }
                     if (kFp8) sc *= kscale;   // positive per-key scale factors out of the ReLU sum
                     if (s <= row_pos[j]) scores[(int64_t)(g * G + j) * ld + s] = sc;
                 }
                 tc::tc_fence_before();
                 __syncwarp();
                 if (lane == 0) tc::mbar_arrive(&acc_empty[acc]);
-                acc ^= 1;
-                if (acc == 0) acc_phase ^= 1;
+                if (++acc == (uint32_t)C::kAcc) {
+                    acc = 0;
+                    acc_phase ^= 1;
+                }
             }
         } else if (kBs) {
             // ------------------------------------------------------------ key scales -> TMEM
@@ -512,9 +537,9 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
             uint32_t stage = 0, phase = 0;
             uint32_t n = 0;
             for (int64_t f = f_begin; f < f_end; ++f, ++n) {
-                if (!tc::mbar_wait(&raw_full[n & 3], (n >> 2) & 1, abort_flag)) break;
+                if (!tc::mbar_wait(&raw_full[n % C::kR], (n / C::kR) & 1, abort_flag)) break;
                 if (!tc::mbar_wait(&empty[stage], phase ^ 1, abort_flag)) break;
-                const uint8_t* src = raw + (size_t)(n & 3) * (kBM * kDI);
+                const uint8_t* src = raw + (size_t)(n % C::kR) * (kBM * kDI);
                 uint8_t* dst = tiles + (size_t)stage * kTileBytes + half * kHalfBytes;
 #pragma unroll 2
                 for (int i = 0; i < 8; ++i) {
@@ -530,7 +555,7 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
                         // exactly; 2^(E_max - 127) is left to the epilogue.  A block more than
                         // 2^246 below the key's largest is flushed to zero.
                         const uint32_t wd = reinterpret_cast<const uint32_t*>(
-                            kscl + (size_t)(n & 3) * C::kScaleStageBytes)[r];
+                            kscl + (size_t)(n % C::kR) * C::kScaleStageBytes)[r];
                         const int emax = (int)max(max(wd & 0xFFu, (wd >> 8) & 0xFFu),
                                                   max((wd >> 16) & 0xFFu, wd >> 24));
                         const int fe = 247 + (int)((wd >> (8 * (c >> 1))) & 0xFFu) - emax;
@@ -568,7 +593,7 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
                         make_uint4(outw[4], outw[5], outw[6], outw[7]);
                 }
                 tc::fence_async_smem();
-                tc::mbar_arrive(&raw_empty[n & 3]);
+                tc::mbar_arrive(&raw_empty[n % C::kR]);
                 tc::mbar_arrive(&full[stage]);
                 if (++stage == (uint32_t)S) {
                     stage = 0;

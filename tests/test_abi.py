@@ -69,6 +69,14 @@ def test_validation_without_gpu():
                              0.04, fake, hsa.HSA_BF16, None)
     rc = L.hsa_fused_decode_noalloc(ctypes.byref(big), ctypes.byref(ia), ctypes.byref(at), 2048, None)
     assert rc == hsa.HSA_ERR_WORKSPACE and b"scratch" in L.hsa_last_error_message()
+    # the chunked prefill checks its chunk list and score buffers before enqueuing anything
+    pf = hsa.hsa_paged_seq_t(1, fake, fake, 64, 64, 64, 4096, 64, fake, fake, 1, None)
+    bufs = (ctypes.c_void_p * 2)(0x1000, 0x2000)
+    for chunks, rows in (([0, 100], 128), ([32, 32], 128), ([0, 64], 32)):
+        arr = (ctypes.c_int32 * 2)(*chunks)
+        rc = L.hsa_prefill_chunked(ctypes.byref(pf), ctypes.byref(ia), ctypes.byref(at), 2048, arr, 1,
+                                   bufs, rows, 4096, fake, None, None, None)
+        assert rc == hsa.HSA_ERR_INVALID_ARG and b"chunk" in L.hsa_last_error_message(), chunks
     rc = L.hsa_quantize_index(fake, hsa.HSA_BF16, 10, 128, 48, None, 10, fake, fake, None)
     assert rc == hsa.HSA_ERR_INVALID_ARG                       # group does not divide D
     # E4M3 latent cache: the scale group must be a multiple of 16 that divides D_v
