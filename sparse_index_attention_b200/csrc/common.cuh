@@ -84,6 +84,28 @@ __device__ __forceinline__ int64_t paged_slot(const SeqView& v, int32_t b, int32
     return (int64_t)page * v.page_size + (s - lp * v.page_size);
 }
 
+// The same lookup without a branch on the loaded page: an out-of-range page reads slot 0 of page
+// 0 and sets `bad`, which the caller reports once (flag_status) after its loop.  The load's
+// result is not needed until the slot is used, so several lookups can be in flight at once.
+__device__ __forceinline__ int64_t paged_slot_nb(const SeqView& v, int32_t b, int32_t s, bool& bad) {
+    const int32_t lp = s / v.page_size;
+    const int32_t page = __ldg(v.block_table + (int64_t)b * v.bt_stride + lp);
+    const bool out = (uint32_t)page >= (uint32_t)v.num_pages;
+    bad |= out;
+    return (int64_t)(out ? 0 : page) * v.page_size + (s - lp * v.page_size);
+}
+
+// paged_slot for a page size known to be 2^pshift (pshift >= 0): shifts instead of a division.
+__device__ __forceinline__ int64_t paged_slot_pow2(const SeqView& v, int32_t b, int32_t s, int pshift) {
+    const int32_t lp = s >> pshift;
+    int32_t page = __ldg(v.block_table + (int64_t)b * v.bt_stride + lp);
+    if (page < 0 || page >= v.num_pages) {
+        flag_status(v, HSA_DEV_BAD_PAGE);
+        page = 0;
+    }
+    return ((int64_t)page << pshift) + (s & ((1 << pshift) - 1));
+}
+
 __device__ __forceinline__ float to_f32(float x) { return x; }
 __device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
 

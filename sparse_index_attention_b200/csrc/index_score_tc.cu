@@ -240,6 +240,10 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
                 int g = first_group(prefix, n_groups, f_begin), kt, cur = -1;
                 uint32_t stage = 0, phase = 0, qe_phase = 0;
                 GroupInfo gi{0, -1};
+                // box_rows is a power of two (the page size, 8..128, or 128); so usually is the page
+                // size: shifts keep this one thread's per-tile work short
+                const int box_shift = __ffs(box_rows) - 1;
+                const int pshift = (v.page_size & (v.page_size - 1)) == 0 ? __ffs(v.page_size) - 1 : -1;
                 for (int64_t f = f_begin; f < f_end; ++f) {
                     locate(prefix, n_groups, f, g, kt);
                     if (g != cur) {
@@ -256,7 +260,7 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
                     }
                     const int s0 = kt * kBM;
                     const int n_keys = min(kBM, gi.pos_max + 1 - s0);
-                    const int n_boxes = (int)ceil_div(n_keys, box_rows);
+                    const int n_boxes = (n_keys + box_rows - 1) >> box_shift;
                     uint64_t* bar = kFp8 ? &raw_full[stage % C::kR] : &full[stage];
                     if (kFp8) {
                         if (!tc::mbar_wait(&raw_empty[stage % C::kR], ((stage / C::kR) & 1) ^ 1, abort_flag)) break;
@@ -267,7 +271,8 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
                         bar, (uint32_t)(n_boxes * box_rows * (kFp8 ? (kMx ? 132 : 128) : kBs ? 132 : 256)));
                     for (int j = 0; j < n_boxes; ++j) {
                         const int s = s0 + j * box_rows;
-                        const int32_t row = (int32_t)paged_slot(v, gi.b, s);
+                        const int32_t row = (int32_t)(pshift >= 0 ? paged_slot_pow2(v, gi.b, s, pshift)
+                                                                  : paged_slot(v, gi.b, s));
                         if (kFp8) {
                             uint8_t* dst = raw + (size_t)(stage % C::kR) * (kBM * kDI) + (size_t)j * box_rows * 128;
                             tc::tma_load_2d(dst, &tmap_k, bar, 0, row);

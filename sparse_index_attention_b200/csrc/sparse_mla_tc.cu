@@ -215,13 +215,22 @@ sparse_mla_tc_kernel(SeqView v,
                             const int k = (j + e / 16) * kBN + warp * 16 + (e % 16);
                             nn[u] = k < K ? __ldg(idx_row + k) : -1;
                         }
+                        // the eight block-table reads are all in flight before any is used
+                        bool bad_page = false, bad_pos = false;
+                        int32_t sl[8];
 #pragma unroll
                         for (int u = 0; u < 8; ++u) {
-                            int32_t sl = -1;
-                            if (nn[u] >= 0 && nn[u] <= r.pos) sl = (int32_t)paged_slot(v, r.b, nn[u]);
-                            else if (nn[u] != -1 && rank == 0) flag_status(v, HSA_DEV_BAD_POS);
-                            my_slots[e0 + lane + 32 * u] = sl;
+                            const bool ok = nn[u] >= 0 && nn[u] <= r.pos;
+                            bad_pos |= !ok && nn[u] != -1;
+                            bool bp = false;
+                            sl[u] = (int32_t)paged_slot_nb(v, r.b, ok ? nn[u] : 0, bp);
+                            bad_page |= ok && bp;
+                            if (!ok) sl[u] = -1;
                         }
+#pragma unroll
+                        for (int u = 0; u < 8; ++u) my_slots[e0 + lane + 32 * u] = sl[u];
+                        if (bad_page) flag_status(v, HSA_DEV_BAD_PAGE);
+                        if (bad_pos && rank == 0) flag_status(v, HSA_DEV_BAD_POS);
                     }
                     __syncwarp();
                 }
