@@ -30,8 +30,8 @@
 // block-scaled MMA (kind::mxf8f6f4) that reads the E8M0 scales from TMEM.
 //
 // Warp roles: 0 TMA producer, 1 MMA issuer (one elected thread each), 2-5 epilogue
-// (TMEM lane quarters 2,3,0,1), 6-9 FP8 converters (FP8 keys) or key-scale writers
-// (block-scaled MMA).
+// (TMEM lane quarters 2,3,0,1), 6-9 (6-13 for E4M3 keys with one row per tile) FP8
+// converters, or 6-9 key-scale writers (block-scaled MMA).
 #include <algorithm>
 
 #include "kernels.h"
@@ -69,7 +69,10 @@ struct Cfg {
     static constexpr int kTmemCols = kBs ? 512 : kAcc * N;   // 256 or 512
     static_assert(!kBs || kSfbCol + N / 32 <= kTmemCols, "TMEM budget");
     static_assert(kAcc * N <= kTmemCols, "TMEM budget");
-    static constexpr int kThreads = (kFp8 || kBs) ? 320 : 192;
+    // FP8 converter warps: eight for E4M3 keys with one query row per tile (the widening sets the
+    // pace of the key stream there), four otherwise (measured: the MX widening is slower with eight)
+    static constexpr int kConv = kFp8 ? ((G == 1 && !kMx) ? 8 : 4) : 0;
+    static constexpr int kThreads = kFp8 ? 192 + 32 * kConv : (kBs ? 320 : 192);
     static constexpr int kBarBytes = 512;
     static constexpr size_t kSmem = 1024 + (size_t)kStages * kTile + (size_t)kRawStages * (kBM * kDI) +
                                     (size_t)kScaleStages * kScaleStageBytes + kQBytes +
@@ -173,7 +176,7 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
 
     if (tid == 0) {
         for (int i = 0; i < S; ++i) {
-            tc::mbar_init(&full[i], kFp8 ? 128 : 1);
+            tc::mbar_init(&full[i], kFp8 ? 32 * C::kConv : 1);
             tc::mbar_init(&empty[i], 1);
             tc::mbar_init(&sf_full[i], 4);
         }
@@ -185,7 +188,7 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
         tc::mbar_init(q_empty, 1);
         for (int i = 0; i < C::kR; ++i) {
             tc::mbar_init(&raw_full[i], 1);
-            tc::mbar_init(&raw_empty[i], 128);
+            tc::mbar_init(&raw_empty[i], 32 * C::kConv);
         }
         tc::mbar_init(epi_bar, 4);
         tc::mbar_init(q_ready, 4);
@@ -367,6 +370,7 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
             uint32_t acc = 0, acc_phase = 0;
             int32_t row_pos[G];
             int32_t seq_b = 0;
+            const int epi_pshift = (v.page_size & (v.page_size - 1)) == 0 ? __ffs(v.page_size) - 1 : -1;
             uint32_t qf_phase = 0;
             tc::WarpSetSync epi_sync{epi_bar, 0};
             for (int64_t f = f_begin; f < f_end; ++f) {
@@ -462,7 +466,8 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
 #pragma unroll
                     for (int j = 0; j < G; ++j) pmax = max(pmax, row_pos[j]);
                     if (s <= pmax) {
-                        const int64_t slot = paged_slot(v, seq_b, s);
+                        const int64_t slot = epi_pshift >= 0 ? paged_slot_pow2(v, seq_b, s, epi_pshift)
+                                                             : paged_slot(v, seq_b, s);
                         if (kMx) {
                             // the largest of the key's four block exponents; the converters
                             // scaled every block relative to it
@@ -535,7 +540,8 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
             // instruction, into the two 64-column swizzled halves of the bf16 tile the MMA reads
             // (e4m3 -> f16 -> bf16 is exact); a row's eight lanes read 128 contiguous bytes, so
             // the staging reads are free of bank conflicts
-            const int cw = (tid - 192) >> 5;           // converter warp 0..3: rows 32cw..32cw+31
+            constexpr int kRowsPerWarp = kBM / (C::kConv > 0 ? C::kConv : 4);   // 16 or 32
+            const int cw = (tid - 192) >> 5;           // converter warp: rows kRowsPerWarp x cw ..
             const int c = lane & 7;                    // 16-code chunk of the row
             const int half = c >> 2;                   // which 64-column half it lands in
             const int chunk = (c & 3) * 2;             // first of its two 16-byte chunks there
@@ -546,9 +552,9 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
                 if (!tc::mbar_wait(&empty[stage], phase ^ 1, abort_flag)) break;
                 const uint8_t* src = raw + (size_t)(n % C::kR) * (kBM * kDI);
                 uint8_t* dst = tiles + (size_t)stage * kTileBytes + half * kHalfBytes;
-#pragma unroll 2
-                for (int i = 0; i < 8; ++i) {
-                    const int r = 32 * cw + 4 * i + (lane >> 3);
+#pragma unroll
+                for (int i = 0; i < kRowsPerWarp / 4; ++i) {
+                    const int r = kRowsPerWarp * cw + 4 * i + (lane >> 3);
                     const uint4 in = *reinterpret_cast<const uint4*>(src + r * 128 + c * 16);
                     const uint32_t words[4] = {in.x, in.y, in.z, in.w};
                     uint32_t outw[8];
