@@ -17,8 +17,10 @@
  *
  * Conventions shared by every call
  *  - Memory: every tensor is caller-owned device memory, row-major and contiguous unless a
- *    stride is given.  The library never allocates device memory.  Calls that need scratch take
- *    a workspace pointer and size; hsa_*_workspace_size() reports the bytes needed.
+ *    stride is given.  The library never allocates device memory at run time.  Calls that need
+ *    scratch take a workspace pointer and size; hsa_*_workspace_size() reports the bytes needed.
+ *    The one exception is hsa_fused_decode_noalloc, whose scratch is a fixed array of the library
+ *    itself (see there).
  *  - Streams: every call is asynchronous on the cudaStream_t passed in as `stream` (NULL = the
  *    legacy default stream).  Host-side argument checks happen before anything is enqueued.
  *  - Errors: every call returns an hsa_status_t.  HSA_ERR_INVALID_ARG: null pointer, size out of
@@ -32,8 +34,9 @@
  *    context stays usable.  Bits: HSA_DEV_BAD_PAGE, HSA_DEV_BAD_POS, HSA_DEV_BAD_GROUP,
  *    HSA_DEV_TIMEOUT (every wait inside a kernel is bounded; one that gives up makes the kernel
  *    leave early and sets this bit instead of hanging the GPU).
- *  - Threading: no mutable global state beyond a per-thread error message; calls on different
- *    streams may be issued from different host threads.
+ *  - Threading: no mutable global state beyond a per-thread error message, a launch counter
+ *    and hsa_fused_decode_noalloc's scratch (shared by its calls); calls on different streams
+ *    may be issued from different host threads.
  */
 #ifndef HSA_H_
 #define HSA_H_
