@@ -226,8 +226,8 @@ def hsa_sparse_mla_workspace_size(seq: PagedSeq, H: int, D_qk: int, D_v: int, K:
 
 
 def _workspace(nbytes: int, device, ws):
-    """Workspace of nbytes (zero-filled: the attention's split schedule keeps row counters there,
-    which must start at zero and which every call leaves at zero)."""
+    """Workspace of nbytes (at least one byte; the current attention kernels report 0 and use
+    none), zero-filled, or the caller's own `ws`."""
     if ws is not None:
         return ws
     return torch.zeros(max(nbytes, 1), dtype=torch.uint8, device=device)

@@ -202,8 +202,7 @@ size_t attn_ws_bytes(const hsa::SparseMlaArgs& a) {
 hsa_status_t run_attn(const hsa::SparseMlaArgs& a, cudaStream_t st) {
     if (a.seq.T_q == 0) return HSA_OK;
     if (hsa::sparse_mla_tc_supported(a)) {
-        // a workspace smaller than the split schedule needs (or none) selects whole rows per
-        // cluster; a given workspace must be 256-byte aligned
+        // the tensor-core kernel needs no workspace; one that is given must be 256-byte aligned
         HSA_REQUIRE(a.ws == nullptr || a.ws_bytes == 0 || aligned(a.ws, 256), HSA_ERR_WORKSPACE,
                     "workspace must be 256-byte aligned");
         return cuda_status(hsa::launch_sparse_mla_tc(a, st), "sparse_mla_attn (tensor core)");
