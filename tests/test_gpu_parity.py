@@ -73,6 +73,10 @@ def test_index_score_mx_block_scaled_vs_oracle(name, kw):
     """MXFP8 queries and keys as codes + E8M0 scales (hsa_index_score_mx: the block-scaled MMA on
     the codes), against the float64 score of the oracle's own MX quantization of both, and
     against the bf16-query MX path on the same rounded queries."""
+    _index_mx_bs_vs_oracle(name, kw)
+
+
+def _index_mx_bs_vs_oracle(name, kw):
     wl = workloads.make(name, DEV, **kw)
     wl.index_fp8 = wl.index_mx = True
     seq = paged_seq(wl)
@@ -146,10 +150,13 @@ def test_index_score_row_groupings(q_run, T):
     _index_vs_oracle(wl, rows=sorted(set(range(0, T, 7)) | {T - 1}))
 
 
-@pytest.mark.parametrize("page_size", [16, 128, 256])
+@pytest.mark.parametrize("page_size", [16, 128, 256, 384])
 def test_index_score_page_sizes(page_size):
+    """Page sizes below, at and above the 128-key tile (384: not a power of two, so the kernel's
+    page arithmetic takes its division path), for bf16, E4M3 and block-scaled MXFP8 keys."""
     _index_vs_oracle(workloads.make("decode_bf16", DEV, B=4, L_min=200, L_max=1300, page_size=page_size))
     _index_vs_oracle(workloads.make("decode_fp8", DEV, B=2, L=900, page_size=page_size))
+    _index_mx_bs_vs_oracle("decode_bf16", dict(B=3, L_min=300, L_max=1200, page_size=page_size))
 
 
 def test_index_score_integer_inputs_bit_exact():
@@ -364,6 +371,14 @@ def _attn_vs_oracle(wl, tol, idx=None, kv_group=None):
 ])
 def test_sparse_mla_vs_oracle(name, kw, tol):
     _attn_vs_oracle(workloads.make(name, DEV, **kw), tol)
+
+
+@pytest.mark.parametrize("page_size", [16, 384])
+def test_sparse_mla_page_sizes(page_size):
+    """The gather's slot lookups with small pages and with a page size that is not a power of
+    two, bf16 and FP8 caches."""
+    _attn_vs_oracle(workloads.make("decode_bf16", DEV, B=3, L_min=2200, L_max=4000, page_size=page_size), 2e-2)
+    _attn_vs_oracle(workloads.make("decode_fp8", DEV, B=2, L=2600, page_size=page_size), 6e-2)
 
 
 @pytest.mark.parametrize("name,kw,block", [
