@@ -31,7 +31,8 @@
 //
 // Warp roles: 0 TMA producer, 1 MMA issuer (one elected thread each), 2-5 epilogue
 // (TMEM lane quarters 2,3,0,1), 6-9 (6-13 for E4M3 keys with one row per tile) FP8
-// converters, or 6-9 key-scale writers (block-scaled MMA).
+// converters, or 6-9 key-scale writers (block-scaled MMA); with two or four rows per tile
+// four more epilogue warps after those, each pair of a lane quarter summing half of the rows.
 #include <algorithm>
 
 #include "kernels.h"
@@ -72,7 +73,12 @@ struct Cfg {
     // FP8 converter warps: eight for E4M3 keys with one query row per tile (the widening sets the
     // pace of the key stream there), four otherwise (measured: the MX widening is slower with eight)
     static constexpr int kConv = kFp8 ? ((G == 1 && !kMx) ? 8 : 4) : 0;
-    static constexpr int kThreads = kFp8 ? 192 + 32 * kConv : (kBs ? 320 : 192);
+    // epilogue warps: four (one per TMEM lane quarter), or eight with two or four rows per tile
+    // (two warps per quarter, each summing half of the rows: there the epilogue sets the pace);
+    // the second four come after the converter / key-scale warps
+    static constexpr int kEpiWarps = (G >= 2 && !kBs) ? 8 : 4;
+    static constexpr int kEpiB0 = 6 + (kFp8 ? kConv : (kBs ? 4 : 0));
+    static constexpr int kThreads = 32 * (kEpiB0 + (kEpiWarps == 8 ? 4 : 0));
     static constexpr int kBarBytes = 512;
     static constexpr size_t kSmem = 1024 + (size_t)kStages * kTile + (size_t)kRawStages * (kBM * kDI) +
                                     (size_t)kScaleStages * kScaleStageBytes + kQBytes +
@@ -182,7 +188,7 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
         }
         for (int i = 0; i < C::kAcc; ++i) {
             tc::mbar_init(&acc_full[i], 1);
-            tc::mbar_init(&acc_empty[i], 4);
+            tc::mbar_init(&acc_empty[i], C::kEpiWarps);
         }
         tc::mbar_init(q_full, 1);
         tc::mbar_init(q_empty, 1);
@@ -190,8 +196,8 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
             tc::mbar_init(&raw_full[i], 1);
             tc::mbar_init(&raw_empty[i], 32 * C::kConv);
         }
-        tc::mbar_init(epi_bar, 4);
-        tc::mbar_init(q_ready, 4);
+        tc::mbar_init(epi_bar, C::kEpiWarps);
+        tc::mbar_init(q_ready, C::kEpiWarps);
         *abort_flag = 0;
         tc::fence_barrier_init();
     }
@@ -361,11 +367,16 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
                 }
             }
             __syncwarp();
-        } else if (warp < 6) {
+        } else if (warp < 6 || (C::kEpiWarps == 8 && warp >= C::kEpiB0)) {
             // ------------------------------------------------------------ epilogue
             const int quarter = warp & 3;
             const int r_in_tile = quarter * 32 + lane;
-            const int et = tid - 64;  // 0..127
+            constexpr int kEpiThreads = 32 * C::kEpiWarps;
+            const int ehalf = warp >= 6 ? 1 : 0;      // second epilogue warp of its lane quarter
+            const int et = ehalf ? 128 + tid - 32 * C::kEpiB0 : tid - 64;   // 0 .. kEpiThreads - 1
+            // the row groups this warp sums: all, or its half of them
+            const int jlo = C::kEpiWarps == 8 ? ehalf * (G / 2) : 0;
+            const int jhi = C::kEpiWarps == 8 ? jlo + G / 2 : G;
             int g = first_group(prefix, n_groups, f_begin), kt, cur = -1;
             uint32_t acc = 0, acc_phase = 0;
             int32_t row_pos[G];
@@ -385,7 +396,7 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
                         if (!tc::mbar_wait(q_full, qf_phase, abort_flag)) break;
                         qf_phase ^= 1;
                         const int hf = et & 1;
-                        for (int i = et >> 1; i < N; i += 64) {
+                        for (int i = et >> 1; i < N; i += kEpiThreads / 2) {
                             uint4* rowp = reinterpret_cast<uint4*>(qbuf + (size_t)hf * (N * 128) + (size_t)i * 128);
                             uint4 x[8];
                             float mx = 0.f;
@@ -422,7 +433,7 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
                         }
                         tc::fence_async_smem();   // the f16 queries -> the tensor core
                     } else {
-                        for (int i = et; i < N; i += 128) {
+                        for (int i = et; i < N; i += kEpiThreads) {
                             const int t = g * G + i / kHI;
                             w_s[i] = t < v.T_q ? w[(int64_t)t * kHI + (i % kHI)] : 0.f;
                         }
@@ -482,6 +493,7 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
                 }
 #pragma unroll
                 for (int j = 0; j < G; ++j) {
+                    if (j < jlo || j >= jhi) continue;
                     float a[64];
                     const float* wj = w_s + j * kHI;
                     float sc = 0.f;
