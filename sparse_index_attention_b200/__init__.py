@@ -554,8 +554,11 @@ def hsa_prefill_chunked(seq: PagedSeq, q_I, w, k_cache, k_scale, q, kv, kv_scale
     bufs = list(prefill_score_buffers(seq, chunks, dev, 2) if own else score_bufs)
     rows_max = max(r1 - r0 for r0, r1 in chunks)
     if len(bufs) < 2 or bufs[0].shape != bufs[1].shape or bufs[0].shape[0] < rows_max or \
-            bufs[0].shape[1] < seq.max_seq_len or not all(b.is_contiguous() for b in bufs[:2]):
-        raise ValueError("two contiguous score buffers of at least [max chunk rows, max_seq_len]")
+            bufs[0].shape[1] < seq.max_seq_len or \
+            not all(b.is_contiguous() and b.dtype == torch.float32 for b in bufs[:2]):
+        raise ValueError("two contiguous fp32 score buffers of at least [max chunk rows, max_seq_len]")
+    if len(streams) != 2:
+        raise ValueError("streams must be a pair (the chunks alternate between them)")
     T_qI, H_I, D_I = q_I.shape
     ia = hsa_index_args_t(_ptr(q_I), _dtype(q_I), _ptr(w), H_I, D_I, _ptr(k_cache),
                           _key_dtype(k_cache, k_scale), _ptr(k_scale), None)
