@@ -36,6 +36,10 @@ constexpr int kThreads = 1024;
 constexpr int kWarps = kThreads / 32;
 constexpr int kBins = 2048;
 constexpr int kSample = 4096;
+// 32-key groups per warp step of the candidate sweeps: sixteen for rows read from L2 (all
+// sixteen reads in flight before the first is used; those sweeps are latency-bound), four for
+// rows staged in shared memory (measured faster there)
+template <bool kStaged> constexpr int kSweep = kStaged ? 4 : 16;
 constexpr int kSampleMinRow = 2 * kSample;     // shorter rows go straight to the exact steps
 constexpr int kSmemKeys = 40 * 1024;           // staged keys (160 KB)
 constexpr int kMaxSmem = 227 * 1024;
@@ -245,15 +249,21 @@ topk_kernel(SeqView v, const float* __restrict__ scores, int64_t ld, int K, int 
             __syncthreads();
             const uint32_t L = radix_select<2>([&](int i) { return sample[i]; }, kSample,
                                                (uint32_t)rank, hist, wsum, misc).key;
-            // warp segments of whole 128-key chunks, swept four keys per lane at a time
+            // warp segments of whole 128-key chunks, swept kSweep keys per lane at a time
             const int seg = ((n + kWarps * 128 - 1) / (kWarps * 128)) * 128;
             const int s0 = min(n, warp * seg), s1 = min(n, s0 + seg);
             uint32_t c = 0u;
-            for (int j = s0; j < s1; j += 128) {
+            for (int j = s0; j < s1; j += 32 * kSweep<kStaged>) {
+                uint32_t u[kSweep<kStaged>];
 #pragma unroll
-                for (int a = 0; a < 4; ++a) {
+                for (int a = 0; a < kSweep<kStaged>; ++a) {
                     const int i = j + 32 * a + lane;
-                    c += (uint32_t)__popc(__ballot_sync(0xffffffffu, i < s1 && key_at(i) >= L));
+                    u[a] = i < s1 ? key_at(i) : 0u;
+                }
+#pragma unroll
+                for (int a = 0; a < kSweep<kStaged>; ++a) {
+                    const int i = j + 32 * a + lane;
+                    c += (uint32_t)__popc(__ballot_sync(0xffffffffu, i < s1 && u[a] >= L));
                 }
             }
             if (lane == 0) wsum[warp] = c;
@@ -268,16 +278,20 @@ topk_kernel(SeqView v, const float* __restrict__ scores, int64_t ld, int K, int 
             __syncthreads();
             if (total >= (uint32_t)K && total <= (uint32_t)cand_cap) {     // the same in every thread
                 const uint32_t lt = lanemask_lt();
-                for (int j = s0; j < s1; j += 128) {
-                    uint32_t u[4], bal[4];
+                for (int j = s0; j < s1; j += 32 * kSweep<kStaged>) {
+                    uint32_t u[kSweep<kStaged>], bal[kSweep<kStaged>];
 #pragma unroll
-                    for (int a = 0; a < 4; ++a) {
+                    for (int a = 0; a < kSweep<kStaged>; ++a) {
                         const int i = j + 32 * a + lane;
                         u[a] = i < s1 ? key_at(i) : 0u;
+                    }
+#pragma unroll
+                    for (int a = 0; a < kSweep<kStaged>; ++a) {
+                        const int i = j + 32 * a + lane;
                         bal[a] = __ballot_sync(0xffffffffu, i < s1 && u[a] >= L);
                     }
 #pragma unroll
-                    for (int a = 0; a < 4; ++a) {
+                    for (int a = 0; a < kSweep<kStaged>; ++a) {
                         if ((bal[a] >> lane) & 1u) {
                             const uint32_t p = before + (uint32_t)__popc(bal[a] & lt);
                             cand_key[p] = u[a];
