@@ -65,6 +65,35 @@ int main(void) {
     CHECK(hsa_dequantize_mx((const uint8_t*)fake, (const uint8_t*)fake, 10, 64, (void*)fake,
                             HSA_E4M3, NULL) == HSA_ERR_UNSUPPORTED);
 
+    /* MXFP8 queries: their scale bytes must be given, 16-byte aligned */
+    st = hsa_index_score_mx(&seq, (const uint8_t*)fake, NULL, (const float*)fake, 4, 32,
+                            (const uint8_t*)fake, (const uint8_t*)fake, (float*)fake, 64, NULL);
+    CHECK(st == HSA_ERR_INVALID_ARG);
+
+    /* the chunked prefill checks its chunk list: [0, 100) lies outside T_q = 2 */
+    {
+        hsa_index_args_t ia;
+        hsa_attn_args_t at;
+        int32_t chunks[2] = {0, 100};
+        float* bufs[2] = {(float*)0x1000, (float*)0x2000};
+        memset(&ia, 0, sizeof ia);
+        memset(&at, 0, sizeof at);
+        ia.q_I = fake; ia.q_dtype = HSA_BF16; ia.w = (const float*)fake; ia.H_I = 4; ia.D_I = 32;
+        ia.k_cache = fake; ia.k_dtype = HSA_BF16;
+        at.q = fake; at.q_dtype = HSA_BF16; at.H = 8; at.D_qk = 80; at.D_v = 64; at.kv = fake;
+        at.kv_dtype = HSA_BF16; at.kv_scale_group = 64; at.softmax_scale = 0.1f;
+        at.out = (void*)fake; at.out_dtype = HSA_BF16;
+        st = hsa_prefill_chunked(&seq, &ia, &at, 32, chunks, 1, bufs, 128, 64, (int32_t*)fake, NULL,
+                                 NULL, NULL);
+        CHECK(st == HSA_ERR_INVALID_ARG);
+        /* the no-allocation decode step rejects a step larger than its scratch before anything
+           touches the device: 2 rows x 2^23 positions of fp32 scores */
+        empty = seq;
+        empty.max_seq_len = 1 << 23;
+        st = hsa_fused_decode_noalloc(&empty, &ia, &at, 32, NULL);
+        CHECK(st == HSA_ERR_WORKSPACE);
+    }
+
     /* zero query rows is a no-op, not an error */
     empty = seq;
     empty.T_q = 0;
