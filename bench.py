@@ -729,6 +729,32 @@ def run_profile_case(args):
     print(json.dumps({"profile_case": "prefill_bf16", "rows": wl.T_q, "launches_per_kernel": 3}))
 
 
+def run_profile_decode_fp8(args):
+    """The FP8 decode batch's shapes with --profile-fp8-seqs sequences of 65536 keys (E4M3 index
+    keys with fp32 scales, FP8 latent cache): index score, Top-K and sparse MLA, each called
+    three times on one stream, nothing timed.  For one-kernel ncu captures."""
+    import sparse_index_attention_b200 as hsa
+    dev = "cuda"
+    wl = workloads.make("decode_fp8", dev, B=args.profile_fp8_seqs)
+    seq = hsa.PagedSeq(wl.seq_lens, wl.block_table, wl.page_size, wl.num_pages, wl.q_seq, wl.q_pos,
+                       q_run=wl.q_run)
+    k8, ks = hsa.hsa_quantize_index(wl.k_I, wl.D_I)
+    ks = ks.view(-1)
+    kv8, kvs, rope = hsa.hsa_quantize_kv(wl.kv, wl.D_v, wl.D_v)
+    kvs = kvs.view(-1)
+    sc = hsa.hsa_index_score(seq, wl.q_I, wl.w, k8, ks)
+    idx = hsa.hsa_topk(seq, sc, wl.K)
+    out, lse = hsa.hsa_sparse_mla_attn(seq, wl.q, kv8, idx, wl.D_v, wl.softmax_scale, kv_scale=kvs,
+                                       kv_rope=rope)
+    for _ in range(2):
+        hsa.hsa_index_score(seq, wl.q_I, wl.w, k8, ks, scores=sc)
+        hsa.hsa_topk(seq, sc, wl.K, idx=idx)
+        hsa.hsa_sparse_mla_attn(seq, wl.q, kv8, idx, wl.D_v, wl.softmax_scale, kv_scale=kvs,
+                                kv_rope=rope, out=out, lse=lse)
+    torch.cuda.synchronize()
+    print(json.dumps({"profile_case": "decode_fp8", "sequences": wl.B, "launches_per_kernel": 3}))
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -744,9 +770,15 @@ def main():
     ap.add_argument("--profile-rows", type=int, default=0,
                     help="only run a small prefill of this many rows (three calls of each kernel, "
                          "for ncu captures) and exit")
+    ap.add_argument("--profile-fp8-seqs", type=int, default=0,
+                    help="only run the FP8 decode kernels on this many 65536-key sequences (three "
+                         "calls each, for ncu captures) and exit")
     args = ap.parse_args()
     if args.profile_rows > 0:
         run_profile_case(args)
+        return
+    if args.profile_fp8_seqs > 0:
+        run_profile_decode_fp8(args)
         return
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

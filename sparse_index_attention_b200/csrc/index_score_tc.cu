@@ -17,10 +17,14 @@
 // changes.  Every CTA derives the list itself from q_pos (prefix sum in shared memory).
 //
 // Data movement.  Keys come through the block table page by page with 2D TMA loads (128-byte
-// swizzle, two 64-column halves per page); FP8 keys are loaded raw and widened in shared memory
-// by four converter warps (E4M3 -> f16 in one conversion, exact; the MMA then runs in f16, the
-// queries rescaled into f16's range per head), and the per-key fp32 scale multiplies the
-// finished score (the scale is positive, so it commutes with the ReLU sum).  MXFP8 keys (one
+// swizzle, two 64-column halves per page).  E4M3 keys with one query row per tile (and a
+// 16-byte-aligned scale array) go straight from TMA to an 8-bit MMA (kind::f8f6f4): each bf16 query row x head is split exactly into two
+// E4M3 code rows, hi and lo / 16 (scaled per head by a power of two folded into its weight), so
+// one MMA of N = 128 gives hi . k and lo . k per head, and the per-key fp32 scales are
+// bulk-copied beside the codes for the epilogue.  Otherwise the E4M3 codes are loaded raw and widened in shared memory by four converter warps (E4M3 -> f16 in one
+// conversion, exact; the MMA then runs in f16, the queries rescaled into f16's range per head).
+// Either way the per-key fp32 scale multiplies the finished score (the scale is positive, so it
+// commutes with the ReLU sum).  MXFP8 keys (one
 // E8M0 byte per 32 dims; "Inference Adaptation and Performance Optimization for a Domestically
 // Developed LLM's New Architecture", section 4 table) with bf16 queries take the same path: the
 // producer bulk-copies each box's scale words beside its codes, the converters place the codes'
@@ -30,9 +34,10 @@
 // block-scaled MMA (kind::mxf8f6f4) that reads the E8M0 scales from TMEM.
 //
 // Warp roles: 0 TMA producer, 1 MMA issuer (one elected thread each), 2-5 epilogue
-// (TMEM lane quarters 2,3,0,1), 6-9 (6-13 for E4M3 keys with one row per tile) FP8
-// converters, or 6-9 key-scale writers (block-scaled MMA); with two or four rows per tile
-// four more epilogue warps after those, each pair of a lane quarter summing half of the rows.
+// (TMEM lane quarters 2,3,0,1), 6-9 (6-13 for E4M3 keys with one row per tile) FP8 converters
+// when the codes are widened, or 6-9 key-scale writers (block-scaled MMA); with two or four
+// rows per tile four more epilogue warps after those, each pair of a lane quarter summing half
+// of the rows.
 #include <algorithm>
 
 #include "kernels.h"
@@ -48,28 +53,32 @@ constexpr int kHI = 64;                  // index heads
 constexpr int kHalfBytes = kBM * 128;    // one 64-column swizzled half of a key tile: 16 KB
 constexpr int kTileBytes = 2 * kHalfBytes;
 
-template <int G, bool kFp8, bool kMx = false, bool kBs = false>
+template <int G, bool kFp8, bool kMx = false, bool kBs = false, bool kSp = false>
 struct Cfg {
     static_assert(!kBs || (G <= 2 && !kFp8 && !kMx), "block-scaled: codes straight to the MMA, G <= 2");
+    static_assert(!kSp || (G == 1 && !kFp8 && !kMx && !kBs), "split queries: E4M3 codes straight to the MMA, G = 1");
     static constexpr int N = G * kHI;
-    static constexpr int kTile = kBs ? kBM * kDI : kTileBytes;  // one MMA stage: 16 KB codes or 32 KB bf16
+    // MMA N = TMEM columns per accumulator: the split-query path holds two code rows per head
+    static constexpr int kNm = kSp ? 2 * N : N;
+    static constexpr int kTile = (kBs || kSp) ? kBM * kDI : kTileBytes;  // one MMA stage: 16 KB codes or 32 KB bf16
     static constexpr int kQBytes = N * kDI * (kBs ? 1 : 2);
-    static constexpr int kStages = kBs ? (G == 1 ? 8 : 6)
+    static constexpr int kStages = kSp ? 12 : kBs ? (G == 1 ? 8 : 6)
                                        : kFp8 ? (G == 1 ? 4 : (G == 2 ? 3 : 2)) : (G == 1 ? 6 : (G == 2 ? 5 : 4));
     static constexpr int kRawStages = kFp8 ? 4 : 0;          // FP8 staging tiles (16 KB each)
     static constexpr int kR = kRawStages > 0 ? kRawStages : 1;
-    static constexpr int kScaleStageBytes = (kMx || kBs) ? kBM * 4 : 0;  // 4 E8M0 bytes per key
-    static constexpr int kScaleStages = kBs ? kStages : kRawStages;
+    // 4 E8M0 bytes or one fp32 scale per key
+    static constexpr int kScaleStageBytes = (kMx || kBs || kSp) ? kBM * 4 : 0;
+    static constexpr int kScaleStages = (kBs || kSp) ? kStages : kRawStages;
     static constexpr int kMaxGroups = G == 1 ? 2048 : 4096;
     // TMEM: kAcc accumulators of N columns (four for N <= 128, so the MMA may run up to four
     // tiles ahead of the epilogue; two for N = 256); block-scaled adds the key scales (4 columns
     // per stage) and the query scales (N / 32 columns) after them
-    static constexpr int kAcc = (N <= 64 || (N == 128 && !kBs)) ? 4 : 2;
-    static constexpr int kSfaCol = kAcc * N;
+    static constexpr int kAcc = (kNm <= 64 || (kNm == 128 && !kBs)) ? 4 : 2;
+    static constexpr int kSfaCol = kAcc * kNm;
     static constexpr int kSfbCol = kSfaCol + 4 * kStages;
-    static constexpr int kTmemCols = kBs ? 512 : kAcc * N;   // 256 or 512
+    static constexpr int kTmemCols = kBs ? 512 : kAcc * kNm;   // 256 or 512
     static_assert(!kBs || kSfbCol + N / 32 <= kTmemCols, "TMEM budget");
-    static_assert(kAcc * N <= kTmemCols, "TMEM budget");
+    static_assert(kAcc * kNm <= kTmemCols, "TMEM budget");
     // FP8 converter warps: eight for E4M3 keys with one query row per tile (the widening sets the
     // pace of the key stream there), four otherwise (measured: the MX widening is slower with eight)
     static constexpr int kConv = kFp8 ? ((G == 1 && !kMx) ? 8 : 4) : 0;
@@ -79,7 +88,7 @@ struct Cfg {
     static constexpr int kEpiWarps = (G >= 2 && !kBs) ? 8 : 4;
     static constexpr int kEpiB0 = 6 + (kFp8 ? kConv : (kBs ? 4 : 0));
     static constexpr int kThreads = 32 * (kEpiB0 + (kEpiWarps == 8 ? 4 : 0));
-    static constexpr int kBarBytes = 512;
+    static constexpr int kBarBytes = kStages > 10 ? 640 : 512;
     static constexpr size_t kSmem = 1024 + (size_t)kStages * kTile + (size_t)kRawStages * (kBM * kDI) +
                                     (size_t)kScaleStages * kScaleStageBytes + kQBytes +
                                     4 * (kMaxGroups + 1) + 4 * N + kBarBytes;
@@ -131,21 +140,27 @@ __device__ __forceinline__ int first_group(const int32_t* prefix, int n_groups, 
     return lo;
 }
 
-template <int G, bool kFp8, bool kMx, bool kBs = false>
-__global__ void __launch_bounds__(Cfg<G, kFp8, kMx, kBs>::kThreads, 1)
+template <int G, bool kFp8, bool kMx, bool kBs = false, bool kSp = false>
+__global__ void __launch_bounds__(Cfg<G, kFp8, kMx, kBs, kSp>::kThreads, 1)
 index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_q,
                       SeqView v, int32_t q_row0, const float* __restrict__ w,
                       const void* __restrict__ k_scale, const uint32_t* __restrict__ q_scale,
                       float* __restrict__ scores, int64_t ld, int32_t box_rows) {
-    using C = Cfg<G, kFp8, kMx, kBs>;
+    using C = Cfg<G, kFp8, kMx, kBs, kSp>;
     static_assert(!kMx || kFp8, "MXFP8 keys go through the FP8 staging path");
+    // kSp (E4M3 keys with fp32 scales, one query row per tile): the key codes go from TMA straight
+    // to a kind::f8f6f4 MMA.  Each bf16 query row x head is split exactly into two E4M3 code rows
+    // (hi and lo / 16, below), so one MMA of N = 128 gives both partial dot products per head.
+    constexpr bool kKeyScale = kFp8 || kSp;   // a per-key scale multiplies the finished score
+    constexpr bool kCodes = kBs || kSp;       // 8-bit codes straight into the MMA stages
     // E4M3 keys with fp32 scales run the MMA in f16: a code widens to f16 in one conversion
     // (exact), and the queries are rescaled per head by a power of two into f16's range, the
     // inverse power folded into the head weight, which leaves every product and sum as in bf16.
     constexpr bool kF16 = kFp8 && !kMx;
     constexpr int N = C::N;
     constexpr int S = C::kStages;
-    constexpr uint32_t kIdesc = kF16 ? tc::idesc_f16_f32(kBM, N) : tc::idesc_bf16_f32(kBM, N, 0, 0);
+    constexpr uint32_t kIdesc = kSp ? tc::idesc_e4m3_f32(kBM, C::kNm)
+                              : kF16 ? tc::idesc_f16_f32(kBM, N) : tc::idesc_bf16_f32(kBM, N, 0, 0);
     // kBs (MXFP8 queries and keys): the codes go from TMA straight to a block-scaled MMA
     // (kind::mxf8f6f4, K = 32 per instruction, one E8M0 scale per 32 dims of every key and
     // query row, read from TMEM); warps 6-9 place each tile's key scales in TMEM, the epilogue
@@ -170,7 +185,8 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
     uint64_t* epi_bar = raw_empty + 8;     // the four epilogue warps
     uint64_t* q_ready = epi_bar + 1;       // f16 MMA: the group's queries converted; block-scaled:
                                            // the group's query scales in TMEM (4 warps)
-    uint64_t* sf_full = q_ready + 1;       // [S] block-scaled: the tile's key scales in TMEM (4 warps)
+    uint64_t* sf_full = q_ready + 1;       // [S] block-scaled: the tile's key scales in TMEM (4 warps);
+                                           // split queries: the epilogue is done with them (4 warps)
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(sf_full + S);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
     static_assert((3 * S + 4 + 4 + 2 + 16 + 2) * 8 + 8 <= C::kBarBytes && C::kR <= 8 && C::kAcc <= 4, "barrier block");
@@ -275,9 +291,11 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
                         if (!tc::mbar_wait(&raw_empty[stage % C::kR], ((stage / C::kR) & 1) ^ 1, abort_flag)) break;
                     } else {
                         if (!tc::mbar_wait(&empty[stage], phase ^ 1, abort_flag)) break;
+                        // the stage's key scales outlive the MMA: the epilogue reads them
+                        if (kSp && !tc::mbar_wait(&sf_full[stage], phase ^ 1, abort_flag)) break;
                     }
                     tc::mbar_arrive_expect_tx(
-                        bar, (uint32_t)(n_boxes * box_rows * (kFp8 ? (kMx ? 132 : 128) : kBs ? 132 : 256)));
+                        bar, (uint32_t)(n_boxes * box_rows * (kFp8 ? (kMx ? 132 : 128) : kCodes ? 132 : 256)));
                     for (int j = 0; j < n_boxes; ++j) {
                         const int s = s0 + j * box_rows;
                         const int32_t row = (int32_t)(pshift >= 0 ? paged_slot_pow2(v, gi.b, s, pshift)
@@ -289,7 +307,9 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
                                 tc::bulk_load(kscl + (size_t)(stage % C::kR) * C::kScaleStageBytes + (size_t)j * box_rows * 4,
                                               static_cast<const uint8_t*>(k_scale) + (int64_t)row * 4,
                                               (uint32_t)box_rows * 4, bar);
-                        } else if (kBs) {   // codes straight into the MMA stage, scale words beside
+                        } else if (kCodes) {   // codes straight into the MMA stage, scales beside
+                            // (E8M0 words or fp32, 4 bytes per key; row is a multiple of box_rows,
+                            // so the copy is 32-byte aligned and ends inside the scale array)
                             uint8_t* dst = tiles + (size_t)stage * C::kTile + (size_t)j * box_rows * 128;
                             tc::tma_load_2d(dst, &tmap_k, bar, 0, row);
                             tc::bulk_load(kscl + (size_t)stage * C::kScaleStageBytes + (size_t)j * box_rows * 4,
@@ -319,7 +339,7 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
                 for (int64_t f = f_begin; f < f_end; ++f) {
                     locate(prefix, n_groups, f, g, kt);
                     if (g != cur) {
-                        if (!tc::mbar_wait(kF16 ? q_ready : q_full, q_phase, abort_flag)) break;
+                        if (!tc::mbar_wait((kF16 || kSp) ? q_ready : q_full, q_phase, abort_flag)) break;
                         if (kBs && !tc::mbar_wait(q_ready, q_phase, abort_flag)) break;
                         q_phase ^= 1;
                         cur = g;
@@ -329,8 +349,15 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
                     if (!tc::mbar_wait(&acc_empty[acc], acc_phase ^ 1, abort_flag)) break;
                     tc::tc_fence_after();
                     const uint32_t a_addr = tc::smem_u32(tiles + (size_t)stage * C::kTile);
-                    const uint32_t d = tmem_base + acc * N;
-                    if (kBs) {
+                    const uint32_t d = tmem_base + acc * C::kNm;
+                    if (kSp) {
+                        // four K = 32 steps through the 128-byte code rows of the keys and of the
+                        // 2N query code rows (hi rows 0..N-1, lo rows N..2N-1)
+#pragma unroll
+                        for (int k = 0; k < kDI / 32; ++k)
+                            tc::mma_f8(d, tc::sw128_desc(a_addr + k * 32, 16, 1024),
+                                       tc::sw128_desc(q_addr + k * 32, 16, 1024), kIdesc, k > 0 ? 1u : 0u);
+                    } else if (kBs) {
                         // four K = 32 steps through the 128-byte code rows; step k reads byte k
                         // of every key's and query row's scale word
 #pragma unroll
@@ -383,6 +410,7 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
             int32_t seq_b = 0;
             const int epi_pshift = (v.page_size & (v.page_size - 1)) == 0 ? __ffs(v.page_size) - 1 : -1;
             uint32_t qf_phase = 0;
+            uint32_t es = 0, ephase = 0;   // split queries: the key-scale slot of tile f
             tc::WarpSetSync epi_sync{epi_bar, 0};
             for (int64_t f = f_begin; f < f_end; ++f) {
                 locate(prefix, n_groups, f, g, kt);
@@ -432,6 +460,82 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
                             }
                         }
                         tc::fence_async_smem();   // the f16 queries -> the tensor core
+                    } else if (kSp) {
+                        // the group's queries (TMA-landed bf16, two 64-dim swizzled halves) become
+                        // E4M3 code rows in place.  Row i (query row x head) is scaled by 2^-e so
+                        // that its largest magnitude x_max lies in [2^7, 2^8), its weight by 2^e;
+                        // then hi = E4M3(x) and lo = E4M3(16 (x - hi)).  A bf16 x has 8 significant
+                        // bits and hi keeps the top 4, so x - hi is a multiple of x's last bit of at
+                        // most 4 bits, and x = hi + lo / 16 exactly wherever |x| >= 2^-6 (below,
+                        // the error is under 2^-14, 2^-21 of x_max).  Code row i takes hi and row
+                        // N + i takes lo: the bytes of bf16 half 0 and half 1 of row i, which the
+                        // row's two threads (one per half, adjacent lanes) both read before either
+                        // writes.
+                        if (!tc::mbar_wait(q_full, qf_phase, abort_flag)) break;
+                        qf_phase ^= 1;
+                        const int hf = et & 1;
+                        static_assert(N % (kEpiThreads / 2) == 0, "every lane takes the same rows");
+                        for (int i = et >> 1; i < N; i += kEpiThreads / 2) {
+                            const int sw = i & 7;   // 128-byte swizzle: chunk c of row i at c ^ (i & 7)
+                            const uint8_t* src = qbuf + (size_t)hf * (N * 128) + (size_t)i * 128;
+                            uint4 x[8];          // x[L]: dims 64 hf + 8 L .. + 7
+                            float mx = 0.f;
+#pragma unroll
+                            for (int L = 0; L < 8; ++L) {
+                                x[L] = *reinterpret_cast<const uint4*>(src + ((L ^ sw) * 16));
+                                const uint32_t wv[4] = {x[L].x, x[L].y, x[L].z, x[L].w};
+#pragma unroll
+                                for (int qq = 0; qq < 4; ++qq) {
+                                    const float2 f2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&wv[qq]));
+                                    mx = fmaxf(mx, fmaxf(fabsf(f2.x), fabsf(f2.y)));
+                                }
+                            }
+                            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+                            const int e = mx > 0.f ? min(100, max(-100, floor_log2_f(mx) - 7)) : 0;
+                            const float f = __uint_as_float((uint32_t)(127 - e) << 23);
+                            uint32_t hi[16], lo[16];   // this thread's 64 codes of each, 4 per word
+#pragma unroll
+                            for (int L = 0; L < 8; ++L) {
+                                const uint32_t wv[4] = {x[L].x, x[L].y, x[L].z, x[L].w};
+#pragma unroll
+                                for (int qq = 0; qq < 4; ++qq) {
+                                    const float2 f2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&wv[qq]));
+                                    const float2 xs = make_float2(f2.x * f, f2.y * f);
+                                    const __nv_fp8x2_storage_t h = __nv_cvt_float2_to_fp8x2(xs, __NV_SATFINITE, __NV_E4M3);
+                                    const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(h, __NV_E4M3);
+                                    const float2 hv = __half22float2(*reinterpret_cast<const __half2*>(&hr));
+                                    const float2 rs = make_float2((xs.x - hv.x) * 16.f, (xs.y - hv.y) * 16.f);
+                                    const __nv_fp8x2_storage_t l = __nv_cvt_float2_to_fp8x2(rs, __NV_SATFINITE, __NV_E4M3);
+                                    // codes 8 L + 2 qq and + 1 of this thread's 64
+                                    if ((qq & 1) == 0) {
+                                        hi[2 * L + (qq >> 1)] = (uint32_t)h;
+                                        lo[2 * L + (qq >> 1)] = (uint32_t)l;
+                                    } else {
+                                        hi[2 * L + (qq >> 1)] |= (uint32_t)h << 16;
+                                        lo[2 * L + (qq >> 1)] |= (uint32_t)l << 16;
+                                    }
+                                }
+                            }
+                            __syncwarp();   // both halves of row i are in registers
+                            uint8_t* hrow = qbuf + (size_t)i * 128;
+                            uint8_t* lrow = qbuf + (size_t)(N + i) * 128;   // (N + i) & 7 == i & 7
+#pragma unroll
+                            for (int j = 0; j < 4; ++j) {   // 16-code chunk 4 hf + j of the code rows
+                                const int cc = ((4 * hf + j) ^ sw) * 16;
+                                *reinterpret_cast<uint4*>(hrow + cc) =
+                                    make_uint4(hi[4 * j], hi[4 * j + 1], hi[4 * j + 2], hi[4 * j + 3]);
+                                *reinterpret_cast<uint4*>(lrow + cc) =
+                                    make_uint4(lo[4 * j], lo[4 * j + 1], lo[4 * j + 2], lo[4 * j + 3]);
+                            }
+                            __syncwarp();
+                            if (hf == 0) {
+                                const int t = g * G + i / kHI;
+                                w_s[i] = t < v.T_q ? w[(int64_t)t * kHI + (i % kHI)] *
+                                                         __uint_as_float((uint32_t)(127 + e) << 23)
+                                                   : 0.f;
+                            }
+                        }
+                        tc::fence_async_smem();   // the query codes -> the tensor core
                     } else {
                         for (int i = et; i < N; i += kEpiThreads) {
                             const int t = g * G + i / kHI;
@@ -464,15 +568,26 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
                         }
                     }
                     if (!epi_sync.sync(abort_flag)) break;   // the new weights are in place
-                    if ((kF16 || kBs) && lane == 0) tc::mbar_arrive(q_ready);
+                    if ((kF16 || kBs || kSp) && lane == 0) tc::mbar_arrive(q_ready);
                     cur = g;
                 }
                 if (!tc::mbar_wait(&acc_full[acc], acc_phase, abort_flag)) break;
                 tc::tc_fence_after();
                 const int s = kt * kBM + r_in_tile;
-                const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + acc * N;
+                const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + acc * C::kNm;
                 float kscale = 1.f;
-                if (kFp8) {
+                if (kSp) {
+                    // the key's fp32 scale, bulk-copied with the codes into the stage's slot
+                    // (waiting on the stage's own barrier makes the copy visible here)
+                    if (!tc::mbar_wait(&full[es], ephase, abort_flag)) break;
+                    kscale = reinterpret_cast<const float*>(kscl + (size_t)es * C::kScaleStageBytes)[r_in_tile];
+                    __syncwarp();
+                    if (lane == 0) tc::mbar_arrive(&sf_full[es]);
+                    if (++es == (uint32_t)S) {
+                        es = 0;
+                        ephase ^= 1;
+                    }
+                } else if (kKeyScale) {
                     int pmax = -1;
 #pragma unroll
                     for (int j = 0; j < G; ++j) pmax = max(pmax, row_pos[j]);
@@ -497,7 +612,21 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
                     float a[64];
                     const float* wj = w_s + j * kHI;
                     float sc = 0.f;
-                    if constexpr (G == 1) {
+                    if constexpr (kSp) {
+                        // head h: hi . k in column h, lo . k in column 64 + h; q . k = hi + lo / 16
+                        float p0 = 0.f, p1 = 0.f;
+#pragma unroll
+                        for (int hh = 0; hh < 2; ++hh) {
+                            tc::tmem_ld32(taddr + 32 * hh, a);
+                            tc::tmem_ld32(taddr + kHI + 32 * hh, a + 32);
+#pragma unroll
+                            for (int h = 0; h < 32; h += 2) {
+                                p0 = fmaf(wj[32 * hh + h], fmaxf(fmaf(a[32 + h], 0.0625f, a[h]), 0.f), p0);
+                                p1 = fmaf(wj[32 * hh + h + 1], fmaxf(fmaf(a[33 + h], 0.0625f, a[h + 1]), 0.f), p1);
+                            }
+                        }
+                        sc = p0 + p1;
+                    } else if constexpr (G == 1) {
                         tc::tmem_ld32(taddr, a);
                         tc::tmem_ld32(taddr + 32, a + 32);
 #pragma unroll
@@ -516,7 +645,7 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
                         }
                         sc = (p0 + p1) + (p2 + p3);
                     }
-                    if (kFp8) sc *= kscale;   // positive per-key scale factors out of the ReLU sum
+                    if (kKeyScale) sc *= kscale;   // positive per-key scale factors out of the ReLU sum
                     if (s <= row_pos[j]) scores[(int64_t)(g * G + j) * ld + s] = sc;
                 }
                 tc::tc_fence_before();
@@ -644,9 +773,9 @@ int num_sms() {
     return n;
 }
 
-template <int G, bool kFp8, bool kMx, bool kBs = false>
+template <int G, bool kFp8, bool kMx, bool kBs = false, bool kSp = false>
 cudaError_t launch_g(const IndexScoreArgs& a, cudaStream_t st) {
-    using C = Cfg<G, kFp8, kMx, kBs>;
+    using C = Cfg<G, kFp8, kMx, kBs, kSp>;
     const int box_rows = a.seq.page_size <= kBM ? a.seq.page_size : kBM;
     const uint64_t slots = (uint64_t)a.seq.num_pages * a.seq.page_size;
     CUtensorMap tk, tq;
@@ -657,7 +786,9 @@ cudaError_t launch_g(const IndexScoreArgs& a, cudaStream_t st) {
              make_tensor_map_2d(&tq, a.q_I, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)a.seq.T_q * kHI,
                                 kDI, kDI, kDI, C::N, CU_TENSOR_MAP_SWIZZLE_128B);
     } else {
-        ok = kFp8 ? make_tensor_map_2d(&tk, a.k_cache, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, slots, kDI,
+        ok = kSp ? make_tensor_map_2d(&tk, a.k_cache, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, slots, kDI, kDI,
+                                      kDI, box_rows, CU_TENSOR_MAP_SWIZZLE_128B)
+           : kFp8 ? make_tensor_map_2d(&tk, a.k_cache, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, slots, kDI,
                                        kDI, kDI, box_rows, CU_TENSOR_MAP_SWIZZLE_NONE)
                   : make_tensor_map_2d(&tk, a.k_cache, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, slots,
                                        kDI, kDI * 2, 64, box_rows, CU_TENSOR_MAP_SWIZZLE_128B);
@@ -666,7 +797,7 @@ cudaError_t launch_g(const IndexScoreArgs& a, cudaStream_t st) {
                                       CU_TENSOR_MAP_SWIZZLE_128B);
     }
     if (!ok) return cudaErrorInvalidValue;
-    auto kern = index_score_tc_kernel<G, kFp8, kMx, kBs>;
+    auto kern = index_score_tc_kernel<G, kFp8, kMx, kBs, kSp>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::kSmem);
     if (e != cudaSuccess) return e;
     const int rows_per_launch = C::kMaxGroups * G;
@@ -715,6 +846,8 @@ cudaError_t launch_index_score_tc(const IndexScoreArgs& a, cudaStream_t st) {
         return mx ? launch_g<4, true, true>(a, st) : fp8 ? launch_g<4, true, false>(a, st) : launch_g<4, false, false>(a, st);
     if (a.q_run % 2 == 0)
         return mx ? launch_g<2, true, true>(a, st) : fp8 ? launch_g<2, true, false>(a, st) : launch_g<2, false, false>(a, st);
+    if (fp8 && (reinterpret_cast<uintptr_t>(a.k_scale) & 15) == 0)   // split queries: scales by bulk copy
+        return launch_g<1, false, false, false, true>(a, st);
     return mx ? launch_g<1, true, true>(a, st) : fp8 ? launch_g<1, true, false>(a, st) : launch_g<1, false, false>(a, st);
 }
 

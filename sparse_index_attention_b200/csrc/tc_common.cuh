@@ -195,6 +195,24 @@ __host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N) {
            | ((uint32_t)(M >> 4) << 24); // M / 16
 }
 
+// Instruction descriptor for kind::f8f6f4: E4M3 A and B (both K-major), fp32 D, M x N tile.
+__host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N) {
+    return (1u << 4)                     // D format: f32
+           | ((uint32_t)(N >> 3) << 17)  // N / 8 (A and B format 0: E4M3)
+           | ((uint32_t)(M >> 4) << 24); // M / 16
+}
+
+// D[tmem] (+)= A[smem] * B[smem]^T, kind::f8f6f4 (8-bit inputs, fp32 accumulate, K = 32 per
+// instruction), one CTA.
+__device__ __forceinline__ void mma_f8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                       uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+        " tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n}\n" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
 // Instruction descriptor for kind::mxf8f6f4 with block scaling: E4M3 A and B (both K-major),
 // fp32 D, E8M0 scale factors, one per 32 consecutive K elements.  One MMA covers K = 32, so it
 // reads one scale per row of A and one per row of B: byte a_sf (b_sf) of the 32-bit TMEM words

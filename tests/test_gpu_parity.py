@@ -204,6 +204,37 @@ def test_index_score_fp8_every_code_bit_exact():
     assert np.array_equal(sc[0, :n].cpu().numpy(), ref)
 
 
+def test_index_score_fp8_integer_inputs_bit_exact_both_paths():
+    """E4M3 keys holding small integers with power-of-two scales, integer bf16 queries and
+    power-of-two weights: every product and partial sum is exact in fp32 in any order, so the
+    score must equal the float64 oracle bit for bit.  Through the 8-bit MMA on split queries
+    (hi + lo / 16; the scale array 16-byte aligned) and through the widening path (the same
+    scales one float off 16-byte alignment)."""
+    wl = workloads.make("decode_fp8", DEV, B=3, L=900)
+    g = torch.Generator(device=DEV).manual_seed(78)
+    slots = wl.num_pages * wl.page_size
+    q = torch.randint(-31, 32, wl.q_I.shape, generator=g, device=DEV).to(torch.bfloat16)
+    kint = torch.randint(-4, 5, (slots, wl.D_I), generator=g, device=DEV)
+    lut = torch.from_numpy(oracle.e4m3_encode(np.arange(-4, 5)).astype(np.uint8)).to(DEV)
+    k8 = lut[kint + 4].contiguous()
+    scale = torch.exp2(torch.randint(0, 2, (slots,), generator=g, device=DEV).float())
+    e = torch.randint(-2, 1, wl.w.shape, generator=g, device=DEV).float()
+    w = torch.exp2(e) * torch.where(torch.rand(wl.w.shape, generator=g, device=DEV) < 0.5, -1.0, 1.0)
+    seq = paged_seq(wl)
+    k_exact = oracle.e4m3_decode(k8.cpu().numpy()) * scale.cpu().double().numpy()[:, None]
+    off = torch.zeros(slots + 1, dtype=torch.float32, device=DEV)
+    off[1:] = scale
+    for ks in (scale, off[1:]):
+        assert (ks.data_ptr() % 16 == 0) == (ks is scale)
+        sc = hsa.hsa_index_score(seq, q, w, k8, ks)
+        check_status(seq)
+        ref = oracle.index_score(oracle_paging(wl), q.cpu(), w.cpu(), k_exact, ld=sc.shape[1])
+        got = sc.cpu().numpy()
+        for t in range(wl.T_q):
+            n = int(wl.q_pos[t]) + 1
+            assert np.array_equal(got[t, :n].astype(np.float64), ref[t, :n]), t
+
+
 def test_index_score_mxfp8_every_code_bit_exact():
     """Every finite E4M3 code through the MXFP8 key path of the tensor-core kernel, with the four
     block exponents of a key all different and the largest one in any of the four blocks.  Key s
