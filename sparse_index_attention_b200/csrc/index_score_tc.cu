@@ -17,21 +17,22 @@
 // changes.  Every CTA derives the list itself from q_pos (prefix sum in shared memory).
 //
 // Data movement.  Keys come through the block table page by page with 2D TMA loads (128-byte
-// swizzle, two 64-column halves per page).  E4M3 keys with one query row per tile (and a
-// 16-byte-aligned scale array) go straight from TMA to an 8-bit MMA (kind::f8f6f4): each bf16 query row x head is split exactly into two
-// E4M3 code rows, hi and lo / 16 (scaled per head by a power of two folded into its weight), so
-// one MMA of N = 128 gives hi . k and lo . k per head, and the per-key fp32 scales are
-// bulk-copied beside the codes for the epilogue.  Otherwise the E4M3 codes are loaded raw and widened in shared memory by four converter warps (E4M3 -> f16 in one
-// conversion, exact; the MMA then runs in f16, the queries rescaled into f16's range per head).
-// Either way the per-key fp32 scale multiplies the finished score (the scale is positive, so it
-// commutes with the ReLU sum).  MXFP8 keys (one
-// E8M0 byte per 32 dims; "Inference Adaptation and Performance Optimization for a Domestically
-// Developed LLM's New Architecture", section 4 table) with bf16 queries take the same path: the
-// producer bulk-copies each box's scale words beside its codes, the converters place the codes'
-// bits in bf16s and scale each 32-dim block by 2^(E_block - E_max) with one packed multiply
-// (exact), and the epilogue multiplies the score by 2^(E_max - 127), the key's largest block
-// scale.  MXFP8 keys with MXFP8 queries skip the converters: the codes go straight to a
-// block-scaled MMA (kind::mxf8f6f4) that reads the E8M0 scales from TMEM.
+// swizzle, two 64-column halves per page).  E4M3 keys (with a 16-byte-aligned scale array) go
+// straight from TMA to 8-bit MMAs (kind::f8f6f4): each bf16 query row x head is split into two
+// E4M3 code rows, hi and lo (scaled per head by a power of two folded into its weight), and the
+// MMAs of both accumulate into one accumulator, hi . k + lo . k = q . k; the per-key fp32
+// scales are bulk-copied beside the codes for the epilogue.  Otherwise the E4M3 codes are
+// loaded raw and widened in shared memory by converter warps (E4M3 -> f16 in one conversion,
+// exact; the MMA then runs in f16, the queries rescaled into f16's range per head).  Either way
+// the per-key fp32 scale multiplies the finished score (the scale is positive, so it commutes
+// with the ReLU sum).  MXFP8 keys (one E8M0 byte per 32 dims; "Inference Adaptation and
+// Performance Optimization for a Domestically Developed LLM's New Architecture", section 4
+// table) with bf16 queries are widened too: the producer bulk-copies each box's scale words
+// beside its codes, the converters place the codes' bits in bf16s and scale each 32-dim block
+// by 2^(E_block - E_max) with one packed multiply (exact), and the epilogue multiplies the score
+// by 2^(E_max - 127), the key's largest block scale.  MXFP8 keys with MXFP8 queries skip the
+// converters: the codes go straight to a block-scaled MMA (kind::mxf8f6f4) that reads the E8M0
+// scales from TMEM.
 //
 // Warp roles: 0 TMA producer, 1 MMA issuer (one elected thread each), 2-5 epilogue
 // (TMEM lane quarters 2,3,0,1), 6-9 (6-13 for E4M3 keys with one row per tile) FP8 converters
@@ -56,13 +57,12 @@ constexpr int kTileBytes = 2 * kHalfBytes;
 template <int G, bool kFp8, bool kMx = false, bool kBs = false, bool kSp = false>
 struct Cfg {
     static_assert(!kBs || (G <= 2 && !kFp8 && !kMx), "block-scaled: codes straight to the MMA, G <= 2");
-    static_assert(!kSp || (G == 1 && !kFp8 && !kMx && !kBs), "split queries: E4M3 codes straight to the MMA, G = 1");
+    static_assert(!kSp || (!kFp8 && !kMx && !kBs), "split queries: E4M3 codes straight to the MMA");
     static constexpr int N = G * kHI;
-    // MMA N = TMEM columns per accumulator: the split-query path holds two code rows per head
-    static constexpr int kNm = kSp ? 2 * N : N;
+    static constexpr int kNm = N;   // MMA N = TMEM columns per accumulator
     static constexpr int kTile = (kBs || kSp) ? kBM * kDI : kTileBytes;  // one MMA stage: 16 KB codes or 32 KB bf16
     static constexpr int kQBytes = N * kDI * (kBs ? 1 : 2);
-    static constexpr int kStages = kSp ? 12 : kBs ? (G == 1 ? 8 : 6)
+    static constexpr int kStages = kSp ? (G == 1 ? 12 : (G == 2 ? 10 : 8)) : kBs ? (G == 1 ? 8 : 6)
                                        : kFp8 ? (G == 1 ? 4 : (G == 2 ? 3 : 2)) : (G == 1 ? 6 : (G == 2 ? 5 : 4));
     static constexpr int kRawStages = kFp8 ? 4 : 0;          // FP8 staging tiles (16 KB each)
     static constexpr int kR = kRawStages > 0 ? kRawStages : 1;
@@ -148,9 +148,9 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
                       float* __restrict__ scores, int64_t ld, int32_t box_rows) {
     using C = Cfg<G, kFp8, kMx, kBs, kSp>;
     static_assert(!kMx || kFp8, "MXFP8 keys go through the FP8 staging path");
-    // kSp (E4M3 keys with fp32 scales, one query row per tile): the key codes go from TMA straight
-    // to a kind::f8f6f4 MMA.  Each bf16 query row x head is split exactly into two E4M3 code rows
-    // (hi and lo / 16, below), so one MMA of N = 128 gives both partial dot products per head.
+    // kSp (E4M3 keys with fp32 scales, bf16 queries): the key codes go from TMA straight to
+    // kind::f8f6f4 MMAs.  Each bf16 query row x head is split into two E4M3 code rows, hi and lo
+    // (below), and both MMAs accumulate into one accumulator: hi . k + lo . k = q . k.
     constexpr bool kKeyScale = kFp8 || kSp;   // a per-key scale multiplies the finished score
     constexpr bool kCodes = kBs || kSp;       // 8-bit codes straight into the MMA stages
     // E4M3 keys with fp32 scales run the MMA in f16: a code widens to f16 in one conversion
@@ -159,7 +159,7 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
     constexpr bool kF16 = kFp8 && !kMx;
     constexpr int N = C::N;
     constexpr int S = C::kStages;
-    constexpr uint32_t kIdesc = kSp ? tc::idesc_e4m3_f32(kBM, C::kNm)
+    constexpr uint32_t kIdesc = kSp ? tc::idesc_e4m3_f32(kBM, N)
                               : kF16 ? tc::idesc_f16_f32(kBM, N) : tc::idesc_bf16_f32(kBM, N, 0, 0);
     // kBs (MXFP8 queries and keys): the codes go from TMA straight to a block-scaled MMA
     // (kind::mxf8f6f4, K = 32 per instruction, one E8M0 scale per 32 dims of every key and
@@ -200,7 +200,7 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
         for (int i = 0; i < S; ++i) {
             tc::mbar_init(&full[i], kFp8 ? 32 * C::kConv : 1);
             tc::mbar_init(&empty[i], 1);
-            tc::mbar_init(&sf_full[i], 4);
+            tc::mbar_init(&sf_full[i], kSp ? C::kEpiWarps : 4);
         }
         for (int i = 0; i < C::kAcc; ++i) {
             tc::mbar_init(&acc_full[i], 1);
@@ -351,12 +351,14 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
                     const uint32_t a_addr = tc::smem_u32(tiles + (size_t)stage * C::kTile);
                     const uint32_t d = tmem_base + acc * C::kNm;
                     if (kSp) {
-                        // four K = 32 steps through the 128-byte code rows of the keys and of the
-                        // 2N query code rows (hi rows 0..N-1, lo rows N..2N-1)
+                        // four K = 32 steps through the 128-byte code rows of the keys against the
+                        // hi query rows, then four against the lo rows (N rows further on), all
+                        // into the one accumulator
 #pragma unroll
-                        for (int k = 0; k < kDI / 32; ++k)
-                            tc::mma_f8(d, tc::sw128_desc(a_addr + k * 32, 16, 1024),
-                                       tc::sw128_desc(q_addr + k * 32, 16, 1024), kIdesc, k > 0 ? 1u : 0u);
+                        for (int k = 0; k < 2 * (kDI / 32); ++k)
+                            tc::mma_f8(d, tc::sw128_desc(a_addr + (k & 3) * 32, 16, 1024),
+                                       tc::sw128_desc(q_addr + (k >> 2) * (N * 128) + (k & 3) * 32, 16, 1024),
+                                       kIdesc, k > 0 ? 1u : 0u);
                     } else if (kBs) {
                         // four K = 32 steps through the 128-byte code rows; step k reads byte k
                         // of every key's and query row's scale word
@@ -464,13 +466,13 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
                         // the group's queries (TMA-landed bf16, two 64-dim swizzled halves) become
                         // E4M3 code rows in place.  Row i (query row x head) is scaled by 2^-e so
                         // that its largest magnitude x_max lies in [2^7, 2^8), its weight by 2^e;
-                        // then hi = E4M3(x) and lo = E4M3(16 (x - hi)).  A bf16 x has 8 significant
-                        // bits and hi keeps the top 4, so x - hi is a multiple of x's last bit of at
-                        // most 4 bits, and x = hi + lo / 16 exactly wherever |x| >= 2^-6 (below,
-                        // the error is under 2^-14, 2^-21 of x_max).  Code row i takes hi and row
-                        // N + i takes lo: the bytes of bf16 half 0 and half 1 of row i, which the
-                        // row's two threads (one per half, adjacent lanes) both read before either
-                        // writes.
+                        // then hi = E4M3(x) and lo = E4M3(x - hi).  A bf16 x has 8 significant
+                        // bits and hi keeps the top 4, so x - hi is at most 8 times x's last bit,
+                        // a multiple of it: x = hi + lo exactly wherever |x| >= 2^-2, which E4M3's
+                        // smallest step (2^-9) reaches; below, the error is under 2^-10, 2^-17 of
+                        // x_max.  Code row i takes hi and row N + i takes lo: the bytes of bf16
+                        // half 0 and half 1 of row i, which the row's two threads (one per half,
+                        // adjacent lanes) both read before either writes.
                         if (!tc::mbar_wait(q_full, qf_phase, abort_flag)) break;
                         qf_phase ^= 1;
                         const int hf = et & 1;
@@ -504,7 +506,7 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
                                     const __nv_fp8x2_storage_t h = __nv_cvt_float2_to_fp8x2(xs, __NV_SATFINITE, __NV_E4M3);
                                     const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(h, __NV_E4M3);
                                     const float2 hv = __half22float2(*reinterpret_cast<const __half2*>(&hr));
-                                    const float2 rs = make_float2((xs.x - hv.x) * 16.f, (xs.y - hv.y) * 16.f);
+                                    const float2 rs = make_float2(xs.x - hv.x, xs.y - hv.y);
                                     const __nv_fp8x2_storage_t l = __nv_cvt_float2_to_fp8x2(rs, __NV_SATFINITE, __NV_E4M3);
                                     // codes 8 L + 2 qq and + 1 of this thread's 64
                                     if ((qq & 1) == 0) {
@@ -612,21 +614,7 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
                     float a[64];
                     const float* wj = w_s + j * kHI;
                     float sc = 0.f;
-                    if constexpr (kSp) {
-                        // head h: hi . k in column h, lo . k in column 64 + h; q . k = hi + lo / 16
-                        float p0 = 0.f, p1 = 0.f;
-#pragma unroll
-                        for (int hh = 0; hh < 2; ++hh) {
-                            tc::tmem_ld32(taddr + 32 * hh, a);
-                            tc::tmem_ld32(taddr + kHI + 32 * hh, a + 32);
-#pragma unroll
-                            for (int h = 0; h < 32; h += 2) {
-                                p0 = fmaf(wj[32 * hh + h], fmaxf(fmaf(a[32 + h], 0.0625f, a[h]), 0.f), p0);
-                                p1 = fmaf(wj[32 * hh + h + 1], fmaxf(fmaf(a[33 + h], 0.0625f, a[h + 1]), 0.f), p1);
-                            }
-                        }
-                        sc = p0 + p1;
-                    } else if constexpr (G == 1) {
+                    if constexpr (G == 1) {
                         tc::tmem_ld32(taddr, a);
                         tc::tmem_ld32(taddr + 32, a + 32);
 #pragma unroll
@@ -846,8 +834,11 @@ cudaError_t launch_index_score_tc(const IndexScoreArgs& a, cudaStream_t st) {
         return mx ? launch_g<4, true, true>(a, st) : fp8 ? launch_g<4, true, false>(a, st) : launch_g<4, false, false>(a, st);
     if (a.q_run % 2 == 0)
         return mx ? launch_g<2, true, true>(a, st) : fp8 ? launch_g<2, true, false>(a, st) : launch_g<2, false, false>(a, st);
-    if (fp8 && (reinterpret_cast<uintptr_t>(a.k_scale) & 15) == 0)   // split queries: scales by bulk copy
+    if (fp8 && (reinterpret_cast<uintptr_t>(a.k_scale) & 15) == 0) {   // split queries: scales by bulk copy
+        if (a.q_run % 4 == 0) return launch_g<4, false, false, false, true>(a, st);
+        if (a.q_run % 2 == 0) return launch_g<2, false, false, false, true>(a, st);
         return launch_g<1, false, false, false, true>(a, st);
+    }
     return mx ? launch_g<1, true, true>(a, st) : fp8 ? launch_g<1, true, false>(a, st) : launch_g<1, false, false>(a, st);
 }
 

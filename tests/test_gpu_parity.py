@@ -204,13 +204,19 @@ def test_index_score_fp8_every_code_bit_exact():
     assert np.array_equal(sc[0, :n].cpu().numpy(), ref)
 
 
-def test_index_score_fp8_integer_inputs_bit_exact_both_paths():
+@pytest.mark.parametrize("name,kw,q_run", [
+    ("decode_fp8", dict(B=3, L=900), 1),                      # one query row per tile
+    ("prefill_long_zigzag", dict(T=700, n_chunks=4), 2),      # two rows per tile
+    ("prefill_long_zigzag", dict(T=700, n_chunks=4), 4),      # four rows per tile
+])
+def test_index_score_fp8_integer_inputs_bit_exact_both_paths(name, kw, q_run):
     """E4M3 keys holding small integers with power-of-two scales, integer bf16 queries and
     power-of-two weights: every product and partial sum is exact in fp32 in any order, so the
-    score must equal the float64 oracle bit for bit.  Through the 8-bit MMA on split queries
-    (hi + lo / 16; the scale array 16-byte aligned) and through the widening path (the same
-    scales one float off 16-byte alignment)."""
-    wl = workloads.make("decode_fp8", DEV, B=3, L=900)
+    score must equal the float64 oracle bit for bit.  Through the 8-bit MMAs on split queries
+    (hi + lo; the scale array 16-byte aligned) and through the widening path (the same scales
+    one float off 16-byte alignment), for one, two and four query rows per tile."""
+    wl = workloads.make(name, DEV, **kw)
+    wl.q_run = q_run
     g = torch.Generator(device=DEV).manual_seed(78)
     slots = wl.num_pages * wl.page_size
     q = torch.randint(-31, 32, wl.q_I.shape, generator=g, device=DEV).to(torch.bfloat16)
