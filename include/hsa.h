@@ -116,7 +116,9 @@ typedef struct hsa_paged_seq {
  * cache, summed with per-head weights); fifth page 3.1 (LI); BF16 and
  * quantized index paths, second page 3.1; MXFP8 index keys, fifth page 4 (table).  The
  * tensor-core kernel serves q BF16, k BF16/E4M3/MXE4M3, H_I = 64, D_I = 128, page_size a
- * multiple of 8; other shapes use a CUDA-core kernel. */
+ * multiple of 8; other shapes use a CUDA-core kernel.  With E4M3 keys a 16-byte-aligned k_scale
+ * lets the codes go straight to 8-bit MMAs (each bf16 query split into two E4M3 parts); a
+ * k_scale aligned to 4 bytes only is served by widening the codes, with the same contract. */
 HSA_API hsa_status_t hsa_index_score(const hsa_paged_seq_t* seq, const void* q_I, hsa_dtype_t q_dtype,
                              const float* w, int32_t H_I, int32_t D_I, const void* k_cache,
                              hsa_dtype_t k_dtype, const void* k_scale, float* scores,
