@@ -14,8 +14,11 @@
 //   sample    4096 evenly spaced keys; a two-pass radix select on them gives a threshold L a few
 //             standard deviations below the sample's estimate of T, so that the row holds K or
 //             more keys >= L with overwhelming probability;
-//   collect   warps sweep contiguous segments of the row: a ballot count, a scan over the warps,
-//             and a second sweep that writes every key >= L with its position, in position order;
+//   collect   warps sweep contiguous segments of the row and keep every key >= L with its
+//             position, in position order: a staged row takes a ballot count, a scan over the
+//             warps and a second sweep that writes at the scanned offsets; a row read from L2
+//             takes one sweep that appends to a stretch per warp, then the stretches are moved
+//             down end to end (the two-sweep form if a stretch overflows);
 //   select    a three-pass radix select (digits of 11, 11 and 10 bits) over the candidates finds
 //             T exactly and how many elements equal to T are selected;
 //   write     a ballot sweep over the candidates places each selected position.
@@ -252,6 +255,16 @@ topk_kernel(SeqView v, const float* __restrict__ scores, int64_t ld, int K, int 
             // warp segments of whole 128-key chunks, swept kSweep keys per lane at a time
             const int seg = ((n + kWarps * 128 - 1) / (kWarps * 128)) * 128;
             const int s0 = min(n, warp * seg), s1 = min(n, s0 + seg);
+            // Rows read from L2: one sweep both counts and collects.  Each warp appends its keys
+            // >= L, in position order, to its own stretch of the upper half of the candidate
+            // arrays (a key past the end of the stretch is counted, not stored), and the
+            // stretches are then moved down end to end.  If a stretch overflowed (heavy ties),
+            // the second sweep below collects instead.  Staged rows count, then collect.
+            constexpr bool kOneSweep = !kStaged;
+            const int cap_w = kOneSweep ? (cand_cap / 2) / kWarps : 0;
+            uint32_t* own_key = cand_key + cand_cap / 2 + warp * cap_w;
+            uint32_t* own_pos = cand_pos + cand_cap / 2 + warp * cap_w;
+            const uint32_t lt = lanemask_lt();
             uint32_t c = 0u;
             for (int j = s0; j < s1; j += 32 * kSweep<kStaged>) {
                 uint32_t u[kSweep<kStaged>];
@@ -263,11 +276,19 @@ topk_kernel(SeqView v, const float* __restrict__ scores, int64_t ld, int K, int 
 #pragma unroll
                 for (int a = 0; a < kSweep<kStaged>; ++a) {
                     const int i = j + 32 * a + lane;
-                    c += (uint32_t)__popc(__ballot_sync(0xffffffffu, i < s1 && u[a] >= L));
+                    const uint32_t bal = __ballot_sync(0xffffffffu, i < s1 && u[a] >= L);
+                    if constexpr (kOneSweep) {
+                        const uint32_t p = c + (uint32_t)__popc(bal & lt);
+                        if (((bal >> lane) & 1u) && p < (uint32_t)cap_w) {
+                            own_key[p] = u[a];
+                            own_pos[p] = (uint32_t)i;
+                        }
+                    }
+                    c += (uint32_t)__popc(bal);
                 }
             }
             if (lane == 0) wsum[warp] = c;
-            __syncthreads();
+            const bool spilled = __syncthreads_or(kOneSweep && c > (uint32_t)cap_w);
             uint32_t before = lane < warp ? (uint32_t)wsum[lane] : 0u;
             uint32_t total = (uint32_t)wsum[lane];
 #pragma unroll
@@ -276,8 +297,15 @@ topk_kernel(SeqView v, const float* __restrict__ scores, int64_t ld, int K, int 
                 total += __shfl_xor_sync(0xffffffffu, total, o);
             }
             __syncthreads();
-            if (total >= (uint32_t)K && total <= (uint32_t)cand_cap) {     // the same in every thread
-                const uint32_t lt = lanemask_lt();
+            // (every condition below is the same in every thread)
+            if (kOneSweep && !spilled && total >= (uint32_t)K && total <= (uint32_t)(cand_cap / 2)) {
+                for (uint32_t k = lane; k < c; k += 32) {   // stretch -> [before, before + c)
+                    cand_key[before + k] = own_key[k];
+                    cand_pos[before + k] = own_pos[k];
+                }
+                n_cand = (int)total;
+                __syncthreads();
+            } else if (total >= (uint32_t)K && total <= (uint32_t)cand_cap) {
                 for (int j = s0; j < s1; j += 32 * kSweep<kStaged>) {
                     uint32_t u[kSweep<kStaged>], bal[kSweep<kStaged>];
 #pragma unroll
