@@ -355,12 +355,15 @@ def test_topk_vs_oracle_bit_exact(ties):
     (10, 131072, 2048),   # read from L2, the longest prefill context
     (80, 60003, 512),     # read from L2, small K
 ])
-@pytest.mark.parametrize("dist", ["normal", "ties", "narrow", "constant"])
+@pytest.mark.parametrize("dist", ["normal", "ties", "narrow", "constant", "clustered"])
 def test_topk_launch_variants_bit_exact(T, ld, K, dist):
     """Every path of the Top-K kernel (rows staged in shared memory or read from L2, aligned or
     unaligned row starts, sampled candidates or the whole row) on score distributions that
     stress each step: spread values, heavy ties with +-0.0, values that all share their top 22
-    key bits, and constant rows whose candidates overflow shared memory."""
+    key bits, constant rows whose candidates overflow shared memory, and the best keys packed
+    into one window of 3 K positions (on rows read from L2 the candidates of the few warps
+    that sweep the window overflow their stretches, so those rows are collected again by the
+    count-then-collect sweeps)."""
     g = torch.Generator().manual_seed(T * 7 + ld)
     lens = torch.randint(1, ld + 1, (T,), generator=g)
     lens[0], lens[1], lens[2], lens[3] = ld, K, K + 1, min(ld, 3 * K + 5)
@@ -370,6 +373,9 @@ def test_topk_launch_variants_bit_exact(T, ld, K, dist):
     elif dist == "constant":
         sc = torch.full_like(sc, 0.75)
         sc[1::2] = -0.0
+    elif dist == "clustered":
+        w0 = ld // 3
+        sc[:, w0:w0 + 3 * K] += 1000.0
     seq = hsa.PagedSeq(torch.tensor([ld], device=DEV), torch.zeros((1, ld), dtype=torch.int32, device=DEV),
                        1, ld, torch.zeros(T, dtype=torch.int32, device=DEV),
                        (lens - 1).to(torch.int32).to(DEV), max_seq_len=ld,
