@@ -58,8 +58,7 @@ template <int G, bool kFp8, bool kMx = false, bool kBs = false, bool kSp = false
 struct Cfg {
     static_assert(!kBs || (G <= 2 && !kFp8 && !kMx), "block-scaled: codes straight to the MMA, G <= 2");
     static_assert(!kSp || (!kFp8 && !kMx && !kBs), "split queries: E4M3 codes straight to the MMA");
-    static constexpr int N = G * kHI;
-    static constexpr int kNm = N;   // MMA N = TMEM columns per accumulator
+    static constexpr int N = G * kHI;   // MMA N = TMEM columns per accumulator
     static constexpr int kTile = (kBs || kSp) ? kBM * kDI : kTileBytes;  // one MMA stage: 16 KB codes or 32 KB bf16
     static constexpr int kQBytes = N * kDI * (kBs ? 1 : 2);
     static constexpr int kStages = kSp ? (G == 1 ? 12 : (G == 2 ? 10 : 8)) : kBs ? (G == 1 ? 8 : 6)
@@ -73,12 +72,12 @@ struct Cfg {
     // TMEM: kAcc accumulators of N columns (four for N <= 128, so the MMA may run up to four
     // tiles ahead of the epilogue; two for N = 256); block-scaled adds the key scales (4 columns
     // per stage) and the query scales (N / 32 columns) after them
-    static constexpr int kAcc = (kNm <= 64 || (kNm == 128 && !kBs)) ? 4 : 2;
-    static constexpr int kSfaCol = kAcc * kNm;
+    static constexpr int kAcc = (N <= 64 || (N == 128 && !kBs)) ? 4 : 2;
+    static constexpr int kSfaCol = kAcc * N;
     static constexpr int kSfbCol = kSfaCol + 4 * kStages;
-    static constexpr int kTmemCols = kBs ? 512 : kAcc * kNm;   // 256 or 512
+    static constexpr int kTmemCols = kBs ? 512 : kAcc * N;   // 256 or 512
     static_assert(!kBs || kSfbCol + N / 32 <= kTmemCols, "TMEM budget");
-    static_assert(kAcc * kNm <= kTmemCols, "TMEM budget");
+    static_assert(kAcc * N <= kTmemCols, "TMEM budget");
     // FP8 converter warps: eight for E4M3 keys with one query row per tile (the widening sets the
     // pace of the key stream there), four otherwise (measured: the MX widening is slower with eight)
     static constexpr int kConv = kFp8 ? ((G == 1 && !kMx) ? 8 : 4) : 0;
@@ -349,7 +348,7 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
                     if (!tc::mbar_wait(&acc_empty[acc], acc_phase ^ 1, abort_flag)) break;
                     tc::tc_fence_after();
                     const uint32_t a_addr = tc::smem_u32(tiles + (size_t)stage * C::kTile);
-                    const uint32_t d = tmem_base + acc * C::kNm;
+                    const uint32_t d = tmem_base + acc * N;
                     if (kSp) {
                         // four K = 32 steps through the 128-byte code rows of the keys against the
                         // hi query rows, then four against the lo rows (N rows further on), all
@@ -576,7 +575,7 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
                 if (!tc::mbar_wait(&acc_full[acc], acc_phase, abort_flag)) break;
                 tc::tc_fence_after();
                 const int s = kt * kBM + r_in_tile;
-                const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + acc * C::kNm;
+                const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + acc * N;
                 float kscale = 1.f;
                 if (kSp) {
                     // the key's fp32 scale, bulk-copied with the codes into the stage's slot
